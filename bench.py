@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of libkda's chunked KDA forward at the 64K context stage.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {libkda,reference}]
+
+One step = one kda_chunk_fwd over the 64K-stage batch (B=1, H=32, T=65536,
+dk=dv=128, bf16 inputs, fp32 state, the 5% a=+8 slice): gate, cumulative decay,
+dense 16-token tile products, WY/UT solve and the state scan, i.e. the whole hot path.
+Inputs (2.69 GB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job tokens/s with inputs resident in
+HBM; ``e2e`` is the same metric through the C ABI with pinned host buffers (H2D of every
+input and D2H of o and S_T inside the timed region).  The decode step (N=256, H=32,
+d=128, fp32 state) is measured in the same run and reported under ``decode``.
+
+Multi-GPU (torchrun): every rank runs its own 64K batch (independent sequences, no
+data-path collective: weak scaling); the step time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle (the only reference this method has) on
+a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunked_linear_attention_chunk_b200 import synth  # noqa: E402
+
+METRIC = "KDA chunk-fwd tokens/s & TFLOP/s (% of B200 BF16 peak) at T=64K; decode HBM GB/s"
+UNIT = "tokens/s"
+G_MIN = -5.0
+# Algorithmic cost of the path per token-head at d = 128 (bf16 token tensors):
+# q, k, v, a (256 B each), beta (2 B), o (256 B); states add 2 * dk*dv*4 B per head.
+BYTES_PER_TOKEN_HEAD = 4 * 256 + 2 + 256
+# Triangle-aware flops per token-head at the 16-token tile (state products W S, Qbar S,
+# Khat^T U: 6 dk dv; tile products and W: dk (3C - 1); Utilde and P U: 2 C dv; solve
+# C^2/3; Gamma scaling dk dv / C), C = 16.
+FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 128 * (3 * 16 - 1) + 2 * 16 * 128 + 16 * 16 / 3 + 128 * 128 / 16
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "chunk_fwd_traffic.json")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunked_linear_attention_chunk_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic_per_token_head():
+    """DRAM bytes per token-head of one kda_chunk_fwd from the committed ncu summary, or
+    None when the kernels changed since it was captured."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    d = json.load(open(PROFILE_TRAFFIC))
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return float(d["dram_bytes_per_token_head"])
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{self.gpu}_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- dist
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling over sequences)."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------- arms
+def time_steps(fn, steps: int, warmup: int, world: int, device):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    ms = e0.elapsed_time(e1) / steps
+    return max_over_ranks(ms, world, device)
+
+
+def cpu_baseline(x, sample_tokens: int):
+    """The fp64 oracle, as it stands, on the first ``sample_tokens`` tokens of every head."""
+    import oracle
+    from chunked_linear_attention_chunk_b200.synth import to_numpy32
+    names = ("q", "k", "v", "a", "beta")
+    arrs = [to_numpy32(x[n][:, :sample_tokens]) for n in names]
+    S0 = x["S0"].numpy().astype("float64")
+    B, _, H, _ = arrs[0].shape
+    cores = min(os.cpu_count() or 1, B * H)
+    oracle.recurrence(*(a[:, :16] for a in arrs), G_MIN, S0=S0)  # build/load outside timing
+    t = time.perf_counter()
+    oracle.recurrence(*arrs, G_MIN, S0=S0, nthreads=cores)
+    dt = time.perf_counter() - t
+    return {"value": B * sample_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {sample_tokens} of {x['q'].shape[1]} tokens, all {B * H} (batch, head) pairs "
+                      f"of the 64K stage; fp64 token-by-token recurrence, {dt:.2f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = synth.STAGE_64K
+    sample = 2048
+    x = synth.make_inputs(w.B, sample, w.H, w.dk, w.dv, w.dtype, w.seed, w.s0_std, False)
+    import oracle
+    from chunked_linear_attention_chunk_b200.synth import to_numpy32
+    names = ("q", "k", "v", "a", "beta")
+    arrs = [to_numpy32(x[n]) for n in names]
+    S0 = x["S0"].numpy().astype("float64")
+    cores = min(os.cpu_count() or 1, w.B * w.H)
+    for _ in range(args.warmup):
+        oracle.recurrence(*(a[:, :64] for a in arrs), G_MIN, S0=S0, nthreads=cores)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrence(*arrs, G_MIN, S0=S0, nthreads=cores)
+    dt = (time.perf_counter() - t) / args.steps
+    value = w.B * sample / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample_tokens_per_step": sample, "note":
+                   "fp64 CPU oracle of the recurrence; each step is a bounded sample of the 64K workload"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {sample} tokens x {w.B * w.H} (batch, head) pairs per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_libkda(args):
+    import chunked_linear_attention_chunk_b200 as kda
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    hbm_peak, bf16_peak, peak_kind = peaks()
+
+    w = synth.STAGE_64K
+    x = synth.make_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), w.s0_std, w.adversarial)
+    names = ("q", "k", "v", "a", "beta")
+    d = {n: x[n].to(device) for n in names}
+    S0 = x["S0"].to(device)
+    B, T, H, D = w.B, w.T, w.H, w.dk
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=device)
+    S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=device)
+    need = kda.kda_chunk_fwd_workspace(B, T, H, D, D)
+    ws = torch.empty(need, dtype=torch.uint8, device=device)
+
+    def step():
+        kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, o=o, S_T=S_T, workspace=ws)
+
+    with ClockSampler(local) as clk:
+        ms = time_steps(step, args.steps, args.warmup, world, device)
+    assert kda.kda_device_status(device) == 0
+    clocks = clk.summary()
+    tokens = B * T
+    value = world * tokens / (ms * 1e-3)
+    token_heads = B * T * H
+    alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+    achieved_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    tflops = token_heads * FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    traffic_pth = measured_traffic_per_token_head()
+
+    # ---- end to end through the C ABI with pinned host buffers
+    hx = {n: x[n].pin_memory() for n in names}
+    hS0 = x["S0"].pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hST = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+
+    def e2e_step():
+        for n in names:
+            d[n].copy_(hx[n], non_blocking=True)
+        S0.copy_(hS0, non_blocking=True)
+        kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, o=o, S_T=S_T, workspace=ws)
+        ho.copy_(o, non_blocking=True)
+        hST.copy_(S_T, non_blocking=True)
+
+    e2e_ms = time_steps(e2e_step, max(2, min(args.steps, 5)), max(3, min(args.warmup, 3)), world, device)
+    h2d = sum(hx[n].numel() * hx[n].element_size() for n in names) + hS0.numel() * 4
+    d2h = ho.numel() * ho.element_size() + hST.numel() * 4
+
+    # ---- decode step: N=256, H=32, d=128, fp32 state, chained steps
+    dw = synth.DECODE
+    S = synth.decode_state(dw).to(device)
+    n_sets = 50
+    toks = []
+    for s in range(n_sets):
+        t = synth.decode_tokens(dw, rank_seed(s, rank))
+        toks.append({n: t[n].to(device) for n in names})
+    od = torch.empty((dw.N, dw.H, dw.dv), dtype=torch.bfloat16, device=device)
+    counter = [0]
+
+    def dec_step():
+        t = toks[counter[0] % n_sets]
+        counter[0] += 1
+        kda.kda_decode_step(*(t[n] for n in names), S, G_MIN, o=od)
+
+    dec_steps = 200
+    with ClockSampler(local) as dclk:
+        dec_ms = time_steps(dec_step, dec_steps, 10, world, device)
+    assert kda.kda_device_status(device) == 0
+    units = dw.N * dw.H
+    dec_bytes = units * (2 * dw.dk * dw.dv * 4 + 3 * dw.dk * 2 + dw.dv * 2 + 2 + dw.dv * 2)
+    dec_gbs = world * dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": D, "dv": D, "chunk": 64, "tile": 16,
+                   "g_min": G_MIN, "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
+                   "l2": "inputs (2.69 GB) exceed L2; no flush"},
+        "clocks": clocks,
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "peak_kind": peak_kind,
+                     "kernel": "kda_chunk_fwd (prep + scan launches of one call)",
+                     "traffic": None if traffic_pth is None else traffic_pth * token_heads,
+                     "algorithmic_bytes": alg_bytes},
+        "chunk_fwd": {"tflops": tflops, "pct_bf16_peak": tflops / bf16_peak, "bf16_peak_tflops": bf16_peak,
+                      "flops_per_token_head": FLOPS_PER_TOKEN_HEAD},
+        "decode": {"metric": "decode HBM GB/s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": dec_ms,
+                   "steps": dec_steps, "workload": dw.name, "gpu_launches": dec_steps,
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
+                                "frac": dec_gbs / world / hbm_peak, "peak_kind": peak_kind},
+                   "clocks": dclk.summary()},
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("libkda", "reference"), default="libkda")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_libkda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,189 @@
-"""libkda: chunked KDA forward (bounded-decay gated delta rule) for B200 -- placeholder."""
+"""libkda Python binding: chunked KDA forward (bounded-decay gated delta rule) on B200.
+
+A thin ctypes layer over ``libkda.so`` (built in-tree by ``build.py``).  Each function
+has the name of the C entry point it calls and does argument marshalling only: it
+checks tensor devices, dtypes, shapes and contiguity, then passes raw device pointers
+and the current CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels; there is no fallback.  If ``libkda.so`` is missing or the library returns
+an error, these functions raise.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda.so")
+
+KDA_BF16 = 0
+KDA_F32 = 1
+KDA_CHUNK = 64
+KDA_TILE = 16
+KDA_G_MIN_LOWEST = -5.4
+
+STATUS = {
+    0: "KDA_OK",
+    1: "KDA_ERR_INVALID_ARG",
+    2: "KDA_ERR_UNSUPPORTED",
+    3: "KDA_ERR_ALIGNMENT",
+    4: "KDA_ERR_ALIAS",
+    5: "KDA_ERR_CUDA",
+    6: "KDA_ERR_DEVICE_TIMEOUT",
+    7: "KDA_ERR_WORKSPACE",
+}
+
+EXPORTS = (
+    "kda_gate_fwd",
+    "kda_chunk_fwd_workspace",
+    "kda_chunk_fwd",
+    "kda_decode_step",
+    "kda_device_status",
+    "kda_status_string",
+    "kda_version",
+)
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call} failed: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libkda.so not found at {LIB_PATH}; build it with "
+            "`python -m chunked_linear_attention_chunk_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, L64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
+    L.kda_gate_fwd.argtypes = [P, I, F, P, L64, P]
+    L.kda_gate_fwd.restype = I
+    L.kda_chunk_fwd_workspace.argtypes = [I, I, I, I, I, I]
+    L.kda_chunk_fwd_workspace.restype = S
+    L.kda_chunk_fwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, S, P]
+    L.kda_chunk_fwd.restype = I
+    L.kda_decode_step.argtypes = [I, I, I, I, I, P, P, P, P, P, F, P, P, P]
+    L.kda_decode_step.restype = I
+    L.kda_device_status.argtypes = [P]
+    L.kda_device_status.restype = I
+    L.kda_status_string.argtypes = [I]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    L.kda_version.restype = I
+    _lib = L
+    return L
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("libkda takes CUDA tensors only")
+        if not t.is_contiguous():
+            raise ValueError("libkda takes contiguous tensors only")
+
+
+def _raise(st: int, call: str):
+    if st != 0:
+        raise KdaError(st, call)
+
+
+def kda_gate_fwd(a: torch.Tensor, g_min: float = -5.0, out: torch.Tensor | None = None) -> torch.Tensor:
+    """g = g_min * sigmoid(a) as float32 (fp64 evaluation, one rounding)."""
+    _check_cuda(a, out)
+    g = out if out is not None else torch.empty(a.shape, dtype=torch.float32, device=a.device)
+    st = lib().kda_gate_fwd(_ptr(a), _dtype_code(a), float(g_min), _ptr(g), a.numel(), _stream(a.device))
+    _raise(st, "kda_gate_fwd")
+    return g
+
+
+def kda_chunk_fwd_workspace(B: int, T: int, H: int, dk: int, dv: int, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(lib().kda_chunk_fwd_workspace(B, T, H, dk, dv, code))
+
+
+def kda_chunk_fwd(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=None,
+                  workspace=None, return_state: bool = True):
+    """Chunked forward.  q, k, a [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H] (bf16 or f32).
+    S0 [B,H,dk,dv] float32 or None (zeros).  Returns (o, S_T); S_T is None when
+    ``return_state`` is False and no S_T buffer is given.  S_T may be S0 (in place)."""
+    _check_cuda(q, k, v, a, beta, S0, o, S_T, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    for t in (k, v, a, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, a, beta must share one dtype")
+    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(lib().kda_chunk_fwd_workspace(B, T, H, dk, dv, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd(B, T, H, dk, dv, code, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
+                             float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+                             _stream(q.device))
+    _raise(st, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_decode_step(q, k, v, a, beta, S, g_min: float = -5.0, o=None):
+    """One decode token.  q, k, a [N,H,dk]; v [N,H,dv]; beta [N,H]; S [N,H,dk,dv] float32,
+    updated in place.  Returns o [N,H,dv]."""
+    _check_cuda(q, k, v, a, beta, S, o)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if S.dtype != torch.float32 or S.shape != (N, H, dk, dv):
+        raise ValueError("S must be float32 [N,H,dk,dv]")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    st = lib().kda_decode_step(N, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
+                               float(g_min), _ptr(S), _ptr(o), _stream(q.device))
+    _raise(st, "kda_decode_step")
+    return o
+
+
+def kda_device_status(device=None) -> int:
+    """Synchronise the current stream and return/clear the device status word."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return int(lib().kda_device_status(_stream(dev)))
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return int(lib().kda_version())

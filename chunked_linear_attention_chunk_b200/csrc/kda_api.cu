@@ -1,0 +1,239 @@
+// kda_api.cu -- the extern "C" boundary of libkda: argument validation, aliasing
+// checks, workspace sizing and dispatch to the kernels.  See include/kda.h for the
+// contract of every entry point.
+#include <cmath>
+#include <cstring>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+__device__ unsigned int g_device_status = 0;
+
+int num_sms()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
+        return 148;
+    if (dev < 64 && cache[dev] > 0)
+        return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64)
+        cache[dev] = n;
+    return n;
+}
+
+namespace {
+
+constexpr int64_t kMaxElems = (int64_t)1 << 40;
+
+struct Range {
+    uintptr_t lo = 0, hi = 0;  // [lo, hi)
+    Range() = default;
+    Range(const void *p, int64_t bytes) : lo((uintptr_t)p), hi((uintptr_t)p + (uintptr_t)(bytes > 0 ? bytes : 0)) {}
+    bool empty() const { return lo == 0 || hi <= lo; }
+};
+
+bool overlaps(const Range &x, const Range &y)
+{
+    if (x.empty() || y.empty())
+        return false;
+    return x.lo < y.hi && y.lo < x.hi;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int elem_size(kda_dtype dt) { return dt == KDA_BF16 ? 2 : 4; }
+
+bool dtype_ok(kda_dtype dt) { return dt == KDA_BF16 || dt == KDA_F32; }
+
+kda_status check_gmin(float g_min)
+{
+    if (!std::isfinite(g_min) || !(g_min < 0.0f))
+        return KDA_ERR_INVALID_ARG;
+    if (g_min < KDA_G_MIN_LOWEST)
+        return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Product of non-negative ints with an overflow bound; -1 when it exceeds kMaxElems.
+int64_t safe_prod(std::initializer_list<int64_t> xs)
+{
+    int64_t p = 1;
+    for (int64_t x : xs) {
+        if (x < 0)
+            return -1;
+        if (x != 0 && p > kMaxElems / x)
+            return -1;
+        p *= x;
+    }
+    return p;
+}
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(kda_status s)
+{
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT";
+    case KDA_ERR_ALIAS: return "KDA_ERR_ALIAS";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+kda_status kda_gate_fwd(const void *a, kda_dtype a_dtype, float g_min, float *g, int64_t n, kda_stream_t stream)
+{
+    if (!dtype_ok(a_dtype) || n < 0 || n > kMaxElems)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    if (n == 0)
+        return KDA_OK;
+    if (!a || !g)
+        return KDA_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(g))
+        return KDA_ERR_ALIGNMENT;
+    if (overlaps(Range(a, n * elem_size(a_dtype)), Range(g, n * 4)))
+        return KDA_ERR_ALIAS;
+    return from_cuda(launch_gate(a, a_dtype, (double)g_min, g, n, (cudaStream_t)stream));
+}
+
+size_t kda_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (B < 1 || H < 1 || T < 0 || dk != dv || (dk != 64 && dk != 128) || !dtype_ok(dtype))
+        return 0;
+    if (dtype != KDA_BF16 || T == 0)
+        return 0;
+    return chunk_bf16_workspace(B, T, H, dk);
+}
+
+kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *S0, void *o,
+                         float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    if (!dtype_ok(dtype) || B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    if (dk != dv || (dk != 64 && dk != 128))
+        return KDA_ERR_UNSUPPORTED;
+    const int64_t ntok = safe_prod({B, T, H});
+    const int64_t nk = safe_prod({B, T, H, dk});
+    const int64_t nv = safe_prod({B, T, H, dv});
+    const int64_t ns = safe_prod({B, H, dk, dv});
+    if (ntok < 0 || nk < 0 || nv < 0 || ns < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (dtype == KDA_BF16 && (int64_t)B * H > 65535)
+        return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!q || !k || !v || !a || !beta || !o))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, a, beta, S0, o, S_T, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return KDA_ERR_ALIGNMENT;
+    const size_t need = kda_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return KDA_ERR_WORKSPACE;
+
+    const int es = elem_size(dtype);
+    const Range rq(q, nk * es), rk(k, nk * es), rv(v, nv * es), ra(a, nk * es), rb(beta, ntok * es);
+    const Range rS0(S0, ns * 4), ro(T > 0 ? o : nullptr, nv * es), rST(S_T, ns * 4);
+    const Range rws(need > 0 ? workspace : nullptr, (int64_t)need);
+    for (const Range &in : {rq, rk, rv, ra, rb, rS0, rST, rws})
+        if (overlaps(ro, in))
+            return KDA_ERR_ALIAS;
+    for (const Range &in : {rq, rk, rv, ra, rb, rws})
+        if (overlaps(rST, in))
+            return KDA_ERR_ALIAS;
+    if (overlaps(rST, rS0) && S_T != S0)
+        return KDA_ERR_ALIAS;
+    for (const Range &in : {rq, rk, rv, ra, rb, rS0})
+        if (overlaps(rws, in))
+            return KDA_ERR_ALIAS;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) {
+        if (!S_T || S_T == S0)
+            return KDA_OK;
+        if (S0)
+            return from_cuda(cudaMemcpyAsync(S_T, S0, (size_t)ns * 4, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(S_T, 0, (size_t)ns * 4, s));
+    }
+    if (dtype == KDA_F32)
+        return from_cuda(launch_chunk_f32(B, T, H, dk, static_cast<const float *>(q), static_cast<const float *>(k),
+                                          static_cast<const float *>(v), static_cast<const float *>(a),
+                                          static_cast<const float *>(beta), g_min, S0, static_cast<float *>(o), S_T,
+                                          s));
+    return from_cuda(launch_chunk_bf16(B, T, H, dk, q, k, v, a, beta, g_min, S0, o, S_T, workspace, s));
+}
+
+kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k, const void *v,
+                           const void *a, const void *beta, float g_min, float *S, void *o, kda_stream_t stream)
+{
+    if (!dtype_ok(dtype) || N < 1 || H < 1 || dk < 1 || dv < 1)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    if (dk != dv || (dk != 64 && dk != 128))
+        return KDA_ERR_UNSUPPORTED;
+    const int64_t nh = safe_prod({N, H});
+    const int64_t ns = safe_prod({N, H, dk, dv});
+    if (nh < 0 || ns < 0 || nh > 0x7fffffff)
+        return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !a || !beta || !S || !o)
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, a, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return KDA_ERR_ALIGNMENT;
+    const int es = elem_size(dtype);
+    const Range rq(q, nh * dk * es), rk(k, nh * dk * es), rv(v, nh * dv * es), ra(a, nh * dk * es),
+        rb(beta, nh * es), rS(S, ns * 4), ro(o, nh * dv * es);
+    for (const Range &in : {rq, rk, rv, ra, rb, rS})
+        if (overlaps(ro, in))
+            return KDA_ERR_ALIAS;
+    for (const Range &in : {rq, rk, rv, ra, rb})
+        if (overlaps(rS, in))
+            return KDA_ERR_ALIAS;
+    return from_cuda(launch_decode(N, H, dk, dtype, q, k, v, a, beta, g_min, S, o, (cudaStream_t)stream));
+}
+
+kda_status kda_device_status(kda_stream_t stream)
+{
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        return (kda_status)v;
+    }
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// kda_internal.h -- host-side launch declarations shared by the libkda translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+int num_sms();  // SM count of the current device (cached per device)
+
+// K1: g = g_min * sigmoid(a), fp64-exact, n elements.
+cudaError_t launch_gate(const void *a, kda_dtype dt, double g_min, float *g, int64_t n, cudaStream_t s);
+
+// K5: float32 CUDA-core chunked forward (16-token chunks).
+cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const float *k, const float *v,
+                             const float *a, const float *beta, float g_min, const float *S0, float *o,
+                             float *S_T, cudaStream_t s);
+
+// K2 + K3: bfloat16 tensor-core chunked forward.
+size_t chunk_bf16_workspace(int B, int T, int H, int D);
+cudaError_t launch_chunk_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                              const void *a, const void *beta, float g_min, const float *S0, void *o,
+                              float *S_T, void *workspace, cudaStream_t s);
+
+// K4: single-token decode step.
+cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,
+                          const void *a, const void *beta, float g_min, float *S, void *o, cudaStream_t s);
+
+}  // namespace kda

@@ -14,14 +14,17 @@ library's contract asks for:
   (deliberately not 16-aligned) has a = +8 on every head and channel, so g sits at the
   lower bound there and tiles straddle the run's edges.
 
-Every tensor comes from its own numpy ``default_rng([seed, stream_id])`` stream, so a
-tensor does not depend on which other tensors were drawn.  bf16 rounding is
+Every tensor comes from its own numpy ``default_rng([seed, stream_id, block])`` streams
+(one per block of 2^22 elements), so a tensor depends neither on which other tensors
+were drawn nor on how many threads drew it.  bf16 rounding is
 round-to-nearest-even (torch's float32 -> bfloat16 cast).  All tensors are returned on
 the CPU; bf16 values are exact in float32, which is what the oracle consumes.
 """
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -72,15 +75,29 @@ ADV_FRACTION = 0.05
 ADV_VALUE = 8.0
 
 
-def _rng(seed: int, stream: int):
-    return np.random.default_rng([int(seed), int(stream)])
+_BLOCK = 1 << 22  # elements per independently seeded block
 
 
 def _normal(seed, stream, shape, std=1.0):
-    x = _rng(seed, stream).standard_normal(size=shape, dtype=np.float32)
-    if std != 1.0:
-        x *= np.float32(std)
-    return x
+    """N(0, std^2) float32 draws; block i of the flattened array comes from
+    default_rng([seed, stream, i]), so the values do not depend on the thread count."""
+    n = int(np.prod(shape))
+    x = np.empty(n, np.float32)
+
+    def fill(i):
+        lo, hi = i * _BLOCK, min(n, (i + 1) * _BLOCK)
+        np.random.default_rng([int(seed), int(stream), i]).standard_normal(out=x[lo:hi], dtype=np.float32)
+        if std != 1.0:
+            x[lo:hi] *= np.float32(std)
+
+    nb = (n + _BLOCK - 1) // _BLOCK
+    if nb <= 1:
+        for i in range(nb):
+            fill(i)
+    else:
+        with ThreadPoolExecutor(max_workers=min(nb, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(nb)))
+    return x.reshape(shape)
 
 
 def _unit_rows(x: np.ndarray) -> np.ndarray:

@@ -1,0 +1,162 @@
+/*
+ * kda.h -- C ABI of libkda: the chunked forward of KDA incremental linear attention
+ * (a gated delta rule with per-channel decay) with the lower-bounded decay gate, and
+ * its single-token decode step, for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  The pages ("Trillion-Scale MoE Multimodal Models: Practical
+ * Techniques for Ultra-Long Context ...", section 3; "Breaking Through
+ * Trillion-Parameter Multimodal MoE ...", section 2.1; "Trillion-Parameter MoE
+ * Multimodal Models: Engineering Long-Context ...", section 3.2) describe a linear
+ * attention whose state is updated incrementally token by token and computed in
+ * chunks with a cumulative decay Gamma, with the log-decay bounded below:
+ *
+ *     g_t = g_min * sigmoid(a_t)                                   (per key channel)
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * S is a dk x dv matrix per (batch, head).  No 1/sqrt(dk) scale is applied; q and k
+ * are expected L2-normalised by the caller (the library does not normalise), beta is
+ * passed post-activation in (0, 1), and a is the gate pre-activation (the projection
+ * that produces it lives upstream).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major (innermost index last) and 16-byte aligned.  The library allocates
+ *     no device memory; scratch space is passed in by the caller.
+ *   - Token tensors are [B, T, H, d]; beta is [B, T, H]; states are [B, H, dk, dv]
+ *     float32.  dtype KDA_BF16 means q, k, v, a, beta and o are bfloat16 (state and
+ *     accumulation stay float32); KDA_F32 means they are float32 (a CUDA-core path
+ *     kept for debugging at tight tolerance).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream).  Arguments are validated synchronously before any launch; an invalid
+ *     call launches nothing and returns an error status.  Calls keep no state between
+ *     invocations and may be made from several host threads.
+ *   - Errors detected inside a kernel (a bounded wait that ran out) are recorded in a
+ *     per-device status word and reported by kda_device_status().
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_BF16 = 0, /* bfloat16 token tensors, float32 state and accumulation */
+    KDA_F32 = 1   /* float32 everywhere (CUDA-core debug path)              */
+} kda_dtype;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,    /* null pointer, negative size, bad dtype, bad g_min  */
+    KDA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (head dim, g_min range)  */
+    KDA_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned                   */
+    KDA_ERR_ALIAS = 4,          /* an output overlaps an input it must not overlap    */
+    KDA_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed        */
+    KDA_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out (kda_device_status) */
+    KDA_ERR_WORKSPACE = 7       /* workspace pointer missing or smaller than required */
+} kda_status;
+
+/* Supported range of g_min: finite, KDA_G_MIN_LOWEST <= g_min < 0.  The pages fix
+ * g_min = -5 so that 1/Gamma inside any 16-token tile stays in range; with the tile's
+ * middle token as reference the largest exponent is 8*|g_min| <= 43.2, far inside
+ * float32/bfloat16's range (e^88.7).                                                 */
+#define KDA_G_MIN_LOWEST (-5.4f)
+
+/* Token chunk of the bfloat16 path (state carried every KDA_CHUNK tokens) and the
+ * decay tile inside it (the pages' 16-token tile). */
+#define KDA_CHUNK 64
+#define KDA_TILE 16
+
+/*
+ * kda_gate_fwd -- the bounded gate on its own: g[i] = g_min * sigmoid(a[i]).
+ * Passage: "Trillion-Scale ..." section 3.2 (g = g_min * Sigmoid(...), g_min = -5) and
+ * "Breaking Through ..." section 2.1 (g_t = g_min * sigma(w x_t + b), range [g_min, 0)).
+ *   a      device, n elements of a_dtype (bf16 or f32), any shape flattened.
+ *   g      device, n float32 outputs.  Evaluated in float64 and rounded once to
+ *          float32 (round-to-nearest-even), so the result is bit-exact against an
+ *          fp64 reference.  NaN propagates; a = +inf gives g_min; a = -inf gives -0.
+ *   n      number of elements (0 is a no-op).
+ * Errors: INVALID_ARG (null pointer with n > 0, bad dtype, g_min not finite or >= 0),
+ * UNSUPPORTED (g_min < KDA_G_MIN_LOWEST), ALIGNMENT, ALIAS (g overlaps a), CUDA.
+ */
+kda_status kda_gate_fwd(const void *a, kda_dtype a_dtype, float g_min, float *g, int64_t n,
+                        kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_workspace -- bytes of device scratch kda_chunk_fwd needs for this
+ * shape (0 when none).  Pure host computation; never fails (returns 0 for invalid
+ * shapes, which kda_chunk_fwd then rejects).
+ */
+size_t kda_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype);
+
+/*
+ * kda_chunk_fwd -- chunked forward over a whole sequence batch (prefill / training
+ * forward), state carried in and out.
+ * Passages: chunked computation with cumulative decay Gamma and its inverse
+ * ("Trillion-Scale ..." section 3.1), all 16-token tiles as dense tensor-core GEMMs
+ * thanks to the bound ("Trillion-Scale ..." section 3.3; "Breaking Through ..."
+ * section 2.1), Delta-Net-style state update ("Breaking Through ..." section 2.1),
+ * chunk recursion with a constant-size state ("Trillion-Parameter MoE ... Engineering"
+ * section 3.2).
+ *   B, T, H    batch, tokens, heads (B, H >= 1; T >= 0; T need not be a multiple of
+ *              anything).  T == 0 copies S0 (or zeros) to S_T and writes no o.
+ *   dk, dv     head dims; supported: dk == dv, 64 or 128.
+ *   dtype      KDA_BF16 or KDA_F32 (applies to q, k, v, a, beta, o).
+ *   q, k, a    [B, T, H, dk];  v: [B, T, H, dv];  beta: [B, T, H].
+ *   g_min      gate lower bound, KDA_G_MIN_LOWEST <= g_min < 0 (the pages use -5).
+ *   S0         [B, H, dk, dv] float32 initial state, or NULL for zeros.
+ *   o          [B, T, H, dv] output (dtype).  Must not overlap any input or S_T.
+ *   S_T        [B, H, dk, dv] float32 final state, or NULL to skip.  May be the same
+ *              pointer as S0 (in-place carry across segment calls); partial overlap
+ *              is rejected.
+ *   workspace  device scratch of at least kda_chunk_fwd_workspace(...) bytes, 16-byte
+ *              aligned, overlapping no tensor argument (may be NULL when that size is
+ *              0).  Its contents on entry are ignored and on exit unspecified.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.
+ */
+kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q,
+                         const void *k, const void *v, const void *a, const void *beta,
+                         float g_min, const float *S0, void *o, float *S_T, void *workspace,
+                         size_t ws_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one token for N independent sequences, state updated in place.
+ * Passage: the incremental state of constant size used at inference ("Trillion-
+ * Parameter MoE ... Engineering" section 3.2).  Per (n, h):
+ *     S_dec = Diag(exp g) S;  u = beta (v - S_dec^T k);  S' = S_dec + k u^T;
+ *     o = S'^T q                     (the recurrence above for a single token)
+ *   N, H       sequences and heads (>= 1); dk == dv in {64, 128}.
+ *   q, k, a    [N, H, dk];  v: [N, H, dv];  beta: [N, H]   (dtype)
+ *   S          [N, H, dk, dv] float32, read and overwritten with S'.
+ *   o          [N, H, dv] (dtype); must not overlap S or any input.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, CUDA.
+ */
+kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const void *q,
+                           const void *k, const void *v, const void *a, const void *beta,
+                           float g_min, float *S, void *o, kda_stream_t stream);
+
+/*
+ * kda_device_status -- synchronise `stream`, then return and clear the current
+ * device's kernel status word: KDA_OK, or KDA_ERR_DEVICE_TIMEOUT if a kernel gave up
+ * on a bounded wait since the last call; KDA_ERR_CUDA if the synchronisation failed.
+ */
+kda_status kda_device_status(kda_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

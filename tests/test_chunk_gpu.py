@@ -1,0 +1,178 @@
+"""kda_chunk_fwd on the GPU against the fp64 oracle (same seeded inputs).
+
+Tolerances (normwise per head, see helpers.py): bf16 path o <= 2e-2, S_T <= 1e-2;
+float32 debug path <= 1e-4 on both."""
+import numpy as np
+import pytest
+import torch
+
+import chunked_linear_attention_chunk_b200 as kda
+from chunked_linear_attention_chunk_b200 import synth
+from helpers import (G_MIN, NAMES, TOL_BF16_O, TOL_BF16_S, TOL_F32, err_o, err_s, oracle_run, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(x, S0=True, **kw):
+    d = to_dev(x)
+    o, ST = kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=d["S0"] if S0 else None, **kw)
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    return o, ST
+
+
+def _check(x, tol_o, tol_s, S0=True):
+    o, ST = _gpu(x, S0)
+    o_ref, S_ref = oracle_run(x, x["S0"] if S0 else None)
+    eo, es = err_o(o.float().cpu().numpy(), o_ref), err_s(ST.cpu().numpy(), S_ref)
+    assert np.isfinite(o.float().cpu().numpy()).all()
+    assert eo <= tol_o and es <= tol_s, (eo, es)
+    return eo, es
+
+
+# ------------------------------------------------------------------ float32 debug path
+def test_f32_tiny_config():
+    """B=1, H=2, T=256, dk=dv=64, fp32, S0 = 0."""
+    x = synth.workload_inputs(synth.TINY)
+    _check(x, TOL_F32, TOL_F32, S0=False)
+
+
+@pytest.mark.parametrize("T,D", [(1, 64), (17, 64), (100, 128), (33, 128)])
+def test_f32_ragged(T, D):
+    x = synth.make_inputs(2, T, 2, D, D, "f32", seed=200 + T, s0_std=0.1)
+    _check(x, TOL_F32, TOL_F32)
+
+
+# ------------------------------------------------------------------ bf16 tensor-core path
+@pytest.mark.parametrize("B,T,H,D", [(2, 300, 3, 128), (1, 129, 2, 64), (1, 512, 1, 128)])
+def test_bf16_several_chunks_ragged_tail(B, T, H, D):
+    x = synth.make_inputs(B, T, H, D, D, "bf16", seed=300 + T, s0_std=0.1)
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65, 127, 128, 129])
+def test_bf16_edge_lengths(T):
+    x = synth.make_inputs(1, T, 2, 128, 128, "bf16", seed=400 + T, s0_std=0.1)
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_saturated_gate_everywhere():
+    """a = +8 on every token (g ~ g_min): the largest 1/Gamma span in every tile."""
+    x = synth.make_inputs(1, 256, 2, 128, 128, "bf16", seed=500, s0_std=0.1)
+    x["a"] = torch.full_like(x["a"], 8.0)
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_no_decay_limit():
+    """a = -inf on every token: g = -0, no decay at all (pure delta rule)."""
+    x = synth.make_inputs(1, 200, 2, 128, 128, "bf16", seed=501, s0_std=0.1)
+    x["a"] = torch.full_like(x["a"], float("-inf"))
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_beta_zero_is_pure_decay():
+    x = synth.make_inputs(1, 130, 2, 128, 128, "bf16", seed=502, s0_std=0.1)
+    x["beta"] = torch.zeros_like(x["beta"])
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_null_state_equals_zero_state():
+    x = synth.make_inputs(2, 150, 2, 128, 128, "bf16", seed=503, s0_std=0.0)
+    o1, S1 = _gpu(x, S0=False)
+    o2, S2 = _gpu(x, S0=True)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_bf16_inplace_state_carry():
+    x = synth.make_inputs(2, 150, 2, 128, 128, "bf16", seed=504, s0_std=0.1)
+    o1, S1 = _gpu(x)
+    d = to_dev(x)
+    S = d["S0"].clone()
+    o2, S2 = kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=S, S_T=S)
+    torch.cuda.synchronize()
+    assert S2.data_ptr() == S.data_ptr()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_bf16_segments_equal_one_call_bitwise():
+    """Segment boundaries on chunk multiples: state carried in fp32 gives identical bits."""
+    x = synth.make_inputs(1, 320, 2, 128, 128, "bf16", seed=505, s0_std=0.1)
+    o, ST = _gpu(x)
+    d = to_dev(x)
+    S = d["S0"].clone()
+    outs = []
+    for lo, hi in ((0, 128), (128, 192), (192, 320)):
+        seg = [d[n][:, lo:hi].contiguous() for n in NAMES]
+        oo, _ = kda.kda_chunk_fwd(*seg, G_MIN, S0=S, S_T=S)
+        outs.append(oo)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(outs, 1), o) and torch.equal(S, ST)
+
+
+def test_empty_sequence_copies_state():
+    x = synth.make_inputs(1, 0, 2, 128, 128, "bf16", seed=506, s0_std=0.1)
+    o, ST = _gpu(x)
+    assert o.numel() == 0 and torch.equal(ST.cpu(), x["S0"])
+    o, ST = _gpu(x, S0=False)
+    assert (ST == 0).all()
+
+
+def test_output_rows_past_T_untouched():
+    """The ragged tail chunk writes no o rows beyond T."""
+    x = synth.make_inputs(1, 70, 1, 128, 128, "bf16", seed=507, s0_std=0.1)
+    d = to_dev(x)
+    big = torch.full((1, 128, 1, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    o = big[:, :70]
+    assert o.is_contiguous()
+    kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=d["S0"], o=o)
+    torch.cuda.synchronize()
+    assert (big[:, 70:] == 3.0).all()
+
+
+# ------------------------------------------------------------------ full workloads
+def test_stage_8k_full():
+    """B=4, H=16, T=8192, d=128, bf16 -- every output against the oracle."""
+    x = synth.workload_inputs(synth.STAGE_8K)
+    _check(x, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_stage_64k_sampled_heads():
+    """B=1, H=32, T=65536 with the 5% a=+8 slice, run whole in the benchmark's launch
+    configuration; heads 0, 13 and 31 checked in full against the oracle, every output
+    finite."""
+    x = synth.workload_inputs(synth.STAGE_64K)
+    o, ST = _gpu(x)
+    oc = o.float().cpu().numpy()
+    assert np.isfinite(oc).all() and torch.isfinite(ST).all()
+    heads = [0, 13, 31]
+    o_ref, S_ref = oracle_run(x, x["S0"], heads=heads)
+    eo = err_o(oc[:, :, heads], o_ref)
+    es = err_s(ST.cpu().numpy()[:, heads], S_ref)
+    assert eo <= TOL_BF16_O and es <= TOL_BF16_S, (eo, es)
+    # the adversarial slice itself, tighter view
+    s, e = synth.adversarial_range(x["q"].shape[1])
+    assert err_o(oc[:, s:e][:, :, heads], o_ref[:, s:e]) <= TOL_BF16_O
+
+
+@pytest.mark.slow
+def test_stage_1m_segmented():
+    """B=1, H=16, T=1M as 16 calls of 64K tokens with S carried in place; o checked on the
+    first 65536 tokens and S after every segment against the streamed oracle."""
+    w = synth.STAGE_1M
+    S = None
+    S_ref = None
+    S_gpu = None
+    for seg in range(w.T // w.segment):
+        x = synth.workload_inputs(w, segment_index=seg)
+        if seg == 0:
+            S_ref = x["S0"].numpy().astype(np.float64)
+            S_gpu = x["S0"].cuda()
+        d = to_dev(x)
+        o, _ = kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=S_gpu, S_T=S_gpu)
+        torch.cuda.synchronize()
+        o_ref, S_ref = oracle_run(x, S_ref)
+        if seg == 0:
+            assert err_o(o.float().cpu().numpy(), o_ref) <= TOL_BF16_O
+        es = err_s(S_gpu.cpu().numpy(), S_ref)
+        assert es <= TOL_BF16_S, (seg, es)
+    assert kda.kda_device_status() == 0

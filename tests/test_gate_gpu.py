@@ -1,0 +1,63 @@
+"""K1 gate on the GPU against the fp64 oracle: bit-exact g."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import chunked_linear_attention_chunk_b200 as kda
+from chunked_linear_attention_chunk_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _all_bf16():
+    bits = torch.arange(65536, dtype=torch.int32)
+    bits = torch.where(bits >= 32768, bits - 65536, bits).to(torch.int16)
+    return bits.view(torch.bfloat16)
+
+
+def _same_bits(g_gpu: np.ndarray, g_ref: np.ndarray):
+    nan = np.isnan(g_ref)
+    assert (np.isnan(g_gpu) == nan).all()
+    a = g_gpu[~nan].view(np.uint32)
+    b = g_ref[~nan].view(np.uint32)
+    bad = np.nonzero(a != b)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first at {bad[:5]}"
+
+
+@pytest.mark.parametrize("g_min", [-5.0, -1.0, -5.4, -0.25])
+def test_gate_bf16_exhaustive_bit_exact(g_min):
+    a = _all_bf16()
+    g = kda.kda_gate_fwd(a.cuda(), g_min).cpu().numpy()
+    ref = oracle.gate(a.float().numpy(), g_min)
+    _same_bits(g, ref)
+    fin = ~np.isnan(ref)
+    assert (g[fin] >= np.float32(g_min)).all() and (g[fin] <= 0).all()
+
+
+def test_gate_f32_bit_exact():
+    rng = np.random.default_rng(7)
+    a = np.concatenate([
+        rng.standard_normal(1 << 20).astype(np.float32) * 2,
+        rng.standard_normal(1 << 16).astype(np.float32) * 40,
+        np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 1e-30, -1e-30, 88.0, -88.0, 104.0, -104.0], np.float32),
+    ])
+    x = synth.workload_inputs(synth.TINY)["a"].numpy().reshape(-1)
+    a = np.concatenate([a, x])
+    g = kda.kda_gate_fwd(torch.from_numpy(a).cuda(), -5.0).cpu().numpy()
+    _same_bits(g, oracle.gate(a, -5.0))
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 1000003])
+def test_gate_ragged_lengths(n):
+    a = _all_bf16()[:n] if n <= 65536 else _all_bf16().repeat(n // 65536 + 1)[:n]
+    a = a.clone()
+    g = kda.kda_gate_fwd(a.cuda(), -5.0).cpu().numpy()
+    _same_bits(g, oracle.gate(a.float().numpy(), -5.0))
+
+
+def test_gate_writes_nothing_past_n():
+    a = torch.randn(13, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((32,), 7.0, device="cuda")
+    kda.kda_gate_fwd(a, -5.0, out=out[:13])
+    assert (out[13:] == 7.0).all()

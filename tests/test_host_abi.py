@@ -1,0 +1,162 @@
+"""Host-side checks of the C ABI (CPU only): the library loads, exports every entry
+point include/kda.h declares, sizes workspaces, and rejects bad arguments with the
+documented status before any CUDA call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import chunked_linear_attention_chunk_b200 as kda
+from chunked_linear_attention_chunk_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, ALIAS, CUDA, TIMEOUT, WS = range(8)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kda.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(kda_[a-z0-9_]+)\s*\(", text, re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("kda_gate_fwd", "kda_chunk_fwd_workspace", "kda_chunk_fwd", "kda_decode_step",
+              "kda_device_status", "kda_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", kda.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT\s+(kda_[a-z0-9_]+)$", out, re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(L, n)
+    assert set(kda.EXPORTS) <= set(declared_functions())
+
+
+def test_status_strings(L):
+    for code, name in kda.STATUS.items():
+        assert L.kda_status_string(code).decode() == name
+    assert L.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
+    assert L.kda_version() >= 100
+
+
+def test_workspace_size(L):
+    f = L.kda_chunk_fwd_workspace
+    rec128 = 4 * 64 * 128 * 2 + 64 * 64 * 2 + 128 * 4
+    assert f(1, 64, 1, 128, 128, kda.KDA_BF16) == rec128
+    assert f(2, 65, 3, 128, 128, kda.KDA_BF16) == 2 * 3 * 2 * rec128
+    assert f(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec128
+    rec64 = 4 * 64 * 64 * 2 + 64 * 64 * 2 + 64 * 4
+    assert f(1, 100, 1, 64, 64, kda.KDA_BF16) == 2 * rec64
+    assert f(1, 100, 1, 64, 64, kda.KDA_F32) == 0
+    assert f(1, 0, 1, 128, 128, kda.KDA_BF16) == 0
+    assert f(0, 64, 1, 128, 128, kda.KDA_BF16) == 0
+    assert f(1, 64, 1, 96, 96, kda.KDA_BF16) == 0
+
+
+# Fake, never-dereferenced device addresses: validation must reject before any launch.
+BASE = 1 << 40
+
+
+def _chunk(L, B=1, T=64, H=1, dk=128, dv=128, dt=kda.KDA_BF16, q=None, k=None, v=None, a=None, beta=None,
+           g_min=-5.0, S0=None, o=None, ST=None, ws=None, ws_bytes=None):
+    es = 2 if dt == kda.KDA_BF16 else 4
+    n = B * T * H * max(dk, 1) * es
+    q = BASE if q is None else q
+    k = BASE + 1 * (n + 4096) if k is None else k
+    v = BASE + 2 * (n + 4096) if v is None else v
+    a = BASE + 3 * (n + 4096) if a is None else a
+    beta = BASE + 4 * (n + 4096) if beta is None else beta
+    o = BASE + 5 * (n + 4096) if o is None else o
+    if ws is None:
+        ws = BASE + 6 * (n + 4096)
+    need = L.kda_chunk_fwd_workspace(B, T, H, dk, dv, dt)
+    ws_bytes = need if ws_bytes is None else ws_bytes
+    P = ctypes.c_void_p
+    return L.kda_chunk_fwd(B, T, H, dk, dv, dt, P(q), P(k), P(v), P(a), P(beta), ctypes.c_float(g_min),
+                           P(S0), P(o), P(ST), P(ws), ws_bytes, None)
+
+
+def test_chunk_fwd_rejects_bad_arguments(L):
+    assert _chunk(L, B=0) == INVALID
+    assert _chunk(L, T=-1) == INVALID
+    assert _chunk(L, dt=7) == INVALID
+    assert _chunk(L, g_min=0.0) == INVALID
+    assert _chunk(L, g_min=1.0) == INVALID
+    assert _chunk(L, g_min=float("nan")) == INVALID
+    assert _chunk(L, g_min=float("-inf")) == INVALID
+    assert _chunk(L, g_min=-6.0) == UNSUPPORTED
+    assert _chunk(L, dk=96, dv=96) == UNSUPPORTED
+    assert _chunk(L, dk=128, dv=64) == UNSUPPORTED
+    assert _chunk(L, q=0) == INVALID  # null input with T > 0
+    assert _chunk(L, o=0) == INVALID
+    assert _chunk(L, q=BASE + 8) == ALIGN
+    assert _chunk(L, S0=BASE * 3 + 4) == ALIGN
+    assert _chunk(L, ws=0) == WS
+    assert _chunk(L, ws_bytes=100) == WS
+    assert _chunk(L, B=300, H=300) == UNSUPPORTED  # B*H beyond the grid limit
+
+
+def test_chunk_fwd_rejects_aliasing(L):
+    n = 64 * 128 * 2
+    assert _chunk(L, o=BASE) == ALIAS                       # o is q
+    assert _chunk(L, o=BASE + 16) == ALIAS                  # o overlaps q
+    S = BASE * 2
+    assert _chunk(L, S0=S, ST=S + 4096) == ALIAS            # partial overlap of states
+    assert _chunk(L, ST=BASE + n + 4096) == ALIAS            # S_T overlaps k
+    assert _chunk(L, ws=BASE + 2 * (n + 4096)) == ALIAS      # workspace overlaps v
+    assert _chunk(L, o=BASE * 3, ST=BASE * 3 + 1024) == ALIAS
+
+
+def _decode(L, N=2, H=2, dk=128, dv=128, dt=kda.KDA_BF16, g_min=-5.0, S=None, o=None, q=None):
+    P = ctypes.c_void_p
+    step = 1 << 24
+    q = BASE if q is None else q
+    S = BASE + 6 * step if S is None else S
+    o = BASE + 5 * step if o is None else o
+    return L.kda_decode_step(N, H, dk, dv, dt, P(q), P(BASE + step), P(BASE + 2 * step), P(BASE + 3 * step),
+                             P(BASE + 4 * step), ctypes.c_float(g_min), P(S), P(o), None)
+
+
+def test_decode_rejects_bad_arguments(L):
+    assert _decode(L, N=0) == INVALID
+    assert _decode(L, g_min=0.5) == INVALID
+    assert _decode(L, g_min=-10.0) == UNSUPPORTED
+    assert _decode(L, dk=32, dv=32) == UNSUPPORTED
+    assert _decode(L, S=0) == INVALID
+    assert _decode(L, S=BASE + 6 * (1 << 24) + 8) == ALIGN
+    assert _decode(L, o=BASE) == ALIAS
+    assert _decode(L, S=BASE + (1 << 24)) == ALIAS
+
+
+def test_gate_rejects_bad_arguments(L):
+    P = ctypes.c_void_p
+    assert L.kda_gate_fwd(P(BASE), kda.KDA_BF16, ctypes.c_float(-5.0), P(BASE * 2), -1, None) == INVALID
+    assert L.kda_gate_fwd(P(BASE), kda.KDA_BF16, ctypes.c_float(-5.0), P(BASE * 2), 0, None) == OK
+    assert L.kda_gate_fwd(P(BASE), 3, ctypes.c_float(-5.0), P(BASE * 2), 16, None) == INVALID
+    assert L.kda_gate_fwd(P(BASE), kda.KDA_BF16, ctypes.c_float(0.0), P(BASE * 2), 16, None) == INVALID
+    assert L.kda_gate_fwd(P(BASE), kda.KDA_BF16, ctypes.c_float(-5.5), P(BASE * 2), 16, None) == UNSUPPORTED
+    assert L.kda_gate_fwd(P(0), kda.KDA_BF16, ctypes.c_float(-5.0), P(BASE * 2), 16, None) == INVALID
+    assert L.kda_gate_fwd(P(BASE + 2), kda.KDA_BF16, ctypes.c_float(-5.0), P(BASE * 2), 16, None) == ALIGN
+    assert L.kda_gate_fwd(P(BASE), kda.KDA_BF16, ctypes.c_float(-5.0), P(BASE + 16), 16, None) == ALIAS
+
+
+def test_python_binding_has_no_cpu_fallback():
+    """The binding refuses CPU tensors instead of computing anything itself."""
+    import torch
+    x = torch.zeros(16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kda.kda_gate_fwd(x)

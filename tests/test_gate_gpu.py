@@ -27,6 +27,8 @@ def _same_bits(g_gpu: np.ndarray, g_ref: np.ndarray):
 
 @pytest.mark.parametrize("g_min", [-5.0, -1.0, -5.4, -0.25])
 def test_gate_bf16_exhaustive_bit_exact(g_min):
+    """g_min crosses the C ABI as float32, so the oracle gets the same float32 value."""
+    g_min = float(np.float32(g_min))
     a = _all_bf16()
     g = kda.kda_gate_fwd(a.cuda(), g_min).cpu().numpy()
     ref = oracle.gate(a.float().numpy(), g_min)

@@ -47,6 +47,7 @@ BYTES_PER_TOKEN_HEAD = 4 * 256 + 2 + 256
 # C^2/3; Gamma scaling dk dv / C), C = 16.
 FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 128 * (3 * 16 - 1) + 2 * 16 * 128 + 16 * 16 / 3 + 128 * 128 / 16
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "chunk_fwd_traffic.json")
+WORKLOADS = {"64k": synth.STAGE_64K, "8k": synth.STAGE_8K}
 
 
 def peaks():
@@ -246,7 +247,7 @@ def run_libkda(args):
     torch.cuda.set_device(device)
     hbm_peak, bf16_peak, peak_kind = peaks()
 
-    w = synth.STAGE_64K
+    w = WORKLOADS[args.workload]
     x = synth.make_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), w.s0_std, w.adversarial)
     names = ("q", "k", "v", "a", "beta")
     d = {n: x[n].to(device) for n in names}
@@ -260,10 +261,14 @@ def run_libkda(args):
     def step():
         kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, o=o, S_T=S_T, workspace=ws)
 
-    with ClockSampler(local) as clk:
-        ms = time_steps(step, args.steps, args.warmup, world, device)
-    assert kda.kda_device_status(device) == 0
-    clocks = clk.summary()
+    if args.only == "decode":
+        ms = float("nan")
+        clocks = {}
+    else:
+        with ClockSampler(local) as clk:
+            ms = time_steps(step, args.steps, args.warmup, world, device)
+        assert kda.kda_device_status(device) == 0
+        clocks = clk.summary()
     tokens = B * T
     value = world * tokens / (ms * 1e-3)
     token_heads = B * T * H
@@ -286,30 +291,35 @@ def run_libkda(args):
         ho.copy_(o, non_blocking=True)
         hST.copy_(S_T, non_blocking=True)
 
-    e2e_ms = time_steps(e2e_step, max(2, min(args.steps, 5)), max(3, min(args.warmup, 3)), world, device)
+    e2e_ms = float("nan")
+    if not args.no_e2e and args.only != "decode":
+        e2e_ms = time_steps(e2e_step, max(2, min(args.steps, 5)), max(3, min(args.warmup, 3)), world, device)
     h2d = sum(hx[n].numel() * hx[n].element_size() for n in names) + hS0.numel() * 4
     d2h = ho.numel() * ho.element_size() + hST.numel() * 4
 
     # ---- decode step: N=256, H=32, d=128, fp32 state, chained steps
     dw = synth.DECODE
-    S = synth.decode_state(dw).to(device)
-    n_sets = 50
-    toks = []
-    for s in range(n_sets):
-        t = synth.decode_tokens(dw, rank_seed(s, rank))
-        toks.append({n: t[n].to(device) for n in names})
-    od = torch.empty((dw.N, dw.H, dw.dv), dtype=torch.bfloat16, device=device)
-    counter = [0]
+    dec_steps = 200 if args.only != "decode" else max(args.steps, 1)
+    dec_ms = float("nan")
+    dclk = None
+    if args.only != "chunk":
+        S = synth.decode_state(dw).to(device)
+        n_sets = 50
+        toks = []
+        for s in range(n_sets):
+            t = synth.decode_tokens(dw, rank_seed(s, rank))
+            toks.append({n: t[n].to(device) for n in names})
+        od = torch.empty((dw.N, dw.H, dw.dv), dtype=torch.bfloat16, device=device)
+        counter = [0]
 
-    def dec_step():
-        t = toks[counter[0] % n_sets]
-        counter[0] += 1
-        kda.kda_decode_step(*(t[n] for n in names), S, G_MIN, o=od)
+        def dec_step():
+            t = toks[counter[0] % n_sets]
+            counter[0] += 1
+            kda.kda_decode_step(*(t[n] for n in names), S, G_MIN, o=od)
 
-    dec_steps = 200
-    with ClockSampler(local) as dclk:
-        dec_ms = time_steps(dec_step, dec_steps, 10, world, device)
-    assert kda.kda_device_status(device) == 0
+        with ClockSampler(local) as dclk:
+            dec_ms = time_steps(dec_step, dec_steps, max(args.warmup, 3), world, device)
+        assert kda.kda_device_status(device) == 0
     units = dw.N * dw.H
     dec_bytes = units * (2 * dw.dk * dw.dv * 4 + 3 * dw.dk * 2 + dw.dv * 2 + 2 + dw.dv * 2)
     dec_gbs = world * dec_bytes / (dec_ms * 1e-3) / 1e9
@@ -320,7 +330,7 @@ def run_libkda(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": D, "dv": D, "chunk": 64, "tile": 16,
                    "g_min": G_MIN, "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
-                   "l2": "inputs (2.69 GB) exceed L2; no flush"},
+                   "l2": "inputs exceed the 126 MB L2; no flush"},
         "clocks": clocks,
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -336,9 +346,9 @@ def run_libkda(args):
                    "steps": dec_steps, "workload": dw.name, "gpu_launches": dec_steps,
                    "roofline": {"bound": "hbm", "achieved": dec_gbs / world, "peak": hbm_peak, "unit": "GB/s",
                                 "frac": dec_gbs / world / hbm_peak, "peak_kind": peak_kind},
-                   "clocks": dclk.summary()},
+                   "clocks": dclk.summary() if dclk is not None else {}},
     }
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -356,6 +366,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("libkda", "reference"), default="libkda")
     ap.add_argument("--cpu-sample-tokens", type=int, default=65536)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="64k",
+                    help="64k (the benchmark workload) or 8k (a smaller case for profiler captures)")
+    ap.add_argument("--only", choices=("all", "chunk", "decode"), default="all")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

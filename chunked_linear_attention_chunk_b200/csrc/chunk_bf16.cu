@@ -7,8 +7,12 @@
 //   A_rj = beta_r sum_c k_rc k_jc e^{G_rc - G_jc}   (j < r),  T = (I + A)^{-1}
 //   P_rj =        sum_c q_rc k_jc e^{G_rc - G_jc}   (j <= r)
 //   W = T diag(beta) Kbar,  Utilde = T diag(beta) V,   Kbar = k e^{G}
-//   U = Utilde - W S;  O = Qbar S + P U;  S <- Diag(e^{G_last}) S + Khat^T U
+//   U = Utilde - W S;  O = Qbar S + P U;  S' = Diag(e^{G_last}) S + Khat^T U
 //   with Qbar = q e^{G} and Khat = k e^{G_last - G} (every factor <= 1).
+// Substituting U once, per chunk, gives the form the scan walks with a single tensor-core
+// round per chunk:
+//   S' = Diag(Gamma) S - N S + Bm,   O = Q' S + O',
+//   N = Khat^T W (D x D),  Bm = Khat^T Utilde (D x D),  Q' = Qbar - P W,  O' = P Utilde.
 //
 // The only unbounded factor is the inverse decay 1/Gamma inside A and P ("Trillion-
 // Scale MoE Multimodal Models ..." section 3.1).  With g >= g_min = -5 ("... section
@@ -18,12 +22,19 @@
 // so every operand stays below e^{40} and ALL tiles, diagonal ones included, are dense
 // tensor-core products ("... section 3.3": no element-wise diagonal path).
 //
-// K2 runs one CTA per (chunk, batch*head), fully parallel, and writes per chunk
-// W, Utilde, Qbar, Khat (bf16, C x D), P (bf16, C x C) and Gamma_C = e^{G_last} (f32)
-// to the caller's workspace.  K3 runs one CTA per (value-column block, batch*head) and
-// walks the chunks in order with the fp32 state block in registers.
+// K2 (prep) runs one CTA per (chunk, batch*head), two CTAs per SM.  The 16-token tile
+// products A and P are warp-level MMAs; the dense contractions W | Utilde = (T beta)
+// [Kbar | V], then Khat^T [W | Utilde] and P [W | Utilde], are 5th-generation tensor
+// core MMAs (tcgen05) with fp32 accumulators in tensor memory.  It writes one record per
+// chunk (N, Q', Gamma, Bm, O') to the caller's workspace in the swizzled layouts the
+// tensor core reads, so a linear bulk copy is directly an MMA operand.
+// K3 (scan) runs one CTA per (32-column block of the value dim, batch*head); a producer
+// warp streams the records through a 3-stage mbarrier pipeline with bulk copies, and per
+// chunk one tcgen05 round computes [N S, Q' S] while four consumer warps, one TMEM lane
+// (= one state row or chunk row) per thread, keep the fp32 state block in registers.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "tcgen05.cuh"
 
 namespace kda {
 
@@ -32,229 +43,366 @@ namespace {
 constexpr int kC = KDA_CHUNK;  // tokens per chunk (state carried every kC tokens)
 constexpr int kTile = KDA_TILE;
 constexpr int kTiles = kC / kTile;
-constexpr int kRef = 7;        // reference token inside each 16-token tile (its middle)
+constexpr int kRef = 7;   // reference token inside each 16-token tile (its middle)
+constexpr int kBV = 32;   // value columns per scan CTA
 
 // ------------------------------------------------------------------ workspace record
+// One record per (batch*head, chunk):
+//   Nm   N = Khat^T W, D x D, K-major 128-byte swizzle (row = key channel)
+//   Qp   Q' = Qbar - P W, 64 x D, K-major 128-byte swizzle (row = token)
+//   Gam  Gamma = e^{G_last}, D floats
+//   then, per 32-column value block b: Bm[:, block b] (D x 32) and O'[:, block b]
+//   (64 x 32), both MN-major 64-byte swizzle.
+// An M = 128 MMA over Nm (D = 64) or Qp reads 64 rows past the operand: those rows fall on
+// the following fields of the same record and only feed accumulator lanes never read.
 template <int D>
 struct Rec {
-    static constexpr size_t kMat = (size_t)kC * D * 2;  // one C x D bf16 matrix
-    static constexpr size_t W = 0;
-    static constexpr size_t U = kMat;
-    static constexpr size_t Qb = 2 * kMat;
-    static constexpr size_t Kh = 3 * kMat;
-    static constexpr size_t P = 4 * kMat;                // C x C bf16
-    static constexpr size_t Gam = P + (size_t)kC * kC * 2;  // D x f32
-    static constexpr size_t Bytes = Gam + (size_t)D * 4;
-    static_assert(Bytes % 128 == 0, "records stay 128-byte aligned");
+    static constexpr uint32_t Nm = 0;
+    static constexpr uint32_t Qp = (uint32_t)D * D * 2;
+    static constexpr uint32_t Gam = Qp + (uint32_t)kC * D * 2;
+    static constexpr uint32_t Shared = Gam + (uint32_t)D * 4;  // bytes every scan CTA needs
+    static constexpr uint32_t BmBlk = (uint32_t)D * kBV * 2;
+    static constexpr uint32_t OpBlk = (uint32_t)kC * kBV * 2;
+    static constexpr uint32_t Blk = BmBlk + OpBlk;             // per value block
+    static constexpr uint32_t Bytes = Shared + (uint32_t)(D / kBV) * Blk;
+    static_assert(Bytes % 128 == 0 && Shared % 16 == 0 && Blk % 16 == 0, "record alignment");
+    static_assert(Qp % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+    // the padded rows of the scan's M = 128 reads stay inside a stage
+    static_assert(Qp + (D / 64 - 1) * kC * 128 + 2 * kC * 128 <= Shared + Blk, "padded rows in bounds");
 };
 
 // ------------------------------------------------------------------ K2: prep
 constexpr int kPrepThreads = 256;
 
 template <int D>
-struct PrepSmem {
-    static constexpr int LDB = D + 8;   // bf16 row stride (16-byte pad: conflict-free ldmatrix)
-    static constexpr int LDG = D + 8;   // f32 row stride (conflict-free float2 fragment reads)
-    static constexpr int LDA = kC + 1;  // f32 C x C matrices
-    static constexpr int LDT = kC + 8;  // bf16 C x C matrices
-    __nv_bfloat16 k[kC * LDB];
-    __nv_bfloat16 q[kC * LDB];   // later: W staging
-    __nv_bfloat16 v[kC * LDB];
-    __nv_bfloat16 ec[kC * LDB];  // k_j e^{G_{m(j)} - G_j}; later: Utilde staging
-    __nv_bfloat16 kb[kC * LDB];  // Kbar = k e^{G}
-    float G[kC * LDG];
-    float A[kC * LDA];
-    float Tm[kC * LDA];
-    __nv_bfloat16 tb[kC * LDT];  // bf16(T diag(beta))
-    __nv_bfloat16 pst[kC * LDT]; // P staging
-    float beta[kC];
-    float X[4][kTile][kTile + 1];  // triangular-solve scratch, one per warp
+struct PrepLayout {
+    static constexpr uint32_t kMat = (uint32_t)kC * D * 2;  // one 64 x D bf16 operand
+    // token-major operands (row = token, MN-major 128-byte swizzle by 64-channel block)
+    static constexpr uint32_t RQ = 0;          // q -> Qr = q E -> Qbar
+    static constexpr uint32_t RK = RQ + kMat;  // k -> Kr = k E -> Kbar   } adjacent: the B
+    static constexpr uint32_t RV = RK + kMat;  // v                       } operand [Kbar | V]
+    static constexpr uint32_t RX = RV + kMat;  // a -> Ec = k / E -> Khat
+    static constexpr uint32_t RP = RX + kMat;  // P, K-major 128-byte swizzle (64 x 64)
+    // G: fp32 [64][D] -> A [64][65] | T [64][65] | solve scratch -> T beta -> [W | Utilde]
+    static constexpr uint32_t RG = RP + (uint32_t)kC * kC * 2;
+    static constexpr uint32_t kGBytes = 2u * kC * D * 2 > (uint32_t)kC * D * 4 ? 2u * kC * D * 2 : (uint32_t)kC * D * 4;
+    static constexpr uint32_t kSolveBytes = 2u * kC * (kC + 1) * 4 + 3u * kTile * (kTile + 1) * 4;
+    static constexpr uint32_t kRGBytes = ((kGBytes > kSolveBytes ? kGBytes : kSolveBytes) + 1023) / 1024 * 1024;
+    static constexpr uint32_t RA = RG;                                // f32 [64][65]
+    static constexpr uint32_t RT = RG + (uint32_t)kC * (kC + 1) * 4;  // f32 [64][65]
+    static constexpr uint32_t RXS = RT + (uint32_t)kC * (kC + 1) * 4; // f32 [3][16][17]
+    // small tables
+    static constexpr uint32_t RBeta = RG + kRGBytes;       // f32 [64]
+    static constexpr uint32_t REm = RBeta + kC * 4;        // bf16 [4][D]  e^{G_{m_I}}
+    static constexpr uint32_t REl = REm + kTiles * D * 2;  // bf16 [4][D]  e^{G_last - G_{m_I}}
+    static constexpr uint32_t RDd = REl + kTiles * D * 2;  // bf16 [6][D]  e^{G_{m_I} - G_{m_J}}
+    static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarrier
+    static constexpr uint32_t RTmem = RBar + 8;
+    static constexpr uint32_t Bytes = RTmem + 8;
+    static_assert(RG % 1024 == 0 && RP % 1024 == 0, "operand alignment");
 };
 
-// One 16x16 output block of the level-L block substitution, done by one warp:
-//   T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ
-__device__ __forceinline__ void solve_offdiag_block(float *A, float *Tm, float (*X)[kTile + 1], int I, int J,
-                                                    int lane)
+// 16-byte chunk address of (token r, channels c8..c8+7) in a token-major operand.
+__device__ __forceinline__ uint32_t tok_off(int r, int c8) { return tc::mnmaj_sw128(r, c8, kC); }
+
+// One 16x16 output block of the block substitution, by two warps (rows split in halves):
+//   X = sum_{K=J}^{I-1} A_IK T_KJ  (phase 0),   T_IJ = -T_II X  (phase 1)
+__device__ __forceinline__ void solve_block_phase(const float *A, float *Tm, float (*X)[kTile + 1], int I, int J,
+                                                  int half, int lane, int phase)
 {
     constexpr int LDA = kC + 1;
     const int cc = lane % kTile;
-    const int r0 = (lane / kTile) * 8;
+    const int rbase = half * 8 + (lane / kTile) * 4;
+    if (phase == 0) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = J; K < I; ++K)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = r0 + i;
-        float s = 0.0f;
-        for (int K = J; K < I; ++K) {
+            for (int x = 0; x < kTile; ++x) {
+                const float t = Tm[(K * kTile + x) * LDA + J * kTile + cc];
 #pragma unroll
-            for (int x = 0; x < kTile; ++x)
-                s += A[(kTile * I + rr) * LDA + kTile * K + x] * Tm[(kTile * K + x) * LDA + kTile * J + cc];
+                for (int i = 0; i < 4; ++i)
+                    s[i] = fmaf(A[(I * kTile + rbase + i) * LDA + K * kTile + x], t, s[i]);
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            X[rbase + i][cc] = s[i];
+    } else {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int x = 0; x < kTile; ++x) {
+            const float xv = X[x][cc];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                s[i] = fmaf(Tm[(I * kTile + rbase + i) * LDA + I * kTile + x], xv, s[i]);
         }
-        X[rr][cc] = s;
-    }
-    __syncwarp();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = r0 + i;
-        float s = 0.0f;
-#pragma unroll
-        for (int x = 0; x < kTile; ++x)
-            s += Tm[(kTile * I + rr) * LDA + kTile * I + x] * X[x][cc];
-        Tm[(kTile * I + rr) * LDA + kTile * J + cc] = -s;
+        for (int i = 0; i < 4; ++i)
+            Tm[(I * kTile + rbase + i) * LDA + J * kTile + cc] = -s[i];
     }
-    __syncwarp();
+}
+
+// Multiply 8 packed bf16 by 8 packed bf16 scalars.
+__device__ __forceinline__ uint4 mul8(uint4 x, uint4 s)
+{
+    __nv_bfloat162 *xa = reinterpret_cast<__nv_bfloat162 *>(&x);
+    const __nv_bfloat162 *sa = reinterpret_cast<const __nv_bfloat162 *>(&s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        xa[i] = __hmul2(xa[i], sa[i]);
+    return x;
+}
+
+__device__ __forceinline__ uint4 pack8(const uint32_t *x)
+{
+    return make_uint4(pack_bf16x2(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                      pack_bf16x2(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                      pack_bf16x2(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                      pack_bf16x2(__uint_as_float(x[6]), __uint_as_float(x[7])));
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads, 1)
+__global__ void __launch_bounds__(kPrepThreads, 2)
     prep_kernel(int T, int H, int NT, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
-                const __nv_bfloat16 *__restrict__ beta, float g_min, unsigned char *__restrict__ ws)
+                const __nv_bfloat16 *__restrict__ beta, float g_min, unsigned char *__restrict__ ws,
+                unsigned int *status)
 {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    using SM = PrepSmem<D>;
-    SM &sm = *reinterpret_cast<SM *>(smem_raw);
-    constexpr int LDB = SM::LDB, LDG = SM::LDG, LDA = SM::LDA, LDT = SM::LDT;
+    extern __shared__ __align__(1024) unsigned char prep_smem[];
+    using L = PrepLayout<D>;
+    using R = Rec<D>;
+    // Two CTAs share an SM only without alignment slack: the swizzled operands need a
+    // 1024-byte aligned base, which the dynamic shared window provides; refuse otherwise.
+    if (smem_u32(prep_smem) & 1023u) {
+        if (threadIdx.x == 0)
+            report_device_error(status, KDA_ERR_UNSUPPORTED);
+        return;
+    }
+    unsigned char *sm = prep_smem;
+    constexpr int LDA = kC + 1;
+    constexpr int CPR = D / 8;  // 16-byte chunks per token row
+    float *sG = reinterpret_cast<float *>(sm + L::RG);   // [64][D]
+    float *sA = reinterpret_cast<float *>(sm + L::RA);   // [64][65]
+    float *sT = reinterpret_cast<float *>(sm + L::RT);   // [64][65]
+    float(*sX)[kTile][kTile + 1] = reinterpret_cast<float(*)[kTile][kTile + 1]>(sm + L::RXS);
+    float *sBeta = reinterpret_cast<float *>(sm + L::RBeta);
+    __nv_bfloat16 *sEm = reinterpret_cast<__nv_bfloat16 *>(sm + L::REm);
+    __nv_bfloat16 *sEl = reinterpret_cast<__nv_bfloat16 *>(sm + L::REl);
+    __nv_bfloat16 *sDd = reinterpret_cast<__nv_bfloat16 *>(sm + L::RDd);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::RBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::RTmem);
+
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = lane >> 2, tq = lane & 3;
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / H, h = bh % H;
     const int t0 = chunk * kC;
     const int n = min(kC, T - t0);
-    unsigned char *rec = ws + ((size_t)bh * NT + chunk) * Rec<D>::Bytes;
+    unsigned char *rec = ws + ((size_t)bh * NT + chunk) * R::Bytes;
     const int64_t rowstride = (int64_t)H * D;  // elements between consecutive tokens
     const int64_t base = (((int64_t)b * T + t0) * H + h) * D;
 
-    // -- 1. async loads of k, q, v (zero-filled past the end of the sequence)
-    for (int i = tid; i < kC * (D / 8); i += kPrepThreads) {
-        const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
+    // -- 0. async loads of q, k, v, a into the swizzled token-major operands (zero past T)
+    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
+        const int r = i / CPR, c8 = (i % CPR) * 8;
         const bool ok = r < n;
         const int64_t off = base + (ok ? (int64_t)r * rowstride : 0) + c8;
-        cp_async_16_zfill(&sm.k[r * LDB + c8], k + off, ok);
-        cp_async_16_zfill(&sm.q[r * LDB + c8], q + off, ok);
-        cp_async_16_zfill(&sm.v[r * LDB + c8], v + off, ok);
+        const uint32_t d = tok_off(r, c8);
+        cp_async_16_zfill(sm + L::RQ + d, q + off, ok);
+        cp_async_16_zfill(sm + L::RK + d, k + off, ok);
+        cp_async_16_zfill(sm + L::RV + d, v + off, ok);
+        cp_async_16_zfill(sm + L::RX + d, a + off, ok);
     }
     cp_async_commit();
     if (tid < kC)
-        sm.beta[tid] = tid < n ? __bfloat162float(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.0f;
+        sBeta[tid] = tid < n ? __bfloat162float(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.0f;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 0)
+        tc::tmem_alloc(tslot, 2 * D);
+    cp_async_wait<0>();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tslot;
 
-    // -- 2. gate and inclusive cumulative log-decay; kPrepThreads/D threads per channel
+    // -- 1. gate g = g_min sigmoid(a) (0 past T), then inclusive cumulative sum over tokens
+    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
+        const int r = i / CPR, c8 = (i % CPR) * 8;
+        const uint4 au = *reinterpret_cast<const uint4 *>(sm + L::RX + tok_off(r, c8));
+        const uint32_t w[4] = {au.x, au.y, au.z, au.w};
+        float gv[8];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 f = unpack_bf16x2(w[p]);
+            gv[2 * p] = r < n ? gate_bounded_fast(f.x, g_min) : 0.0f;
+            gv[2 * p + 1] = r < n ? gate_bounded_fast(f.y, g_min) : 0.0f;
+        }
+        float4 *dst = reinterpret_cast<float4 *>(&sG[r * D + c8]);
+        dst[0] = make_float4(gv[0], gv[1], gv[2], gv[3]);
+        dst[1] = make_float4(gv[4], gv[5], gv[6], gv[7]);
+    }
+    __syncthreads();
     {
         constexpr int TPC = kPrepThreads / D;
-        constexpr int L = kC / TPC;
+        constexpr int LEN = kC / TPC;
         const int c = tid % D, part = tid / D;
         float acc = 0.0f;
-        for (int r = part * L; r < part * L + L; ++r) {
-            float g = 0.0f;
-            if (r < n)
-                g = gate_bounded_fast(__bfloat162float(a[base + (int64_t)r * rowstride + c]), g_min);
-            acc += g;
-            sm.G[r * LDG + c] = acc;
+#pragma unroll 8
+        for (int r = part * LEN; r < part * LEN + LEN; ++r) {
+            acc += sG[r * D + c];
+            sG[r * D + c] = acc;
         }
         __syncthreads();
         float off = 0.0f;
         for (int p = 0; p < part; ++p)
-            off += sm.G[(p * L + L - 1) * LDG + c];
+            off += sG[(p * LEN + LEN - 1) * D + c];
         __syncthreads();
         if (part > 0)
-            for (int r = part * L; r < part * L + L; ++r)
-                sm.G[r * LDG + c] += off;
+#pragma unroll 8
+            for (int r = part * LEN; r < part * LEN + LEN; ++r)
+                sG[r * D + c] += off;
     }
-    cp_async_wait<0>();
     __syncthreads();
 
-    // -- 3. elementwise decay factors; Qbar, Khat, Gamma_C go straight to the workspace
+    // -- 2. per-(tile, channel) decay scalars (bf16) and Gamma_C (record)
+    for (int i = tid; i < kTiles * D; i += kPrepThreads) {
+        const int I = i / D, c = i % D;
+        const float Gm = sG[(I * kTile + kRef) * D + c];
+        sEm[i] = __float2bfloat16(__expf(Gm));
+        sEl[i] = __float2bfloat16(__expf(sG[(kC - 1) * D + c] - Gm));
+    }
+    for (int i = tid; i < 6 * D; i += kPrepThreads) {
+        const int p = i / D, c = i % D;
+        const int I = p < 1 ? 1 : (p < 3 ? 2 : 3);
+        const int J = p - I * (I - 1) / 2;
+        sDd[i] = __float2bfloat16(__expf(sG[(I * kTile + kRef) * D + c] - sG[(J * kTile + kRef) * D + c]));
+    }
     {
-        __nv_bfloat16 *gQb = reinterpret_cast<__nv_bfloat16 *>(rec + Rec<D>::Qb);
-        __nv_bfloat16 *gKh = reinterpret_cast<__nv_bfloat16 *>(rec + Rec<D>::Kh);
-        for (int i = tid; i < kC * (D / 8); i += kPrepThreads) {
-            const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-            const int m = (r / kTile) * kTile + kRef;
-            const uint4 ku = *reinterpret_cast<const uint4 *>(&sm.k[r * LDB + c8]);
-            const uint4 qu = *reinterpret_cast<const uint4 *>(&sm.q[r * LDB + c8]);
-            const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w};
-            const uint32_t qw[4] = {qu.x, qu.y, qu.z, qu.w};
-            uint32_t ec[4], kb[4], qb[4], kh[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const int c = c8 + 2 * p;
-                const float2 kk = unpack_bf16x2(kw[p]), qq = unpack_bf16x2(qw[p]);
-                const float G0 = sm.G[r * LDG + c], G1 = sm.G[r * LDG + c + 1];
-                const float M0 = sm.G[m * LDG + c], M1 = sm.G[m * LDG + c + 1];
-                const float L0 = sm.G[(kC - 1) * LDG + c], L1 = sm.G[(kC - 1) * LDG + c + 1];
-                const float e0 = __expf(G0), e1 = __expf(G1);
-                ec[p] = pack_bf16x2(kk.x * __expf(M0 - G0), kk.y * __expf(M1 - G1));
-                kb[p] = pack_bf16x2(kk.x * e0, kk.y * e1);
-                qb[p] = pack_bf16x2(qq.x * e0, qq.y * e1);
-                kh[p] = pack_bf16x2(kk.x * __expf(L0 - G0), kk.y * __expf(L1 - G1));
-            }
-            *reinterpret_cast<uint4 *>(&sm.ec[r * LDB + c8]) = make_uint4(ec[0], ec[1], ec[2], ec[3]);
-            *reinterpret_cast<uint4 *>(&sm.kb[r * LDB + c8]) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
-            *reinterpret_cast<uint4 *>(&gQb[r * D + c8]) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
-            *reinterpret_cast<uint4 *>(&gKh[r * D + c8]) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-        }
-        float *gGam = reinterpret_cast<float *>(rec + Rec<D>::Gam);
+        float *gGam = reinterpret_cast<float *>(rec + R::Gam);
         for (int c = tid; c < D; c += kPrepThreads)
-            gGam[c] = __expf(sm.G[(kC - 1) * LDG + c]);
-        for (int i = tid; i < kC * kC; i += kPrepThreads)
-            sm.pst[(i / kC) * LDT + (i % kC)] = __float2bfloat16(0.0f);
+            gGam[c] = __expf(sG[(kC - 1) * D + c]);
+    }
+
+    // -- 3. decay factors with the tile's middle token as reference: E = e^{G - G_m}
+    //       Kr = k E and Qr = q E in place of k and q, Ec = k / E in place of a
+    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
+        const int r = i / CPR, c8 = (i % CPR) * 8;
+        const int m = (r / kTile) * kTile + kRef;
+        const uint32_t d = tok_off(r, c8);
+        const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + d);
+        const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + d);
+        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w};
+        const uint32_t qw[4] = {qu.x, qu.y, qu.z, qu.w};
+        const float4 G0 = *reinterpret_cast<const float4 *>(&sG[r * D + c8]);
+        const float4 G1 = *reinterpret_cast<const float4 *>(&sG[r * D + c8 + 4]);
+        const float4 M0 = *reinterpret_cast<const float4 *>(&sG[m * D + c8]);
+        const float4 M1 = *reinterpret_cast<const float4 *>(&sG[m * D + c8 + 4]);
+        const float x[8] = {G0.x - M0.x, G0.y - M0.y, G0.z - M0.z, G0.w - M0.w,
+                            G1.x - M1.x, G1.y - M1.y, G1.z - M1.z, G1.w - M1.w};
+        uint32_t kr[4], qr[4], ec[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 kk = unpack_bf16x2(kw[p]), qq = unpack_bf16x2(qw[p]);
+            const float e0 = __expf(x[2 * p]), e1 = __expf(x[2 * p + 1]);
+            const float i0 = __expf(-x[2 * p]), i1 = __expf(-x[2 * p + 1]);
+            kr[p] = pack_bf16x2(kk.x * e0, kk.y * e1);
+            qr[p] = pack_bf16x2(qq.x * e0, qq.y * e1);
+            ec[p] = pack_bf16x2(kk.x * i0, kk.y * i1);
+        }
+        *reinterpret_cast<uint4 *>(sm + L::RK + d) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
+        *reinterpret_cast<uint4 *>(sm + L::RQ + d) = make_uint4(qr[0], qr[1], qr[2], qr[3]);
+        *reinterpret_cast<uint4 *>(sm + L::RX + d) = make_uint4(ec[0], ec[1], ec[2], ec[3]);
+    }
+    // upper blocks of P are zero
+    for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
+        const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+        if (j / kTile > r / kTile)
+            *reinterpret_cast<uint32_t *>(sm + L::RP + tc::kmaj_sw128(r, j, kC)) = 0u;
     }
     __syncthreads();
 
-    // -- 4. dense tile products A and P: one warp per (row tile I, column tile J <= I).
-    //       Row operands k_r e^{G_r - G_{m_J}} and q_r e^{G_r - G_{m_J}} are built in
-    //       registers from G; the column operand is ec (tile J, referenced at m_J).
-    {
-        const int grp = lane >> 2, tq = lane & 3;
-        for (int pidx = warp; pidx < kTiles * (kTiles + 1) / 2; pidx += kPrepThreads / 32) {
-            int I = 0, J = pidx;
-            while (J > I) {  // pidx -> (I, J): 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) ...
-                J -= I + 1;
-                ++I;
-            }
-            const int m = J * kTile + kRef;
-            float accA[2][4] = {}, accP[2][4] = {};
+    // -- 4. dense 16-token tile products A and P, one warp per (row tile I, column tile
+    //       J <= I): row operands Kr, Qr of tile I (scaled by e^{G_{m_I} - G_{m_J}} when
+    //       I > J), column operand Ec of tile J.  A (fp32, beta-scaled, strictly lower)
+    //       goes over G, which is no longer needed; P (bf16, lower) to its operand slot.
+    for (int pidx = warp; pidx < kTiles * (kTiles + 1) / 2; pidx += kPrepThreads / 32) {
+        int I = 0, J = pidx;
+        while (J > I) {  // pidx -> (I, J): 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) ...
+            J -= I + 1;
+            ++I;
+        }
+        const __nv_bfloat16 *dsc = I > J ? &sDd[(I * (I - 1) / 2 + J) * D] : nullptr;
+        float accA[2][4] = {}, accP[2][4] = {};
 #pragma unroll 2
-            for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t ak[4], aq[4];
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t ak[4], aq[4], bf[4];
+            const int mi = lane >> 3;
+            {
+                const int row = I * kTile + (lane & 7) + 8 * (mi & 1);
+                const int col = ks * 16 + 8 * (mi >> 1);
+                ldmatrix_x4(ak, sm + L::RK + tok_off(row, col));
+                ldmatrix_x4(aq, sm + L::RQ + tok_off(row, col));
+            }
+            if (dsc) {
 #pragma unroll
                 for (int reg = 0; reg < 4; ++reg) {
-                    const int r = I * kTile + grp + 8 * (reg & 1);
                     const int c = ks * 16 + 2 * tq + 8 * (reg >> 1);
-                    const float2 Gr = *reinterpret_cast<const float2 *>(&sm.G[r * LDG + c]);
-                    const float2 Gm = *reinterpret_cast<const float2 *>(&sm.G[m * LDG + c]);
-                    const float e0 = __expf(Gr.x - Gm.x), e1 = __expf(Gr.y - Gm.y);
-                    const float2 kk = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(&sm.k[r * LDB + c]));
-                    const float2 qq = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(&sm.q[r * LDB + c]));
-                    ak[reg] = pack_bf16x2(kk.x * e0, kk.y * e1);
-                    aq[reg] = pack_bf16x2(qq.x * e0, qq.y * e1);
+                    const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162 *>(&dsc[c]);
+                    __nv_bfloat162 kk = *reinterpret_cast<__nv_bfloat162 *>(&ak[reg]);
+                    __nv_bfloat162 qq = *reinterpret_cast<__nv_bfloat162 *>(&aq[reg]);
+                    kk = __hmul2(kk, s2);
+                    qq = __hmul2(qq, s2);
+                    ak[reg] = *reinterpret_cast<uint32_t *>(&kk);
+                    aq[reg] = *reinterpret_cast<uint32_t *>(&qq);
                 }
-                uint32_t bf[4];
-                {
-                    const int mi = lane >> 3;
-                    const int row = J * kTile + (lane & 7) + 8 * (mi >> 1);
-                    const int col = ks * 16 + 8 * (mi & 1);
-                    ldmatrix_x4(bf, &sm.ec[row * LDB + col]);
-                }
-                const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-                mma_bf16_16816(accA[0], ak, b0);
-                mma_bf16_16816(accA[1], ak, b1);
-                mma_bf16_16816(accP[0], aq, b0);
-                mma_bf16_16816(accP[1], aq, b1);
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = I * kTile + grp + 8 * (e >> 1);
-                    const int j = J * kTile + nt * 8 + 2 * tq + (e & 1);
-                    const bool lowA = I > J || j < r, lowP = I > J || j <= r;
-                    sm.A[r * LDA + j] = lowA ? sm.beta[r] * accA[nt][e] : 0.0f;
-                    sm.pst[r * LDT + j] = __float2bfloat16(lowP ? accP[nt][e] : 0.0f);
-                }
+            {
+                const int row = J * kTile + (lane & 7) + 8 * (mi >> 1);
+                const int col = ks * 16 + 8 * (mi & 1);
+                ldmatrix_x4(bf, sm + L::RX + tok_off(row, col));
+            }
+            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+            mma_bf16_16816(accA[0], ak, b0);
+            mma_bf16_16816(accA[1], ak, b1);
+            mma_bf16_16816(accP[0], aq, b0);
+            mma_bf16_16816(accP[1], aq, b1);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = I * kTile + grp + 8 * hh;
+                const int j = J * kTile + nt * 8 + 2 * tq;
+                const bool lo0 = I > J || j < r, lo1 = I > J || j + 1 < r;
+                const bool lp0 = I > J || j <= r, lp1 = I > J || j + 1 <= r;
+                sA[r * LDA + j] = lo0 ? sBeta[r] * accA[nt][2 * hh] : 0.0f;
+                sA[r * LDA + j + 1] = lo1 ? sBeta[r] * accA[nt][2 * hh + 1] : 0.0f;
+                *reinterpret_cast<uint32_t *>(sm + L::RP + tc::kmaj_sw128(r, j, kC)) =
+                    pack_bf16x2(lp0 ? accP[nt][2 * hh] : 0.0f, lp1 ? accP[nt][2 * hh + 1] : 0.0f);
+            }
     }
     __syncthreads();
 
-    // -- 5. T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution, then block
-    //       substitution level by level.
+    // -- 4b. chunk-referenced operands in place: Kbar = Kr e^{G_m}, Qbar = Qr e^{G_m},
+    //        Khat = Ec e^{G_last - G_m}
+    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
+        const int r = i / CPR, c8 = (i % CPR) * 8;
+        const int tile = r / kTile;
+        const uint32_t d = tok_off(r, c8);
+        const uint4 em = *reinterpret_cast<const uint4 *>(&sEm[tile * D + c8]);
+        const uint4 el = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
+        uint4 *pk = reinterpret_cast<uint4 *>(sm + L::RK + d);
+        uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + d);
+        uint4 *px = reinterpret_cast<uint4 *>(sm + L::RX + d);
+        *pk = mul8(*pk, em);
+        *pq = mul8(*pq, em);
+        *px = mul8(*px, el);
+    }
+
+    // -- 5. T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (one lane per
+    //       column), then block substitution level by level, two warps per block.
     if (warp < kTiles && lane < kTile) {
         const int I = warp, c = lane;
         float x[kTile];
@@ -266,331 +414,356 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             float s = 0.0f;
 #pragma unroll
             for (int y = 0; y < r; ++y)
-                s += sm.A[(I * kTile + r) * LDA + I * kTile + y] * x[y];
+                s = fmaf(sA[(I * kTile + r) * LDA + I * kTile + y], x[y], s);
             if (r > c)
                 x[r] = -s;
         }
 #pragma unroll
         for (int r = 0; r < kTile; ++r)
-            sm.Tm[(I * kTile + r) * LDA + I * kTile + c] = x[r];
+            sT[(I * kTile + r) * LDA + I * kTile + c] = x[r];
     }
-    // upper blocks of T are zero
     for (int i = tid; i < kC * kC; i += kPrepThreads) {
         const int r = i / kC, j = i % kC;
         if (j / kTile > r / kTile)
-            sm.Tm[r * LDA + j] = 0.0f;
+            sT[r * LDA + j] = 0.0f;
     }
     __syncthreads();
     for (int lvl = 1; lvl < kTiles; ++lvl) {
-        if (warp < kTiles - lvl)
-            solve_offdiag_block(sm.A, sm.Tm, sm.X[warp], warp + lvl, warp, lane);
+        const int nblk = kTiles - lvl;
+        const int blk = warp >> 1, half = warp & 1;
+        if (blk < nblk)
+            solve_block_phase(sA, sT, sX[blk], blk + lvl, blk, half, lane, 0);
+        __syncthreads();
+        if (blk < nblk)
+            solve_block_phase(sA, sT, sX[blk], blk + lvl, blk, half, lane, 1);
         __syncthreads();
     }
-    // bf16(T diag(beta)); P staging -> workspace
-    for (int i = tid; i < kC * kC; i += kPrepThreads) {
-        const int r = i / kC, j = i % kC;
-        sm.tb[r * LDT + j] = __float2bfloat16(sm.Tm[r * LDA + j] * sm.beta[j]);
+    // T diag(beta) as the K-major A operand (over A's place; the 8 KB after it are the
+    // don't-care rows of the M = 128 MMA)
+    for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
+        const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) =
+            pack_bf16x2(sT[r * LDA + j] * sBeta[j], sT[r * LDA + j + 1] * sBeta[j + 1]);
     }
-    {
-        __nv_bfloat16 *gP = reinterpret_cast<__nv_bfloat16 *>(rec + Rec<D>::P);
-        for (int i = tid; i < kC * (kC / 8); i += kPrepThreads) {
-            const int r = i / (kC / 8), c8 = (i % (kC / 8)) * 8;
-            *reinterpret_cast<uint4 *>(&gP[r * kC + c8]) = *reinterpret_cast<const uint4 *>(&sm.pst[r * LDT + c8]);
-        }
-    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
     __syncthreads();
+    tc::fence_after_sync();
 
-    // -- 6. W = (T beta) Kbar, Utilde = (T beta) V: warp -> (row tile I, half of D)
-    {
-        const int grp = lane >> 2, tq = lane & 3;
-        const int I = warp % kTiles, nh = warp / kTiles;
-        constexpr int NTL = D / 16;  // n8 tiles per warp (half of D)
-        float accW[NTL][4] = {}, accU[NTL][4] = {};
-        for (int ks = 0; ks <= I; ++ks) {
-            uint32_t af[4];
-            {
-                const int mi = lane >> 3;
-                const int row = I * kTile + (lane & 7) + 8 * (mi & 1);
-                const int col = ks * 16 + 8 * (mi >> 1);
-                ldmatrix_x4(af, &sm.tb[row * LDT + col]);
-            }
-#pragma unroll
-            for (int np = 0; np < NTL / 2; ++np) {
-                const int mi = lane >> 3;
-                const int row = ks * 16 + (lane & 7) + 8 * (mi & 1);
-                const int col = nh * (D / 2) + np * 16 + 8 * (mi >> 1);
-                uint32_t bk[4], bv[4];
-                ldmatrix_x4_trans(bk, &sm.kb[row * LDB + col]);
-                ldmatrix_x4_trans(bv, &sm.v[row * LDB + col]);
-                const uint32_t k0[2] = {bk[0], bk[1]}, k1[2] = {bk[2], bk[3]};
-                const uint32_t v0[2] = {bv[0], bv[1]}, v1[2] = {bv[2], bv[3]};
-                mma_bf16_16816(accW[2 * np], af, k0);
-                mma_bf16_16816(accW[2 * np + 1], af, k1);
-                mma_bf16_16816(accU[2 * np], af, v0);
-                mma_bf16_16816(accU[2 * np + 1], af, v1);
-            }
-        }
-        // stage in shared memory (q and ec are free now), then coalesced copies out
-#pragma unroll
-        for (int nt = 0; nt < NTL; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = I * kTile + grp + 8 * hh;
-                const int c = nh * (D / 2) + nt * 8 + 2 * tq;
-                *reinterpret_cast<uint32_t *>(&sm.q[r * LDB + c]) =
-                    pack_bf16x2(accW[nt][2 * hh], accW[nt][2 * hh + 1]);
-                *reinterpret_cast<uint32_t *>(&sm.ec[r * LDB + c]) =
-                    pack_bf16x2(accU[nt][2 * hh], accU[nt][2 * hh + 1]);
-            }
-    }
-    __syncthreads();
-    {
-        __nv_bfloat16 *gW = reinterpret_cast<__nv_bfloat16 *>(rec + Rec<D>::W);
-        __nv_bfloat16 *gU = reinterpret_cast<__nv_bfloat16 *>(rec + Rec<D>::U);
-        for (int i = tid; i < kC * (D / 8); i += kPrepThreads) {
-            const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-            *reinterpret_cast<uint4 *>(&gW[r * D + c8]) = *reinterpret_cast<const uint4 *>(&sm.q[r * LDB + c8]);
-            *reinterpret_cast<uint4 *>(&gU[r * D + c8]) = *reinterpret_cast<const uint4 *>(&sm.ec[r * LDB + c8]);
-        }
-    }
-}
-
-// ------------------------------------------------------------------ K3: scan
-constexpr int kScanThreads = 128;  // 4 warps: warp w owns chunk rows [16w, 16w+16)
-
-template <int D, int BV>
-struct ScanStage {
-    static constexpr int LDB = D + 8;
-    static constexpr int LDP = kC + 8;
-    static constexpr int LDU = BV + 8;
-    __nv_bfloat16 W[kC * LDB];
-    __nv_bfloat16 Qb[kC * LDB];
-    __nv_bfloat16 Kh[kC * LDB];
-    __nv_bfloat16 P[kC * LDP];
-    __nv_bfloat16 U[kC * LDU];
-    float gam[D];
-};
-
-template <int D, int BV>
-struct ScanSmem {
-    static constexpr int LDU = BV + 8;
-    ScanStage<D, BV> st[2];
-    __nv_bfloat16 Sb[D * LDU];  // current state block, bf16 (B operand)
-    __nv_bfloat16 Uc[kC * LDU]; // corrected U = Utilde - W S, bf16 (B operand)
-};
-
-template <int D, int BV>
-__device__ __forceinline__ void scan_load_stage(ScanStage<D, BV> &st, const unsigned char *rec, int col0, int tid)
-{
-    constexpr int LDB = ScanStage<D, BV>::LDB, LDP = ScanStage<D, BV>::LDP, LDU = ScanStage<D, BV>::LDU;
-    const __nv_bfloat16 *gW = reinterpret_cast<const __nv_bfloat16 *>(rec + Rec<D>::W);
-    const __nv_bfloat16 *gQ = reinterpret_cast<const __nv_bfloat16 *>(rec + Rec<D>::Qb);
-    const __nv_bfloat16 *gK = reinterpret_cast<const __nv_bfloat16 *>(rec + Rec<D>::Kh);
-    const __nv_bfloat16 *gP = reinterpret_cast<const __nv_bfloat16 *>(rec + Rec<D>::P);
-    const __nv_bfloat16 *gU = reinterpret_cast<const __nv_bfloat16 *>(rec + Rec<D>::U);
-    const float *gG = reinterpret_cast<const float *>(rec + Rec<D>::Gam);
-    for (int i = tid; i < kC * (D / 8); i += kScanThreads) {
-        const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-        cp_async_16(&st.W[r * LDB + c8], gW + r * D + c8);
-        cp_async_16(&st.Qb[r * LDB + c8], gQ + r * D + c8);
-        cp_async_16(&st.Kh[r * LDB + c8], gK + r * D + c8);
-    }
-    for (int i = tid; i < kC * (kC / 8); i += kScanThreads) {
-        const int r = i / (kC / 8), c8 = (i % (kC / 8)) * 8;
-        cp_async_16(&st.P[r * LDP + c8], gP + r * kC + c8);
-    }
-    for (int i = tid; i < kC * (BV / 8); i += kScanThreads) {
-        const int r = i / (BV / 8), c8 = (i % (BV / 8)) * 8;
-        cp_async_16(&st.U[r * LDU + c8], gU + r * D + col0 + c8);
-    }
-    for (int i = tid; i < D / 4; i += kScanThreads)
-        cp_async_16(&st.gam[4 * i], gG + 4 * i);
-}
-
-template <int D, int BV>
-__global__ void __launch_bounds__(kScanThreads, 1)
-    scan_kernel(int T, int H, int NT, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
-                __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T)
-{
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    using SM = ScanSmem<D, BV>;
-    SM &sm = *reinterpret_cast<SM *>(smem_raw);
-    constexpr int LDB = ScanStage<D, BV>::LDB, LDP = ScanStage<D, BV>::LDP, LDU = SM::LDU;
-    constexpr int MT = D / 64;   // 16-row state tiles per warp (warp owns D/4 state rows)
-    constexpr int NTL = BV / 8;  // n8 tiles across the value block
-    constexpr int KS = D / 16;   // k16 steps over the key dim
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int grp = lane >> 2, tq = lane & 3;
-    const int col0 = blockIdx.x * BV, bh = blockIdx.y;
-    const int b = bh / H, h = bh % H;
-    const unsigned char *recs = ws + (size_t)bh * NT * Rec<D>::Bytes;
-    const int srow0 = warp * (D / 4);
-
-    // state block in registers (C-fragment layout): rows srow0 + 16 mt + grp (+8)
-    float S[MT][NTL][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NTL; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = srow0 + 16 * mt + grp + 8 * hh;
-                const int c = col0 + nt * 8 + 2 * tq;
-                float2 s = make_float2(0.0f, 0.0f);
-                if (S0)
-                    s = *reinterpret_cast<const float2 *>(&S0[((size_t)bh * D + r) * D + c]);
-                S[mt][nt][2 * hh] = s.x;
-                S[mt][nt][2 * hh + 1] = s.y;
-                *reinterpret_cast<uint32_t *>(&sm.Sb[r * LDU + nt * 8 + 2 * tq]) = pack_bf16x2(s.x, s.y);
-            }
-
-    scan_load_stage<D, BV>(sm.st[0], recs, col0, tid);
-    cp_async_commit();
-
-    for (int c = 0; c < NT; ++c) {
-        if (c + 1 < NT) {
-            scan_load_stage<D, BV>(sm.st[(c + 1) & 1], recs + (size_t)(c + 1) * Rec<D>::Bytes, col0, tid);
-            cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        ScanStage<D, BV> &st = sm.st[c & 1];
-
-        // (1) X = W S and Y = Qbar S for chunk rows [16 warp, +16)
-        float X[NTL][4] = {}, Y[NTL][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            uint32_t aw[4], aq[4];
-            {
-                const int mi = lane >> 3;
-                const int row = warp * 16 + (lane & 7) + 8 * (mi & 1);
-                const int col = ks * 16 + 8 * (mi >> 1);
-                ldmatrix_x4(aw, &st.W[row * LDB + col]);
-                ldmatrix_x4(aq, &st.Qb[row * LDB + col]);
-            }
-#pragma unroll
-            for (int np = 0; np < NTL / 2; ++np) {
-                const int mi = lane >> 3;
-                const int row = ks * 16 + (lane & 7) + 8 * (mi & 1);
-                const int col = np * 16 + 8 * (mi >> 1);
-                uint32_t bs[4];
-                ldmatrix_x4_trans(bs, &sm.Sb[row * LDU + col]);
-                const uint32_t s0[2] = {bs[0], bs[1]}, s1[2] = {bs[2], bs[3]};
-                mma_bf16_16816(X[2 * np], aw, s0);
-                mma_bf16_16816(X[2 * np + 1], aw, s1);
-                mma_bf16_16816(Y[2 * np], aq, s0);
-                mma_bf16_16816(Y[2 * np + 1], aq, s1);
-            }
-        }
-        // (2) U = Utilde - X -> Uc (bf16)
-#pragma unroll
-        for (int nt = 0; nt < NTL; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = warp * 16 + grp + 8 * hh;
-                const int cc = nt * 8 + 2 * tq;
-                const float2 ut = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(&st.U[r * LDU + cc]));
-                *reinterpret_cast<uint32_t *>(&sm.Uc[r * LDU + cc]) =
-                    pack_bf16x2(ut.x - X[nt][2 * hh], ut.y - X[nt][2 * hh + 1]);
-            }
-        __syncthreads();
-
-        // (3) B fragments of U (tokens x value block), shared by P U and Khat^T U
-        uint32_t bu[kC / 16][NTL][2];
-#pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks)
-#pragma unroll
-            for (int np = 0; np < NTL / 2; ++np) {
-                const int mi = lane >> 3;
-                const int row = ks * 16 + (lane & 7) + 8 * (mi & 1);
-                const int col = np * 16 + 8 * (mi >> 1);
-                uint32_t r4[4];
-                ldmatrix_x4_trans(r4, &sm.Uc[row * LDU + col]);
-                bu[ks][2 * np][0] = r4[0];
-                bu[ks][2 * np][1] = r4[1];
-                bu[ks][2 * np + 1][0] = r4[2];
-                bu[ks][2 * np + 1][1] = r4[3];
-            }
-        // O = Y + P U (P is lower triangular: k-steps 0..warp)
+    // -- 6. tensor core round 1: [W | Utilde] = (T beta) [Kbar | V]  (64 x 2D, TMEM cols 0..2D)
+    uint32_t phase = 0;
+    if (tid == 0) {
+        const uint32_t id = tc::idesc_bf16(128, 2 * D, false, true);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
-            if (ks > warp)
-                break;
-            uint32_t ap[4];
-            const int mi = lane >> 3;
-            const int row = warp * 16 + (lane & 7) + 8 * (mi & 1);
-            const int col = ks * 16 + 8 * (mi >> 1);
-            ldmatrix_x4(ap, &st.P[row * LDP + col]);
-#pragma unroll
-            for (int nt = 0; nt < NTL; ++nt)
-                mma_bf16_16816(Y[nt], ap, bu[ks][nt]);
+            const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RG) + ks * 32, 16, 1024, tc::kSw128);
+            const uint64_t bd = tc::smem_desc(smem_u32(sm + L::RK) + ks * 2048, kC * 128, 1024, tc::kSw128);
+            tc::mma_bf16(tmem, ad, bd, id, ks > 0 ? 1u : 0u);
         }
-        {
-            const int tbase = c * kC + warp * 16;
+        tc::commit(bar);
+    }
+    mbar_wait_bounded(bar, phase, status);
+    phase ^= 1;
+    tc::fence_after_sync();
+    // [W | Utilde] (chunk rows 0..63 = TMEM lanes 0..63) -> bf16 token-major operand over G
+    if ((warp & 3) < 2) {
+        const int r = (warp & 3) * 32 + lane;
+        const int cbase = (warp >> 2) * D;  // warps 0,1: W; warps 4,5: Utilde
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int t = tbase + grp + 8 * hh;
-                if (t < T) {
-                    __nv_bfloat16 *orow = o + (((int64_t)b * T + t) * H + h) * D + col0;
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t x[32];
+            tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cbase + c0), x);
+            tc::wait_ld();
 #pragma unroll
-                    for (int nt = 0; nt < NTL; ++nt)
-                        *reinterpret_cast<uint32_t *>(&orow[nt * 8 + 2 * tq]) =
-                            pack_bf16x2(Y[nt][2 * hh], Y[nt][2 * hh + 1]);
-                }
-            }
+            for (int j = 0; j < 32; j += 8)  // [W | Utilde] column; 64-column blocks 8 KB apart
+                *reinterpret_cast<uint4 *>(sm + L::RG + tok_off(r, cbase + c0 + j)) = pack8(&x[j]);
         }
-        // (4) S <- Diag(Gamma_C) S + Khat^T U
+        tc::fence_smem_to_async();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+
+    // -- 7. rounds 2 and 3: Khat^T X (TMEM cols 0..D) and P X (cols D..2D) for X = W, then
+    //       X = Utilde.  Epilogues: N, Q' = Qbar - P W; then Bm, O' = P Utilde.
+#pragma unroll 1
+    for (int round = 0; round < 2; ++round) {
+        if (tid == 0) {
+            const uint32_t id_kt = tc::idesc_bf16(128, D, true, true);  // A = Khat^T (MN-major)
+            const uint32_t id_p = tc::idesc_bf16(128, D, false, true);  // A = P (K-major)
+            const uint32_t xb = smem_u32(sm + L::RG) + round * (D / 64) * (kC * 128);
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const float g0 = st.gam[srow0 + 16 * mt + grp], g1 = st.gam[srow0 + 16 * mt + grp + 8];
-#pragma unroll
-            for (int nt = 0; nt < NTL; ++nt) {
-                S[mt][nt][0] *= g0;
-                S[mt][nt][1] *= g0;
-                S[mt][nt][2] *= g1;
-                S[mt][nt][3] *= g1;
+            for (int ks = 0; ks < kC / 16; ++ks) {
+                const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RX) + ks * 2048, kC * 128, 1024, tc::kSw128);
+                const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
+                tc::mma_bf16(tmem, ad, bd, id_kt, ks > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int ks = 0; ks < kC / 16; ++ks) {
-                uint32_t ak[4];
-                const int mi = lane >> 3;
-                const int row = ks * 16 + (lane & 7) + 8 * (mi >> 1);   // token
-                const int col = srow0 + 16 * mt + 8 * (mi & 1);        // key channel
-                ldmatrix_x4_trans(ak, &st.Kh[row * LDB + col]);
+                const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RP) + ks * 32, 16, 1024, tc::kSw128);
+                const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
+                tc::mma_bf16(tmem + D, ad, bd, id_p, ks > 0 ? 1u : 0u);
+            }
+            tc::commit(bar);
+        }
+        mbar_wait_bounded(bar, phase, status);
+        phase ^= 1;
+        tc::fence_after_sync();
+        // Khat^T X: row i (key channel) = TMEM lane i; warp w reads the lanes of quarter
+        // w % 4 and half w / 4 of the columns
+        {
+            const int i = (warp & 3) * 32 + lane;
+            if ((warp & 3) * 32 < D) {
+                const int cb = (warp >> 2) * (D / 2);
 #pragma unroll
-                for (int nt = 0; nt < NTL; ++nt)
-                    mma_bf16_16816(S[mt][nt], ak, bu[ks][nt]);
+                for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                    uint32_t x[32];
+                    tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cb + c0), x);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        const int col = cb + c0 + j;
+                        if (round == 0)
+                            *reinterpret_cast<uint4 *>(rec + R::Nm + tc::kmaj_sw128(i, col, D)) = pack8(&x[j]);
+                        else
+                            *reinterpret_cast<uint4 *>(rec + R::Shared + (col / kBV) * R::Blk +
+                                                       tc::mnmaj_sw64(i, col % kBV)) = pack8(&x[j]);
+                    }
+                }
             }
         }
-        // (5) bf16 copy of the new state for the next chunk
+        // P X: chunk row r = TMEM lane r (< 64)
+        if ((warp & 3) < 2) {
+            const int r = (warp & 3) * 32 + lane;
+            const int cb = (warp >> 2) * (D / 2);
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                uint32_t x[32];
+                tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, D + cb + c0), x);
+                tc::wait_ld();
 #pragma unroll
-            for (int nt = 0; nt < NTL; ++nt)
+                for (int j = 0; j < 32; j += 8) {
+                    const int col = cb + c0 + j;
+                    if (round == 0) {  // Q' = Qbar - P W
+                        const uint4 qb = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(r, col));
+                        const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
+                        uint32_t o4[4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = srow0 + 16 * mt + grp + 8 * hh;
-                    *reinterpret_cast<uint32_t *>(&sm.Sb[r * LDU + nt * 8 + 2 * tq]) =
-                        pack_bf16x2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
+                        for (int p = 0; p < 4; ++p) {
+                            const float2 f = unpack_bf16x2(qw[p]);
+                            o4[p] = pack_bf16x2(f.x - __uint_as_float(x[j + 2 * p]),
+                                                f.y - __uint_as_float(x[j + 2 * p + 1]));
+                        }
+                        *reinterpret_cast<uint4 *>(rec + R::Qp + tc::kmaj_sw128(r, col, kC)) =
+                            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    } else {  // O' = P Utilde
+                        *reinterpret_cast<uint4 *>(rec + R::Shared + (col / kBV) * R::Blk + R::BmBlk +
+                                                   tc::mnmaj_sw64(r, col % kBV)) = pack8(&x[j]);
+                    }
                 }
+            }
+        }
+        tc::fence_before_sync();
         __syncthreads();
+        tc::fence_after_sync();
     }
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, 2 * D);
+}
 
-    if (S_T) {
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < NTL; ++nt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = srow0 + 16 * mt + grp + 8 * hh;
-                    const int cc = col0 + nt * 8 + 2 * tq;
-                    *reinterpret_cast<float2 *>(&S_T[((size_t)bh * D + r) * D + cc]) =
-                        make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
-                }
+// ------------------------------------------------------------------ K3: scan
+constexpr int kScanWarps = 4;                        // consumer warps (one TMEM lane quarter each)
+constexpr int kScanThreads = (kScanWarps + 1) * 32;  // + one producer warp
+constexpr int kStages = 3;
+
+template <int D>
+struct ScanSmem {
+    static constexpr uint32_t kStageBytes = Rec<D>::Shared + Rec<D>::Blk;  // shared part + own value block
+    static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+    alignas(1024) unsigned char stage[kStages][kStageStride];
+    alignas(1024) unsigned char sbuf[D * kBV * 2];  // S block, bf16, MN-major 64-byte swizzle (row = key channel)
+    uint64_t full[kStages];                         // stage filled (arrive + bytes)
+    uint64_t empty[kStages];                        // stage released by the consumers
+    uint64_t mma_bar;                               // tcgen05 MMA batch completed
+    uint32_t tmem_slot;
+};
+
+__device__ __forceinline__ void consumer_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_local(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kScanThreads, 1)
+    scan_kernel(int T, int H, int NT, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
+                __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, unsigned int *status)
+{
+    extern __shared__ __align__(1024) unsigned char scan_smem[];
+    using SM = ScanSmem<D>;
+    using R = Rec<D>;
+    SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
+    constexpr uint32_t kTmemCols = 2 * kBV;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int blk = blockIdx.x, col0 = blk * kBV, bh = blockIdx.y;
+    const int b = bh / H, h = bh % H;
+    const unsigned char *recs = ws + (size_t)bh * NT * R::Bytes;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.mma_bar, 1);
+        fence_mbar_init_cluster();
     }
+    if (warp == 0)
+        tc::tmem_alloc(&sm.tmem_slot, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_slot;  // columns [0, kBV): N S; [kBV, 2 kBV): Q' S
+
+    if (warp == kScanWarps) {
+        // ---------------- producer: one lane issues the bulk copies
+        if (lane == 0) {
+            for (int c = 0; c < NT; ++c) {
+                const int s = c % kStages;
+                if (c >= kStages)
+                    mbar_wait_bounded(&sm.empty[s], ((c / kStages) - 1) & 1, status);
+                mbar_arrive_expect_tx(&sm.full[s], SM::kStageBytes);
+                const unsigned char *rec = recs + (size_t)c * R::Bytes;
+                bulk_g2s(sm.stage[s], rec, R::Shared, &sm.full[s]);
+                bulk_g2s(sm.stage[s] + R::Shared, rec + R::Shared + blk * R::Blk, R::Blk, &sm.full[s]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- consumers: thread `row` owns TMEM lane `row`
+        const int row = warp * 32 + lane;
+        const bool srow = row < D;  // owns state row `row` (key channel)
+        const uint32_t lane_addr = tc::taddr(tmem, (uint32_t)warp * 32, 0);
+        float S[kBV];
+        if (srow) {
+#pragma unroll
+            for (int j = 0; j < kBV; j += 4) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (S0)
+                    v = *reinterpret_cast<const float4 *>(&S0[((size_t)bh * D + row) * D + col0 + j]);
+                S[j] = v.x;
+                S[j + 1] = v.y;
+                S[j + 2] = v.z;
+                S[j + 3] = v.w;
+            }
+#pragma unroll
+            for (int j = 0; j < kBV; j += 8)
+                *reinterpret_cast<uint4 *>(sm.sbuf + tc::mnmaj_sw64(row, j)) =
+                    make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
+                               pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        consumer_sync();
+        tc::fence_after_sync();
+
+        const uint32_t id_k = tc::idesc_bf16(128, kBV, false, true);  // A K-major, B MN-major
+        const uint32_t sbuf_a = smem_u32(sm.sbuf);
+        uint32_t mma_phase = 0;
+        for (int c = 0; c < NT; ++c) {
+            const int s = c % kStages;
+            mbar_wait_bounded(&sm.full[s], (c / kStages) & 1, status);
+            const unsigned char *st = sm.stage[s];
+            const uint32_t st_a = smem_u32(st);
+
+            // [N S | Q' S] in one round (rows past N (D = 64) and past Q' are don't-cares)
+            if (tid == 0) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
+                    const uint64_t an =
+                        tc::smem_desc(st_a + R::Nm + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
+                    const uint64_t aq =
+                        tc::smem_desc(st_a + R::Qp + (ks >> 2) * (kC * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
+                    tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(&sm.mma_bar);
+            }
+            mbar_wait_bounded(&sm.mma_bar, mma_phase, status);
+            mma_phase ^= 1;
+            tc::fence_after_sync();
+
+            const unsigned char *blkp = st + R::Shared;
+            // S <- Diag(Gamma) S - N S + Bm; bf16 copy for the next chunk
+            if (srow) {
+                uint32_t d[kBV];
+                tc::ld_32x32b_x32(lane_addr, d);
+                tc::wait_ld();
+                const float g = reinterpret_cast<const float *>(st + R::Gam)[row];
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8) {
+                    const uint4 bu = *reinterpret_cast<const uint4 *>(blkp + tc::mnmaj_sw64(row, j));
+                    const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 bf = unpack_bf16x2(bw[p]);
+                        S[j + 2 * p] = fmaf(g, S[j + 2 * p], bf.x - __uint_as_float(d[j + 2 * p]));
+                        S[j + 2 * p + 1] = fmaf(g, S[j + 2 * p + 1], bf.y - __uint_as_float(d[j + 2 * p + 1]));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8)
+                    *reinterpret_cast<uint4 *>(sm.sbuf + tc::mnmaj_sw64(row, j)) =
+                        make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
+                                   pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+                tc::fence_smem_to_async();
+            }
+            // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
+            if (warp < 2) {
+                uint32_t y[kBV];
+                tc::ld_32x32b_x32(lane_addr + kBV, y);
+                tc::wait_ld();
+                const int t = c * kC + row;
+                if (t < T) {
+                    uint4 *orow = reinterpret_cast<uint4 *>(o + (((int64_t)b * T + t) * H + h) * D + col0);
+#pragma unroll
+                    for (int j = 0; j < kBV; j += 8) {
+                        const uint4 ou = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
+                        const uint32_t ow[4] = {ou.x, ou.y, ou.z, ou.w};
+                        uint32_t r4[4];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const float2 of = unpack_bf16x2(ow[p]);
+                            r4[p] = pack_bf16x2(of.x + __uint_as_float(y[j + 2 * p]),
+                                                of.y + __uint_as_float(y[j + 2 * p + 1]));
+                        }
+                        orow[j / 8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            consumer_sync();
+            tc::fence_after_sync();
+            if (tid == 0)
+                mbar_arrive_local(&sm.empty[s]);
+        }
+
+        if (S_T && srow)
+#pragma unroll
+            for (int j = 0; j < kBV; j += 4)
+                *reinterpret_cast<float4 *>(&S_T[((size_t)bh * D + row) * D + col0 + j]) =
+                    make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 template <int D>
@@ -598,30 +771,31 @@ cudaError_t launch_bf16_d(int B, int T, int H, const void *q, const void *k, con
                           const void *beta, float g_min, const float *S0, void *o, float *S_T, void *ws,
                           cudaStream_t s)
 {
-    constexpr int BV = 32;
     const int NT = (T + kC - 1) / kC;
     const int BH = B * H;
     unsigned char *w = static_cast<unsigned char *>(ws);
+    unsigned int *status = device_status_ptr();
+    if (!status)
+        return cudaErrorInvalidDevice;
     {
-        const size_t smem = sizeof(PrepSmem<D>);
+        const size_t smem = PrepLayout<D>::Bytes;
         cudaError_t e = cudaFuncSetAttribute(prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
         prep_kernel<D><<<dim3(NT, BH), kPrepThreads, smem, s>>>(
             T, H, NT, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
             static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-            static_cast<const __nv_bfloat16 *>(beta), g_min, w);
+            static_cast<const __nv_bfloat16 *>(beta), g_min, w, status);
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
     }
     {
-        const size_t smem = sizeof(ScanSmem<D, BV>);
-        cudaError_t e =
-            cudaFuncSetAttribute(scan_kernel<D, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
+        cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
-        scan_kernel<D, BV><<<dim3(D / BV, BH), kScanThreads, smem, s>>>(
-            T, H, NT, w, S0, static_cast<__nv_bfloat16 *>(o), S_T);
+        scan_kernel<D><<<dim3(D / kBV, BH), kScanThreads, smem, s>>>(T, H, NT, w, S0,
+                                                                    static_cast<__nv_bfloat16 *>(o), S_T, status);
         return cudaGetLastError();
     }
 }

@@ -27,6 +27,22 @@ int num_sms()
     return n;
 }
 
+unsigned int *device_status_ptr()
+{
+    static unsigned int *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
+        return nullptr;
+    if (dev < 64 && cache[dev])
+        return cache[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess)
+        return nullptr;
+    if (dev < 64)
+        cache[dev] = static_cast<unsigned int *>(p);
+    return static_cast<unsigned int *>(p);
+}
+
 namespace {
 
 constexpr int64_t kMaxElems = (int64_t)1 << 40;

@@ -11,6 +11,9 @@ namespace kda {
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Device address of the current device's kernel status word (see kda_device_status).
+unsigned int *device_status_ptr();
+
 // K1: g = g_min * sigmoid(a), fp64-exact, n elements.
 cudaError_t launch_gate(const void *a, kda_dtype dt, double g_min, float *g, int64_t n, cudaStream_t s);
 

@@ -55,11 +55,12 @@ def test_status_strings(L):
 
 def test_workspace_size(L):
     f = L.kda_chunk_fwd_workspace
-    rec128 = 4 * 64 * 128 * 2 + 64 * 64 * 2 + 128 * 4
+    # per chunk record: N (D x D) + Q' (64 x D) bf16, Gamma (D f32), Bm (D x D) + O' (64 x D) bf16
+    rec128 = 128 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 128 * 128 * 2 + 64 * 128 * 2
     assert f(1, 64, 1, 128, 128, kda.KDA_BF16) == rec128
     assert f(2, 65, 3, 128, 128, kda.KDA_BF16) == 2 * 3 * 2 * rec128
     assert f(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec128
-    rec64 = 4 * 64 * 64 * 2 + 64 * 64 * 2 + 64 * 4
+    rec64 = 64 * 64 * 2 + 64 * 64 * 2 + 64 * 4 + 64 * 64 * 2 + 64 * 64 * 2
     assert f(1, 100, 1, 64, 64, kda.KDA_BF16) == 2 * rec64
     assert f(1, 100, 1, 64, 64, kda.KDA_F32) == 0
     assert f(1, 0, 1, 128, 128, kda.KDA_BF16) == 0

@@ -86,11 +86,10 @@ struct PrepLayout {
     // G: fp32 [64][D] -> A [64][65] | T [64][65] | solve scratch -> T beta -> [W | Utilde]
     static constexpr uint32_t RG = RP + (uint32_t)kC * kC * 2;
     static constexpr uint32_t kGBytes = 2u * kC * D * 2 > (uint32_t)kC * D * 4 ? 2u * kC * D * 2 : (uint32_t)kC * D * 4;
-    static constexpr uint32_t kSolveBytes = 2u * kC * (kC + 1) * 4 + 3u * kTile * (kTile + 1) * 4;
+    static constexpr uint32_t kSolveBytes = 2u * kC * (kC + 1) * 4;
     static constexpr uint32_t kRGBytes = ((kGBytes > kSolveBytes ? kGBytes : kSolveBytes) + 1023) / 1024 * 1024;
-    static constexpr uint32_t RA = RG;                                // f32 [64][65]
-    static constexpr uint32_t RT = RG + (uint32_t)kC * (kC + 1) * 4;  // f32 [64][65]
-    static constexpr uint32_t RXS = RT + (uint32_t)kC * (kC + 1) * 4; // f32 [3][16][17]
+    static constexpr uint32_t RA = RG;                                // f32 [64][65]; its upper
+    static constexpr uint32_t RT = RG + (uint32_t)kC * (kC + 1) * 4;  // blocks hold the solve scratch
     // small tables
     static constexpr uint32_t RBeta = RG + kRGBytes;       // f32 [64]
     static constexpr uint32_t REm = RBeta + kC * 4;        // bf16 [4][D]  e^{G_{m_I}}
@@ -107,8 +106,9 @@ __device__ __forceinline__ uint32_t tok_off(int r, int c8) { return tc::mnmaj_sw
 
 // One 16x16 output block of the block substitution, by two warps (rows split in halves):
 //   X = sum_{K=J}^{I-1} A_IK T_KJ  (phase 0),   T_IJ = -T_II X  (phase 1)
-__device__ __forceinline__ void solve_block_phase(const float *A, float *Tm, float (*X)[kTile + 1], int I, int J,
-                                                  int half, int lane, int phase)
+// X is a 16x16 scratch with row stride kC + 1 (an unused upper block of A).
+__device__ __forceinline__ void solve_block_phase(const float *A, float *Tm, float *X, int I, int J, int half,
+                                                  int lane, int phase)
 {
     constexpr int LDA = kC + 1;
     const int cc = lane % kTile;
@@ -125,12 +125,12 @@ __device__ __forceinline__ void solve_block_phase(const float *A, float *Tm, flo
             }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            X[rbase + i][cc] = s[i];
+            X[(rbase + i) * LDA + cc] = s[i];
     } else {
         float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int x = 0; x < kTile; ++x) {
-            const float xv = X[x][cc];
+            const float xv = X[x * LDA + cc];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 s[i] = fmaf(Tm[(I * kTile + rbase + i) * LDA + I * kTile + x], xv, s[i]);
@@ -183,7 +183,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     float *sG = reinterpret_cast<float *>(sm + L::RG);   // [64][D]
     float *sA = reinterpret_cast<float *>(sm + L::RA);   // [64][65]
     float *sT = reinterpret_cast<float *>(sm + L::RT);   // [64][65]
-    float(*sX)[kTile][kTile + 1] = reinterpret_cast<float(*)[kTile][kTile + 1]>(sm + L::RXS);
     float *sBeta = reinterpret_cast<float *>(sm + L::RBeta);
     __nv_bfloat16 *sEm = reinterpret_cast<__nv_bfloat16 *>(sm + L::REm);
     __nv_bfloat16 *sEl = reinterpret_cast<__nv_bfloat16 *>(sm + L::REl);
@@ -248,21 +247,25 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         constexpr int TPC = kPrepThreads / D;
         constexpr int LEN = kC / TPC;
         const int c = tid % D, part = tid / D;
-        float acc = 0.0f;
-#pragma unroll 8
-        for (int r = part * LEN; r < part * LEN + LEN; ++r) {
-            acc += sG[r * D + c];
-            sG[r * D + c] = acc;
-        }
+        float gv[LEN];
+#pragma unroll
+        for (int r = 0; r < LEN; ++r)
+            gv[r] = sG[(part * LEN + r) * D + c];
+#pragma unroll
+        for (int r = 1; r < LEN; ++r)
+            gv[r] += gv[r - 1];
+#pragma unroll
+        for (int r = 0; r < LEN; ++r)
+            sG[(part * LEN + r) * D + c] = gv[r];
         __syncthreads();
         float off = 0.0f;
         for (int p = 0; p < part; ++p)
             off += sG[(p * LEN + LEN - 1) * D + c];
         __syncthreads();
         if (part > 0)
-#pragma unroll 8
-            for (int r = part * LEN; r < part * LEN + LEN; ++r)
-                sG[r * D + c] += off;
+#pragma unroll
+            for (int r = 0; r < LEN; ++r)
+                sG[(part * LEN + r) * D + c] = gv[r] + off;
     }
     __syncthreads();
 
@@ -431,11 +434,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     for (int lvl = 1; lvl < kTiles; ++lvl) {
         const int nblk = kTiles - lvl;
         const int blk = warp >> 1, half = warp & 1;
+        float *scratch = sA + (blk + 1) * kTile;  // upper block (0, blk + 1) of A is never read
         if (blk < nblk)
-            solve_block_phase(sA, sT, sX[blk], blk + lvl, blk, half, lane, 0);
+            solve_block_phase(sA, sT, scratch, blk + lvl, blk, half, lane, 0);
         __syncthreads();
         if (blk < nblk)
-            solve_block_phase(sA, sT, sX[blk], blk + lvl, blk, half, lane, 1);
+            solve_block_phase(sA, sT, scratch, blk + lvl, blk, half, lane, 1);
         __syncthreads();
     }
     // T diag(beta) as the K-major A operand (over A's place; the 8 KB after it are the

@@ -23,10 +23,11 @@ __device__ __forceinline__ float gate_bounded_exact(float a, double g_min)
     return __double2float_rn(g_min / (1.0 + exp(-(double)a)));
 }
 
-// Same gate in float32 (fast path inside the chunk kernels; |err| <= a few ulp).
+// Same gate in float32 with the hardware exponential and divide (the chunk kernels'
+// fast path; a few ulp from the fp64 value, saturating to g_min / -0 like it).
 __device__ __forceinline__ float gate_bounded_fast(float a, float g_min)
 {
-    return g_min * __frcp_rn(1.0f + __expf(-a));
+    return __fdividef(g_min, 1.0f + __expf(-a));
 }
 
 // ------------------------------------------------------------------ bf16 helpers

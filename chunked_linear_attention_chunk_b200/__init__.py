@@ -44,6 +44,8 @@ EXPORTS = (
     "kda_device_status",
     "kda_status_string",
     "kda_version",
+    "kda_chunk_fwd_noalloc",
+    "kda_chunk_fwd_noalloc_max_scratch",
 )
 
 
@@ -81,6 +83,10 @@ def lib() -> ctypes.CDLL:
     L.kda_status_string.restype = ctypes.c_char_p
     L.kda_version.argtypes = []
     L.kda_version.restype = I
+    L.kda_chunk_fwd_noalloc.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P]
+    L.kda_chunk_fwd_noalloc.restype = I
+    L.kda_chunk_fwd_noalloc_max_scratch.argtypes = []
+    L.kda_chunk_fwd_noalloc_max_scratch.restype = S
     _lib = L
     return L
 
@@ -156,6 +162,23 @@ def kda_chunk_fwd(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=No
                              float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
                              _stream(q.device))
     _raise(st, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_chunk_fwd_noalloc(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=None,
+                          return_state: bool = True):
+    """Like ``kda_chunk_fwd`` but with the library's built-in scratch instead of a
+    workspace (for callers that cannot allocate device memory; see include/kda.h)."""
+    _check_cuda(q, k, v, a, beta, S0, o, S_T)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = lib().kda_chunk_fwd_noalloc(B, T, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                     _ptr(beta), float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _stream(q.device))
+    _raise(st, "kda_chunk_fwd_noalloc")
     return o, S_T
 
 

@@ -143,6 +143,34 @@ kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const 
                            float g_min, float *S, void *o, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for the library's users.
+ * Code that runs during CUDA graph capture (allocation is not allowed there), serving
+ * loops that must never call cudaMalloc (it can synchronise the device), and hosts whose
+ * device memory is owned by another allocator cannot provide the workspace that
+ * kda_chunk_fwd takes.  This entry point takes the same arguments minus the workspace and
+ * uses a fixed scratch array built into the library instead: kda_chunk_fwd_noalloc_max_
+ * scratch() bytes (64 MiB) of device memory on every GPU that loads the library, held
+ * until the process exits.  It allocates nothing and computes exactly what kda_chunk_fwd
+ * computes: inputs longer than the scratch holds are processed in stretches of whole
+ * 64-token chunks with the float32 state carried between them.
+ *   - The first call on a device looks up the scratch array's device address (once per
+ *     device, with that device current); make that first call before any stream capture.
+ *   - All calls share the one array, and it keeps whatever the last call left there;
+ *     nothing in it needs to start at zero.  Calls whose GPU work overlaps (other
+ *     streams, other host threads) race on the array: serialise them.
+ *   - Errors: as kda_chunk_fwd, plus WORKSPACE when even one 64-token chunk of all heads
+ *     (with the state carry slot) does not fit the scratch (roughly H > 600 at
+ *     dk = dv = 128), and CUDA if the scratch address cannot be looked up.
+ */
+kda_status kda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q,
+                                 const void *k, const void *v, const void *a, const void *beta,
+                                 float g_min, const float *S0, void *o, float *S_T, kda_stream_t stream);
+
+/* Size in bytes of the built-in scratch array kda_chunk_fwd_noalloc uses. */
+size_t kda_chunk_fwd_noalloc_max_scratch(void);
+
+/*
  * kda_device_status -- synchronise `stream`, then return and clear the current
  * device's kernel status word: KDA_OK, or KDA_ERR_DEVICE_TIMEOUT if a kernel gave up
  * on a bounded wait since the last call; KDA_ERR_CUDA if the synchronisation failed.

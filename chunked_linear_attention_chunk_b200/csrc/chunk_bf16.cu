@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         }
         const __nv_bfloat16 *dsc = I > J ? &sDd[(I * (I - 1) / 2 + J) * D] : nullptr;
         float accA[2][4] = {}, accP[2][4] = {};
-#pragma unroll 2
+#pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             uint32_t ak[4], aq[4], bf[4];
             const int mi = lane >> 3;
@@ -388,25 +388,25 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     __syncthreads();
 
-    // -- 4b. chunk-referenced operands in place: Kbar = Kr e^{G_m}, Qbar = Qr e^{G_m},
-    //        Khat = Ec e^{G_last - G_m}
-    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
-        const int r = i / CPR, c8 = (i % CPR) * 8;
-        const int tile = r / kTile;
-        const uint32_t d = tok_off(r, c8);
-        const uint4 em = *reinterpret_cast<const uint4 *>(&sEm[tile * D + c8]);
-        const uint4 el = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
-        uint4 *pk = reinterpret_cast<uint4 *>(sm + L::RK + d);
-        uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + d);
-        uint4 *px = reinterpret_cast<uint4 *>(sm + L::RX + d);
-        *pk = mul8(*pk, em);
-        *pq = mul8(*pq, em);
-        *px = mul8(*px, el);
-    }
-
-    // -- 5. T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution (one lane per
-    //       column), then block substitution level by level, two warps per block.
-    if (warp < kTiles && lane < kTile) {
+    // -- 4b/5. warps 4..7: chunk-referenced operands in place (Kbar = Kr e^{G_m},
+    //         Qbar = Qr e^{G_m}, Khat = Ec e^{G_last - G_m}); at the same time warps 0..3
+    //         start T = (I + A)^{-1} with the 16x16 diagonal blocks (forward substitution,
+    //         one lane per column).  Then block substitution level by level.
+    if (warp >= kPrepThreads / 64) {
+        for (int i = tid - kPrepThreads / 2; i < kC * CPR; i += kPrepThreads / 2) {
+            const int r = i / CPR, c8 = (i % CPR) * 8;
+            const int tile = r / kTile;
+            const uint32_t d = tok_off(r, c8);
+            const uint4 em = *reinterpret_cast<const uint4 *>(&sEm[tile * D + c8]);
+            const uint4 el = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
+            uint4 *pk = reinterpret_cast<uint4 *>(sm + L::RK + d);
+            uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + d);
+            uint4 *px = reinterpret_cast<uint4 *>(sm + L::RX + d);
+            *pk = mul8(*pk, em);
+            *pq = mul8(*pq, em);
+            *px = mul8(*px, el);
+        }
+    } else if (lane < kTile) {
         const int I = warp, c = lane;
         float x[kTile];
 #pragma unroll
@@ -489,7 +489,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     tc::fence_after_sync();
 
     // -- 7. rounds 2 and 3: Khat^T X (TMEM cols 0..D) and P X (cols D..2D) for X = W, then
-    //       X = Utilde.  Epilogues: N, Q' = Qbar - P W; then Bm, O' = P Utilde.
+    //       X = Utilde.  The results are staged in shared memory in record order (round 2:
+    //       N over [Kbar | V], Q' = Qbar - P W in place of Qbar; round 3: Bm and O' over
+    //       [Qbar | Kbar | V]) and written with bulk copies.
+    static_assert(R::Qp - R::Nm <= 2 * L::kMat && R::Bytes - R::Shared <= 3 * L::kMat, "staging fits");
 #pragma unroll 1
     for (int round = 0; round < 2; ++round) {
         if (tid == 0) {
@@ -513,26 +516,31 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         mbar_wait_bounded(bar, phase, status);
         phase ^= 1;
         tc::fence_after_sync();
+        if (round == 1) {  // the round-2 stores must have read their staging before reuse
+            if (tid == 0)
+                bulk_wait_read_all();
+            __syncthreads();
+        }
+        unsigned char *stage2 = sm + L::RK;  // round 2: N (D x D) over [Kbar | V]
+        unsigned char *stage3 = sm + L::RQ;  // round 3: per value block Bm | O' over [Qbar | Kbar | V]
         // Khat^T X: row i (key channel) = TMEM lane i; warp w reads the lanes of quarter
         // w % 4 and half w / 4 of the columns
-        {
+        if ((warp & 3) * 32 < D) {
             const int i = (warp & 3) * 32 + lane;
-            if ((warp & 3) * 32 < D) {
-                const int cb = (warp >> 2) * (D / 2);
+            const int cb = (warp >> 2) * (D / 2);
 #pragma unroll
-                for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                    uint32_t x[32];
-                    tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cb + c0), x);
-                    tc::wait_ld();
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                uint32_t x[32];
+                tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cb + c0), x);
+                tc::wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const int col = cb + c0 + j;
-                        if (round == 0)
-                            *reinterpret_cast<uint4 *>(rec + R::Nm + tc::kmaj_sw128(i, col, D)) = pack8(&x[j]);
-                        else
-                            *reinterpret_cast<uint4 *>(rec + R::Shared + (col / kBV) * R::Blk +
-                                                       tc::mnmaj_sw64(i, col % kBV)) = pack8(&x[j]);
-                    }
+                for (int j = 0; j < 32; j += 8) {
+                    const int col = cb + c0 + j;
+                    if (round == 0)
+                        *reinterpret_cast<uint4 *>(stage2 + tc::kmaj_sw128(i, col, D)) = pack8(&x[j]);
+                    else
+                        *reinterpret_cast<uint4 *>(stage3 + (col / kBV) * R::Blk + tc::mnmaj_sw64(i, col % kBV)) =
+                            pack8(&x[j]);
                 }
             }
         }
@@ -548,8 +556,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
                     const int col = cb + c0 + j;
-                    if (round == 0) {  // Q' = Qbar - P W
-                        const uint4 qb = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(r, col));
+                    if (round == 0) {  // Q' = Qbar - P W, in place (same layout as the record)
+                        uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + tok_off(r, col));
+                        const uint4 qb = *pq;
                         const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
                         uint32_t o4[4];
 #pragma unroll
@@ -558,19 +567,31 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                             o4[p] = pack_bf16x2(f.x - __uint_as_float(x[j + 2 * p]),
                                                 f.y - __uint_as_float(x[j + 2 * p + 1]));
                         }
-                        *reinterpret_cast<uint4 *>(rec + R::Qp + tc::kmaj_sw128(r, col, kC)) =
-                            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                        *pq = make_uint4(o4[0], o4[1], o4[2], o4[3]);
                     } else {  // O' = P Utilde
-                        *reinterpret_cast<uint4 *>(rec + R::Shared + (col / kBV) * R::Blk + R::BmBlk +
+                        *reinterpret_cast<uint4 *>(stage3 + (col / kBV) * R::Blk + R::BmBlk +
                                                    tc::mnmaj_sw64(r, col % kBV)) = pack8(&x[j]);
                     }
                 }
             }
         }
+        tc::fence_smem_to_async();
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
+        if (tid == 0) {
+            if (round == 0) {
+                bulk_s2g(rec + R::Nm, stage2, D * D * 2);
+                bulk_s2g(rec + R::Qp, sm + L::RQ, kC * D * 2);
+            } else {
+                bulk_s2g(rec + R::Shared, stage3, R::Bytes - R::Shared);
+            }
+            bulk_commit();
+        }
     }
+    if (tid == 0)
+        bulk_wait_read_all();  // staging must stay valid until the stores have read it
+    __syncthreads();
     if (warp == 0)
         tc::tmem_dealloc(tmem, 2 * D);
 }

@@ -3,10 +3,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {libkda,reference}]
 
-One step = one kda_chunk_fwd over the 64K-stage batch (B=1, H=32, T=65536,
+One step = one chunked forward over the 64K-stage batch (B=1, H=32, T=65536,
 dk=dv=128, bf16 inputs, fp32 state, the 5% a=+8 slice): gate, cumulative decay,
 dense 16-token tile products, WY/UT solve and the state scan, i.e. the whole hot path.
+It is issued as kda_chunk_fwd_prep + kda_chunk_fwd_scan (the two launches kda_chunk_fwd
+makes) so that CUDA events between them time each kernel during the timed steps.
 Inputs (2.69 GB) exceed the 126 MB L2, so no flush is needed between steps.
+The log-sigmoid ablation (element-wise diagonal tiles) is timed on the same inputs and
+reported under ``ablation``.
 
 Prints ONE JSON line (rank 0).  ``value`` is whole-job tokens/s with inputs resident in
 HBM; ``e2e`` is the same metric through the C ABI with pinned host buffers (H2D of every
@@ -42,6 +46,9 @@ G_MIN = -5.0
 # Algorithmic cost of the path per token-head at d = 128 (bf16 token tensors):
 # q, k, v, a (256 B each), beta (2 B), o (256 B); states add 2 * dk*dv*4 B per head.
 BYTES_PER_TOKEN_HEAD = 4 * 256 + 2 + 256
+# The prep kernel's share of them (it reads the inputs; the scan writes o and the states).
+# The workspace records between the two kernels are the implementation's own traffic.
+PREP_BYTES_PER_TOKEN_HEAD = 4 * 256 + 2
 # Triangle-aware flops per token-head at the 16-token tile (state products W S, Qbar S,
 # Khat^T U: 6 dk dv; tile products and W: dk (3C - 1); Utilde and P U: 2 C dv; solve
 # C^2/3; Gamma scaling dk dv / C), C = 16.
@@ -58,23 +65,27 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+KERNEL_SOURCES = ("chunk_bf16.cu", "kda_common.cuh", "tcgen05.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the chunk kernels' sources: a traffic figure is valid only for these."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_linear_attention_chunk_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic_per_token_head():
-    """DRAM bytes per token-head of one kda_chunk_fwd from the committed ncu summary, or
-    None when the kernels changed since it was captured."""
+def measured_traffic_per_token_head(kernel: str):
+    """DRAM bytes (read + write) per token-head of one launch of ``kernel`` ("prep" or
+    "scan") from the committed ncu summary, or None when the kernels changed since."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     d = json.load(open(PROFILE_TRAFFIC))
-    if d.get("source_hash") != kernel_source_hash():
+    if d.get("source_hash") != kernel_source_hash() or kernel not in d:
         return None
-    return float(d["dram_bytes_per_token_head"])
+    return float(d[kernel]["dram_bytes_per_token_head"])
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -163,9 +174,11 @@ def barrier(world: int):
 
 
 # ---------------------------------------------------------------------------- arms
-def time_steps(fn, steps: int, warmup: int, world: int, device):
+def time_steps(fn, steps: int, warmup: int, world: int, device, timed_flag=None):
     for _ in range(warmup):
         fn()
+    if timed_flag is not None:
+        timed_flag["on"] = True
     torch.cuda.synchronize(device)
     barrier(world)
     torch.cuda.synchronize(device)
@@ -258,24 +271,57 @@ def run_libkda(args):
     need = kda.kda_chunk_fwd_workspace(B, T, H, D, D)
     ws = torch.empty(need, dtype=torch.uint8, device=device)
 
-    def step():
-        kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, o=o, S_T=S_T, workspace=ws)
+    # One step is kda_chunk_fwd issued as its two stages (the same two launches the single
+    # call makes), with CUDA events around each on the launching stream during the timed
+    # steps, so each kernel's own duration is measured live.
+    stream = torch.cuda.current_stream(device)
+    timed = {"on": False, "ev": []}
 
+    def step():
+        ev = None
+        if timed["on"]:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(stream)
+        kda.kda_chunk_fwd_prep(*(d[n] for n in names), ws, G_MIN)
+        if ev:
+            ev[1].record(stream)
+        kda.kda_chunk_fwd_scan(ws, B, T, H, D, D, S0=S0, o=o, S_T=S_T)
+        if ev:
+            ev[2].record(stream)
+            timed["ev"].append(ev)
+
+    prep_ms = scan_ms = float("nan")
     if args.only == "decode":
         ms = float("nan")
         clocks = {}
     else:
         with ClockSampler(local) as clk:
-            ms = time_steps(step, args.steps, args.warmup, world, device)
+            ms = time_steps(step, args.steps, args.warmup, world, device, timed)
         assert kda.kda_device_status(device) == 0
         clocks = clk.summary()
+        prep_ms = max_over_ranks(statistics.fmean(e[0].elapsed_time(e[1]) for e in timed["ev"]), world, device)
+        scan_ms = max_over_ranks(statistics.fmean(e[1].elapsed_time(e[2]) for e in timed["ev"]), world, device)
     tokens = B * T
     value = world * tokens / (ms * 1e-3)
     token_heads = B * T * H
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
     achieved_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    prep_bytes = token_heads * PREP_BYTES_PER_TOKEN_HEAD
+    prep_gbs = prep_bytes / (prep_ms * 1e-3) / 1e9
     tflops = token_heads * FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
-    traffic_pth = measured_traffic_per_token_head()
+    prep_traffic = measured_traffic_per_token_head("prep")
+    scan_traffic = measured_traffic_per_token_head("scan")
+
+    # ---- the ablation: unbounded log-sigmoid gate, element-wise diagonal tiles (same inputs)
+    abl = None
+    if args.only != "decode" and not args.no_ablation:
+        def abl_step():
+            kda.kda_chunk_fwd_logsigmoid(*(d[n] for n in names), S0=S0, o=o, S_T=S_T, workspace=ws)
+
+        abl_ms = time_steps(abl_step, max(2, min(args.steps, 5)), 3, world, device)
+        assert kda.kda_device_status(device) == 0
+        abl = {"gate": "g = log sigmoid(a), diagonal 16x16 tiles element by element", "ms_per_step": abl_ms,
+               "value": world * tokens / (abl_ms * 1e-3), "unit": UNIT, "slowdown_vs_bounded": abl_ms / ms}
 
     # ---- end to end through the C ABI with pinned host buffers
     hx = {n: x[n].pin_memory() for n in names}
@@ -335,11 +381,16 @@ def run_libkda(args):
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm_peak, "peak_kind": peak_kind,
-                     "kernel": "kda_chunk_fwd (prep + scan launches of one call)",
-                     "traffic": None if traffic_pth is None else traffic_pth * token_heads,
-                     "algorithmic_bytes": alg_bytes},
+        "roofline": {"bound": "hbm", "achieved": prep_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": prep_gbs / hbm_peak, "peak_kind": peak_kind,
+                     "kernel": "prep_kernel (dominant; one launch per step)",
+                     "algorithmic_bytes_per_launch": prep_bytes, "ms_per_launch": prep_ms,
+                     "traffic": None if prep_traffic is None else prep_traffic * token_heads,
+                     "path": {"kernels": "prep + scan (one kda_chunk_fwd)", "achieved": achieved_gbs,
+                              "frac": achieved_gbs / hbm_peak, "algorithmic_bytes": alg_bytes}},
+        "kernels": {"prep_kernel": {"ms_per_launch": prep_ms, "share": prep_ms / (prep_ms + scan_ms)},
+                    "scan_kernel": {"ms_per_launch": scan_ms, "share": scan_ms / (prep_ms + scan_ms),
+                                    "traffic": None if scan_traffic is None else scan_traffic * token_heads}},
         "chunk_fwd": {"tflops": tflops, "pct_bf16_peak": tflops / bf16_peak, "bf16_peak_tflops": bf16_peak,
                       "flops_per_token_head": FLOPS_PER_TOKEN_HEAD},
         "decode": {"metric": "decode HBM GB/s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": dec_ms,
@@ -348,6 +399,8 @@ def run_libkda(args):
                                 "frac": dec_gbs / world / hbm_peak, "peak_kind": peak_kind},
                    "clocks": dclk.summary() if dclk is not None else {}},
     }
+    if abl is not None:
+        line["ablation"] = abl
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
     if rank == 0:
@@ -370,6 +423,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="64k",
                     help="64k (the benchmark workload) or 8k (a smaller case for profiler captures)")
     ap.add_argument("--only", choices=("all", "chunk", "decode"), default="all")
+    ap.add_argument("--no-ablation", action="store_true", help="skip timing the log-sigmoid ablation path")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

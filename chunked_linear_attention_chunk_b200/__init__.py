@@ -24,6 +24,8 @@ KDA_F32 = 1
 KDA_CHUNK = 64
 KDA_TILE = 16
 KDA_G_MIN_LOWEST = -5.4
+KDA_GATE_BOUNDED = 0
+KDA_GATE_LOGSIGMOID = 1
 
 STATUS = {
     0: "KDA_OK",
@@ -46,6 +48,9 @@ EXPORTS = (
     "kda_version",
     "kda_chunk_fwd_noalloc",
     "kda_chunk_fwd_noalloc_max_scratch",
+    "kda_chunk_fwd_logsigmoid",
+    "kda_chunk_fwd_prep",
+    "kda_chunk_fwd_scan",
 )
 
 
@@ -87,6 +92,12 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_fwd_noalloc.restype = I
     L.kda_chunk_fwd_noalloc_max_scratch.argtypes = []
     L.kda_chunk_fwd_noalloc_max_scratch.restype = S
+    L.kda_chunk_fwd_logsigmoid.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_fwd_logsigmoid.restype = I
+    L.kda_chunk_fwd_prep.argtypes = [I, I, I, I, I, I, F, P, P, P, P, P, P, S, P]
+    L.kda_chunk_fwd_prep.restype = I
+    L.kda_chunk_fwd_scan.argtypes = [I, I, I, I, I, P, S, P, P, P, P]
+    L.kda_chunk_fwd_scan.restype = I
     _lib = L
     return L
 
@@ -162,6 +173,65 @@ def kda_chunk_fwd(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=No
                              float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
                              _stream(q.device))
     _raise(st, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_chunk_fwd_logsigmoid(q, k, v, a, beta, S0=None, o=None, S_T=None, workspace=None,
+                             return_state: bool = True):
+    """The ablation path: ``kda_chunk_fwd`` with the unbounded gate g = log(sigmoid(a)) and
+    element-wise diagonal tiles (bf16 only).  Same shapes and return value."""
+    _check_cuda(q, k, v, a, beta, S0, o, S_T, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    for t in (k, v, a, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, a, beta must share one dtype")
+    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(lib().kda_chunk_fwd_workspace(B, T, H, dk, dv, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_logsigmoid(B, T, H, dk, dv, code, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
+                                        _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+                                        _stream(q.device))
+    _raise(st, "kda_chunk_fwd_logsigmoid")
+    return o, S_T
+
+
+def kda_chunk_fwd_prep(q, k, v, a, beta, workspace, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED):
+    """First stage of the bf16 chunked forward: one record per (batch*head, chunk) into
+    ``workspace`` (uint8, at least ``kda_chunk_fwd_workspace`` bytes)."""
+    _check_cuda(q, k, v, a, beta, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16 or any(t.dtype != torch.bfloat16 for t in (k, v, a, beta)):
+        raise TypeError("kda_chunk_fwd_prep takes bfloat16 tensors")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_prep(B, T, H, dk, dv, int(gate), float(g_min), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                  _ptr(beta), _ptr(workspace), ws_bytes, _stream(q.device))
+    _raise(st, "kda_chunk_fwd_prep")
+
+
+def kda_chunk_fwd_scan(workspace, B: int, T: int, H: int, dk: int, dv: int, S0=None, o=None, S_T=None,
+                       return_state: bool = True):
+    """Second stage: the chunk recursion over the records of ``kda_chunk_fwd_prep``.
+    Returns (o, S_T) like ``kda_chunk_fwd``."""
+    _check_cuda(workspace, S0, o, S_T)
+    dev = workspace.device
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_scan(B, T, H, dk, dv, _ptr(workspace), ws_bytes, _ptr(S0), _ptr(o), _ptr(S_T),
+                                  _stream(dev))
+    _raise(st, "kda_chunk_fwd_scan")
     return o, S_T
 
 

@@ -104,40 +104,51 @@ struct PrepLayout {
 // 16-byte chunk address of (token r, channels c8..c8+7) in a token-major operand.
 __device__ __forceinline__ uint32_t tok_off(int r, int c8) { return tc::mnmaj_sw128(r, c8, kC); }
 
-// One 16x16 output block of the block substitution, by two warps (rows split in halves):
-//   X = sum_{K=J}^{I-1} A_IK T_KJ  (phase 0),   T_IJ = -T_II X  (phase 1)
-// X is a 16x16 scratch with row stride kC + 1 (an unused upper block of A).
-__device__ __forceinline__ void solve_block_phase(const float *A, float *Tm, float *X, int I, int J, int half,
-                                                  int lane, int phase)
+// One 16x16 output block of the block substitution, by one warp with tf32 tensor-core
+// MMAs:  X = sum_{K=J}^{I-1} A_IK T_KJ,  T_IJ = -T_II X.  A and T are fp32 [64][kC + 1];
+// X goes through a 16x16 scratch (row stride kC + 1, an unused upper block of A) to turn
+// the accumulator layout into an operand layout.
+__device__ __forceinline__ void solve_block_tf32(const float *A, float *Tm, float *X, int I, int J, int lane)
 {
-    constexpr int LDA = kC + 1;
-    const int cc = lane % kTile;
-    const int rbase = half * 8 + (lane / kTile) * 4;
-    if (phase == 0) {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int K = J; K < I; ++K)
+    constexpr int LD = kC + 1;
+    const int g = lane >> 2, t = lane & 3;
+    float acc[2][4] = {};
+    auto product = [&](const float *Am, int arow, int acol, const float *Bm, int brow, int bcol, int bld) {
 #pragma unroll
-            for (int x = 0; x < kTile; ++x) {
-                const float t = Tm[(K * kTile + x) * LDA + J * kTile + cc];
+        for (int kk = 0; kk < kTile; kk += 8) {
+            uint32_t af[4];
+            af[0] = to_tf32(Am[(arow + g) * LD + acol + kk + t]);
+            af[1] = to_tf32(Am[(arow + g + 8) * LD + acol + kk + t]);
+            af[2] = to_tf32(Am[(arow + g) * LD + acol + kk + t + 4]);
+            af[3] = to_tf32(Am[(arow + g + 8) * LD + acol + kk + t + 4]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    s[i] = fmaf(A[(I * kTile + rbase + i) * LDA + K * kTile + x], t, s[i]);
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bf[2];
+                bf[0] = to_tf32(Bm[(brow + kk + t) * bld + bcol + nt * 8 + g]);
+                bf[1] = to_tf32(Bm[(brow + kk + t + 4) * bld + bcol + nt * 8 + g]);
+                mma_tf32_1688(acc[nt], af, bf);
             }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            X[(rbase + i) * LDA + cc] = s[i];
-    } else {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int x = 0; x < kTile; ++x) {
-            const float xv = X[x * LDA + cc];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                s[i] = fmaf(Tm[(I * kTile + rbase + i) * LDA + I * kTile + x], xv, s[i]);
         }
+    };
+    for (int K = J; K < I; ++K)
+        product(A, I * kTile, K * kTile, Tm, K * kTile, J * kTile, LD);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            Tm[(I * kTile + rbase + i) * LDA + J * kTile + cc] = -s[i];
+    for (int nt = 0; nt < 2; ++nt) {
+        X[g * LD + nt * 8 + 2 * t] = acc[nt][0];
+        X[g * LD + nt * 8 + 2 * t + 1] = acc[nt][1];
+        X[(g + 8) * LD + nt * 8 + 2 * t] = acc[nt][2];
+        X[(g + 8) * LD + nt * 8 + 2 * t + 1] = acc[nt][3];
+        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+    }
+    __syncwarp();
+    product(Tm, I * kTile, I * kTile, X, 0, 0, LD);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        float *o = Tm + (I * kTile + g) * LD + J * kTile + nt * 8 + 2 * t;
+        o[0] = -acc[nt][0];
+        o[1] = -acc[nt][1];
+        o[8 * LD] = -acc[nt][2];
+        o[8 * LD + 1] = -acc[nt][3];
     }
 }
 
@@ -160,7 +171,23 @@ __device__ __forceinline__ uint4 pack8(const uint32_t *x)
                       pack_bf16x2(__uint_as_float(x[6]), __uint_as_float(x[7])));
 }
 
-template <int D>
+// Diagonal 16x16 tiles of the ablation path (unbounded gate), computed element by
+// element: 4 tiles x 136 lower (r, j) pairs, one exponential per (r, j, channel).  Thread
+// `tid` owns pairs p = (tid % 64) + 64 s, s < 3, of tile tid / 64; pair p <-> (r, j) with
+// r (r + 1) / 2 <= p < (r + 1) (r + 2) / 2, j = p - r (r + 1) / 2 <= r.
+constexpr int kDiagPairs = kTile * (kTile + 1) / 2;
+constexpr int kDiagSlots = 3;
+static_assert(kTiles * 64 == 256 && 64 * kDiagSlots >= kDiagPairs, "diagonal pair mapping");
+
+__device__ __forceinline__ void diag_pair(int p, int &r, int &j)
+{
+    r = 0;
+    while ((r + 1) * (r + 2) / 2 <= p)
+        ++r;
+    j = p - r * (r + 1) / 2;
+}
+
+template <int D, bool kLogSig>
 __global__ void __launch_bounds__(kPrepThreads, 2)
     prep_kernel(int T, int H, int NT, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
@@ -235,8 +262,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const float2 f = unpack_bf16x2(w[p]);
-            gv[2 * p] = r < n ? gate_bounded_fast(f.x, g_min) : 0.0f;
-            gv[2 * p + 1] = r < n ? gate_bounded_fast(f.y, g_min) : 0.0f;
+            if constexpr (kLogSig) {
+                gv[2 * p] = r < n ? gate_logsigmoid_fast(f.x) : 0.0f;
+                gv[2 * p + 1] = r < n ? gate_logsigmoid_fast(f.y) : 0.0f;
+            } else {
+                gv[2 * p] = r < n ? gate_bounded_fast(f.x, g_min) : 0.0f;
+                gv[2 * p + 1] = r < n ? gate_bounded_fast(f.y, g_min) : 0.0f;
+            }
         }
         float4 *dst = reinterpret_cast<float4 *>(&sG[r * D + c8]);
         dst[0] = make_float4(gv[0], gv[1], gv[2], gv[3]);
@@ -270,17 +302,32 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     __syncthreads();
 
     // -- 2. per-(tile, channel) decay scalars (bf16) and Gamma_C (record)
+    //       Bounded gate: one reference per tile, its middle token m_I (row and column
+    //       role alike).  Unbounded gate: the row role of tile I takes G just before the
+    //       tile (b_I; 0 for I = 0), the column role of tile J the tile's last token
+    //       (e_J), so every off-diagonal factor is at most 1 whatever g is.
+    auto row_ref = [&](int I, int c) -> float {
+        if constexpr (kLogSig)
+            return I > 0 ? sG[(I * kTile - 1) * D + c] : 0.0f;
+        else
+            return sG[(I * kTile + kRef) * D + c];
+    };
+    auto col_ref = [&](int J, int c) -> float {
+        if constexpr (kLogSig)
+            return sG[(J * kTile + kTile - 1) * D + c];
+        else
+            return sG[(J * kTile + kRef) * D + c];
+    };
     for (int i = tid; i < kTiles * D; i += kPrepThreads) {
         const int I = i / D, c = i % D;
-        const float Gm = sG[(I * kTile + kRef) * D + c];
-        sEm[i] = __float2bfloat16(__expf(Gm));
-        sEl[i] = __float2bfloat16(__expf(sG[(kC - 1) * D + c] - Gm));
+        sEm[i] = __float2bfloat16(__expf(row_ref(I, c)));
+        sEl[i] = __float2bfloat16(__expf(sG[(kC - 1) * D + c] - col_ref(I, c)));
     }
     for (int i = tid; i < 6 * D; i += kPrepThreads) {
         const int p = i / D, c = i % D;
         const int I = p < 1 ? 1 : (p < 3 ? 2 : 3);
         const int J = p - I * (I - 1) / 2;
-        sDd[i] = __float2bfloat16(__expf(sG[(I * kTile + kRef) * D + c] - sG[(J * kTile + kRef) * D + c]));
+        sDd[i] = __float2bfloat16(__expf(row_ref(I, c) - col_ref(J, c)));
     }
     {
         float *gGam = reinterpret_cast<float *>(rec + R::Gam);
@@ -288,11 +335,50 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             gGam[c] = __expf(sG[(kC - 1) * D + c]);
     }
 
-    // -- 3. decay factors with the tile's middle token as reference: E = e^{G - G_m}
-    //       Kr = k E and Qr = q E in place of k and q, Ec = k / E in place of a
+    // -- 3a. unbounded gate only: the diagonal tiles element by element from the raw q, k
+    //        and G (their decay cannot be factored), held in registers until step 4
+    float dA[kDiagSlots] = {}, dP[kDiagSlots] = {};
+    if constexpr (kLogSig) {
+        const int I = tid >> 6;
+#pragma unroll
+        for (int s = 0; s < kDiagSlots; ++s) {
+            const int p = (tid & 63) + 64 * s;
+            if (p < kDiagPairs) {
+                int r, j;
+                diag_pair(p, r, j);
+                const int tr = I * kTile + r, tj = I * kTile + j;
+                float sa = 0.0f, sp = 0.0f;
+                for (int c8 = 0; c8 < D; c8 += 8) {
+                    const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tr, c8));
+                    const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(tr, c8));
+                    const uint4 ju = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tj, c8));
+                    const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w},
+                                   jw[4] = {ju.x, ju.y, ju.z, ju.w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float2 kr = unpack_bf16x2(kw[w]), qr = unpack_bf16x2(qw[w]), kj = unpack_bf16x2(jw[w]);
+                        const float2 gr = *reinterpret_cast<const float2 *>(&sG[tr * D + c8 + 2 * w]);
+                        const float2 gj = *reinterpret_cast<const float2 *>(&sG[tj * D + c8 + 2 * w]);
+                        const float e0 = __expf(gr.x - gj.x), e1 = __expf(gr.y - gj.y);
+                        sa = fmaf(kr.x * kj.x, e0, sa);
+                        sa = fmaf(kr.y * kj.y, e1, sa);
+                        sp = fmaf(qr.x * kj.x, e0, sp);
+                        sp = fmaf(qr.y * kj.y, e1, sp);
+                    }
+                }
+                dA[s] = j < r ? sBeta[tr] * sa : 0.0f;
+                dP[s] = sp;
+            }
+        }
+        __syncthreads();  // raw q, k are overwritten next
+    }
+
+    // -- 3. decay factors E = e^{G - G_ref} (row role) and e^{G_ref' - G} (column role):
+    //       Kr = k E and Qr = q E in place of k and q, Ec in place of a
     for (int i = tid; i < kC * CPR; i += kPrepThreads) {
         const int r = i / CPR, c8 = (i % CPR) * 8;
-        const int m = (r / kTile) * kTile + kRef;
+        const int m = kLogSig ? (r / kTile) * kTile - 1 : (r / kTile) * kTile + kRef;  // row reference token
+        const int mc = kLogSig ? (r / kTile) * kTile + kTile - 1 : m;                   // column reference token
         const uint32_t d = tok_off(r, c8);
         const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + d);
         const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + d);
@@ -300,16 +386,31 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         const uint32_t qw[4] = {qu.x, qu.y, qu.z, qu.w};
         const float4 G0 = *reinterpret_cast<const float4 *>(&sG[r * D + c8]);
         const float4 G1 = *reinterpret_cast<const float4 *>(&sG[r * D + c8 + 4]);
-        const float4 M0 = *reinterpret_cast<const float4 *>(&sG[m * D + c8]);
-        const float4 M1 = *reinterpret_cast<const float4 *>(&sG[m * D + c8 + 4]);
+        const float4 zero4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        const float4 M0 = m >= 0 ? *reinterpret_cast<const float4 *>(&sG[m * D + c8]) : zero4;
+        const float4 M1 = m >= 0 ? *reinterpret_cast<const float4 *>(&sG[m * D + c8 + 4]) : zero4;
         const float x[8] = {G0.x - M0.x, G0.y - M0.y, G0.z - M0.z, G0.w - M0.w,
                             G1.x - M1.x, G1.y - M1.y, G1.z - M1.z, G1.w - M1.w};
+        float y[8];  // column exponent G_{mc} - G
+        if constexpr (kLogSig) {
+            const float4 C0 = *reinterpret_cast<const float4 *>(&sG[mc * D + c8]);
+            const float4 C1 = *reinterpret_cast<const float4 *>(&sG[mc * D + c8 + 4]);
+            const float yy[8] = {C0.x - G0.x, C0.y - G0.y, C0.z - G0.z, C0.w - G0.w,
+                                 C1.x - G1.x, C1.y - G1.y, C1.z - G1.z, C1.w - G1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                y[e] = yy[e];
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                y[e] = -x[e];
+        }
         uint32_t kr[4], qr[4], ec[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const float2 kk = unpack_bf16x2(kw[p]), qq = unpack_bf16x2(qw[p]);
             const float e0 = __expf(x[2 * p]), e1 = __expf(x[2 * p + 1]);
-            const float i0 = __expf(-x[2 * p]), i1 = __expf(-x[2 * p + 1]);
+            const float i0 = __expf(y[2 * p]), i1 = __expf(y[2 * p + 1]);
             kr[p] = pack_bf16x2(kk.x * e0, kk.y * e1);
             qr[p] = pack_bf16x2(qq.x * e0, qq.y * e1);
             ec[p] = pack_bf16x2(kk.x * i0, kk.y * i1);
@@ -330,10 +431,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     //       J <= I): row operands Kr, Qr of tile I (scaled by e^{G_{m_I} - G_{m_J}} when
     //       I > J), column operand Ec of tile J.  A (fp32, beta-scaled, strictly lower)
     //       goes over G, which is no longer needed; P (bf16, lower) to its operand slot.
-    for (int pidx = warp; pidx < kTiles * (kTiles + 1) / 2; pidx += kPrepThreads / 32) {
-        int I = 0, J = pidx;
-        while (J > I) {  // pidx -> (I, J): 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) ...
-            J -= I + 1;
+    //       Unbounded gate: off-diagonal tiles only (the diagonal ones come from step 3a).
+    constexpr int kTilePairs = kLogSig ? kTiles * (kTiles - 1) / 2 : kTiles * (kTiles + 1) / 2;
+    for (int pidx = warp; pidx < kTilePairs; pidx += kPrepThreads / 32) {
+        int I = kLogSig ? 1 : 0, J = pidx;
+        while (kLogSig ? J >= I : J > I) {  // pidx -> (I, J): 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) ...
+            J -= kLogSig ? I : I + 1;       //   or, off-diagonal only: 0:(1,0) 1:(2,0) 2:(2,1) ...
             ++I;
         }
         const __nv_bfloat16 *dsc = I > J ? &sDd[(I * (I - 1) / 2 + J) * D] : nullptr;
@@ -386,6 +489,26 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                     pack_bf16x2(lp0 ? accP[nt][2 * hh] : 0.0f, lp1 ? accP[nt][2 * hh + 1] : 0.0f);
             }
     }
+    if constexpr (kLogSig) {  // the element-wise diagonal tiles (G, now overwritten, is no longer read)
+        const int I = tid >> 6;
+#pragma unroll
+        for (int s = 0; s < kDiagSlots; ++s) {
+            const int p = (tid & 63) + 64 * s;
+            if (p < kDiagPairs) {
+                int r, j;
+                diag_pair(p, r, j);
+                const int tr = I * kTile + r, tj = I * kTile + j;
+                sA[tr * LDA + tj] = dA[s];
+                *reinterpret_cast<__nv_bfloat16 *>(sm + L::RP + tc::kmaj_sw128(tr, tj, kC)) = __float2bfloat16(dP[s]);
+            }
+        }
+        for (int i = tid; i < kTiles * kTile * kTile; i += kPrepThreads) {  // P above the diagonal
+            const int I = i / (kTile * kTile), r = (i / kTile) % kTile, j = i % kTile;
+            if (j > r)
+                *reinterpret_cast<__nv_bfloat16 *>(sm + L::RP + tc::kmaj_sw128(I * kTile + r, I * kTile + j, kC)) =
+                    __float2bfloat16(0.0f);
+        }
+    }
     __syncthreads();
 
     // -- 4b/5. warps 4..7: chunk-referenced operands in place (Kbar = Kr e^{G_m},
@@ -425,29 +548,20 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         for (int r = 0; r < kTile; ++r)
             sT[(I * kTile + r) * LDA + I * kTile + c] = x[r];
     }
-    for (int i = tid; i < kC * kC; i += kPrepThreads) {
-        const int r = i / kC, j = i % kC;
-        if (j / kTile > r / kTile)
-            sT[r * LDA + j] = 0.0f;
-    }
     __syncthreads();
-    for (int lvl = 1; lvl < kTiles; ++lvl) {
-        const int nblk = kTiles - lvl;
-        const int blk = warp >> 1, half = warp & 1;
-        float *scratch = sA + (blk + 1) * kTile;  // upper block (0, blk + 1) of A is never read
-        if (blk < nblk)
-            solve_block_phase(sA, sT, scratch, blk + lvl, blk, half, lane, 0);
-        __syncthreads();
-        if (blk < nblk)
-            solve_block_phase(sA, sT, scratch, blk + lvl, blk, half, lane, 1);
+    for (int lvl = 1; lvl < kTiles; ++lvl) {  // level lvl: blocks (J + lvl, J), one warp each
+        if (warp < kTiles - lvl)
+            solve_block_tf32(sA, sT, sA + (warp + 1) * kTile /* upper block (0, warp+1) of A */, warp + lvl,
+                             warp, lane);
         __syncthreads();
     }
     // T diag(beta) as the K-major A operand (over A's place; the 8 KB after it are the
     // don't-care rows of the M = 128 MMA)
     for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
         const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+        const bool upper = j / kTile > r / kTile;  // those blocks of T are zero and never written
         *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) =
-            pack_bf16x2(sT[r * LDA + j] * sBeta[j], sT[r * LDA + j + 1] * sBeta[j + 1]);
+            upper ? 0u : pack_bf16x2(sT[r * LDA + j] * sBeta[j], sT[r * LDA + j + 1] * sBeta[j + 1]);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -719,28 +833,35 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 }
                 tc::commit(&sm.mma_bar);
             }
+            // Diag(Gamma) S + Bm while the tensor core runs (stage data is in since `full`)
+            if (srow) {
+                const float g = reinterpret_cast<const float *>(st + R::Gam)[row];
+                const unsigned char *bmp = st + R::Shared;
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8) {
+                    const uint4 bu = *reinterpret_cast<const uint4 *>(bmp + tc::mnmaj_sw64(row, j));
+                    const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 bf = unpack_bf16x2(bw[q]);
+                        S[j + 2 * q] = fmaf(g, S[j + 2 * q], bf.x);
+                        S[j + 2 * q + 1] = fmaf(g, S[j + 2 * q + 1], bf.y);
+                    }
+                }
+            }
             mbar_wait_bounded(&sm.mma_bar, mma_phase, status);
             mma_phase ^= 1;
             tc::fence_after_sync();
 
             const unsigned char *blkp = st + R::Shared;
-            // S <- Diag(Gamma) S - N S + Bm; bf16 copy for the next chunk
+            // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk
             if (srow) {
                 uint32_t d[kBV];
                 tc::ld_32x32b_x32(lane_addr, d);
                 tc::wait_ld();
-                const float g = reinterpret_cast<const float *>(st + R::Gam)[row];
 #pragma unroll
-                for (int j = 0; j < kBV; j += 8) {
-                    const uint4 bu = *reinterpret_cast<const uint4 *>(blkp + tc::mnmaj_sw64(row, j));
-                    const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float2 bf = unpack_bf16x2(bw[p]);
-                        S[j + 2 * p] = fmaf(g, S[j + 2 * p], bf.x - __uint_as_float(d[j + 2 * p]));
-                        S[j + 2 * p + 1] = fmaf(g, S[j + 2 * p + 1], bf.y - __uint_as_float(d[j + 2 * p + 1]));
-                    }
-                }
+                for (int j = 0; j < kBV; ++j)
+                    S[j] -= __uint_as_float(d[j]);
 #pragma unroll
                 for (int j = 0; j < kBV; j += 8)
                     *reinterpret_cast<uint4 *>(sm.sbuf + tc::mnmaj_sw64(row, j)) =
@@ -791,38 +912,39 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D>
-cudaError_t launch_bf16_d(int B, int T, int H, const void *q, const void *k, const void *v, const void *a,
-                          const void *beta, float g_min, const float *S0, void *o, float *S_T, void *ws,
-                          cudaStream_t s)
+template <int D, bool kLogSig>
+cudaError_t launch_prep_d(int B, int T, int H, const void *q, const void *k, const void *v, const void *a,
+                          const void *beta, float g_min, void *ws, cudaStream_t s)
 {
     const int NT = (T + kC - 1) / kC;
-    const int BH = B * H;
-    unsigned char *w = static_cast<unsigned char *>(ws);
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
-    {
-        const size_t smem = PrepLayout<D>::Bytes;
-        cudaError_t e = cudaFuncSetAttribute(prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        prep_kernel<D><<<dim3(NT, BH), kPrepThreads, smem, s>>>(
-            T, H, NT, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-            static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-            static_cast<const __nv_bfloat16 *>(beta), g_min, w, status);
-        if ((e = cudaGetLastError()) != cudaSuccess)
-            return e;
-    }
-    {
-        const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
-        cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        scan_kernel<D><<<dim3(D / kBV, BH), kScanThreads, smem, s>>>(T, H, NT, w, S0,
-                                                                    static_cast<__nv_bfloat16 *>(o), S_T, status);
-        return cudaGetLastError();
-    }
+    const size_t smem = PrepLayout<D>::Bytes;
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<D, kLogSig>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    prep_kernel<D, kLogSig><<<dim3(NT, B * H), kPrepThreads, smem, s>>>(
+        T, H, NT, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
+        static_cast<const __nv_bfloat16 *>(beta), g_min, static_cast<unsigned char *>(ws), status);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_scan_d(int B, int T, int H, const void *ws, const float *S0, void *o, float *S_T, cudaStream_t s)
+{
+    const int NT = (T + kC - 1) / kC;
+    unsigned int *status = device_status_ptr();
+    if (!status)
+        return cudaErrorInvalidDevice;
+    const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    scan_kernel<D><<<dim3(D / kBV, B * H), kScanThreads, smem, s>>>(
+        T, H, NT, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, status);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -834,13 +956,22 @@ size_t chunk_bf16_workspace(int B, int T, int H, int D)
     return (size_t)B * H * NT * rec;
 }
 
-cudaError_t launch_chunk_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                              const void *a, const void *beta, float g_min, const float *S0, void *o,
-                              float *S_T, void *workspace, cudaStream_t s)
+cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                             const void *a, const void *beta, float g_min, bool logsigmoid, void *workspace,
+                             cudaStream_t s)
 {
-    if (D == 64)
-        return launch_bf16_d<64>(B, T, H, q, k, v, a, beta, g_min, S0, o, S_T, workspace, s);
-    return launch_bf16_d<128>(B, T, H, q, k, v, a, beta, g_min, S0, o, S_T, workspace, s);
+    if (logsigmoid)
+        return D == 64 ? launch_prep_d<64, true>(B, T, H, q, k, v, a, beta, g_min, workspace, s)
+                       : launch_prep_d<128, true>(B, T, H, q, k, v, a, beta, g_min, workspace, s);
+    return D == 64 ? launch_prep_d<64, false>(B, T, H, q, k, v, a, beta, g_min, workspace, s)
+                   : launch_prep_d<128, false>(B, T, H, q, k, v, a, beta, g_min, workspace, s);
+}
+
+cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
+                             float *S_T, cudaStream_t s)
+{
+    return D == 64 ? launch_scan_d<64>(B, T, H, workspace, S0, o, S_T, s)
+                   : launch_scan_d<128>(B, T, H, workspace, S0, o, S_T, s);
 }
 
 }  // namespace kda

@@ -143,65 +143,205 @@ size_t kda_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dt
     return chunk_bf16_workspace(B, T, H, dk);
 }
 
-kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
-                         const void *v, const void *a, const void *beta, float g_min, const float *S0, void *o,
-                         float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// Sizes of one chunk-forward call, checked once.
+struct ChunkShape {
+    int B = 0, T = 0, H = 0, D = 0;
+    kda_dtype dtype = KDA_BF16;
+    int64_t ntok = 0, nk = 0, nv = 0, ns = 0;
+    size_t ws = 0;  // workspace bytes kda_chunk_fwd_workspace reports
+    int es = 2;     // element size of the token tensors
+};
+
+kda_status check_shape(int B, int T, int H, int dk, int dv, kda_dtype dtype, ChunkShape &sh)
 {
     if (!dtype_ok(dtype) || B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
         return KDA_ERR_INVALID_ARG;
-    kda_status st = check_gmin(g_min);
-    if (st != KDA_OK)
-        return st;
     if (dk != dv || (dk != 64 && dk != 128))
         return KDA_ERR_UNSUPPORTED;
-    const int64_t ntok = safe_prod({B, T, H});
-    const int64_t nk = safe_prod({B, T, H, dk});
-    const int64_t nv = safe_prod({B, T, H, dv});
-    const int64_t ns = safe_prod({B, H, dk, dv});
-    if (ntok < 0 || nk < 0 || nv < 0 || ns < 0)
+    sh.ntok = safe_prod({B, T, H});
+    sh.nk = safe_prod({B, T, H, dk});
+    sh.nv = safe_prod({B, T, H, dv});
+    sh.ns = safe_prod({B, H, dk, dv});
+    if (sh.ntok < 0 || sh.nk < 0 || sh.nv < 0 || sh.ns < 0)
         return KDA_ERR_INVALID_ARG;
     if (dtype == KDA_BF16 && (int64_t)B * H > 65535)
         return KDA_ERR_UNSUPPORTED;
-    if (T > 0 && (!q || !k || !v || !a || !beta || !o))
-        return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, a, beta, S0, o, S_T, workspace};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p))
-            return KDA_ERR_ALIGNMENT;
-    const size_t need = kda_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
-    if (need > 0 && (!workspace || ws_bytes < need))
-        return KDA_ERR_WORKSPACE;
+    sh.B = B, sh.T = T, sh.H = H, sh.D = dk, sh.dtype = dtype;
+    sh.ws = kda_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
+    sh.es = elem_size(dtype);
+    return KDA_OK;
+}
 
-    const int es = elem_size(dtype);
-    const Range rq(q, nk * es), rk(k, nk * es), rv(v, nv * es), ra(a, nk * es), rb(beta, ntok * es);
-    const Range rS0(S0, ns * 4), ro(T > 0 ? o : nullptr, nv * es), rST(S_T, ns * 4);
-    const Range rws(need > 0 ? workspace : nullptr, (int64_t)need);
-    for (const Range &in : {rq, rk, rv, ra, rb, rS0, rST, rws})
-        if (overlaps(ro, in))
+kda_status check_gate(kda_gate gate, float g_min, kda_dtype dtype)
+{
+    if (gate == KDA_GATE_BOUNDED)
+        return check_gmin(g_min);
+    if (gate == KDA_GATE_LOGSIGMOID)
+        return dtype == KDA_BF16 ? KDA_OK : KDA_ERR_UNSUPPORTED;
+    return KDA_ERR_INVALID_ARG;
+}
+
+bool all_aligned(std::initializer_list<const void *> ps)
+{
+    for (const void *p : ps)
+        if (p && !aligned16(p))
+            return false;
+    return true;
+}
+
+kda_status check_workspace(const ChunkShape &sh, const void *workspace, size_t ws_bytes)
+{
+    if (sh.ws > 0 && (!workspace || ws_bytes < sh.ws))
+        return KDA_ERR_WORKSPACE;
+    return KDA_OK;
+}
+
+// The inputs of the prep: q, k, v, a, beta present (T > 0), aligned, and not overlapped by
+// the workspace it writes.
+kda_status check_prep_args(const ChunkShape &sh, const void *q, const void *k, const void *v, const void *a,
+                           const void *beta, const void *workspace, size_t ws_bytes)
+{
+    if (sh.T > 0 && (!q || !k || !v || !a || !beta))
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, a, beta, workspace}))
+        return KDA_ERR_ALIGNMENT;
+    kda_status st = check_workspace(sh, workspace, ws_bytes);
+    if (st != KDA_OK)
+        return st;
+    const Range rws(sh.ws > 0 ? workspace : nullptr, (int64_t)sh.ws);
+    const int es = sh.es;
+    for (const Range &in : {Range(q, sh.nk * es), Range(k, sh.nk * es), Range(v, sh.nv * es), Range(a, sh.nk * es),
+                            Range(beta, sh.ntok * es)})
+        if (overlaps(rws, in))
             return KDA_ERR_ALIAS;
-    for (const Range &in : {rq, rk, rv, ra, rb, rws})
-        if (overlaps(rST, in))
+    return KDA_OK;
+}
+
+// The outputs of the scan: o present (T > 0) and overlapping nothing else; S_T either S0
+// itself or disjoint from it, and disjoint from the workspace; S0 disjoint from the
+// workspace.
+kda_status check_scan_args(const ChunkShape &sh, const void *workspace, size_t ws_bytes, const float *S0, void *o,
+                           float *S_T)
+{
+    if (sh.T > 0 && !o)
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({workspace, S0, o, S_T}))
+        return KDA_ERR_ALIGNMENT;
+    kda_status st = check_workspace(sh, workspace, ws_bytes);
+    if (st != KDA_OK)
+        return st;
+    const Range rws(sh.ws > 0 ? workspace : nullptr, (int64_t)sh.ws);
+    const Range rS0(S0, sh.ns * 4), ro(sh.T > 0 ? o : nullptr, sh.nv * sh.es), rST(S_T, sh.ns * 4);
+    for (const Range &r : {rS0, rST, rws})
+        if (overlaps(ro, r))
             return KDA_ERR_ALIAS;
+    if (overlaps(rST, rws) || overlaps(rS0, rws))
+        return KDA_ERR_ALIAS;
     if (overlaps(rST, rS0) && S_T != S0)
         return KDA_ERR_ALIAS;
-    for (const Range &in : {rq, rk, rv, ra, rb, rS0})
-        if (overlaps(rws, in))
+    return KDA_OK;
+}
+
+// T == 0: the final state is the initial one.
+kda_status copy_state(const ChunkShape &sh, const float *S0, float *S_T, cudaStream_t s)
+{
+    if (!S_T || S_T == S0)
+        return KDA_OK;
+    if (S0)
+        return from_cuda(cudaMemcpyAsync(S_T, S0, (size_t)sh.ns * 4, cudaMemcpyDeviceToDevice, s));
+    return from_cuda(cudaMemsetAsync(S_T, 0, (size_t)sh.ns * 4, s));
+}
+
+// Validation and dispatch shared by kda_chunk_fwd and kda_chunk_fwd_logsigmoid.
+kda_status chunk_fwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                          const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                          const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                          kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
+    if (st == KDA_OK)
+        st = check_gate(gate, g_min, dtype);
+    if (st == KDA_OK)
+        st = check_prep_args(sh, q, k, v, a, beta, workspace, ws_bytes);
+    if (st == KDA_OK)
+        st = check_scan_args(sh, workspace, ws_bytes, S0, o, S_T);
+    if (st != KDA_OK)
+        return st;
+    // the outputs must not overlap the inputs either
+    const int es = sh.es;
+    const Range ro(T > 0 ? o : nullptr, sh.nv * es), rST(S_T, sh.ns * 4);
+    for (const Range &in : {Range(q, sh.nk * es), Range(k, sh.nk * es), Range(v, sh.nv * es), Range(a, sh.nk * es),
+                            Range(beta, sh.ntok * es)})
+        if (overlaps(ro, in) || overlaps(rST, in))
             return KDA_ERR_ALIAS;
 
     cudaStream_t s = (cudaStream_t)stream;
-    if (T == 0) {
-        if (!S_T || S_T == S0)
-            return KDA_OK;
-        if (S0)
-            return from_cuda(cudaMemcpyAsync(S_T, S0, (size_t)ns * 4, cudaMemcpyDeviceToDevice, s));
-        return from_cuda(cudaMemsetAsync(S_T, 0, (size_t)ns * 4, s));
-    }
+    if (T == 0)
+        return copy_state(sh, S0, S_T, s);
     if (dtype == KDA_F32)
         return from_cuda(launch_chunk_f32(B, T, H, dk, static_cast<const float *>(q), static_cast<const float *>(k),
                                           static_cast<const float *>(v), static_cast<const float *>(a),
                                           static_cast<const float *>(beta), g_min, S0, static_cast<float *>(o), S_T,
                                           s));
-    return from_cuda(launch_chunk_bf16(B, T, H, dk, q, k, v, a, beta, g_min, S0, o, S_T, workspace, s));
+    st = from_cuda(launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, workspace, s));
+    if (st != KDA_OK)
+        return st;
+    return from_cuda(launch_scan_bf16(B, T, H, dk, workspace, S0, o, S_T, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *S0, void *o,
+                         float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    return chunk_fwd_impl(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, KDA_GATE_BOUNDED, S0, o, S_T, workspace,
+                          ws_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q,
+                                    const void *k, const void *v, const void *a, const void *beta, const float *S0,
+                                    void *o, float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    return chunk_fwd_impl(B, T, H, dk, dv, dtype, q, k, v, a, beta, 0.0f, KDA_GATE_LOGSIGMOID, S0, o, S_T,
+                          workspace, ws_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const void *q,
+                              const void *k, const void *v, const void *a, const void *beta, void *workspace,
+                              size_t ws_bytes, kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, KDA_BF16, sh);
+    if (st == KDA_OK)
+        st = check_gate(gate, g_min, KDA_BF16);
+    if (st == KDA_OK)
+        st = check_prep_args(sh, q, k, v, a, beta, workspace, ws_bytes);
+    if (st != KDA_OK || T == 0)
+        return st;
+    return from_cuda(launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, workspace,
+                                      (cudaStream_t)stream));
+}
+
+kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
+                              const float *S0, void *o, float *S_T, kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, KDA_BF16, sh);
+    if (st == KDA_OK)
+        st = check_scan_args(sh, workspace, ws_bytes, S0, o, S_T);
+    if (st != KDA_OK)
+        return st;
+    if (T == 0)
+        return copy_state(sh, S0, S_T, (cudaStream_t)stream);
+    return from_cuda(launch_scan_bf16(B, T, H, dk, workspace, S0, o, S_T, (cudaStream_t)stream));
 }
 
 kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k, const void *v,

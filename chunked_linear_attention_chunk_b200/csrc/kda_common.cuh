@@ -30,6 +30,14 @@ __device__ __forceinline__ float gate_bounded_fast(float a, float g_min)
     return __fdividef(g_min, 1.0f + __expf(-a));
 }
 
+// Unbounded gate g = log sigmoid(a) = min(a, 0) - log(1 + e^{-|a|}) in float32: the form
+// without the lower bound ("Breaking Through ..." section 2.1), used by the ablation path.
+// Neither term overflows for finite a; large negative a gives g ~ a.
+__device__ __forceinline__ float gate_logsigmoid_fast(float a)
+{
+    return fminf(a, 0.0f) - log1pf(__expf(-fabsf(a)));
+}
+
 // ------------------------------------------------------------------ bf16 helpers
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -57,6 +65,23 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D = A(16x8, row) * B(8x8, col) + C with tf32 inputs (10-bit mantissa), fp32 accumulate.
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

@@ -22,11 +22,15 @@ cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const f
                              const float *a, const float *beta, float g_min, const float *S0, float *o,
                              float *S_T, cudaStream_t s);
 
-// K2 + K3: bfloat16 tensor-core chunked forward.
+// K2 + K3: bfloat16 tensor-core chunked forward.  The prep writes one record per (b*h,
+// chunk) into the workspace; the scan walks them.  `logsigmoid` selects the unbounded gate
+// g = log sigmoid(a) with element-wise diagonal tiles (g_min is then not used).
 size_t chunk_bf16_workspace(int B, int T, int H, int D);
-cudaError_t launch_chunk_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                              const void *a, const void *beta, float g_min, const float *S0, void *o,
-                              float *S_T, void *workspace, cudaStream_t s);
+cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                             const void *a, const void *beta, float g_min, bool logsigmoid, void *workspace,
+                             cudaStream_t s);
+cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
+                             float *S_T, cudaStream_t s);
 
 // K4: single-token decode step.
 cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,

@@ -63,6 +63,12 @@ typedef enum {
     KDA_ERR_WORKSPACE = 7       /* workspace pointer missing or smaller than required */
 } kda_status;
 
+/* The decay gate of the chunked forward. */
+typedef enum {
+    KDA_GATE_BOUNDED = 0,   /* g = g_min * sigmoid(a), g_min in [KDA_G_MIN_LOWEST, 0)          */
+    KDA_GATE_LOGSIGMOID = 1 /* g = log(sigmoid(a)), unbounded: the ablation path (see below)  */
+} kda_gate;
+
 /* Supported range of g_min: finite, KDA_G_MIN_LOWEST <= g_min < 0.  The pages fix
  * g_min = -5 so that 1/Gamma inside any 16-token tile stays in range; with the tile's
  * middle token as reference the largest exponent is 8*|g_min| <= 43.2, far inside
@@ -125,6 +131,59 @@ kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
                          const void *k, const void *v, const void *a, const void *beta,
                          float g_min, const float *S0, void *o, float *S_T, void *workspace,
                          size_t ws_bytes, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_logsigmoid -- the ablation of the bounded gate: the same chunked forward
+ * with the unbounded gate g = log(sigmoid(a)) and no g_min.
+ * Passages: the unbounded log-sigmoid gate ("Breaking Through ..." section 2.1), and the
+ * path the bound replaced ("Trillion-Scale ..." sections 3.1 and 3.3; "Breaking Through
+ * ..." section 2.1).  Without a lower bound on g, the inverse decay inside a 16-token
+ * tile cannot be factored into tensor-core operands, so the pairs (r, j) of the diagonal
+ * tiles are computed element by element on CUDA cores, one exponential per pair and key
+ * channel (the slow position-pair path).  The off-diagonal tiles stay dense products,
+ * with references chosen so that every factor is at most 1.  Everything after the tiles
+ * (solve, record, scan) is the kda_chunk_fwd path unchanged.
+ *   Arguments, layouts, workspace (kda_chunk_fwd_workspace), aliasing rules and errors
+ *   are those of kda_chunk_fwd without g_min; only dtype KDA_BF16 is implemented
+ *   (KDA_F32 returns UNSUPPORTED).  Every finite a is accepted; the result is
+ *   unspecified for infinite or NaN a.
+ */
+kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q,
+                                    const void *k, const void *v, const void *a, const void *beta,
+                                    const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                                    kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_prep, kda_chunk_fwd_scan -- the two stages of the bfloat16 kda_chunk_fwd
+ * as separate calls, for callers that schedule them apart (timing each stage, or running
+ * the fully parallel prep of one batch while other work waits for the serial scan).
+ * kda_chunk_fwd(bf16) is exactly kda_chunk_fwd_prep followed by kda_chunk_fwd_scan on the
+ * same stream with the same workspace.
+ *
+ * kda_chunk_fwd_prep: everything inside each 64-token chunk (gate, cumulative decay,
+ * tile products, the delta-rule solve and the chunk's contributions), written as one
+ * record per (batch*head, chunk) into `workspace`.  All chunks are independent.
+ *   gate, g_min  KDA_GATE_BOUNDED with g_min as in kda_chunk_fwd, or KDA_GATE_LOGSIGMOID
+ *                (g_min unused) as in kda_chunk_fwd_logsigmoid.
+ *   q, k, v, a, beta, workspace, ws_bytes: as in kda_chunk_fwd, bfloat16 only.
+ *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS (workspace overlaps an input),
+ *   WORKSPACE, CUDA.  T == 0 does nothing.
+ *
+ * kda_chunk_fwd_scan: the chunk recursion over the records, serial over chunks per
+ * (batch, head, 32-column block of the state): writes o and, if S_T is not NULL, the
+ * final state.
+ *   workspace    the records of a kda_chunk_fwd_prep call with the same B, T, H, dk, dv,
+ *                ordered before this call (same stream, or an event).  Other contents give
+ *                unspecified o and S_T but no access outside the buffers.
+ *   S0, o, S_T   as in kda_chunk_fwd (S_T may be S0; o overlaps nothing else).
+ *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.  T == 0 copies S0
+ *   (or zeros) to S_T.
+ */
+kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const void *q,
+                              const void *k, const void *v, const void *a, const void *beta, void *workspace,
+                              size_t ws_bytes, kda_stream_t stream);
+kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
+                              const float *S0, void *o, float *S_T, kda_stream_t stream);
 
 /*
  * kda_decode_step -- one token for N independent sequences, state updated in place.

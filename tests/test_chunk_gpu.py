@@ -176,3 +176,21 @@ def test_stage_1m_segmented():
         es = err_s(S_gpu.cpu().numpy(), S_ref)
         assert es <= TOL_BF16_S, (seg, es)
     assert kda.kda_device_status() == 0
+
+
+@pytest.mark.parametrize("gate", [kda.KDA_GATE_BOUNDED, kda.KDA_GATE_LOGSIGMOID])
+def test_prep_then_scan_equals_one_call_bitwise(gate):
+    """kda_chunk_fwd (and its log-sigmoid variant) is exactly prep followed by scan."""
+    x = synth.make_inputs(2, 200, 3, 128, 128, "bf16", seed=900 + gate, s0_std=0.1)
+    d = to_dev(x)
+    B, T, H, D = 2, 200, 3, 128
+    if gate == kda.KDA_GATE_BOUNDED:
+        o1, S1 = kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=d["S0"])
+    else:
+        o1, S1 = kda.kda_chunk_fwd_logsigmoid(*(d[n] for n in NAMES), S0=d["S0"])
+    ws = torch.empty(kda.kda_chunk_fwd_workspace(B, T, H, D, D), dtype=torch.uint8, device="cuda")
+    kda.kda_chunk_fwd_prep(*(d[n] for n in NAMES), ws, G_MIN, gate)
+    o2, S2 = kda.kda_chunk_fwd_scan(ws, B, T, H, D, D, S0=d["S0"])
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)

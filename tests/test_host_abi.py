@@ -161,3 +161,62 @@ def test_python_binding_has_no_cpu_fallback():
     x = torch.zeros(16, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         kda.kda_gate_fwd(x)
+
+
+def _chunk_logsig(L, B=1, T=64, H=1, dk=128, dv=128, dt=kda.KDA_BF16, q=None, o=None, S0=None, ST=None, ws=None,
+                  ws_bytes=None):
+    es = 2 if dt == kda.KDA_BF16 else 4
+    n = B * T * H * max(dk, 1) * es
+    q = BASE if q is None else q
+    o = BASE + 5 * (n + 4096) if o is None else o
+    ws = BASE + 6 * (n + 4096) if ws is None else ws
+    need = L.kda_chunk_fwd_workspace(B, T, H, dk, dv, dt)
+    ws_bytes = need if ws_bytes is None else ws_bytes
+    P = ctypes.c_void_p
+    return L.kda_chunk_fwd_logsigmoid(B, T, H, dk, dv, dt, P(q), P(BASE + (n + 4096)), P(BASE + 2 * (n + 4096)),
+                                      P(BASE + 3 * (n + 4096)), P(BASE + 4 * (n + 4096)), P(S0), P(o), P(ST),
+                                      P(ws), ws_bytes, None)
+
+
+def test_logsigmoid_entry_validates_like_chunk_fwd(L):
+    """The ablation entry shares kda_chunk_fwd's checks, takes no g_min, and has no fp32 path."""
+    assert _chunk_logsig(L, B=0) == INVALID
+    assert _chunk_logsig(L, dt=kda.KDA_F32) == UNSUPPORTED
+    assert _chunk_logsig(L, dk=96, dv=96) == UNSUPPORTED
+    assert _chunk_logsig(L, q=0) == INVALID
+    assert _chunk_logsig(L, q=BASE + 8) == ALIGN
+    assert _chunk_logsig(L, ws=0) == WS
+    assert _chunk_logsig(L, o=BASE + 16) == ALIAS
+
+
+def test_prep_and_scan_entries_validate(L):
+    P = ctypes.c_void_p
+    B, T, H, D = 1, 64, 1, 128
+    n = B * T * H * D * 2
+    need = L.kda_chunk_fwd_workspace(B, T, H, D, D, kda.KDA_BF16)
+    ins = [BASE + i * (n + 4096) for i in range(5)]
+    ws = BASE + 6 * (n + 4096)
+
+    def prep(gate=kda.KDA_GATE_BOUNDED, g_min=-5.0, q=ins[0], w=ws, wb=need, dk=D):
+        return L.kda_chunk_fwd_prep(B, T, H, dk, dk, gate, ctypes.c_float(g_min), P(q), P(ins[1]), P(ins[2]),
+                                    P(ins[3]), P(ins[4]), P(w), wb, None)
+
+    def scan(w=ws, wb=need, S0=None, o=BASE + 5 * (n + 4096), ST=None):
+        return L.kda_chunk_fwd_scan(B, T, H, D, D, P(w), wb, P(S0), P(o), P(ST), None)
+
+    assert prep(g_min=0.0) == INVALID
+    assert prep(g_min=-6.0) == UNSUPPORTED
+    assert prep(gate=7) == INVALID
+    assert prep(q=0) == INVALID
+    assert prep(q=BASE + 8) == ALIGN
+    assert prep(w=0) == WS
+    assert prep(wb=need - 1) == WS
+    assert prep(w=ins[2]) == ALIAS                     # workspace over v
+    assert prep(dk=96) == UNSUPPORTED
+    assert scan(o=0) == INVALID
+    assert scan(w=0) == WS
+    assert scan(S0=BASE * 3 + 4) == ALIGN
+    assert scan(o=ws + 1024) == ALIAS                  # o inside the records
+    S = BASE * 2
+    assert scan(S0=S, ST=S + 4096) == ALIAS
+    assert scan(ST=ws) == ALIAS

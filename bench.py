@@ -323,6 +323,28 @@ def run_libkda(args):
         abl = {"gate": "g = log sigmoid(a), diagonal 16x16 tiles element by element", "ms_per_step": abl_ms,
                "value": world * tokens / (abl_ms * 1e-3), "unit": UNIT, "slowdown_vs_bounded": abl_ms / ms}
 
+    # ---- packed variable-length batch: documents of mixed length on the same 64K token axis
+    vl = None
+    if args.only != "decode" and not args.no_varlen and (B, T, H) == (1, synth.VARLEN_64K_T, synth.VARLEN_64K_H):
+        lengths = synth.document_lengths(T)
+        cu = torch.from_numpy(synth.cu_seqlens(lengths)).to(device)
+        Nd = len(lengths)
+        S0v = synth.make_inputs(Nd, 1, H, D, D, "bf16", synth.VARLEN_SEED, 0.1)["S0"].to(device)
+        S_Tv = torch.empty_like(S0v)
+        packed = [d[n][0] for n in names]
+        ws_v = torch.empty(kda.kda_chunk_fwd_varlen_workspace(Nd, T, H, D, D), dtype=torch.uint8, device=device)
+
+        def vl_step():
+            kda.kda_chunk_fwd_varlen(*packed, cu, G_MIN, S0=S0v, o=o[0], S_T=S_Tv, workspace=ws_v)
+
+        vl_ms = time_steps(vl_step, max(3, min(args.steps, 10)), 3, world, device)
+        assert kda.kda_device_status(device) == 0
+        vl = {"workload": f"packed 64K axis, H={H} d={D}: {Nd} documents, log-uniform lengths 16..16384 "
+                          f"(min {int(lengths.min())}, max {int(lengths.max())})",
+              "ms_per_step": vl_ms, "value": world * tokens / (vl_ms * 1e-3), "unit": UNIT, "gpu_launches_per_step": 3,
+              "roofline_path_frac": (token_heads * BYTES_PER_TOKEN_HEAD + 2 * Nd * H * D * D * 4) / (vl_ms * 1e-3)
+              / 1e9 / hbm_peak}
+
     # ---- end to end through the C ABI with pinned host buffers
     hx = {n: x[n].pin_memory() for n in names}
     hS0 = x["S0"].pin_memory()
@@ -401,6 +423,8 @@ def run_libkda(args):
     }
     if abl is not None:
         line["ablation"] = abl
+    if vl is not None:
+        line["varlen"] = vl
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
     if rank == 0:
@@ -424,6 +448,7 @@ def main(argv=None):
                     help="64k (the benchmark workload) or 8k (a smaller case for profiler captures)")
     ap.add_argument("--only", choices=("all", "chunk", "decode"), default="all")
     ap.add_argument("--no-ablation", action="store_true", help="skip timing the log-sigmoid ablation path")
+    ap.add_argument("--no-varlen", action="store_true", help="skip timing the packed variable-length batch")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

@@ -51,6 +51,9 @@ EXPORTS = (
     "kda_chunk_fwd_logsigmoid",
     "kda_chunk_fwd_prep",
     "kda_chunk_fwd_scan",
+    "kda_selftest_device_timeout",
+    "kda_chunk_fwd_varlen_workspace",
+    "kda_chunk_fwd_varlen",
 )
 
 
@@ -98,6 +101,12 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_fwd_prep.restype = I
     L.kda_chunk_fwd_scan.argtypes = [I, I, I, I, I, P, S, P, P, P, P]
     L.kda_chunk_fwd_scan.restype = I
+    L.kda_selftest_device_timeout.argtypes = [ctypes.c_uint32, P]
+    L.kda_selftest_device_timeout.restype = I
+    L.kda_chunk_fwd_varlen_workspace.argtypes = [I, I, I, I, I, I]
+    L.kda_chunk_fwd_varlen_workspace.restype = S
+    L.kda_chunk_fwd_varlen.argtypes = [I, P, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_fwd_varlen.restype = I
     _lib = L
     return L
 
@@ -204,6 +213,35 @@ def kda_chunk_fwd_logsigmoid(q, k, v, a, beta, S0=None, o=None, S_T=None, worksp
     return o, S_T
 
 
+def kda_chunk_fwd_varlen(q, k, v, a, beta, cu_seqlens, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED,
+                         S0=None, o=None, S_T=None, workspace=None, return_state: bool = True):
+    """Chunked forward over a packed batch: q, k, a [T,H,dk]; v [T,H,dv]; beta [T,H] (bf16);
+    cu_seqlens int32 [N+1] on the device (sequence s = tokens cu[s]..cu[s+1]-1).  S0 / S_T
+    are [N,H,dk,dv] float32.  Returns (o [T,H,dv], S_T)."""
+    _check_cuda(q, k, v, a, beta, cu_seqlens, S0, o, S_T, workspace)
+    if q.dim() == 4 and q.shape[0] == 1:
+        q, k, v, a, beta = (t[0] for t in (q, k, v, a, beta))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise TypeError("cu_seqlens must be a 1-D int32 tensor")
+    N = cu_seqlens.numel() - 1
+    code = _dtype_code(q)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(lib().kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_varlen(N, _ptr(cu_seqlens), T, H, dk, dv, code, int(gate), float(g_min), _ptr(q),
+                                    _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
+                                    _ptr(workspace), ws_bytes, _stream(q.device))
+    _raise(st, "kda_chunk_fwd_varlen")
+    return o, S_T
+
+
 def kda_chunk_fwd_prep(q, k, v, a, beta, workspace, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED):
     """First stage of the bf16 chunked forward: one record per (batch*head, chunk) into
     ``workspace`` (uint8, at least ``kda_chunk_fwd_workspace`` bytes)."""
@@ -272,6 +310,13 @@ def kda_device_status(device=None) -> int:
     """Synchronise the current stream and return/clear the device status word."""
     dev = device if device is not None else torch.cuda.current_device()
     return int(lib().kda_device_status(_stream(dev)))
+
+
+def kda_selftest_device_timeout(limit_us: int = 20000, device=None) -> None:
+    """Launch the library's bounded-wait self-test: a kernel whose wait runs out after
+    ``limit_us`` and records KDA_ERR_DEVICE_TIMEOUT (read it with kda_device_status)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    _raise(lib().kda_selftest_device_timeout(int(limit_us), _stream(dev)), "kda_selftest_device_timeout")
 
 
 def kda_status_string(status: int) -> str:

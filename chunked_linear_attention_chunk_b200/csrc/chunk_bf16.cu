@@ -71,6 +71,91 @@ struct Rec {
     static_assert(Qp + (D / 64 - 1) * kC * 128 + 2 * kC * 128 <= Shared + Blk, "padded rows in bounds");
 };
 
+// ------------------------------------------------------------------ where chunks live
+// Regular batch: B sequences of T tokens, record row (b*H + h) of NT = ceil(T/64) records.
+// Packed variable-length batch: N sequences back to back on one token axis of T tokens,
+// sequence s spanning [cu[s], cu[s+1]); its chunks (ceil(len/64), none crossing into the
+// next sequence) are records choff[s] .. choff[s+1]-1 of head h's row of NT records.
+struct SeqMap {
+    const int32_t *cu = nullptr;     // packed batch: N + 1 token offsets; null for a regular batch
+    const int32_t *choff = nullptr;  // packed batch: N + 1 chunk offsets (prefix sums of ceil(len/64))
+    int nseq = 0;                    // B or N
+    int T = 0;                       // tokens per sequence (regular) or on the packed axis
+    int NT = 0;                      // records per row
+};
+
+struct ChunkLoc {
+    int64_t tok0;  // first token of the chunk on the flattened token axis (b*T + t)
+    int n;         // tokens of the chunk that exist (1..64)
+    size_t rec;    // record index
+    int h;
+    bool live;
+};
+
+// The chunk of prep CTA (blockIdx.x, blockIdx.y): regular grid (NT, B*H), packed (NT, H).
+__device__ __forceinline__ ChunkLoc locate_chunk(const SeqMap &m, int H)
+{
+    ChunkLoc L;
+    if (!m.cu) {
+        const int chunk = blockIdx.x, bh = blockIdx.y;
+        const int b = bh / H, t0 = chunk * kC;
+        L.tok0 = (int64_t)b * m.T + t0;
+        L.n = min(kC, m.T - t0);
+        L.rec = (size_t)bh * m.NT + chunk;
+        L.h = bh % H;
+        L.live = true;
+        return L;
+    }
+    const int g = blockIdx.x;
+    L.h = blockIdx.y;
+    L.live = g < m.choff[m.nseq];
+    if (!L.live)
+        return L;
+    int lo = 0, hi = m.nseq;  // the sequence s with choff[s] <= g < choff[s+1]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (m.choff[mid] <= g)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    const int c = g - m.choff[lo];
+    L.tok0 = (int64_t)m.cu[lo] + (int64_t)c * kC;
+    L.n = (int)min((int64_t)kC, (int64_t)m.cu[lo + 1] - L.tok0);
+    L.rec = (size_t)L.h * m.NT + g;
+    return L;
+}
+
+struct SeqLoc {
+    int64_t tok0;  // first token of the sequence on the flattened token axis
+    int len;       // its tokens
+    int nchunks;
+    size_t rec0;   // its first record
+    int sh;        // state index (sequence * H + h)
+    int h;
+};
+
+// The sequence of scan CTA row blockIdx.y = sequence * H + h (both layouts).
+__device__ __forceinline__ SeqLoc locate_seq(const SeqMap &m, int H)
+{
+    SeqLoc L;
+    L.sh = blockIdx.y;
+    const int sq = L.sh / H;
+    L.h = L.sh % H;
+    if (!m.cu) {
+        L.tok0 = (int64_t)sq * m.T;
+        L.len = m.T;
+        L.nchunks = m.NT;
+        L.rec0 = (size_t)L.sh * m.NT;
+    } else {
+        L.tok0 = m.cu[sq];
+        L.len = m.cu[sq + 1] - m.cu[sq];
+        L.nchunks = m.choff[sq + 1] - m.choff[sq];
+        L.rec0 = (size_t)L.h * m.NT + m.choff[sq];
+    }
+    return L;
+}
+
 // ------------------------------------------------------------------ K2: prep
 constexpr int kPrepThreads = 256;
 
@@ -189,7 +274,7 @@ __device__ __forceinline__ void diag_pair(int p, int &r, int &j)
 
 template <int D, bool kLogSig>
 __global__ void __launch_bounds__(kPrepThreads, 2)
-    prep_kernel(int T, int H, int NT, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+    prep_kernel(SeqMap map, int H, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                 const __nv_bfloat16 *__restrict__ beta, float g_min, unsigned char *__restrict__ ws,
                 unsigned int *status)
@@ -219,13 +304,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = lane >> 2, tq = lane & 3;
-    const int chunk = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / H, h = bh % H;
-    const int t0 = chunk * kC;
-    const int n = min(kC, T - t0);
-    unsigned char *rec = ws + ((size_t)bh * NT + chunk) * R::Bytes;
+    const ChunkLoc loc = locate_chunk(map, H);
+    if (!loc.live)  // packed batch: grid slots past the last chunk
+        return;
+    const int n = loc.n, h = loc.h;
+    unsigned char *rec = ws + loc.rec * R::Bytes;
     const int64_t rowstride = (int64_t)H * D;  // elements between consecutive tokens
-    const int64_t base = (((int64_t)b * T + t0) * H + h) * D;
+    const int64_t base = (loc.tok0 * H + h) * D;
 
     // -- 0. async loads of q, k, v, a into the swizzled token-major operands (zero past T)
     for (int i = tid; i < kC * CPR; i += kPrepThreads) {
@@ -240,7 +325,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     cp_async_commit();
     if (tid < kC)
-        sBeta[tid] = tid < n ? __bfloat162float(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.0f;
+        sBeta[tid] = tid < n ? __bfloat162float(beta[(loc.tok0 + tid) * H + h]) : 0.0f;
     if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init_cluster();
@@ -739,7 +824,7 @@ __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar)
 
 template <int D>
 __global__ void __launch_bounds__(kScanThreads, 1)
-    scan_kernel(int T, int H, int NT, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
+    scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char scan_smem[];
@@ -748,9 +833,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
     constexpr uint32_t kTmemCols = 2 * kBV;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int blk = blockIdx.x, col0 = blk * kBV, bh = blockIdx.y;
-    const int b = bh / H, h = bh % H;
-    const unsigned char *recs = ws + (size_t)bh * NT * R::Bytes;
+    const int blk = blockIdx.x, col0 = blk * kBV;
+    const SeqLoc seq = locate_seq(map, H);
+    const int h = seq.h, NT = seq.nchunks, bh = seq.sh;
+    const unsigned char *recs = ws + seq.rec0 * R::Bytes;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -875,8 +961,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 tc::ld_32x32b_x32(lane_addr + kBV, y);
                 tc::wait_ld();
                 const int t = c * kC + row;
-                if (t < T) {
-                    uint4 *orow = reinterpret_cast<uint4 *>(o + (((int64_t)b * T + t) * H + h) * D + col0);
+                if (t < seq.len) {
+                    uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
 #pragma unroll
                     for (int j = 0; j < kBV; j += 8) {
                         const uint4 ou = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
@@ -913,10 +999,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 }
 
 template <int D, bool kLogSig>
-cudaError_t launch_prep_d(int B, int T, int H, const void *q, const void *k, const void *v, const void *a,
-                          const void *beta, float g_min, void *ws, cudaStream_t s)
+cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, const void *k, const void *v,
+                          const void *a, const void *beta, float g_min, void *ws, cudaStream_t s)
 {
-    const int NT = (T + kC - 1) / kC;
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
@@ -924,17 +1009,17 @@ cudaError_t launch_prep_d(int B, int T, int H, const void *q, const void *k, con
     cudaError_t e = cudaFuncSetAttribute(prep_kernel<D, kLogSig>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    prep_kernel<D, kLogSig><<<dim3(NT, B * H), kPrepThreads, smem, s>>>(
-        T, H, NT, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+    prep_kernel<D, kLogSig><<<grid, kPrepThreads, smem, s>>>(
+        m, H, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
         static_cast<const __nv_bfloat16 *>(beta), g_min, static_cast<unsigned char *>(ws), status);
     return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_scan_d(int B, int T, int H, const void *ws, const float *S0, void *o, float *S_T, cudaStream_t s)
+cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S0, void *o, float *S_T,
+                          cudaStream_t s)
 {
-    const int NT = (T + kC - 1) / kC;
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
@@ -942,10 +1027,82 @@ cudaError_t launch_scan_d(int B, int T, int H, const void *ws, const float *S0, 
     cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    scan_kernel<D><<<dim3(D / kBV, B * H), kScanThreads, smem, s>>>(
-        T, H, NT, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, status);
+    scan_kernel<D><<<dim3(D / kBV, m.nseq * H), kScanThreads, smem, s>>>(
+        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, status);
     return cudaGetLastError();
 }
+
+cudaError_t launch_prep(const SeqMap &m, int H, int D, dim3 grid, const void *q, const void *k, const void *v,
+                        const void *a, const void *beta, float g_min, bool logsigmoid, void *ws, cudaStream_t s)
+{
+    if (logsigmoid)
+        return D == 64 ? launch_prep_d<64, true>(m, H, grid, q, k, v, a, beta, g_min, ws, s)
+                       : launch_prep_d<128, true>(m, H, grid, q, k, v, a, beta, g_min, ws, s);
+    return D == 64 ? launch_prep_d<64, false>(m, H, grid, q, k, v, a, beta, g_min, ws, s)
+                   : launch_prep_d<128, false>(m, H, grid, q, k, v, a, beta, g_min, ws, s);
+}
+
+cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const float *S0, void *o, float *S_T,
+                        cudaStream_t s)
+{
+    return D == 64 ? launch_scan_d<64>(m, H, ws, S0, o, S_T, s) : launch_scan_d<128>(m, H, ws, S0, o, S_T, s);
+}
+
+SeqMap regular_map(int B, int T)
+{
+    SeqMap m;
+    m.nseq = B;
+    m.T = T;
+    m.NT = (T + kC - 1) / kC;
+    return m;
+}
+
+// ------------------------------------------------------------------ packed-batch chunk table
+// One CTA: checks cu (cu[0] = 0, non-decreasing, cu[N] = T) and writes choff[s] = sum over
+// earlier sequences of ceil(len/64).  An invalid cu records KDA_ERR_INVALID_ARG and leaves an
+// all-zero table, so the prep and scan that follow touch nothing but S_T (= S0).
+constexpr int kTableThreads = 1024;
+
+__global__ void __launch_bounds__(kTableThreads)
+    seq_table_kernel(const int32_t *__restrict__ cu, int N, int T, int32_t *__restrict__ choff, unsigned int *status)
+{
+    __shared__ int32_t part[kTableThreads];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0)
+        bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
+    __syncthreads();
+    for (int s0 = 0; s0 < N; s0 += kTableThreads) {
+        const int s = s0 + tid;
+        if (s < N && cu[s + 1] < cu[s])
+            bad = 1;
+    }
+    __syncthreads();
+    const bool ok = bad == 0;
+    int carry = 0;
+    if (tid == 0)
+        choff[0] = 0;
+    for (int s0 = 0; s0 < N; s0 += kTableThreads) {
+        const int s = s0 + tid;
+        const int len = (ok && s < N) ? cu[s + 1] - cu[s] : 0;
+        part[tid] = (len + kC - 1) / kC;
+        __syncthreads();
+        for (int d = 1; d < kTableThreads; d <<= 1) {  // inclusive scan (Hillis-Steele)
+            const int x = tid >= d ? part[tid - d] : 0;
+            __syncthreads();
+            part[tid] += x;
+            __syncthreads();
+        }
+        if (s < N)
+            choff[s + 1] = carry + part[tid];
+        carry += part[kTableThreads - 1];
+        __syncthreads();
+    }
+    if (!ok && tid == 0)
+        report_device_error(status, KDA_ERR_INVALID_ARG);
+}
+
+size_t varlen_records(int N, int T) { return ((size_t)T + kC - 1) / kC + (size_t)N; }
 
 }  // namespace
 
@@ -960,18 +1117,46 @@ cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const vo
                              const void *a, const void *beta, float g_min, bool logsigmoid, void *workspace,
                              cudaStream_t s)
 {
-    if (logsigmoid)
-        return D == 64 ? launch_prep_d<64, true>(B, T, H, q, k, v, a, beta, g_min, workspace, s)
-                       : launch_prep_d<128, true>(B, T, H, q, k, v, a, beta, g_min, workspace, s);
-    return D == 64 ? launch_prep_d<64, false>(B, T, H, q, k, v, a, beta, g_min, workspace, s)
-                   : launch_prep_d<128, false>(B, T, H, q, k, v, a, beta, g_min, workspace, s);
+    const SeqMap m = regular_map(B, T);
+    return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, workspace, s);
 }
 
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
                              float *S_T, cudaStream_t s)
 {
-    return D == 64 ? launch_scan_d<64>(B, T, H, workspace, S0, o, S_T, s)
-                   : launch_scan_d<128>(B, T, H, workspace, S0, o, S_T, s);
+    return launch_scan(regular_map(B, T), H, D, workspace, S0, o, S_T, s);
+}
+
+size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D)
+{
+    const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
+    const size_t table = ((size_t)(N + 1) * 4 + 255) / 256 * 256;
+    return (size_t)H * varlen_records(N, T) * rec + table;
+}
+
+cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
+                                     const void *v, const void *a, const void *beta, float g_min, bool logsigmoid,
+                                     const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s)
+{
+    unsigned int *status = device_status_ptr();
+    if (!status)
+        return cudaErrorInvalidDevice;
+    const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
+    SeqMap m;
+    m.cu = cu;
+    m.nseq = N;
+    m.T = T;
+    m.NT = (int)varlen_records(N, T);
+    int32_t *choff = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + (size_t)H * m.NT * rec);
+    m.choff = choff;
+    seq_table_kernel<<<1, kTableThreads, 0, s>>>(cu, N, T, choff, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    e = launch_prep(m, H, D, dim3(m.NT, H), q, k, v, a, beta, g_min, logsigmoid, workspace, s);
+    if (e != cudaSuccess)
+        return e;
+    return launch_scan(m, H, D, workspace, S0, o, S_T, s);
 }
 
 }  // namespace kda

@@ -46,6 +46,7 @@ unsigned int *device_status_ptr()
 namespace {
 
 constexpr int64_t kMaxElems = (int64_t)1 << 40;
+constexpr int kMaxPackedTokens = 0x7fffffff - 64;  // packed axis; cu_seqlens are int32
 
 struct Range {
     uintptr_t lo = 0, hi = 0;  // [lo, hi)
@@ -312,6 +313,52 @@ kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dty
 {
     return chunk_fwd_impl(B, T, H, dk, dv, dtype, q, k, v, a, beta, 0.0f, KDA_GATE_LOGSIGMOID, S0, o, S_T,
                           workspace, ws_bytes, stream);
+}
+
+size_t kda_chunk_fwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (N < 1 || T < 0 || T > kMaxPackedTokens || H < 1 || dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16)
+        return 0;
+    return chunk_bf16_varlen_workspace(N, T, H, dk);
+}
+
+kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
+                                kda_gate gate, float g_min, const void *q, const void *k, const void *v,
+                                const void *a, const void *beta, const float *S0, void *o, float *S_T,
+                                void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    if (!dtype_ok(dtype) || N < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gate(gate, g_min, KDA_BF16);
+    if (st != KDA_OK)
+        return st;
+    if (dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16 || T > kMaxPackedTokens || (int64_t)N * H > 65535)
+        return KDA_ERR_UNSUPPORTED;
+    const int64_t nk = (int64_t)T * H * dk, ntok = (int64_t)T * H, ns = (int64_t)N * H * dk * dv;
+    if (!cu_seqlens || (T > 0 && (!q || !k || !v || !a || !beta || !o)))
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, a, beta, S0, o, S_T, workspace}) || ((uintptr_t)cu_seqlens & 3u))
+        return KDA_ERR_ALIGNMENT;
+    const size_t need = kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, dtype);
+    if (!workspace || ws_bytes < need)
+        return KDA_ERR_WORKSPACE;
+    const Range rq(q, nk * 2), rk(k, nk * 2), rv(v, nk * 2), ra(a, nk * 2), rb(beta, ntok * 2),
+        rcu(cu_seqlens, (int64_t)(N + 1) * 4), rS0(S0, ns * 4), ro(T > 0 ? o : nullptr, nk * 2), rST(S_T, ns * 4),
+        rws(workspace, (int64_t)need);
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rS0, rST, rws})
+        if (overlaps(ro, in))
+            return KDA_ERR_ALIAS;
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rws})
+        if (overlaps(rST, in))
+            return KDA_ERR_ALIAS;
+    if (overlaps(rST, rS0) && S_T != S0)
+        return KDA_ERR_ALIAS;
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rS0})
+        if (overlaps(rws, in))
+            return KDA_ERR_ALIAS;
+    return from_cuda(launch_chunk_bf16_varlen(N, cu_seqlens, T, H, dk, q, k, v, a, beta, g_min,
+                                              gate == KDA_GATE_LOGSIGMOID, S0, o, S_T, workspace,
+                                              (cudaStream_t)stream));
 }
 
 kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const void *q,

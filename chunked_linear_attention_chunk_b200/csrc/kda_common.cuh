@@ -177,14 +177,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity)
 
 // Wait for the phase of `bar` with the given parity to complete, for at most
 // kWaitLimitNs.  Returns false (and records the timeout) when the limit is reached.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, unsigned int *status)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, unsigned int *status,
+                                                  unsigned long long limit_ns = kWaitLimitNs)
 {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report_device_error(status, KDA_ERR_DEVICE_TIMEOUT);
             return false;
         }

@@ -32,6 +32,14 @@ cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const vo
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
                              float *S_T, cudaStream_t s);
 
+// Packed variable-length batch: N sequences on one axis of T tokens, sequence s spanning
+// [cu[s], cu[s+1]) (cu on the device).  A table kernel validates cu and writes the chunk
+// offsets at the end of the workspace; prep and scan follow on the same stream.
+size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D);
+cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
+                                     const void *v, const void *a, const void *beta, float g_min, bool logsigmoid,
+                                     const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s);
+
 // K4: single-token decode step.
 cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,
                           const void *a, const void *beta, float g_min, float *S, void *o, cudaStream_t s);

@@ -167,3 +167,29 @@ def decode_tokens(w: DecodeWorkload, step: int, dtype="bf16"):
 def to_numpy32(t: torch.Tensor) -> np.ndarray:
     """Exact float32 copy of a (bf16 or f32) CPU tensor, for the oracle."""
     return t.detach().to("cpu", torch.float32).contiguous().numpy()
+
+
+# ---------------------------------------------------------------------------- packed batches
+# Packed variable-length stage: documents of mixed length packed back to back to fill one
+# 64K-token axis.  Lengths are log-uniform between 16 and 16384 tokens (most documents are
+# short, most tokens sit in long ones), drawn from their own stream; the last document is
+# cut to fill the axis exactly.  Token tensors are the 64K stage's draw (without the a = +8
+# run); every document starts from its own S0 slice.
+VARLEN_64K_T = 65536
+VARLEN_64K_H = 32
+VARLEN_SEED = 1005
+
+
+def document_lengths(T: int, seed: int = VARLEN_SEED, lo: int = 16, hi: int = 16384) -> np.ndarray:
+    rng = np.random.default_rng([seed, 99])
+    out, total = [], 0
+    while total < T:
+        L = int(np.exp(rng.uniform(np.log(lo), np.log(hi))))
+        L = min(L, T - total)
+        out.append(L)
+        total += L
+    return np.asarray(out, np.int64)
+
+
+def cu_seqlens(lengths) -> np.ndarray:
+    return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)

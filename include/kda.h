@@ -154,6 +154,35 @@ kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dty
                                     kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_varlen -- the chunked forward over a packed batch of variable-length
+ * sequences: N sequences stored back to back on one token axis of T tokens, sequence s
+ * being tokens [cu_seqlens[s], cu_seqlens[s+1]).  Each sequence starts from its own state
+ * S0[s] (or zeros) and ends in S_T[s]; nothing flows across a boundary, and no chunk
+ * spans two sequences.  Equal-length sequences give exactly kda_chunk_fwd's result.
+ * Passage: many documents packed into one long training sequence ("Breaking Through ..."
+ * section 3, the packing used for the long-context stages); the per-sequence recurrence
+ * is kda_chunk_fwd's.
+ *   N            sequences (>= 1; N * H <= 65535).
+ *   cu_seqlens   DEVICE pointer to N + 1 int32 offsets, 4-byte aligned: cu[0] = 0,
+ *                non-decreasing, cu[N] = T (empty sequences allowed).  Checked on the
+ *                device: an invalid array records KDA_ERR_INVALID_ARG in the device status
+ *                word (kda_device_status), writes no o, and S_T gets S0 (or zeros).
+ *   T            tokens on the packed axis (0 .. 2^31 - 65).
+ *   dk, dv       dk == dv in {64, 128}; dtype must be KDA_BF16.
+ *   gate, g_min  as in kda_chunk_fwd_prep.
+ *   q, k, a      [T, H, dk];  v, o: [T, H, dv];  beta: [T, H]   (bfloat16)
+ *   S0, S_T      [N, H, dk, dv] float32, or NULL (zeros / not stored); S_T may be S0.
+ *   workspace    >= kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, dtype) bytes (records
+ *                for ceil(T/64) + N chunks per head, plus the chunk table), 16-byte aligned.
+ *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.
+ */
+size_t kda_chunk_fwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype);
+kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
+                                kda_gate gate, float g_min, const void *q, const void *k, const void *v,
+                                const void *a, const void *beta, const float *S0, void *o, float *S_T,
+                                void *workspace, size_t ws_bytes, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_prep, kda_chunk_fwd_scan -- the two stages of the bfloat16 kda_chunk_fwd
  * as separate calls, for callers that schedule them apart (timing each stage, or running
  * the fully parallel prep of one batch while other work waits for the serial scan).
@@ -231,10 +260,23 @@ size_t kda_chunk_fwd_noalloc_max_scratch(void);
 
 /*
  * kda_device_status -- synchronise `stream`, then return and clear the current
- * device's kernel status word: KDA_OK, or KDA_ERR_DEVICE_TIMEOUT if a kernel gave up
- * on a bounded wait since the last call; KDA_ERR_CUDA if the synchronisation failed.
+ * device's kernel status word: KDA_OK; KDA_ERR_DEVICE_TIMEOUT if a kernel gave up on a
+ * bounded wait since the last call; KDA_ERR_INVALID_ARG if kda_chunk_fwd_varlen found
+ * its cu_seqlens invalid; KDA_ERR_CUDA if the synchronisation failed.  The first error
+ * recorded since the last call is the one reported.
  */
 kda_status kda_device_status(kda_stream_t stream);
+
+/*
+ * kda_selftest_device_timeout -- exercise the kernels' failure path.  Launches one small
+ * kernel whose bounded wait, on an mbarrier that nothing completes, runs out after
+ * `limit_us` microseconds (1 .. 2 000 000); it then records KDA_ERR_DEVICE_TIMEOUT in the
+ * device status word exactly as a real timeout would, and returns.  The GPU and the CUDA
+ * context stay usable: the next kda_device_status() returns KDA_ERR_DEVICE_TIMEOUT and
+ * clears the word.  The pages have no counterpart; it exists to test error handling.
+ * Errors: INVALID_ARG (limit out of range), CUDA.
+ */
+kda_status kda_selftest_device_timeout(uint32_t limit_us, kda_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(kda_status status);

@@ -220,3 +220,38 @@ def test_prep_and_scan_entries_validate(L):
     S = BASE * 2
     assert scan(S0=S, ST=S + 4096) == ALIAS
     assert scan(ST=ws) == ALIAS
+
+
+def test_selftest_timeout_rejects_bad_limits(L):
+    assert L.kda_selftest_device_timeout(0, None) == INVALID
+    assert L.kda_selftest_device_timeout(2000001, None) == INVALID
+
+
+def test_varlen_entry_validates(L):
+    P = ctypes.c_void_p
+    N, T, H, D = 2, 100, 2, 128
+    n = T * H * D * 2
+    ws_need = L.kda_chunk_fwd_varlen_workspace(N, T, H, D, D, kda.KDA_BF16)
+    rec = 128 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 128 * 128 * 2 + 64 * 128 * 2
+    assert ws_need == H * ((T + 63) // 64 + N) * rec + 256
+    assert L.kda_chunk_fwd_varlen_workspace(N, T, H, D, D, kda.KDA_F32) == 0
+    ins = [BASE + i * (n + 4096) for i in range(5)]
+    cu = BASE * 2
+    ws = BASE + 6 * (n + 4096)
+
+    def call(N=N, cu=cu, dt=kda.KDA_BF16, gate=kda.KDA_GATE_BOUNDED, g_min=-5.0, o=BASE + 5 * (n + 4096), w=ws,
+             wb=ws_need, H=H):
+        return L.kda_chunk_fwd_varlen(N, P(cu), T, H, D, D, dt, gate, ctypes.c_float(g_min), *(P(p) for p in ins),
+                                      None, P(o), None, P(w), wb, None)
+
+    assert call(N=0) == INVALID
+    assert call(cu=0) == INVALID
+    assert call(cu=cu + 2) == ALIGN
+    assert call(dt=kda.KDA_F32) == UNSUPPORTED
+    assert call(g_min=-9.0) == UNSUPPORTED
+    assert call(gate=5) == INVALID
+    assert call(N=40000) == UNSUPPORTED          # N * H beyond the grid limit
+    assert call(w=0) == WS
+    assert call(wb=ws_need - 1) == WS
+    assert call(o=ins[1]) == ALIAS
+    assert call(cu=ws + 64) == ALIAS              # cu_seqlens inside the workspace

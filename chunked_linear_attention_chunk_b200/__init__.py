@@ -213,6 +213,11 @@ def kda_chunk_fwd_logsigmoid(q, k, v, a, beta, S0=None, o=None, S_T=None, worksp
     return o, S_T
 
 
+def kda_chunk_fwd_varlen_workspace(N: int, T: int, H: int, dk: int, dv: int, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(lib().kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, code))
+
+
 def kda_chunk_fwd_varlen(q, k, v, a, beta, cu_seqlens, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED,
                          S0=None, o=None, S_T=None, workspace=None, return_state: bool = True):
     """Chunked forward over a packed batch: q, k, a [T,H,dk]; v [T,H,dv]; beta [T,H] (bf16);
@@ -288,6 +293,11 @@ def kda_chunk_fwd_noalloc(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None
                                      _ptr(beta), float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _stream(q.device))
     _raise(st, "kda_chunk_fwd_noalloc")
     return o, S_T
+
+
+def kda_chunk_fwd_noalloc_max_scratch() -> int:
+    """Bytes of the built-in device scratch kda_chunk_fwd_noalloc uses."""
+    return int(lib().kda_chunk_fwd_noalloc_max_scratch())
 
 
 def kda_decode_step(q, k, v, a, beta, S, g_min: float = -5.0, o=None):

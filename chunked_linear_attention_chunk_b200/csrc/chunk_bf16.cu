@@ -180,8 +180,8 @@ struct PrepLayout {
     static constexpr uint32_t REm = RBeta + kC * 4;        // bf16 [4][D]  e^{G_{m_I}}
     static constexpr uint32_t REl = REm + kTiles * D * 2;  // bf16 [4][D]  e^{G_last - G_{m_I}}
     static constexpr uint32_t RDd = REl + kTiles * D * 2;  // bf16 [6][D]  e^{G_{m_I} - G_{m_J}}
-    static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarrier
-    static constexpr uint32_t RTmem = RBar + 8;
+    static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarriers: round 1, then units U1..U4
+    static constexpr uint32_t RTmem = RBar + 5 * 8;
     static constexpr uint32_t Bytes = RTmem + 8;
     static_assert(RG % 1024 == 0 && RP % 1024 == 0, "operand alignment");
 };
@@ -312,7 +312,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const int64_t rowstride = (int64_t)H * D;  // elements between consecutive tokens
     const int64_t base = (loc.tok0 * H + h) * D;
 
-    // -- 0. async loads of q, k, v, a into the swizzled token-major operands (zero past T)
+    // -- 0. async loads into the swizzled token-major operands (zero past the sequence):
+    //       a first (the gate needs it), then q, k, v, which land during steps 1-2
+    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
+        const int r = i / CPR, c8 = (i % CPR) * 8;
+        const bool ok = r < n;
+        const int64_t off = base + (ok ? (int64_t)r * rowstride : 0) + c8;
+        cp_async_16_zfill(sm + L::RX + tok_off(r, c8), a + off, ok);
+    }
+    cp_async_commit();
     for (int i = tid; i < kC * CPR; i += kPrepThreads) {
         const int r = i / CPR, c8 = (i % CPR) * 8;
         const bool ok = r < n;
@@ -321,56 +329,45 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         cp_async_16_zfill(sm + L::RQ + d, q + off, ok);
         cp_async_16_zfill(sm + L::RK + d, k + off, ok);
         cp_async_16_zfill(sm + L::RV + d, v + off, ok);
-        cp_async_16_zfill(sm + L::RX + d, a + off, ok);
     }
     cp_async_commit();
     if (tid < kC)
         sBeta[tid] = tid < n ? __bfloat162float(beta[(loc.tok0 + tid) * H + h]) : 0.0f;
     if (tid == 0) {
-        mbar_init(bar, 1);
+        for (int i = 0; i < 5; ++i)
+            mbar_init(bar + i, 1);
         fence_mbar_init_cluster();
     }
     if (warp == 0)
         tc::tmem_alloc(tslot, 2 * D);
-    cp_async_wait<0>();
+    cp_async_wait<1>();  // a is in; q, k, v may still be in flight
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tslot;
 
-    // -- 1. gate g = g_min sigmoid(a) (0 past T), then inclusive cumulative sum over tokens
-    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
-        const int r = i / CPR, c8 = (i % CPR) * 8;
-        const uint4 au = *reinterpret_cast<const uint4 *>(sm + L::RX + tok_off(r, c8));
-        const uint32_t w[4] = {au.x, au.y, au.z, au.w};
-        float gv[8];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float2 f = unpack_bf16x2(w[p]);
-            if constexpr (kLogSig) {
-                gv[2 * p] = r < n ? gate_logsigmoid_fast(f.x) : 0.0f;
-                gv[2 * p + 1] = r < n ? gate_logsigmoid_fast(f.y) : 0.0f;
-            } else {
-                gv[2 * p] = r < n ? gate_bounded_fast(f.x, g_min) : 0.0f;
-                gv[2 * p + 1] = r < n ? gate_bounded_fast(f.y, g_min) : 0.0f;
-            }
-        }
-        float4 *dst = reinterpret_cast<float4 *>(&sG[r * D + c8]);
-        dst[0] = make_float4(gv[0], gv[1], gv[2], gv[3]);
-        dst[1] = make_float4(gv[4], gv[5], gv[6], gv[7]);
-    }
-    __syncthreads();
+    // -- 1. gate g = g_min sigmoid(a) (0 past the sequence) fused with its inclusive
+    //       cumulative sum over tokens: kPrepThreads / D threads per channel, each summing
+    //       its run of tokens; later runs then add the totals of the earlier ones
     {
         constexpr int TPC = kPrepThreads / D;
         constexpr int LEN = kC / TPC;
         const int c = tid % D, part = tid / D;
         float gv[LEN];
+        float run = 0.0f;
 #pragma unroll
-        for (int r = 0; r < LEN; ++r)
-            gv[r] = sG[(part * LEN + r) * D + c];
-#pragma unroll
-        for (int r = 1; r < LEN; ++r)
-            gv[r] += gv[r - 1];
+        for (int r = 0; r < LEN; ++r) {
+            const int t = part * LEN + r;
+            const float av =
+                __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
+            float g;
+            if constexpr (kLogSig)
+                g = gate_logsigmoid_fast(av);
+            else
+                g = gate_bounded_fast(av, g_min);
+            run += t < n ? g : 0.0f;
+            gv[r] = run;
+        }
 #pragma unroll
         for (int r = 0; r < LEN; ++r)
             sG[(part * LEN + r) * D + c] = gv[r];
@@ -384,6 +381,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             for (int r = 0; r < LEN; ++r)
                 sG[(part * LEN + r) * D + c] = gv[r] + off;
     }
+    cp_async_wait<0>();  // q, k, v are in (read from step 3a on)
     __syncthreads();
 
     // -- 2. per-(tile, channel) decay scalars (bf16) and Gamma_C (record)
@@ -687,109 +685,158 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     __syncthreads();
     tc::fence_after_sync();
 
-    // -- 7. rounds 2 and 3: Khat^T X (TMEM cols 0..D) and P X (cols D..2D) for X = W, then
-    //       X = Utilde.  The results are staged in shared memory in record order (round 2:
-    //       N over [Kbar | V], Q' = Qbar - P W in place of Qbar; round 3: Bm and O' over
-    //       [Qbar | Kbar | V]) and written with bulk copies.
-    static_assert(R::Qp - R::Nm <= 2 * L::kMat && R::Bytes - R::Shared <= 3 * L::kMat, "staging fits");
-#pragma unroll 1
-    for (int round = 0; round < 2; ++round) {
-        if (tid == 0) {
-            const uint32_t id_kt = tc::idesc_bf16(128, D, true, true);  // A = Khat^T (MN-major)
-            const uint32_t id_p = tc::idesc_bf16(128, D, false, true);  // A = P (K-major)
-            const uint32_t xb = smem_u32(sm + L::RG) + round * (D / 64) * (kC * 128);
+    // -- 7. four tensor-core units on the operands in place, each completing on its own
+    //       mbarrier, so the tensor core runs one unit while the warps drain another:
+    //         U1  N = Khat^T W     TMEM cols 0..D    staged over [Kbar | V]
+    //         U2  P W              cols D..2D        Q' = Qbar - P W in place of Qbar
+    //         U3  Bm = Khat^T Ut   cols 0..D         staged over Khat and W
+    //         U4  O' = P Ut        cols D..2D        staged over Utilde
+    //       U3 is issued once U1's columns are read, U4 once U2's are.  Every staging area
+    //       is free when written ([Kbar | V] and Qbar after round 1; Khat and W once U3 is
+    //       done, U4 reading only P and Utilde; Utilde once U4 is done), so no store waits
+    //       for another to finish reading shared memory.
+    constexpr int NB = D / kBV;  // value blocks of the record
+    static_assert((uint32_t)D * D * 2 <= 2 * L::kMat, "N staging fits over [Kbar | V]");
+    static_assert((NB / 2) * R::BmBlk <= L::kMat && NB * R::OpBlk <= L::kMat, "Bm / O' staging fits");
+    uint64_t *bar_u = bar + 1;
+    const uint32_t xw = smem_u32(sm + L::RG), xu = xw + L::kMat;  // W, Utilde (token-major operands)
+    auto issue_kt = [&](uint32_t xb, uint32_t col) {                  // Khat^T X
+        const uint32_t id = tc::idesc_bf16(128, D, true, true);       // A = Khat^T (MN-major)
 #pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks) {
-                const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RX) + ks * 2048, kC * 128, 1024, tc::kSw128);
-                const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
-                tc::mma_bf16(tmem, ad, bd, id_kt, ks > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks) {
-                const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RP) + ks * 32, 16, 1024, tc::kSw128);
-                const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
-                tc::mma_bf16(tmem + D, ad, bd, id_p, ks > 0 ? 1u : 0u);
-            }
-            tc::commit(bar);
+        for (int ks = 0; ks < kC / 16; ++ks) {
+            const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RX) + ks * 2048, kC * 128, 1024, tc::kSw128);
+            const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
+            tc::mma_bf16(tmem + col, ad, bd, id, ks > 0 ? 1u : 0u);
         }
-        mbar_wait_bounded(bar, phase, status);
-        phase ^= 1;
-        tc::fence_after_sync();
-        if (round == 1) {  // the round-2 stores must have read their staging before reuse
-            if (tid == 0)
-                bulk_wait_read_all();
-            __syncthreads();
+    };
+    auto issue_p = [&](uint32_t xb, uint32_t col) {                   // P X
+        const uint32_t id = tc::idesc_bf16(128, D, false, true);      // A = P (K-major)
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) {
+            const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RP) + ks * 32, 16, 1024, tc::kSw128);
+            const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
+            tc::mma_bf16(tmem + col, ad, bd, id, ks > 0 ? 1u : 0u);
         }
-        unsigned char *stage2 = sm + L::RK;  // round 2: N (D x D) over [Kbar | V]
-        unsigned char *stage3 = sm + L::RQ;  // round 3: per value block Bm | O' over [Qbar | Kbar | V]
-        // Khat^T X: row i (key channel) = TMEM lane i; warp w reads the lanes of quarter
-        // w % 4 and half w / 4 of the columns
-        if ((warp & 3) * 32 < D) {
-            const int i = (warp & 3) * 32 + lane;
-            const int cb = (warp >> 2) * (D / 2);
-#pragma unroll
-            for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                uint32_t x[32];
-                tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cb + c0), x);
-                tc::wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    const int col = cb + c0 + j;
-                    if (round == 0)
-                        *reinterpret_cast<uint4 *>(stage2 + tc::kmaj_sw128(i, col, D)) = pack8(&x[j]);
-                    else
-                        *reinterpret_cast<uint4 *>(stage3 + (col / kBV) * R::Blk + tc::mnmaj_sw64(i, col % kBV)) =
-                            pack8(&x[j]);
-                }
-            }
-        }
-        // P X: chunk row r = TMEM lane r (< 64)
-        if ((warp & 3) < 2) {
-            const int r = (warp & 3) * 32 + lane;
-            const int cb = (warp >> 2) * (D / 2);
-#pragma unroll
-            for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                uint32_t x[32];
-                tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, D + cb + c0), x);
-                tc::wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    const int col = cb + c0 + j;
-                    if (round == 0) {  // Q' = Qbar - P W, in place (same layout as the record)
-                        uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + tok_off(r, col));
-                        const uint4 qb = *pq;
-                        const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
-                        uint32_t o4[4];
-#pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            const float2 f = unpack_bf16x2(qw[p]);
-                            o4[p] = pack_bf16x2(f.x - __uint_as_float(x[j + 2 * p]),
-                                                f.y - __uint_as_float(x[j + 2 * p + 1]));
-                        }
-                        *pq = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                    } else {  // O' = P Utilde
-                        *reinterpret_cast<uint4 *>(stage3 + (col / kBV) * R::Blk + R::BmBlk +
-                                                   tc::mnmaj_sw64(r, col % kBV)) = pack8(&x[j]);
-                    }
-                }
-            }
-        }
-        tc::fence_smem_to_async();
+    };
+    auto bm_stage = [&](int blk) -> unsigned char * {  // Bm block blk: over Khat, then W
+        return blk < NB / 2 ? sm + L::RX + blk * R::BmBlk : sm + L::RG + (blk - NB / 2) * R::BmBlk;
+    };
+    auto sync_all = [&]() {
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        if (tid == 0) {
-            if (round == 0) {
-                bulk_s2g(rec + R::Nm, stage2, D * D * 2);
-                bulk_s2g(rec + R::Qp, sm + L::RQ, kC * D * 2);
-            } else {
-                bulk_s2g(rec + R::Shared, stage3, R::Bytes - R::Shared);
-            }
-            bulk_commit();
+    };
+    if (tid == 0) {
+        issue_kt(xw, 0);
+        tc::commit(&bar_u[0]);
+        issue_p(xw, D);
+        tc::commit(&bar_u[1]);
+    }
+    // Khat^T X epilogues: row i (key channel) = TMEM lane i; warp w reads the lanes of
+    // quarter w % 4 and half w / 4 of the columns.  P X epilogues: chunk row r = lane r < 64.
+    const bool kt_rows = (warp & 3) * 32 < D, p_rows = (warp & 3) < 2;
+    const int lrow = (warp & 3) * 32 + lane, chalf = (warp >> 2) * (D / 2);
+
+    // U1 -> N over [Kbar | V]
+    mbar_wait_bounded(&bar_u[0], 0, status);
+    tc::fence_after_sync();
+    if (kt_rows) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t x[32];
+            tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, chalf + c0), x);
+            tc::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4 *>(sm + L::RK + tc::kmaj_sw128(lrow, chalf + c0 + j, D)) = pack8(&x[j]);
         }
     }
-    if (tid == 0)
+    sync_all();
+    if (tid == 0) {
+        issue_kt(xu, 0);
+        tc::commit(&bar_u[2]);
+    }
+    // U2 -> Q' = Qbar - P W, in place (same layout as the record)
+    mbar_wait_bounded(&bar_u[1], 0, status);
+    tc::fence_after_sync();
+    if (p_rows) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t x[32];
+            tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, D + chalf + c0), x);
+            tc::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + tok_off(lrow, chalf + c0 + j));
+                const uint4 qb = *pq;
+                const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 f = unpack_bf16x2(qw[p]);
+                    o4[p] = pack_bf16x2(f.x - __uint_as_float(x[j + 2 * p]), f.y - __uint_as_float(x[j + 2 * p + 1]));
+                }
+                *pq = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+    }
+    tc::fence_smem_to_async();
+    sync_all();
+    if (tid == 0) {
+        issue_p(xu, D);
+        tc::commit(&bar_u[3]);
+        bulk_s2g(rec + R::Nm, sm + L::RK, D * D * 2);
+        bulk_s2g(rec + R::Qp, sm + L::RQ, kC * D * 2);
+        bulk_commit();
+    }
+    // U3 -> Bm blocks over Khat and W
+    mbar_wait_bounded(&bar_u[2], 0, status);
+    tc::fence_after_sync();
+    if (kt_rows) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t x[32];
+            tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, chalf + c0), x);
+            tc::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                const int col = chalf + c0 + j;
+                *reinterpret_cast<uint4 *>(bm_stage(col / kBV) + tc::mnmaj_sw64(lrow, col % kBV)) = pack8(&x[j]);
+            }
+        }
+    }
+    tc::fence_smem_to_async();
+    sync_all();
+    if (tid == 0) {
+        for (int blk = 0; blk < NB; ++blk)
+            bulk_s2g(rec + R::Shared + blk * R::Blk, bm_stage(blk), R::BmBlk);
+        bulk_commit();
+    }
+    // U4 -> O' blocks over Utilde
+    mbar_wait_bounded(&bar_u[3], 0, status);
+    tc::fence_after_sync();
+    if (p_rows) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t x[32];
+            tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, D + chalf + c0), x);
+            tc::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                const int col = chalf + c0 + j;
+                *reinterpret_cast<uint4 *>(sm + L::RG + L::kMat + (col / kBV) * R::OpBlk +
+                                           tc::mnmaj_sw64(lrow, col % kBV)) = pack8(&x[j]);
+            }
+        }
+    }
+    tc::fence_smem_to_async();
+    sync_all();
+    if (tid == 0) {
+        for (int blk = 0; blk < NB; ++blk)
+            bulk_s2g(rec + R::Shared + blk * R::Blk + R::BmBlk, sm + L::RG + L::kMat + blk * R::OpBlk, R::OpBlk);
+        bulk_commit();
         bulk_wait_read_all();  // staging must stay valid until the stores have read it
+    }
     __syncthreads();
     if (warp == 0)
         tc::tmem_dealloc(tmem, 2 * D);

@@ -255,3 +255,10 @@ def test_varlen_entry_validates(L):
     assert call(wb=ws_need - 1) == WS
     assert call(o=ins[1]) == ALIAS
     assert call(cu=ws + 64) == ALIAS              # cu_seqlens inside the workspace
+
+
+def test_binding_has_a_function_for_every_export():
+    """The Python binding carries the C names: one function per exported entry point."""
+    missing = [n for n in kda.EXPORTS if not callable(getattr(kda, n, None))]
+    assert not missing, missing
+    assert set(kda.EXPORTS) == set(declared_functions())

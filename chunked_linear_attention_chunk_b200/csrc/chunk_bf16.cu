@@ -92,12 +92,12 @@ struct ChunkLoc {
     bool live;
 };
 
-// The chunk of prep CTA (blockIdx.x, blockIdx.y): regular grid (NT, B*H), packed (NT, H).
-__device__ __forceinline__ ChunkLoc locate_chunk(const SeqMap &m, int H)
+// The chunk of prep CTA (x, y): regular grid (NT, B*H), packed (NT, H).
+__device__ __forceinline__ ChunkLoc locate_chunk(const SeqMap &m, int H, int x, int y)
 {
     ChunkLoc L;
     if (!m.cu) {
-        const int chunk = blockIdx.x, bh = blockIdx.y;
+        const int chunk = x, bh = y;
         const int b = bh / H, t0 = chunk * kC;
         L.tok0 = (int64_t)b * m.T + t0;
         L.n = min(kC, m.T - t0);
@@ -106,8 +106,8 @@ __device__ __forceinline__ ChunkLoc locate_chunk(const SeqMap &m, int H)
         L.live = true;
         return L;
     }
-    const int g = blockIdx.x;
-    L.h = blockIdx.y;
+    const int g = x;
+    L.h = y;
     L.live = g < m.choff[m.nseq];
     if (!L.live)
         return L;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = lane >> 2, tq = lane & 3;
-    const ChunkLoc loc = locate_chunk(map, H);
+    const ChunkLoc loc = locate_chunk(map, H, blockIdx.x, blockIdx.y);
     if (!loc.live)  // packed batch: grid slots past the last chunk
         return;
     const int n = loc.n, h = loc.h;

@@ -212,18 +212,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
-// Same copy delivered to the same offsets in every CTA of `mask` within the cluster
-// (global memory of this GPU only), each destination's `bar` receiving the bytes.
-__device__ __forceinline__ void bulk_g2s_multicast(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                                   uint16_t mask)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.multicast::cluster [%0], [%1], %2, [%3], "
-        "%4;" ::"r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "h"(mask)
-        : "memory");
-}
-
 // Bulk (non-tensor) async copy shared -> global, tracked by bulk groups.
 __device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes)
 {

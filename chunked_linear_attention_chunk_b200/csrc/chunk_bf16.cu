@@ -157,7 +157,12 @@ __device__ __forceinline__ SeqLoc locate_seq(const SeqMap &m, int H)
 }
 
 // ------------------------------------------------------------------ K2: prep
-constexpr int kPrepThreads = 256;
+constexpr int kPrepWarps = 10;  // one per 16x16 tile pair of the chunk
+constexpr int kPrepThreads = kPrepWarps * 32;
+// The first eight warps take the roles tied to the layout: two TMEM lane quarters x two
+// column halves in the epilogues, two threads per key channel in the cumulative sum.
+constexpr int kCoreThreads = 256;
+static_assert(kPrepWarps >= 8 && kPrepWarps >= kTiles * (kTiles + 1) / 2, "prep warp roles");
 
 template <int D>
 struct PrepLayout {
@@ -350,33 +355,37 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     //       cumulative sum over tokens: kPrepThreads / D threads per channel, each summing
     //       its run of tokens; later runs then add the totals of the earlier ones
     {
-        constexpr int TPC = kPrepThreads / D;
+        constexpr int TPC = kCoreThreads / D;
         constexpr int LEN = kC / TPC;
+        const bool core = tid < kCoreThreads;
         const int c = tid % D, part = tid / D;
         float gv[LEN];
         float run = 0.0f;
+        if (core) {
 #pragma unroll
-        for (int r = 0; r < LEN; ++r) {
-            const int t = part * LEN + r;
-            const float av =
-                __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
-            float g;
-            if constexpr (kLogSig)
-                g = gate_logsigmoid_fast(av);
-            else
-                g = gate_bounded_fast(av, g_min);
-            run += t < n ? g : 0.0f;
-            gv[r] = run;
+            for (int r = 0; r < LEN; ++r) {
+                const int t = part * LEN + r;
+                const float av =
+                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
+                float g;
+                if constexpr (kLogSig)
+                    g = gate_logsigmoid_fast(av);
+                else
+                    g = gate_bounded_fast(av, g_min);
+                run += t < n ? g : 0.0f;
+                gv[r] = run;
+            }
         }
+        if (core)
 #pragma unroll
-        for (int r = 0; r < LEN; ++r)
-            sG[(part * LEN + r) * D + c] = gv[r];
+            for (int r = 0; r < LEN; ++r)
+                sG[(part * LEN + r) * D + c] = gv[r];
         __syncthreads();
         float off = 0.0f;
-        for (int p = 0; p < part; ++p)
+        for (int p = 0; p < part && core; ++p)
             off += sG[(p * LEN + LEN - 1) * D + c];
         __syncthreads();
-        if (part > 0)
+        if (core && part > 0)
 #pragma unroll
             for (int r = 0; r < LEN; ++r)
                 sG[(part * LEN + r) * D + c] = gv[r] + off;
@@ -426,7 +435,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
         for (int s = 0; s < kDiagSlots; ++s) {
             const int p = (tid & 63) + 64 * s;
-            if (p < kDiagPairs) {
+            if (tid < kCoreThreads && p < kDiagPairs) {
                 int r, j;
                 diag_pair(p, r, j);
                 const int tr = I * kTile + r, tj = I * kTile + j;
@@ -516,7 +525,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     //       goes over G, which is no longer needed; P (bf16, lower) to its operand slot.
     //       Unbounded gate: off-diagonal tiles only (the diagonal ones come from step 3a).
     constexpr int kTilePairs = kLogSig ? kTiles * (kTiles - 1) / 2 : kTiles * (kTiles + 1) / 2;
-    for (int pidx = warp; pidx < kTilePairs; pidx += kPrepThreads / 32) {
+    for (int pidx = warp; pidx < kTilePairs; pidx += kPrepWarps) {
         int I = kLogSig ? 1 : 0, J = pidx;
         while (kLogSig ? J >= I : J > I) {  // pidx -> (I, J): 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) ...
             J -= kLogSig ? I : I + 1;       //   or, off-diagonal only: 0:(1,0) 1:(2,0) 2:(2,1) ...
@@ -577,7 +586,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
         for (int s = 0; s < kDiagSlots; ++s) {
             const int p = (tid & 63) + 64 * s;
-            if (p < kDiagPairs) {
+            if (tid < kCoreThreads && p < kDiagPairs) {
                 int r, j;
                 diag_pair(p, r, j);
                 const int tr = I * kTile + r, tj = I * kTile + j;
@@ -594,12 +603,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     __syncthreads();
 
-    // -- 4b/5. warps 4..7: chunk-referenced operands in place (Kbar = Kr e^{G_m},
+    // -- 4b/5. warps 4 and up: chunk-referenced operands in place (Kbar = Kr e^{G_m},
     //         Qbar = Qr e^{G_m}, Khat = Ec e^{G_last - G_m}); at the same time warps 0..3
     //         start T = (I + A)^{-1} with the 16x16 diagonal blocks (forward substitution,
     //         one lane per column).  Then block substitution level by level.
-    if (warp >= kPrepThreads / 64) {
-        for (int i = tid - kPrepThreads / 2; i < kC * CPR; i += kPrepThreads / 2) {
+    if (warp >= kTiles) {
+        for (int i = tid - kTiles * 32; i < kC * CPR; i += kPrepThreads - kTiles * 32) {
             const int r = i / CPR, c8 = (i % CPR) * 8;
             const int tile = r / kTile;
             const uint32_t d = tok_off(r, c8);
@@ -667,7 +676,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     phase ^= 1;
     tc::fence_after_sync();
     // [W | Utilde] (chunk rows 0..63 = TMEM lanes 0..63) -> bf16 token-major operand over G
-    if ((warp & 3) < 2) {
+    if (warp < 8 && (warp & 3) < 2) {
         const int r = (warp & 3) * 32 + lane;
         const int cbase = (warp >> 2) * D;  // warps 0,1: W; warps 4,5: Utilde
 #pragma unroll
@@ -734,7 +743,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     // Khat^T X epilogues: row i (key channel) = TMEM lane i; warp w reads the lanes of
     // quarter w % 4 and half w / 4 of the columns.  P X epilogues: chunk row r = lane r < 64.
-    const bool kt_rows = (warp & 3) * 32 < D, p_rows = (warp & 3) < 2;
+    const bool kt_rows = warp < 8 && (warp & 3) * 32 < D, p_rows = warp < 8 && (warp & 3) < 2;
     const int lrow = (warp & 3) * 32 + lane, chalf = (warp >> 2) * (D / 2);
 
     // U1 -> N over [Kbar | V]

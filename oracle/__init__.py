@@ -75,6 +75,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.oracle_decode.restype = _I
     lib.oracle_tile_factors_f32.argtypes = [_P, _P, _I, _I, _I, _P, _P]
     lib.oracle_tile_factors_f32.restype = _I
+    lib.oracle_gate_heads_f32.argtypes = [_P, _L, _I, _I, _D, _P, _P]
+    lib.oracle_gate_heads_f32.restype = None
     return lib
 
 
@@ -110,6 +112,17 @@ def gate_f64(a, g_min: float = -5.0, kind: int = GATE_BOUNDED, lib=None) -> np.n
     a = _f32(a)
     g = np.empty(a.shape, np.float64)
     _get(lib).oracle_gate_f64(_ptr(a), a.size, float(g_min), int(kind), _ptr(g))
+    return g
+
+
+def gate_heads(a, A_log, g_min: float = -5.0, lib=None) -> np.ndarray:
+    """g = g_min * sigmoid(e^{A_log[h]} * a) for a [..., H, dk] (fp64, rounded once)."""
+    a = _f32(a)
+    A_log = _f32(A_log)
+    H, dk = a.shape[-2], a.shape[-1]
+    assert A_log.shape == (H,), "A_log is one value per head"
+    g = np.empty(a.shape, np.float32)
+    _get(lib).oracle_gate_heads_f32(_ptr(a), a.size // (H * dk), H, dk, float(g_min), _ptr(A_log), _ptr(g))
     return g
 
 

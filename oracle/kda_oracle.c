@@ -72,6 +72,23 @@ void oracle_gate_f32(const float *a, int64_t n, double g_min, int kind, float *g
         g[i] = (float)gate_f64((double)a[i], g_min, kind);
 }
 
+/* Gate with a per-head scale on the pre-activation.  "Trillion-Scale ..." section 3.2
+ * writes the bounded gate as g = g_min * Sigmoid(e^A * h * z): the argument of the sigmoid
+ * is the projection h * z (the caller's `a`) scaled by e^A, one A per head.  a is
+ * [n_tok, H, dk] flattened, A_log is [H]; evaluated in fp64 and rounded once.            */
+void oracle_gate_heads_f32(const float *a, int64_t n_tok, int H, int dk, double g_min, const float *A_log,
+                           float *g)
+{
+    for (int64_t t = 0; t < n_tok; ++t)
+        for (int h = 0; h < H; ++h) {
+            const double scale = exp((double)A_log[h]);
+            for (int c = 0; c < dk; ++c) {
+                const int64_t i = (t * H + h) * dk + c;
+                g[i] = (float)gate_f64((double)a[i] * scale, g_min, ORACLE_GATE_BOUNDED);
+            }
+        }
+}
+
 /* ------------------------------------------------------------------------------ */
 /* Work distribution over independent (b, h) sequences.                           */
 typedef struct {

@@ -294,6 +294,22 @@ def pin_range_claim(lib):
     assert bad > 0
 
 
+def pin_gate_head_scale(lib):
+    """g_min * sigmoid(e^A * a) per head ("Trillion-Scale ..." 3.2): A = 0 is the plain gate
+    bit for bit; other A against scipy's expit of the scaled argument (within one float32
+    ulp: e^{log s} is s only to double rounding)."""
+    rng = np.random.default_rng(77)
+    a = (rng.standard_normal((5, 3, 16)) * 3).astype(np.float32)
+    g0 = oracle.gate_heads(a, np.zeros(3, np.float32), G_MIN, lib=lib)
+    assert np.array_equal(g0, oracle.gate(a, G_MIN, lib=lib))
+    A_log = np.array([np.log(0.5), 0.0, np.log(3.0)], np.float32)
+    g = oracle.gate_heads(a, A_log, G_MIN, lib=lib).astype(np.float64)
+    scale = np.exp(A_log.astype(np.float64))[None, :, None]
+    ref = (G_MIN * scipy.special.expit(a.astype(np.float64) * scale)).astype(np.float32).astype(np.float64)
+    assert np.all(np.abs(g - ref) <= np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)), \
+        "per-head scaled gate differs from g_min*expit(e^A a)"
+
+
 ALL_PINS = [
     pin_gate_special_values,
     pin_gate_vs_library,
@@ -309,4 +325,5 @@ ALL_PINS = [
     pin_segment_carry,
     pin_decode_step,
     pin_range_claim,
+    pin_gate_head_scale,
 ]

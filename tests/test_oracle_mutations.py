@@ -40,6 +40,9 @@ MUTATIONS = [
     ("chunk_pair_transposed", [("exp(G[(int64_t)r * dk + c] - G[(int64_t)s * dk + c]);\n                    A_rs",
                                 "exp(G[(int64_t)s * dk + c] - G[(int64_t)r * dk + c]);\n                    A_rs", 0)]),
     ("tile_col_factor_sign", [("expf(Gf - Gr);", "expf(Gr - Gf);", 0)]),
+    ("head_scale_ignored", [("const double scale = exp((double)A_log[h]);", "const double scale = 1.0;", 0)]),
+    ("head_scale_wrong_head", [("const double scale = exp((double)A_log[h]);",
+                                "const double scale = exp((double)A_log[0]);", 0)]),
 ]
 
 

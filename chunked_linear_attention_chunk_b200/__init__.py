@@ -54,6 +54,7 @@ EXPORTS = (
     "kda_selftest_device_timeout",
     "kda_chunk_fwd_varlen_workspace",
     "kda_chunk_fwd_varlen",
+    "kda_gate_fwd_heads",
 )
 
 
@@ -97,7 +98,7 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_fwd_noalloc_max_scratch.restype = S
     L.kda_chunk_fwd_logsigmoid.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, S, P]
     L.kda_chunk_fwd_logsigmoid.restype = I
-    L.kda_chunk_fwd_prep.argtypes = [I, I, I, I, I, I, F, P, P, P, P, P, P, S, P]
+    L.kda_chunk_fwd_prep.argtypes = [I, I, I, I, I, I, F, P, P, P, P, P, P, P, S, P]
     L.kda_chunk_fwd_prep.restype = I
     L.kda_chunk_fwd_scan.argtypes = [I, I, I, I, I, P, S, P, P, P, P]
     L.kda_chunk_fwd_scan.restype = I
@@ -105,7 +106,9 @@ def lib() -> ctypes.CDLL:
     L.kda_selftest_device_timeout.restype = I
     L.kda_chunk_fwd_varlen_workspace.argtypes = [I, I, I, I, I, I]
     L.kda_chunk_fwd_varlen_workspace.restype = S
-    L.kda_chunk_fwd_varlen.argtypes = [I, P, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_fwd_varlen.argtypes = [I, P, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_gate_fwd_heads.argtypes = [P, I, F, P, L64, I, I, P, P]
+    L.kda_gate_fwd_heads.restype = I
     L.kda_chunk_fwd_varlen.restype = I
     _lib = L
     return L
@@ -148,6 +151,19 @@ def kda_gate_fwd(a: torch.Tensor, g_min: float = -5.0, out: torch.Tensor | None 
     g = out if out is not None else torch.empty(a.shape, dtype=torch.float32, device=a.device)
     st = lib().kda_gate_fwd(_ptr(a), _dtype_code(a), float(g_min), _ptr(g), a.numel(), _stream(a.device))
     _raise(st, "kda_gate_fwd")
+    return g
+
+
+def kda_gate_fwd_heads(a: torch.Tensor, A_log: torch.Tensor, g_min: float = -5.0, out=None) -> torch.Tensor:
+    """g = g_min * sigmoid(e^{A_log[h]} * a) for a [..., H, dk] (fp64 evaluation, one rounding)."""
+    _check_cuda(a, A_log, out)
+    H, dk = a.shape[-2], a.shape[-1]
+    if A_log.dtype != torch.float32 or A_log.shape != (H,):
+        raise ValueError("A_log must be float32 [H]")
+    g = out if out is not None else torch.empty(a.shape, dtype=torch.float32, device=a.device)
+    st = lib().kda_gate_fwd_heads(_ptr(a), _dtype_code(a), float(g_min), _ptr(A_log), a.numel() // (H * dk), H, dk,
+                                  _ptr(g), _stream(a.device))
+    _raise(st, "kda_gate_fwd_heads")
     return g
 
 
@@ -219,11 +235,11 @@ def kda_chunk_fwd_varlen_workspace(N: int, T: int, H: int, dk: int, dv: int, dty
 
 
 def kda_chunk_fwd_varlen(q, k, v, a, beta, cu_seqlens, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED,
-                         S0=None, o=None, S_T=None, workspace=None, return_state: bool = True):
+                         S0=None, o=None, S_T=None, workspace=None, return_state: bool = True, A_log=None):
     """Chunked forward over a packed batch: q, k, a [T,H,dk]; v [T,H,dv]; beta [T,H] (bf16);
     cu_seqlens int32 [N+1] on the device (sequence s = tokens cu[s]..cu[s+1]-1).  S0 / S_T
     are [N,H,dk,dv] float32.  Returns (o [T,H,dv], S_T)."""
-    _check_cuda(q, k, v, a, beta, cu_seqlens, S0, o, S_T, workspace)
+    _check_cuda(q, k, v, a, beta, cu_seqlens, S0, o, S_T, workspace, A_log)
     if q.dim() == 4 and q.shape[0] == 1:
         q, k, v, a, beta = (t[0] for t in (q, k, v, a, beta))
     T, H, dk = q.shape
@@ -240,23 +256,27 @@ def kda_chunk_fwd_varlen(q, k, v, a, beta, cu_seqlens, g_min: float = -5.0, gate
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().kda_chunk_fwd_varlen(N, _ptr(cu_seqlens), T, H, dk, dv, code, int(gate), float(g_min), _ptr(q),
+    st = lib().kda_chunk_fwd_varlen(N, _ptr(cu_seqlens), T, H, dk, dv, code, int(gate), float(g_min), _ptr(A_log),
+                                    _ptr(q),
                                     _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
                                     _ptr(workspace), ws_bytes, _stream(q.device))
     _raise(st, "kda_chunk_fwd_varlen")
     return o, S_T
 
 
-def kda_chunk_fwd_prep(q, k, v, a, beta, workspace, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED):
+def kda_chunk_fwd_prep(q, k, v, a, beta, workspace, g_min: float = -5.0, gate: int = KDA_GATE_BOUNDED,
+                       A_log=None):
     """First stage of the bf16 chunked forward: one record per (batch*head, chunk) into
-    ``workspace`` (uint8, at least ``kda_chunk_fwd_workspace`` bytes)."""
-    _check_cuda(q, k, v, a, beta, workspace)
+    ``workspace`` (uint8, at least ``kda_chunk_fwd_workspace`` bytes).  ``A_log`` (float32
+    [H], optional) scales the gate's argument by e^{A_log[h]}."""
+    _check_cuda(q, k, v, a, beta, workspace, A_log)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if q.dtype != torch.bfloat16 or any(t.dtype != torch.bfloat16 for t in (k, v, a, beta)):
         raise TypeError("kda_chunk_fwd_prep takes bfloat16 tensors")
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = lib().kda_chunk_fwd_prep(B, T, H, dk, dv, int(gate), float(g_min), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+    st = lib().kda_chunk_fwd_prep(B, T, H, dk, dv, int(gate), float(g_min), _ptr(A_log), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(a),
                                   _ptr(beta), _ptr(workspace), ws_bytes, _stream(q.device))
     _raise(st, "kda_chunk_fwd_prep")
 

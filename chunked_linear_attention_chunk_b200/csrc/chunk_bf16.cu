@@ -281,8 +281,8 @@ template <int D, bool kLogSig>
 __global__ void __launch_bounds__(kPrepThreads, 2)
     prep_kernel(SeqMap map, int H, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
-                const __nv_bfloat16 *__restrict__ beta, float g_min, unsigned char *__restrict__ ws,
-                unsigned int *status)
+                const __nv_bfloat16 *__restrict__ beta, float g_min, const float *__restrict__ A_log,
+                unsigned char *__restrict__ ws, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char prep_smem[];
     using L = PrepLayout<D>;
@@ -359,14 +359,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         constexpr int LEN = kC / TPC;
         const bool core = tid < kCoreThreads;
         const int c = tid % D, part = tid / D;
+        const float scale = A_log ? __expf(A_log[h]) : 1.0f;  // e^A on the gate's argument
         float gv[LEN];
         float run = 0.0f;
         if (core) {
 #pragma unroll
             for (int r = 0; r < LEN; ++r) {
                 const int t = part * LEN + r;
-                const float av =
-                    __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
+                const float av = scale * __bfloat162float(
+                                             *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
                 float g;
                 if constexpr (kLogSig)
                     g = gate_logsigmoid_fast(av);
@@ -1056,7 +1057,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 
 template <int D, bool kLogSig>
 cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, const void *k, const void *v,
-                          const void *a, const void *beta, float g_min, void *ws, cudaStream_t s)
+                          const void *a, const void *beta, float g_min, const float *A_log, void *ws, cudaStream_t s)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
@@ -1068,7 +1069,7 @@ cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, cons
     prep_kernel<D, kLogSig><<<grid, kPrepThreads, smem, s>>>(
         m, H, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-        static_cast<const __nv_bfloat16 *>(beta), g_min, static_cast<unsigned char *>(ws), status);
+        static_cast<const __nv_bfloat16 *>(beta), g_min, A_log, static_cast<unsigned char *>(ws), status);
     return cudaGetLastError();
 }
 
@@ -1089,13 +1090,14 @@ cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S
 }
 
 cudaError_t launch_prep(const SeqMap &m, int H, int D, dim3 grid, const void *q, const void *k, const void *v,
-                        const void *a, const void *beta, float g_min, bool logsigmoid, void *ws, cudaStream_t s)
+                        const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log, void *ws,
+                        cudaStream_t s)
 {
     if (logsigmoid)
-        return D == 64 ? launch_prep_d<64, true>(m, H, grid, q, k, v, a, beta, g_min, ws, s)
-                       : launch_prep_d<128, true>(m, H, grid, q, k, v, a, beta, g_min, ws, s);
-    return D == 64 ? launch_prep_d<64, false>(m, H, grid, q, k, v, a, beta, g_min, ws, s)
-                   : launch_prep_d<128, false>(m, H, grid, q, k, v, a, beta, g_min, ws, s);
+        return D == 64 ? launch_prep_d<64, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s)
+                       : launch_prep_d<128, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s);
+    return D == 64 ? launch_prep_d<64, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s)
+                   : launch_prep_d<128, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s);
 }
 
 cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const float *S0, void *o, float *S_T,
@@ -1170,11 +1172,11 @@ size_t chunk_bf16_workspace(int B, int T, int H, int D)
 }
 
 cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                             const void *a, const void *beta, float g_min, bool logsigmoid, void *workspace,
-                             cudaStream_t s)
+                             const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log,
+                             void *workspace, cudaStream_t s)
 {
     const SeqMap m = regular_map(B, T);
-    return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, workspace, s);
+    return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, s);
 }
 
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
@@ -1192,7 +1194,8 @@ size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D)
 
 cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
                                      const void *v, const void *a, const void *beta, float g_min, bool logsigmoid,
-                                     const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s)
+                                     const float *A_log, const float *S0, void *o, float *S_T, void *workspace,
+                                     cudaStream_t s)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
@@ -1209,7 +1212,7 @@ cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    e = launch_prep(m, H, D, dim3(m.NT, H), q, k, v, a, beta, g_min, logsigmoid, workspace, s);
+    e = launch_prep(m, H, D, dim3(m.NT, H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, s);
     if (e != cudaSuccess)
         return e;
     return launch_scan(m, H, D, workspace, S0, o, S_T, s);

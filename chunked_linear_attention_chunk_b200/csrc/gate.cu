@@ -72,6 +72,49 @@ __global__ void __launch_bounds__(256) gate_kernel(const Tin *__restrict__ a, in
     }
 }
 
+// Per-head scaled form g = g_min * sigmoid(e^{A_h} a) on a [n_tok, H, dk] layout: the
+// argument a * e^{A_h} is formed in float64 too, so the result is still one rounding from
+// the fp64 value.  dk is a multiple of the vector width, so a vector never spans two heads.
+template <typename Tin>
+__global__ void __launch_bounds__(256) gate_heads_kernel(const Tin *__restrict__ a, int64_t nvec, int H, int dk,
+                                                         const float *__restrict__ A_log, double g_min,
+                                                         float *__restrict__ g)
+{
+    constexpr int V = GateVec<Tin>::kPerVec;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+        const int head = (int)(((i * V) / dk) % H);
+        const double scale = exp((double)A_log[head]);
+        float x[V];
+        GateVec<Tin>::load(a + i * V, x);
+        float y[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+            y[j] = __double2float_rn(g_min / (1.0 + exp(-((double)x[j] * scale))));
+        float4 *out = reinterpret_cast<float4 *>(g + i * V);
+#pragma unroll
+        for (int j = 0; j < V / 4; ++j)
+            __stcs(out + j, make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]));
+    }
+}
+
+cudaError_t launch_gate_heads(const void *a, kda_dtype dt, double g_min, const float *A_log, int64_t n_tok, int H,
+                              int dk, float *g, cudaStream_t s)
+{
+    const int per = dt == KDA_BF16 ? 8 : 4;
+    const int64_t nvec = n_tok * H * dk / per;
+    int64_t blocks = (nvec + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    blocks = blocks > cap ? cap : (blocks < 1 ? 1 : blocks);
+    if (dt == KDA_BF16)
+        gate_heads_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(a), nvec, H, dk, A_log, g_min, g);
+    else
+        gate_heads_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float *>(a), nvec, H, dk,
+                                                                   A_log, g_min, g);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gate(const void *a, kda_dtype dt, double g_min, float *g, int64_t n, cudaStream_t s)
 {
     const int per = dt == KDA_BF16 ? 8 : 4;

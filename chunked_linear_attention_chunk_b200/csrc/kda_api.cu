@@ -135,6 +135,31 @@ kda_status kda_gate_fwd(const void *a, kda_dtype a_dtype, float g_min, float *g,
     return from_cuda(launch_gate(a, a_dtype, (double)g_min, g, n, (cudaStream_t)stream));
 }
 
+kda_status kda_gate_fwd_heads(const void *a, kda_dtype a_dtype, float g_min, const float *A_log, int64_t n_tok,
+                              int H, int dk, float *g, kda_stream_t stream)
+{
+    if (!dtype_ok(a_dtype) || n_tok < 0 || H < 1 || dk < 1)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    if (dk % 8 != 0)
+        return KDA_ERR_UNSUPPORTED;
+    const int64_t n = safe_prod({n_tok, H, dk});
+    if (n < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (n == 0)
+        return KDA_OK;
+    if (!a || !g || !A_log)
+        return KDA_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(g) || ((uintptr_t)A_log & 3u))
+        return KDA_ERR_ALIGNMENT;
+    const Range rg(g, n * 4);
+    if (overlaps(rg, Range(a, n * elem_size(a_dtype))) || overlaps(rg, Range(A_log, (int64_t)H * 4)))
+        return KDA_ERR_ALIAS;
+    return from_cuda(launch_gate_heads(a, a_dtype, (double)g_min, A_log, n_tok, H, dk, g, (cudaStream_t)stream));
+}
+
 size_t kda_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype)
 {
     if (B < 1 || H < 1 || T < 0 || dk != dv || (dk != 64 && dk != 128) || !dtype_ok(dtype))
@@ -289,7 +314,8 @@ kda_status chunk_fwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, 
                                           static_cast<const float *>(v), static_cast<const float *>(a),
                                           static_cast<const float *>(beta), g_min, S0, static_cast<float *>(o), S_T,
                                           s));
-    st = from_cuda(launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, workspace, s));
+    st = from_cuda(
+        launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, nullptr, workspace, s));
     if (st != KDA_OK)
         return st;
     return from_cuda(launch_scan_bf16(B, T, H, dk, workspace, S0, o, S_T, s));
@@ -323,9 +349,9 @@ size_t kda_chunk_fwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_d
 }
 
 kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
-                                kda_gate gate, float g_min, const void *q, const void *k, const void *v,
-                                const void *a, const void *beta, const float *S0, void *o, float *S_T,
-                                void *workspace, size_t ws_bytes, kda_stream_t stream)
+                                kda_gate gate, float g_min, const float *A_log, const void *q, const void *k,
+                                const void *v, const void *a, const void *beta, const float *S0, void *o,
+                                float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream)
 {
     if (!dtype_ok(dtype) || N < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
         return KDA_ERR_INVALID_ARG;
@@ -337,33 +363,34 @@ kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
     const int64_t nk = (int64_t)T * H * dk, ntok = (int64_t)T * H, ns = (int64_t)N * H * dk * dv;
     if (!cu_seqlens || (T > 0 && (!q || !k || !v || !a || !beta || !o)))
         return KDA_ERR_INVALID_ARG;
-    if (!all_aligned({q, k, v, a, beta, S0, o, S_T, workspace}) || ((uintptr_t)cu_seqlens & 3u))
+    if (!all_aligned({q, k, v, a, beta, S0, o, S_T, workspace}) || ((uintptr_t)cu_seqlens & 3u) ||
+        ((uintptr_t)A_log & 3u))
         return KDA_ERR_ALIGNMENT;
     const size_t need = kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, dtype);
     if (!workspace || ws_bytes < need)
         return KDA_ERR_WORKSPACE;
     const Range rq(q, nk * 2), rk(k, nk * 2), rv(v, nk * 2), ra(a, nk * 2), rb(beta, ntok * 2),
         rcu(cu_seqlens, (int64_t)(N + 1) * 4), rS0(S0, ns * 4), ro(T > 0 ? o : nullptr, nk * 2), rST(S_T, ns * 4),
-        rws(workspace, (int64_t)need);
-    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rS0, rST, rws})
+        rws(workspace, (int64_t)need), rA(A_log, (int64_t)H * 4);
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rA, rS0, rST, rws})
         if (overlaps(ro, in))
             return KDA_ERR_ALIAS;
-    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rws})
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rA, rws})
         if (overlaps(rST, in))
             return KDA_ERR_ALIAS;
     if (overlaps(rST, rS0) && S_T != S0)
         return KDA_ERR_ALIAS;
-    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rS0})
+    for (const Range &in : {rq, rk, rv, ra, rb, rcu, rA, rS0})
         if (overlaps(rws, in))
             return KDA_ERR_ALIAS;
     return from_cuda(launch_chunk_bf16_varlen(N, cu_seqlens, T, H, dk, q, k, v, a, beta, g_min,
-                                              gate == KDA_GATE_LOGSIGMOID, S0, o, S_T, workspace,
+                                              gate == KDA_GATE_LOGSIGMOID, A_log, S0, o, S_T, workspace,
                                               (cudaStream_t)stream));
 }
 
-kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const void *q,
-                              const void *k, const void *v, const void *a, const void *beta, void *workspace,
-                              size_t ws_bytes, kda_stream_t stream)
+kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const float *A_log,
+                              const void *q, const void *k, const void *v, const void *a, const void *beta,
+                              void *workspace, size_t ws_bytes, kda_stream_t stream)
 {
     ChunkShape sh;
     kda_status st = check_shape(B, T, H, dk, dv, KDA_BF16, sh);
@@ -371,10 +398,14 @@ kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate
         st = check_gate(gate, g_min, KDA_BF16);
     if (st == KDA_OK)
         st = check_prep_args(sh, q, k, v, a, beta, workspace, ws_bytes);
+    if (st == KDA_OK && ((uintptr_t)A_log & 3u))
+        st = KDA_ERR_ALIGNMENT;
+    if (st == KDA_OK && sh.ws > 0 && overlaps(Range(workspace, (int64_t)sh.ws), Range(A_log, (int64_t)H * 4)))
+        st = KDA_ERR_ALIAS;
     if (st != KDA_OK || T == 0)
         return st;
-    return from_cuda(launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, workspace,
-                                      (cudaStream_t)stream));
+    return from_cuda(launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, A_log,
+                                      workspace, (cudaStream_t)stream));
 }
 
 kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,

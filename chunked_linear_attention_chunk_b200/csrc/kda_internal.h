@@ -16,6 +16,8 @@ unsigned int *device_status_ptr();
 
 // K1: g = g_min * sigmoid(a), fp64-exact, n elements.
 cudaError_t launch_gate(const void *a, kda_dtype dt, double g_min, float *g, int64_t n, cudaStream_t s);
+cudaError_t launch_gate_heads(const void *a, kda_dtype dt, double g_min, const float *A_log, int64_t n_tok, int H,
+                              int dk, float *g, cudaStream_t s);
 
 // K5: float32 CUDA-core chunked forward (16-token chunks).
 cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const float *k, const float *v,
@@ -24,11 +26,12 @@ cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const f
 
 // K2 + K3: bfloat16 tensor-core chunked forward.  The prep writes one record per (b*h,
 // chunk) into the workspace; the scan walks them.  `logsigmoid` selects the unbounded gate
-// g = log sigmoid(a) with element-wise diagonal tiles (g_min is then not used).
+// g = log sigmoid(a) with element-wise diagonal tiles (g_min is then not used).  A_log
+// (nullable, [H]) scales the gate's argument by e^{A_log[h]}.
 size_t chunk_bf16_workspace(int B, int T, int H, int D);
 cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                             const void *a, const void *beta, float g_min, bool logsigmoid, void *workspace,
-                             cudaStream_t s);
+                             const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log,
+                             void *workspace, cudaStream_t s);
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
                              float *S_T, cudaStream_t s);
 
@@ -38,7 +41,8 @@ cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, 
 size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D);
 cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
                                      const void *v, const void *a, const void *beta, float g_min, bool logsigmoid,
-                                     const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s);
+                                     const float *A_log, const float *S0, void *o, float *S_T, void *workspace,
+                                     cudaStream_t s);
 
 // K4: single-token decode step.
 cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,

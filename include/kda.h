@@ -96,6 +96,21 @@ kda_status kda_gate_fwd(const void *a, kda_dtype a_dtype, float g_min, float *g,
                         kda_stream_t stream);
 
 /*
+ * kda_gate_fwd_heads -- the gate with a per-head scale on its argument:
+ *     g[t, h, c] = g_min * sigmoid(e^{A_log[h]} * a[t, h, c])
+ * Passage: "Trillion-Scale ..." section 3.2 (g = g_min * Sigmoid(e^A * h * z), with `a`
+ * the projection h * z and one A per head).
+ *   a        device, [n_tok, H, dk] of a_dtype (bf16 or f32); dk a multiple of 8.
+ *   A_log    device, H float32 values (4-byte aligned).
+ *   g        device, [n_tok, H, dk] float32.  The scaled argument and the gate are
+ *            evaluated in float64 and rounded once, as in kda_gate_fwd.
+ * Errors: INVALID_ARG, UNSUPPORTED (dk not a multiple of 8, g_min range), ALIGNMENT,
+ * ALIAS (g overlaps a or A_log), CUDA.
+ */
+kda_status kda_gate_fwd_heads(const void *a, kda_dtype a_dtype, float g_min, const float *A_log, int64_t n_tok,
+                              int H, int dk, float *g, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_workspace -- bytes of device scratch kda_chunk_fwd needs for this
  * shape (0 when none).  Pure host computation; never fails (returns 0 for invalid
  * shapes, which kda_chunk_fwd then rejects).
@@ -169,7 +184,7 @@ kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dty
  *                word (kda_device_status), writes no o, and S_T gets S0 (or zeros).
  *   T            tokens on the packed axis (0 .. 2^31 - 65).
  *   dk, dv       dk == dv in {64, 128}; dtype must be KDA_BF16.
- *   gate, g_min  as in kda_chunk_fwd_prep.
+ *   gate, g_min, A_log  as in kda_chunk_fwd_prep.
  *   q, k, a      [T, H, dk];  v, o: [T, H, dv];  beta: [T, H]   (bfloat16)
  *   S0, S_T      [N, H, dk, dv] float32, or NULL (zeros / not stored); S_T may be S0.
  *   workspace    >= kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, dtype) bytes (records
@@ -178,9 +193,9 @@ kda_status kda_chunk_fwd_logsigmoid(int B, int T, int H, int dk, int dv, kda_dty
  */
 size_t kda_chunk_fwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype);
 kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
-                                kda_gate gate, float g_min, const void *q, const void *k, const void *v,
-                                const void *a, const void *beta, const float *S0, void *o, float *S_T,
-                                void *workspace, size_t ws_bytes, kda_stream_t stream);
+                                kda_gate gate, float g_min, const float *A_log, const void *q, const void *k,
+                                const void *v, const void *a, const void *beta, const float *S0, void *o,
+                                float *S_T, void *workspace, size_t ws_bytes, kda_stream_t stream);
 
 /*
  * kda_chunk_fwd_prep, kda_chunk_fwd_scan -- the two stages of the bfloat16 kda_chunk_fwd
@@ -194,6 +209,10 @@ kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
  * record per (batch*head, chunk) into `workspace`.  All chunks are independent.
  *   gate, g_min  KDA_GATE_BOUNDED with g_min as in kda_chunk_fwd, or KDA_GATE_LOGSIGMOID
  *                (g_min unused) as in kda_chunk_fwd_logsigmoid.
+ *   A_log        NULL, or a DEVICE array of H float32 values (4-byte aligned): the gate's
+ *                argument becomes e^{A_log[h]} * a, the per-head scale of g = g_min *
+ *                Sigmoid(e^A * h * z) ("Trillion-Scale ..." section 3.2; `a` is the
+ *                projection h * z), fused here instead of a separate pass over a.
  *   q, k, v, a, beta, workspace, ws_bytes: as in kda_chunk_fwd, bfloat16 only.
  *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS (workspace overlaps an input),
  *   WORKSPACE, CUDA.  T == 0 does nothing.
@@ -208,9 +227,9 @@ kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
  *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.  T == 0 copies S0
  *   (or zeros) to S_T.
  */
-kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const void *q,
-                              const void *k, const void *v, const void *a, const void *beta, void *workspace,
-                              size_t ws_bytes, kda_stream_t stream);
+kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const float *A_log,
+                              const void *q, const void *k, const void *v, const void *a, const void *beta,
+                              void *workspace, size_t ws_bytes, kda_stream_t stream);
 kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
                               const float *S0, void *o, float *S_T, kda_stream_t stream);
 

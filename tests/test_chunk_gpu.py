@@ -194,3 +194,57 @@ def test_prep_then_scan_equals_one_call_bitwise(gate):
     torch.cuda.synchronize()
     assert kda.kda_device_status() == 0
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def _scaled_a(a, A_log):
+    """The gate's argument e^{A_h} a, formed in fp64 and rounded to float32, for the oracle."""
+    x = a.double() * torch.exp(A_log.double())[None, None, :, None]
+    return x.float()
+
+
+def test_head_scaled_gate_matches_oracle():
+    """A_log fused into the prep: the oracle runs the plain gate on e^{A_h} a."""
+    B, T, H, D = 1, 200, 3, 128
+    x = synth.make_inputs(B, T, H, D, D, "bf16", seed=960, s0_std=0.1)
+    A_log = torch.tensor([-0.7, 0.0, 0.9], dtype=torch.float32)
+    d = to_dev(x)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace(B, T, H, D, D), dtype=torch.uint8, device="cuda")
+    kda.kda_chunk_fwd_prep(*(d[n] for n in NAMES), ws, G_MIN, kda.KDA_GATE_BOUNDED, A_log=A_log.cuda())
+    o, ST = kda.kda_chunk_fwd_scan(ws, B, T, H, D, D, S0=d["S0"])
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    xs = dict(x)
+    xs["a"] = _scaled_a(x["a"].float(), A_log)
+    o_ref, S_ref = oracle_run(xs, x["S0"])
+    eo, es = err_o(o.float().cpu().numpy(), o_ref), err_s(ST.cpu().numpy(), S_ref)
+    assert eo <= TOL_BF16_O and es <= TOL_BF16_S, (eo, es)
+    # A_log = 0 is the plain call, bit for bit
+    ws.zero_()
+    kda.kda_chunk_fwd_prep(*(d[n] for n in NAMES), ws, G_MIN, kda.KDA_GATE_BOUNDED,
+                           A_log=torch.zeros(H, device="cuda"))
+    o0, S0_ = kda.kda_chunk_fwd_scan(ws, B, T, H, D, D, S0=d["S0"])
+    o1, S1 = kda.kda_chunk_fwd(*(d[n] for n in NAMES), G_MIN, S0=d["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o0, o1) and torch.equal(S0_, S1)
+
+
+def test_head_scaled_gate_packed_batch():
+    lengths = [90, 0, 130]
+    T, H, D = sum(lengths), 2, 64
+    x = synth.make_inputs(1, T, H, D, D, "bf16", seed=961, s0_std=0.0)
+    S0 = synth.make_inputs(len(lengths), 1, H, D, D, "bf16", seed=962, s0_std=0.1)["S0"]
+    A_log = torch.tensor([0.4, -0.3], dtype=torch.float32)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    d = to_dev(x)
+    o, ST = kda.kda_chunk_fwd_varlen(*(d[n][0] for n in NAMES), cu.cuda(), G_MIN, S0=S0.cuda(), A_log=A_log.cuda())
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    o, ST = o.float().cpu().numpy(), ST.cpu().numpy()
+    for s_, (a0, b0) in enumerate(zip(cu[:-1].tolist(), cu[1:].tolist())):
+        if b0 == a0:
+            continue
+        xs = {n: x[n][:, a0:b0] for n in NAMES}
+        xs["a"] = _scaled_a(xs["a"].float(), A_log)
+        o_ref, S_ref = oracle_run(xs, S0[s_:s_ + 1])
+        eo, es = err_o(o[None, a0:b0], o_ref), err_s(ST[s_:s_ + 1], S_ref)
+        assert eo <= TOL_BF16_O and es <= TOL_BF16_S, (s_, eo, es)

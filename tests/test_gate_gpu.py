@@ -63,3 +63,15 @@ def test_gate_writes_nothing_past_n():
     out = torch.full((32,), 7.0, device="cuda")
     kda.kda_gate_fwd(a, -5.0, out=out[:13])
     assert (out[13:] == 7.0).all()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gate_heads_bit_exact(dtype):
+    """g_min * sigmoid(e^{A_h} a) per head, bit-exact against the fp64 oracle."""
+    gen = torch.Generator().manual_seed(31)
+    a = (torch.randn(37, 6, 128, generator=gen) * 3).to(dtype)
+    A_log = torch.randn(6, generator=gen) * 0.7
+    g = kda.kda_gate_fwd_heads(a.cuda(), A_log.cuda(), -5.0)
+    torch.cuda.synchronize()
+    ref = oracle.gate_heads(a.float().numpy(), A_log.numpy(), -5.0)
+    assert np.array_equal(g.cpu().numpy().view(np.uint32), ref.view(np.uint32))

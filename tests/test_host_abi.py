@@ -198,7 +198,7 @@ def test_prep_and_scan_entries_validate(L):
     ws = BASE + 6 * (n + 4096)
 
     def prep(gate=kda.KDA_GATE_BOUNDED, g_min=-5.0, q=ins[0], w=ws, wb=need, dk=D):
-        return L.kda_chunk_fwd_prep(B, T, H, dk, dk, gate, ctypes.c_float(g_min), P(q), P(ins[1]), P(ins[2]),
+        return L.kda_chunk_fwd_prep(B, T, H, dk, dk, gate, ctypes.c_float(g_min), None, P(q), P(ins[1]), P(ins[2]),
                                     P(ins[3]), P(ins[4]), P(w), wb, None)
 
     def scan(w=ws, wb=need, S0=None, o=BASE + 5 * (n + 4096), ST=None):
@@ -241,7 +241,7 @@ def test_varlen_entry_validates(L):
 
     def call(N=N, cu=cu, dt=kda.KDA_BF16, gate=kda.KDA_GATE_BOUNDED, g_min=-5.0, o=BASE + 5 * (n + 4096), w=ws,
              wb=ws_need, H=H):
-        return L.kda_chunk_fwd_varlen(N, P(cu), T, H, D, D, dt, gate, ctypes.c_float(g_min), *(P(p) for p in ins),
+        return L.kda_chunk_fwd_varlen(N, P(cu), T, H, D, D, dt, gate, ctypes.c_float(g_min), None, *(P(p) for p in ins),
                                       None, P(o), None, P(w), wb, None)
 
     assert call(N=0) == INVALID
@@ -262,3 +262,18 @@ def test_binding_has_a_function_for_every_export():
     missing = [n for n in kda.EXPORTS if not callable(getattr(kda, n, None))]
     assert not missing, missing
     assert set(kda.EXPORTS) == set(declared_functions())
+
+
+def test_gate_heads_validates(L):
+    P = ctypes.c_void_p
+    f = lambda a=BASE, g=BASE * 2, A=BASE * 3, n=10, H=2, dk=64, g_min=-5.0, dt=kda.KDA_BF16: \
+        L.kda_gate_fwd_heads(P(a), dt, ctypes.c_float(g_min), P(A), n, H, dk, P(g), None)
+    assert f(n=0) == OK
+    assert f(H=0) == INVALID
+    assert f(A=0) == INVALID
+    assert f(dk=12) == UNSUPPORTED
+    assert f(g_min=-7.0) == UNSUPPORTED
+    assert f(a=BASE + 8) == ALIGN
+    assert f(A=BASE * 3 + 2) == ALIGN
+    assert f(g=BASE + 64) == ALIAS
+    assert f(A=BASE * 2 + 16) == ALIAS

@@ -345,6 +345,27 @@ def run_libkda(args):
               "roofline_path_frac": (token_heads * BYTES_PER_TOKEN_HEAD + 2 * Nd * H * D * D * 4) / (vl_ms * 1e-3)
               / 1e9 / hbm_peak}
 
+    # ---- sequence parallel: one 64K sequence split into world consecutive segments, one per
+    # rank (the same seeded sequence on every rank; rank r takes its slice)
+    spl = None
+    if args.only != "decode" and not args.no_sp and B == 1 and T % world == 0:
+        from chunked_linear_attention_chunk_b200.sp import sp_chunk_fwd
+        xs = x if world == 1 else synth.make_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.seed, w.s0_std,
+                                                    w.adversarial)
+        seg = T // world
+        sd = [xs[n][:, rank * seg:(rank + 1) * seg].contiguous().to(device) for n in names]
+        S0s = xs["S0"].to(device)
+
+        def sp_step():
+            sp_chunk_fwd(*sd, S0=S0s)
+
+        sp_ms = time_steps(sp_step, max(3, min(args.steps, 10)), 3, world, device)
+        assert kda.kda_device_status(device) == 0
+        spl = {"workload": f"one {T}-token sequence in {world} segment(s) of {seg}, H={H} d={D}",
+               "ms_per_step": sp_ms, "value": tokens / (sp_ms * 1e-3), "unit": UNIT, "segments": world,
+               "gpu_launches_per_step": 4, "collectives_per_step": 2 if world > 1 else 0}
+        del sd
+
     # ---- end to end through the C ABI with pinned host buffers
     hx = {n: x[n].pin_memory() for n in names}
     hS0 = x["S0"].pin_memory()
@@ -425,6 +446,8 @@ def run_libkda(args):
         line["ablation"] = abl
     if vl is not None:
         line["varlen"] = vl
+    if spl is not None:
+        line["sequence_parallel"] = spl
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
     if rank == 0:
@@ -449,6 +472,7 @@ def main(argv=None):
     ap.add_argument("--only", choices=("all", "chunk", "decode"), default="all")
     ap.add_argument("--no-ablation", action="store_true", help="skip timing the log-sigmoid ablation path")
     ap.add_argument("--no-varlen", action="store_true", help="skip timing the packed variable-length batch")
+    ap.add_argument("--no-sp", action="store_true", help="skip timing the sequence-parallel leg")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

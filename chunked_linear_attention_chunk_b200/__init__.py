@@ -55,6 +55,8 @@ EXPORTS = (
     "kda_chunk_fwd_varlen_workspace",
     "kda_chunk_fwd_varlen",
     "kda_gate_fwd_heads",
+    "kda_chunk_fwd_scan_affine",
+    "kda_state_combine",
 )
 
 
@@ -109,6 +111,10 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_fwd_varlen.argtypes = [I, P, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, P, S, P]
     L.kda_gate_fwd_heads.argtypes = [P, I, F, P, L64, I, I, P, P]
     L.kda_gate_fwd_heads.restype = I
+    L.kda_chunk_fwd_scan_affine.argtypes = [I, I, I, I, I, P, S, P, P, P]
+    L.kda_chunk_fwd_scan_affine.restype = I
+    L.kda_state_combine.argtypes = [I, I, I, I, I, P, P, P, P, P]
+    L.kda_state_combine.restype = I
     L.kda_chunk_fwd_varlen.restype = I
     _lib = L
     return L
@@ -296,6 +302,34 @@ def kda_chunk_fwd_scan(workspace, B: int, T: int, H: int, dk: int, dv: int, S0=N
                                   _stream(dev))
     _raise(st, "kda_chunk_fwd_scan")
     return o, S_T
+
+
+def kda_chunk_fwd_scan_affine(workspace, B: int, T: int, H: int, dk: int, dv: int, S_zero=None, M=None):
+    """Affine map of the segment whose records ``workspace`` holds: returns (S_zero, M) with
+    S_out = M S_in + S_zero; S_zero [B,H,dk,dv], M [B,H,dk,dk] (float32)."""
+    _check_cuda(workspace, S_zero, M)
+    dev = workspace.device
+    if S_zero is None:
+        S_zero = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if M is None:
+        M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_scan_affine(B, T, H, dk, dv, _ptr(workspace), ws_bytes, _ptr(S_zero), _ptr(M),
+                                         _stream(dev))
+    _raise(st, "kda_chunk_fwd_scan_affine")
+    return S_zero, M
+
+
+def kda_state_combine(M, S_zero, S0=None, S_in=None):
+    """Incoming states of R consecutive segments from their maps: M, S_zero [R,B,H,d,d];
+    returns S_in [R+1,B,H,d,d] with S_in[0] = S0 (or 0) and S_in[R] the final state."""
+    _check_cuda(M, S_zero, S0, S_in)
+    R, B, H, dk, dv = S_zero.shape
+    if S_in is None:
+        S_in = torch.empty((R + 1, B, H, dk, dv), dtype=torch.float32, device=M.device)
+    st = lib().kda_state_combine(R, B, H, dk, dv, _ptr(M), _ptr(S_zero), _ptr(S0), _ptr(S_in), _stream(M.device))
+    _raise(st, "kda_state_combine")
+    return S_in
 
 
 def kda_chunk_fwd_noalloc(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=None,

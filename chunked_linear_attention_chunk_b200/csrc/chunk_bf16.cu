@@ -182,13 +182,17 @@ struct PrepLayout {
     static constexpr uint32_t RT = RG + (uint32_t)kC * (kC + 1) * 4;  // blocks hold the solve scratch
     // small tables
     static constexpr uint32_t RBeta = RG + kRGBytes;       // f32 [64]
-    static constexpr uint32_t REm = RBeta + kC * 4;        // bf16 [4][D]  e^{G_{m_I}}
-    static constexpr uint32_t REl = REm + kTiles * D * 2;  // bf16 [4][D]  e^{G_last - G_{m_I}}
-    static constexpr uint32_t RDd = REl + kTiles * D * 2;  // bf16 [6][D]  e^{G_{m_I} - G_{m_J}}
+    // scale tables as bf16 hi / lo pairs (hi [4][D], then lo [4][D]): x * (hi + lo) in two
+    // packed bf16 operations with one effective rounding
+    static constexpr uint32_t REm = RBeta + kC * 4;        // e^{G_{m_I}}
+    static constexpr uint32_t REl = REm + kTiles * D * 4;  // e^{G_last - G_{m_I}}
+    static constexpr uint32_t RDd = REl + kTiles * D * 4;  // bf16 [6][D]  e^{G_{m_I} - G_{m_J}}
     static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarriers: round 1, then units U1..U4
     static constexpr uint32_t RTmem = RBar + 5 * 8;
     static constexpr uint32_t Bytes = RTmem + 8;
     static_assert(RG % 1024 == 0 && RP % 1024 == 0, "operand alignment");
+    // two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+    static_assert(2 * (Bytes + 1024) <= 233472, "two prep CTAs fit one SM");
 };
 
 // 16-byte chunk address of (token r, channels c8..c8+7) in a token-major operand.
@@ -242,15 +246,37 @@ __device__ __forceinline__ void solve_block_tf32(const float *A, float *Tm, floa
     }
 }
 
-// Multiply 8 packed bf16 by 8 packed bf16 scalars.
-__device__ __forceinline__ uint4 mul8(uint4 x, uint4 s)
+// Multiply 8 packed bf16 x by scalars given as bf16 hi + lo: rn(x hi + rn(x lo)), which is x (hi
+// + lo) rounded once up to a 2^-17 relative term (a fused packed multiply-add after a packed
+// multiply).
+__device__ __forceinline__ uint4 mul8_hilo(uint4 x, uint4 hi, uint4 lo)
 {
-    __nv_bfloat162 *xa = reinterpret_cast<__nv_bfloat162 *>(&x);
-    const __nv_bfloat162 *sa = reinterpret_cast<const __nv_bfloat162 *>(&s);
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, hs[4] = {hi.x, hi.y, hi.z, hi.w}, ls[4] = {lo.x, lo.y, lo.z, lo.w};
+    uint32_t r[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        xa[i] = __hmul2(xa[i], sa[i]);
-    return x;
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 xv = *reinterpret_cast<const __nv_bfloat162 *>(&xs[i]);
+        const __nv_bfloat162 t = __hmul2(xv, *reinterpret_cast<const __nv_bfloat162 *>(&ls[i]));
+        const __nv_bfloat162 y = __hfma2(xv, *reinterpret_cast<const __nv_bfloat162 *>(&hs[i]), t);
+        r[i] = *reinterpret_cast<const uint32_t *>(&y);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// 8 floats (as bits) -> bf16 hi = rn(x) and lo = rn(x - hi), so hi + lo carries x to about
+// 2^-16 relative.
+__device__ __forceinline__ void pack8_hilo(const uint32_t *x, uint4 &hi, uint4 &lo)
+{
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float a = __uint_as_float(x[2 * p]), b = __uint_as_float(x[2 * p + 1]);
+        h[p] = pack_bf16x2(a, b);
+        const float2 hf = unpack_bf16x2(h[p]);
+        l[p] = pack_bf16x2(a - hf.x, b - hf.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 __device__ __forceinline__ uint4 pack8(const uint32_t *x)
@@ -301,7 +327,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     float *sA = reinterpret_cast<float *>(sm + L::RA);   // [64][65]
     float *sT = reinterpret_cast<float *>(sm + L::RT);   // [64][65]
     float *sBeta = reinterpret_cast<float *>(sm + L::RBeta);
-    __nv_bfloat16 *sEm = reinterpret_cast<__nv_bfloat16 *>(sm + L::REm);
+    __nv_bfloat16 *sEm = reinterpret_cast<__nv_bfloat16 *>(sm + L::REm);  // hi [4][D] | lo [4][D]
     __nv_bfloat16 *sEl = reinterpret_cast<__nv_bfloat16 *>(sm + L::REl);
     __nv_bfloat16 *sDd = reinterpret_cast<__nv_bfloat16 *>(sm + L::RDd);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::RBar);
@@ -413,8 +439,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     };
     for (int i = tid; i < kTiles * D; i += kPrepThreads) {
         const int I = i / D, c = i % D;
-        sEm[i] = __float2bfloat16(__expf(row_ref(I, c)));
-        sEl[i] = __float2bfloat16(__expf(sG[(kC - 1) * D + c] - col_ref(I, c)));
+        const float em = __expf(row_ref(I, c)), el = __expf(sG[(kC - 1) * D + c] - col_ref(I, c));
+        const __nv_bfloat16 emh = __float2bfloat16(em), elh = __float2bfloat16(el);
+        sEm[i] = emh;
+        sEm[kTiles * D + i] = __float2bfloat16(em - __bfloat162float(emh));
+        sEl[i] = elh;
+        sEl[kTiles * D + i] = __float2bfloat16(el - __bfloat162float(elh));
     }
     for (int i = tid; i < 6 * D; i += kPrepThreads) {
         const int p = i / D, c = i % D;
@@ -613,14 +643,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             const int r = i / CPR, c8 = (i % CPR) * 8;
             const int tile = r / kTile;
             const uint32_t d = tok_off(r, c8);
-            const uint4 em = *reinterpret_cast<const uint4 *>(&sEm[tile * D + c8]);
-            const uint4 el = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
+            const uint4 emh = *reinterpret_cast<const uint4 *>(&sEm[tile * D + c8]);
+            const uint4 eml = *reinterpret_cast<const uint4 *>(&sEm[(kTiles + tile) * D + c8]);
+            const uint4 elh = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
+            const uint4 ell = *reinterpret_cast<const uint4 *>(&sEl[(kTiles + tile) * D + c8]);
             uint4 *pk = reinterpret_cast<uint4 *>(sm + L::RK + d);
             uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + d);
             uint4 *px = reinterpret_cast<uint4 *>(sm + L::RX + d);
-            *pk = mul8(*pk, em);
-            *pq = mul8(*pq, em);
-            *px = mul8(*px, el);
+            *pk = mul8_hilo(*pk, emh, eml);
+            *pq = mul8_hilo(*pq, emh, eml);
+            *px = mul8_hilo(*px, elh, ell);
         }
     } else if (lane < kTile) {
         const int I = warp, c = lane;
@@ -648,13 +680,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                              warp, lane);
         __syncthreads();
     }
-    // T diag(beta) as the K-major A operand (over A's place; the 8 KB after it are the
-    // don't-care rows of the M = 128 MMA)
+    // T diag(beta) as the K-major A operand (over A's place), written twice: as rows 0..63
+    // and again as rows 64..127 of the M = 128 MMA, so TMEM lanes 64..127 hold a second copy
+    // of the result and all four lane quarters can drain it
     for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
         const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
         const bool upper = j / kTile > r / kTile;  // those blocks of T are zero and never written
-        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) =
+        const uint32_t tb =
             upper ? 0u : pack_bf16x2(sT[r * LDA + j] * sBeta[j], sT[r * LDA + j + 1] * sBeta[j + 1]);
+        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) = tb;
+        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(kC + r, j, kC)) = tb;
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -676,18 +711,32 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     mbar_wait_bounded(bar, phase, status);
     phase ^= 1;
     tc::fence_after_sync();
-    // [W | Utilde] (chunk rows 0..63 = TMEM lanes 0..63) -> bf16 token-major operand over G
-    if (warp < 8 && (warp & 3) < 2) {
-        const int r = (warp & 3) * 32 + lane;
-        const int cbase = (warp >> 2) * D;  // warps 0,1: W; warps 4,5: Utilde
+    // [W | Utilde] (chunk rows 0..63 = TMEM lanes 0..63) -> bf16 token-major operands over G,
+    // and the remainder Utilde - rn(Utilde) over V (no longer an operand): Bm = Khat^T Utilde
+    // takes both halves, so the term that dominates the next state is not rounded on its way.
+    // Warps 0..3 drain W, warps 4..7 Utilde (hi and lo); lane quarters 0, 1 (chunk rows
+    // 0..63) take the first D / 2 columns, quarters 2, 3 (the same rows, copied) the rest.
+    if (warp < 8) {
+        const int r = (warp & 1) * 32 + lane;
+        const bool ut = warp >= 4;
+        const int cbase = ut ? D : 0;
+        const int cbeg = (warp & 2) ? D / 2 : 0;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = cbeg; c0 < cbeg + D / 2; c0 += 32) {
             uint32_t x[32];
             tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, cbase + c0), x);
             tc::wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 8)  // [W | Utilde] column; 64-column blocks 8 KB apart
-                *reinterpret_cast<uint4 *>(sm + L::RG + tok_off(r, cbase + c0 + j)) = pack8(&x[j]);
+            for (int j = 0; j < 32; j += 8) {  // [W | Utilde] column; 64-column blocks 8 KB apart
+                if (ut) {  // Utilde_lo, at the offsets Utilde has relative to G, over V
+                    uint4 hi, lo;
+                    pack8_hilo(&x[j], hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + L::RG + tok_off(r, cbase + c0 + j)) = hi;
+                    *reinterpret_cast<uint4 *>(sm + L::RK + tok_off(r, cbase + c0 + j)) = lo;
+                } else {
+                    *reinterpret_cast<uint4 *>(sm + L::RG + tok_off(r, c0 + j)) = pack8(&x[j]);
+                }
+            }
         }
         tc::fence_smem_to_async();
     }
@@ -697,28 +746,32 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 
     // -- 7. four tensor-core units on the operands in place, each completing on its own
     //       mbarrier, so the tensor core runs one unit while the warps drain another:
-    //         U1  N = Khat^T W     TMEM cols 0..D    staged over [Kbar | V]
-    //         U2  P W              cols D..2D        Q' = Qbar - P W in place of Qbar
-    //         U3  Bm = Khat^T Ut   cols 0..D         staged over Khat and W
-    //         U4  O' = P Ut        cols D..2D        staged over Utilde
+    //         U1  N = Khat^T W                TMEM cols 0..D    staged over Kbar | W
+    //         U2  P W                         cols D..2D        Q' = Qbar - P W in place of Qbar
+    //         U3  Bm = Khat^T (Ut_hi + Ut_lo) cols 0..D         staged over Khat | Ut_lo
+    //         U4  O' = P Ut_hi                cols D..2D        staged over Ut_hi
     //       U3 is issued once U1's columns are read, U4 once U2's are.  Every staging area
-    //       is free when written ([Kbar | V] and Qbar after round 1; Khat and W once U3 is
-    //       done, U4 reading only P and Utilde; Utilde once U4 is done), so no store waits
-    //       for another to finish reading shared memory.
+    //       is free when written (Kbar after round 1, W once U1 and U2 are done; Qbar is Q'
+    //       itself; Khat and Ut_lo once U3 is done, U4 reading only P and Ut_hi; Ut_hi once
+    //       U4 is done), so no store waits for another to finish reading shared memory.
+    //       O' takes Utilde at bf16 (hi): it only feeds the output.
     constexpr int NB = D / kBV;  // value blocks of the record
-    static_assert((uint32_t)D * D * 2 <= 2 * L::kMat, "N staging fits over [Kbar | V]");
     static_assert((NB / 2) * R::BmBlk <= L::kMat && NB * R::OpBlk <= L::kMat, "Bm / O' staging fits");
+    static_assert((uint32_t)D * 64 * 2 <= L::kMat, "a 64-column block of N fits one operand slot");
     uint64_t *bar_u = bar + 1;
-    const uint32_t xw = smem_u32(sm + L::RG), xu = xw + L::kMat;  // W, Utilde (token-major operands)
-    auto issue_kt = [&](uint32_t xb, uint32_t col) {                  // Khat^T X
+    const uint32_t xw = smem_u32(sm + L::RG), xu = xw + L::kMat;      // W_hi, Ut_hi
+    const uint32_t xu_lo = smem_u32(sm + L::RK) + L::kMat;              // Ut_lo (over V)
+    auto issue_kt = [&](uint32_t xb, uint32_t col, uint32_t acc0) {  // Khat^T X
         const uint32_t id = tc::idesc_bf16(128, D, true, true);       // A = Khat^T (MN-major)
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
             const uint64_t ad = tc::smem_desc(smem_u32(sm + L::RX) + ks * 2048, kC * 128, 1024, tc::kSw128);
             const uint64_t bd = tc::smem_desc(xb + ks * 2048, kC * 128, 1024, tc::kSw128);
-            tc::mma_bf16(tmem + col, ad, bd, id, ks > 0 ? 1u : 0u);
+            tc::mma_bf16(tmem + col, ad, bd, id, ks > 0 ? 1u : acc0);
         }
     };
+    // N's 64-column blocks: block 0 over Kbar, block 1 (D = 128) over W
+    auto n_stage = [&](int blk64) -> unsigned char * { return sm + (blk64 == 0 ? L::RK : L::RG); };
     auto issue_p = [&](uint32_t xb, uint32_t col) {                   // P X
         const uint32_t id = tc::idesc_bf16(128, D, false, true);      // A = P (K-major)
 #pragma unroll
@@ -728,8 +781,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             tc::mma_bf16(tmem + col, ad, bd, id, ks > 0 ? 1u : 0u);
         }
     };
-    auto bm_stage = [&](int blk) -> unsigned char * {  // Bm block blk: over Khat, then W
-        return blk < NB / 2 ? sm + L::RX + blk * R::BmBlk : sm + L::RG + (blk - NB / 2) * R::BmBlk;
+    auto bm_stage = [&](int blk) -> unsigned char * {  // Bm block blk: over Khat, then Ut_lo
+        return blk < NB / 2 ? sm + L::RX + blk * R::BmBlk : sm + L::RK + L::kMat + (blk - NB / 2) * R::BmBlk;
     };
     auto sync_all = [&]() {
         tc::fence_before_sync();
@@ -737,7 +790,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         tc::fence_after_sync();
     };
     if (tid == 0) {
-        issue_kt(xw, 0);
+        issue_kt(xw, 0, 0u);
         tc::commit(&bar_u[0]);
         issue_p(xw, D);
         tc::commit(&bar_u[1]);
@@ -747,8 +800,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const bool kt_rows = warp < 8 && (warp & 3) * 32 < D, p_rows = warp < 8 && (warp & 3) < 2;
     const int lrow = (warp & 3) * 32 + lane, chalf = (warp >> 2) * (D / 2);
 
-    // U1 -> N over [Kbar | V]
+    // U1 -> N over Kbar | W (W is read by U1 and U2, so wait for U2 as well)
     mbar_wait_bounded(&bar_u[0], 0, status);
+    mbar_wait_bounded(&bar_u[1], 0, status);
     tc::fence_after_sync();
     if (kt_rows) {
 #pragma unroll
@@ -757,18 +811,19 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, chalf + c0), x);
             tc::wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 8)
-                *reinterpret_cast<uint4 *>(sm + L::RK + tc::kmaj_sw128(lrow, chalf + c0 + j, D)) = pack8(&x[j]);
+            for (int j = 0; j < 32; j += 8) {
+                const int col = chalf + c0 + j;
+                *reinterpret_cast<uint4 *>(n_stage(col >> 6) + tc::kmaj_sw128(lrow, col & 63, D)) = pack8(&x[j]);
+            }
         }
     }
     sync_all();
     if (tid == 0) {
-        issue_kt(xu, 0);
+        issue_kt(xu, 0, 0u);
+        issue_kt(xu_lo, 0, 1u);
         tc::commit(&bar_u[2]);
     }
     // U2 -> Q' = Qbar - P W, in place (same layout as the record)
-    mbar_wait_bounded(&bar_u[1], 0, status);
-    tc::fence_after_sync();
     if (p_rows) {
 #pragma unroll
         for (int c0 = 0; c0 < D / 2; c0 += 32) {
@@ -795,7 +850,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     if (tid == 0) {
         issue_p(xu, D);
         tc::commit(&bar_u[3]);
-        bulk_s2g(rec + R::Nm, sm + L::RK, D * D * 2);
+        for (int b64 = 0; b64 < D / 64; ++b64)
+            bulk_s2g(rec + R::Nm + b64 * (D * 128), n_stage(b64), D * 128);
         bulk_s2g(rec + R::Qp, sm + L::RQ, kC * D * 2);
         bulk_commit();
     }
@@ -879,18 +935,33 @@ __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int D>
+// Row `row` of the state block as the bf16 MMA operand (MN-major, 64-byte swizzle).
+__device__ __forceinline__ void store_state(unsigned char *sbuf, int row, const float (&S)[kBV])
+{
+#pragma unroll
+    for (int j = 0; j < kBV; j += 8)
+        *reinterpret_cast<uint4 *>(sbuf + tc::mnmaj_sw64(row, j)) =
+            make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
+                       pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+}
+
+template <int D, bool kAffine>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
-                __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, unsigned int *status)
+                __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, float *__restrict__ M_out,
+                unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char scan_smem[];
     using SM = ScanSmem<D>;
     using R = Rec<D>;
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
-    constexpr uint32_t kTmemCols = 2 * kBV;
+    constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N S; [kBV, 2 kBV): Q' S
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int blk = blockIdx.x, col0 = blk * kBV;
+    // Column blocks past D / kBV (affine mode only) carry the transfer map instead of the
+    // state: they start from the identity, add no Bm and write M_out.
+    constexpr int NB = D / kBV;
+    const bool xfer = kAffine && blockIdx.x >= NB;
+    const int blk = xfer ? blockIdx.x - NB : blockIdx.x, col0 = blk * kBV;
     const SeqLoc seq = locate_seq(map, H);
     const int h = seq.h, NT = seq.nchunks, bh = seq.sh;
     const unsigned char *recs = ws + seq.rec0 * R::Bytes;
@@ -934,18 +1005,20 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 #pragma unroll
             for (int j = 0; j < kBV; j += 4) {
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (S0)
+                if (xfer) {  // identity columns col0 .. col0 + kBV of the transfer map
+                    v.x = row == col0 + j ? 1.f : 0.f;
+                    v.y = row == col0 + j + 1 ? 1.f : 0.f;
+                    v.z = row == col0 + j + 2 ? 1.f : 0.f;
+                    v.w = row == col0 + j + 3 ? 1.f : 0.f;
+                } else if (S0) {
                     v = *reinterpret_cast<const float4 *>(&S0[((size_t)bh * D + row) * D + col0 + j]);
+                }
                 S[j] = v.x;
                 S[j + 1] = v.y;
                 S[j + 2] = v.z;
                 S[j + 3] = v.w;
             }
-#pragma unroll
-            for (int j = 0; j < kBV; j += 8)
-                *reinterpret_cast<uint4 *>(sm.sbuf + tc::mnmaj_sw64(row, j)) =
-                    make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
-                               pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+            store_state(sm.sbuf, row, S);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -986,7 +1059,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float2 bf = unpack_bf16x2(bw[q]);
+                        const float2 bf = xfer ? make_float2(0.f, 0.f) : unpack_bf16x2(bw[q]);
                         S[j + 2 * q] = fmaf(g, S[j + 2 * q], bf.x);
                         S[j + 2 * q + 1] = fmaf(g, S[j + 2 * q + 1], bf.y);
                     }
@@ -1005,15 +1078,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kBV; ++j)
                     S[j] -= __uint_as_float(d[j]);
-#pragma unroll
-                for (int j = 0; j < kBV; j += 8)
-                    *reinterpret_cast<uint4 *>(sm.sbuf + tc::mnmaj_sw64(row, j)) =
-                        make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
-                                   pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+                store_state(sm.sbuf, row, S);
                 tc::fence_smem_to_async();
             }
             // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
-            if (warp < 2) {
+            if (o && warp < 2) {
                 uint32_t y[kBV];
                 tc::ld_32x32b_x32(lane_addr + kBV, y);
                 tc::wait_ld();
@@ -1042,10 +1111,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 mbar_arrive_local(&sm.empty[s]);
         }
 
-        if (S_T && srow)
+        float *Sout = xfer ? M_out : S_T;
+        if (Sout && srow)
 #pragma unroll
             for (int j = 0; j < kBV; j += 4)
-                *reinterpret_cast<float4 *>(&S_T[((size_t)bh * D + row) * D + col0 + j]) =
+                *reinterpret_cast<float4 *>(&Sout[((size_t)bh * D + row) * D + col0 + j]) =
                     make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     tc::fence_before_sync();
@@ -1075,17 +1145,19 @@ cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, cons
 
 template <int D>
 cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S0, void *o, float *S_T,
-                          cudaStream_t s)
+                          float *M_out, cudaStream_t s)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
     const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
-    cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // with M_out: the state blocks and, after them, as many transfer-map blocks
+    auto kernel = M_out ? scan_kernel<D, true> : scan_kernel<D, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    scan_kernel<D><<<dim3(D / kBV, m.nseq * H), kScanThreads, smem, s>>>(
-        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, status);
+    kernel<<<dim3((M_out ? 2 : 1) * (D / kBV), m.nseq * H), kScanThreads, smem, s>>>(
+        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, M_out, status);
     return cudaGetLastError();
 }
 
@@ -1101,9 +1173,10 @@ cudaError_t launch_prep(const SeqMap &m, int H, int D, dim3 grid, const void *q,
 }
 
 cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const float *S0, void *o, float *S_T,
-                        cudaStream_t s)
+                        cudaStream_t s, float *M_out = nullptr)
 {
-    return D == 64 ? launch_scan_d<64>(m, H, ws, S0, o, S_T, s) : launch_scan_d<128>(m, H, ws, S0, o, S_T, s);
+    return D == 64 ? launch_scan_d<64>(m, H, ws, S0, o, S_T, M_out, s)
+                   : launch_scan_d<128>(m, H, ws, S0, o, S_T, M_out, s);
 }
 
 SeqMap regular_map(int B, int T)
@@ -1183,6 +1256,76 @@ cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, 
                              float *S_T, cudaStream_t s)
 {
     return launch_scan(regular_map(B, T), H, D, workspace, S0, o, S_T, s);
+}
+
+cudaError_t launch_scan_affine_bf16(int B, int T, int H, int D, const void *workspace, float *S_zero, float *M,
+                                    cudaStream_t s)
+{
+    return launch_scan(regular_map(B, T), H, D, workspace, nullptr, nullptr, S_zero, s, M);
+}
+
+// ------------------------------------------------------------------ segment combine
+// S_in[0] = S0 (or 0); S_in[r + 1] = M[r] S_in[r] + S_zero[r], r < R.  One CTA per
+// (32-column block, b*h) keeps its block of the running state in shared memory; thread t
+// computes row t / 2, columns (t % 2) * 16 .. + 16 of the next one.  Float32 FMAs.
+constexpr int kCombThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kCombThreads)
+    combine_kernel(int R, int BH, const float *__restrict__ M, const float *__restrict__ S_zero,
+                   const float *__restrict__ S0, float *__restrict__ S_in)
+{
+    __shared__ float Sb[D][kBV + 1];
+    const int tid = threadIdx.x, col0 = blockIdx.x * kBV, bh = blockIdx.y;
+    const size_t mstride = (size_t)BH * D * D;  // one segment's maps (and states: dk == dv)
+    for (int i = tid; i < D * kBV; i += kCombThreads) {
+        const int r = i / kBV, c = i % kBV;
+        const float v = S0 ? S0[((size_t)bh * D + r) * D + col0 + c] : 0.0f;
+        Sb[r][c] = v;
+        S_in[((size_t)bh * D + r) * D + col0 + c] = v;
+    }
+    __syncthreads();
+    static_assert(2 * D <= 2 * kCombThreads && kBV == 32, "two threads per row, 16 columns each");
+    for (int seg = 0; seg < R; ++seg) {
+        const float *Mr = M + seg * mstride + (size_t)bh * D * D;
+        const float *Zr = S_zero + seg * mstride + (size_t)bh * D * D;
+        float acc[16];
+        const int row = tid / 2, cb = (tid % 2) * 16;
+        const bool live = row < D;
+        if (live) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                acc[j] = Zr[(size_t)row * D + col0 + cb + j];
+            for (int k4 = 0; k4 < D; k4 += 4) {
+                const float4 m = *reinterpret_cast<const float4 *>(&Mr[(size_t)row * D + k4]);
+                const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        acc[j] = fmaf(mk[kk], Sb[k4 + kk][cb + j], acc[j]);
+            }
+        }
+        __syncthreads();
+        if (live)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                Sb[row][cb + j] = acc[j];
+                S_in[(seg + 1) * mstride + ((size_t)bh * D + row) * D + col0 + cb + j] = acc[j];
+            }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_combine(int R, int BH, int D, const float *M, const float *S_zero, const float *S0, float *S_in,
+                           cudaStream_t s)
+{
+    const dim3 grid(D / kBV, BH);
+    if (D == 64)
+        combine_kernel<64><<<grid, kCombThreads, 0, s>>>(R, BH, M, S_zero, S0, S_in);
+    else
+        combine_kernel<128><<<grid, kCombThreads, 0, s>>>(R, BH, M, S_zero, S0, S_in);
+    return cudaGetLastError();
 }
 
 size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D)

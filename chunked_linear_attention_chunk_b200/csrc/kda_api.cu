@@ -64,6 +64,9 @@ bool overlaps(const Range &x, const Range &y)
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// beta is read one element at a time: its natural alignment is enough.
+bool beta_aligned(const void *beta, int es) { return ((uintptr_t)beta % (uintptr_t)es) == 0; }
+
 int elem_size(kda_dtype dt) { return dt == KDA_BF16 ? 2 : 4; }
 
 bool dtype_ok(kda_dtype dt) { return dt == KDA_BF16 || dt == KDA_F32; }
@@ -233,7 +236,7 @@ kda_status check_prep_args(const ChunkShape &sh, const void *q, const void *k, c
 {
     if (sh.T > 0 && (!q || !k || !v || !a || !beta))
         return KDA_ERR_INVALID_ARG;
-    if (!all_aligned({q, k, v, a, beta, workspace}))
+    if (!all_aligned({q, k, v, a, workspace}) || !beta_aligned(beta, sh.es))
         return KDA_ERR_ALIGNMENT;
     kda_status st = check_workspace(sh, workspace, ws_bytes);
     if (st != KDA_OK)
@@ -363,7 +366,7 @@ kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
     const int64_t nk = (int64_t)T * H * dk, ntok = (int64_t)T * H, ns = (int64_t)N * H * dk * dv;
     if (!cu_seqlens || (T > 0 && (!q || !k || !v || !a || !beta || !o)))
         return KDA_ERR_INVALID_ARG;
-    if (!all_aligned({q, k, v, a, beta, S0, o, S_T, workspace}) || ((uintptr_t)cu_seqlens & 3u) ||
+    if (!all_aligned({q, k, v, a, S0, o, S_T, workspace}) || !beta_aligned(beta, 2) || ((uintptr_t)cu_seqlens & 3u) ||
         ((uintptr_t)A_log & 3u))
         return KDA_ERR_ALIGNMENT;
     const size_t need = kda_chunk_fwd_varlen_workspace(N, T, H, dk, dv, dtype);
@@ -386,6 +389,46 @@ kda_status kda_chunk_fwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
     return from_cuda(launch_chunk_bf16_varlen(N, cu_seqlens, T, H, dk, q, k, v, a, beta, g_min,
                                               gate == KDA_GATE_LOGSIGMOID, A_log, S0, o, S_T, workspace,
                                               (cudaStream_t)stream));
+}
+
+kda_status kda_chunk_fwd_scan_affine(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
+                                     float *S_zero, float *M, kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, KDA_BF16, sh);
+    if (st != KDA_OK)
+        return st;
+    if (!S_zero || !M)
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({workspace, S_zero, M}))
+        return KDA_ERR_ALIGNMENT;
+    if ((st = check_workspace(sh, workspace, ws_bytes)) != KDA_OK)
+        return st;
+    const Range rws(sh.ws > 0 ? workspace : nullptr, (int64_t)sh.ws), rz(S_zero, sh.ns * 4), rm(M, sh.ns * 4);
+    if (overlaps(rz, rm) || overlaps(rz, rws) || overlaps(rm, rws))
+        return KDA_ERR_ALIAS;
+    return from_cuda(launch_scan_affine_bf16(B, T, H, dk, workspace, S_zero, M, (cudaStream_t)stream));
+}
+
+kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M, const float *S_zero,
+                             const float *S0, float *S_in, kda_stream_t stream)
+{
+    if (R < 0 || B < 1 || H < 1 || dk < 1 || dv < 1)
+        return KDA_ERR_INVALID_ARG;
+    if (dk != dv || (dk != 64 && dk != 128) || (int64_t)B * H > 65535)
+        return KDA_ERR_UNSUPPORTED;
+    const int64_t per = safe_prod({B, H, dk, dv});
+    if (per < 0 || safe_prod({R + 1, per}) < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!S_in || (R > 0 && (!M || !S_zero)))
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({M, S_zero, S0, S_in}))
+        return KDA_ERR_ALIGNMENT;
+    const Range rin(S_in, (R + 1) * per * 4);
+    for (const Range &x : {Range(M, R * per * 4), Range(S_zero, R * per * 4), Range(S0, per * 4)})
+        if (overlaps(rin, x))
+            return KDA_ERR_ALIAS;
+    return from_cuda(launch_combine(R, B * H, dk, M, S_zero, S0, S_in, (cudaStream_t)stream));
 }
 
 kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate, float g_min, const float *A_log,
@@ -438,11 +481,13 @@ kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const 
         return KDA_ERR_INVALID_ARG;
     if (!q || !k || !v || !a || !beta || !S || !o)
         return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, a, beta, S, o};
+    const int es = elem_size(dtype);
+    const void *ptrs[] = {q, k, v, a, S, o};
     for (const void *p : ptrs)
         if (!aligned16(p))
             return KDA_ERR_ALIGNMENT;
-    const int es = elem_size(dtype);
+    if (!beta_aligned(beta, es))
+        return KDA_ERR_ALIGNMENT;
     const Range rq(q, nh * dk * es), rk(k, nh * dk * es), rv(v, nh * dv * es), ra(a, nh * dk * es),
         rb(beta, nh * es), rS(S, ns * 4), ro(o, nh * dv * es);
     for (const Range &in : {rq, rk, rv, ra, rb, rS})

@@ -35,6 +35,14 @@ cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const vo
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
                              float *S_T, cudaStream_t s);
 
+// Sequence-parallel pieces: the scan over one segment's records from S = 0 (S_zero) and of
+// the identity without Bm (M, the segment's transfer map), and the prefix combine
+// S_in[r + 1] = M[r] S_in[r] + S_zero[r] over R segments (dk == dv == D).
+cudaError_t launch_scan_affine_bf16(int B, int T, int H, int D, const void *workspace, float *S_zero, float *M,
+                                    cudaStream_t s);
+cudaError_t launch_combine(int R, int BH, int D, const float *M, const float *S_zero, const float *S0, float *S_in,
+                           cudaStream_t s);
+
 // Packed variable-length batch: N sequences on one axis of T tokens, sequence s spanning
 // [cu[s], cu[s+1]) (cu on the device).  A table kernel validates cu and writes the chunk
 // offsets at the end of the workspace; prep and scan follow on the same stream.

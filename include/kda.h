@@ -21,7 +21,8 @@
  *
  * Conventions shared by every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
- *     row-major (innermost index last) and 16-byte aligned.  The library allocates
+ *     row-major (innermost index last) and 16-byte aligned, except beta, which needs only
+ *     its element size (so [T, H] slices at any token offset are accepted).  The library allocates
  *     no device memory; scratch space is passed in by the caller.
  *   - Token tensors are [B, T, H, d]; beta is [B, T, H]; states are [B, H, dk, dv]
  *     float32.  dtype KDA_BF16 means q, k, v, a, beta and o are bfloat16 (state and
@@ -232,6 +233,36 @@ kda_status kda_chunk_fwd_prep(int B, int T, int H, int dk, int dv, kda_gate gate
                               void *workspace, size_t ws_bytes, kda_stream_t stream);
 kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
                               const float *S0, void *o, float *S_T, kda_stream_t stream);
+
+/*
+ * Sequence parallelism: one long sequence split into R consecutive segments, one per GPU
+ * ("Breaking Through ..." section 3: sequence parallelism for the million-token stage).
+ * Over a segment the state map is affine, S_out = M S_in + S_zero, with M the product of
+ * the segments' per-chunk maps Diag(Gamma) - N and S_zero the state the segment reaches
+ * from S_in = 0.  Each GPU preps its segment (kda_chunk_fwd_prep), computes (S_zero, M)
+ * (kda_chunk_fwd_scan_affine), all-gathers them, forms every segment's incoming state
+ * (kda_state_combine), and scans its segment again from its own incoming state
+ * (kda_chunk_fwd_scan) to write o.  The result equals one kda_chunk_fwd over the whole
+ * sequence up to rounding.
+ *
+ * kda_chunk_fwd_scan_affine -- (S_zero, M) of the segment whose records `workspace` holds.
+ *   workspace    the records of kda_chunk_fwd_prep(B, T, H, dk, dv, ...), ordered before.
+ *   S_zero       [B, H, dk, dv] float32 out: the final state from a zero initial state.
+ *   M            [B, H, dk, dk] float32 out: the segment's transfer map (T == 0: identity).
+ *   Writes no o.  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.
+ *
+ * kda_state_combine -- incoming states of R consecutive segments:
+ *     S_in[0] = S0 (or zeros),  S_in[r + 1] = M[r] S_in[r] + S_zero[r],  r < R
+ *   M, S_zero    [R, B, H, dk, dv] float32 (dk == dv), as gathered from the segments.
+ *   S0           [B, H, dk, dv] float32 or NULL.
+ *   S_in         [R + 1, B, H, dk, dv] float32 out; S_in[R] is the whole sequence's final
+ *                state.  Float32 arithmetic.
+ *   Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS (S_in overlaps an input), CUDA.
+ */
+kda_status kda_chunk_fwd_scan_affine(int B, int T, int H, int dk, int dv, const void *workspace, size_t ws_bytes,
+                                     float *S_zero, float *M, kda_stream_t stream);
+kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M, const float *S_zero,
+                             const float *S0, float *S_in, kda_stream_t stream);
 
 /*
  * kda_decode_step -- one token for N independent sequences, state updated in place.

@@ -277,3 +277,25 @@ def test_gate_heads_validates(L):
     assert f(A=BASE * 3 + 2) == ALIGN
     assert f(g=BASE + 64) == ALIAS
     assert f(A=BASE * 2 + 16) == ALIAS
+
+
+def test_sp_entries_validate(L):
+    P = ctypes.c_void_p
+    assert L.kda_chunk_fwd_scan_affine(1, 64, 1, 128, 128, P(BASE), 1 << 20, None, P(BASE * 2), None) == INVALID
+    assert L.kda_chunk_fwd_scan_affine(1, 64, 1, 96, 96, P(BASE), 1 << 20, P(BASE * 3), P(BASE * 2), None) == UNSUPPORTED
+    assert L.kda_chunk_fwd_scan_affine(1, 64, 1, 128, 128, P(BASE), 10, P(BASE * 3), P(BASE * 2), None) == WS
+    assert L.kda_chunk_fwd_scan_affine(1, 64, 1, 128, 128, P(BASE), 1 << 20, P(BASE * 3), P(BASE * 3 + 64), None) == ALIAS
+    assert L.kda_state_combine(-1, 1, 1, 128, 128, P(BASE), P(BASE * 2), None, P(BASE * 3), None) == INVALID
+    assert L.kda_state_combine(2, 1, 1, 128, 128, P(BASE), P(BASE * 2), None, None, None) == INVALID
+    assert L.kda_state_combine(2, 1, 1, 128, 128, P(BASE + 4), P(BASE * 2), None, P(BASE * 3), None) == ALIGN
+    assert L.kda_state_combine(2, 1, 1, 128, 128, P(BASE), P(BASE * 2), None, P(BASE + 4096), None) == ALIAS
+
+
+def test_beta_needs_only_its_element_size():
+    """beta may start at any token offset: 2-byte alignment passes the alignment check (the
+    call then stops on the too-small workspace, before any launch); 1 byte does not."""
+    L = kda.lib()
+    n = 1 * 64 * 1 * 128 * 2
+    beta = BASE + 4 * (n + 4096)
+    assert _chunk(L, beta=beta + 2, ws_bytes=100) == WS
+    assert _chunk(L, beta=beta + 1) == ALIGN

@@ -195,8 +195,19 @@ def time_steps(fn, steps: int, warmup: int, world: int, device, timed_flag=None)
     return max_over_ranks(ms, world, device)
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(x, sample_tokens: int):
-    """The fp64 oracle, as it stands, on the first ``sample_tokens`` tokens of every head."""
+    """The fp64 oracle, as it stands, on the first ``sample_tokens`` tokens of every head,
+    plus its chunked form (C = 16) on a shorter sample as a second CPU figure."""
     import oracle
     from chunked_linear_attention_chunk_b200.synth import to_numpy32
     names = ("q", "k", "v", "a", "beta")
@@ -208,9 +219,16 @@ def cpu_baseline(x, sample_tokens: int):
     t = time.perf_counter()
     oracle.recurrence(*arrs, G_MIN, S0=S0, nthreads=cores)
     dt = time.perf_counter() - t
+    short = min(sample_tokens, 8192)
+    t = time.perf_counter()
+    oracle.chunked(16, *(a[:, :short] for a in arrs), G_MIN, S0=S0, nthreads=cores)
+    dtc = time.perf_counter() - t
     return {"value": B * sample_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
             "sample": f"first {sample_tokens} of {x['q'].shape[1]} tokens, all {B * H} (batch, head) pairs "
-                      f"of the 64K stage; fp64 token-by-token recurrence, {dt:.2f} s"}
+                      f"of the 64K stage; fp64 token-by-token recurrence, {dt:.2f} s",
+            "chunked_c16": {"value": B * short / dtc, "unit": UNIT,
+                            "sample": f"first {short} tokens, fp64 chunked form with C = 16, {dtc:.2f} s"}}
 
 
 def run_reference(args):

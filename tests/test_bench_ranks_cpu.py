@@ -1,0 +1,32 @@
+"""bench.py's multi-rank plumbing over two gloo ranks on CPU: the step time every rank
+reports is the maximum over ranks, and each rank draws its own seed (weak scaling)."""
+import os
+import socket
+
+import numpy as np
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _rank(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(1.0 + rank * 2.5, world, "cpu")
+        bench.barrier(world)
+        np.save(os.path.join(out_dir, f"r{rank}.npy"), np.array([got, bench.rank_seed(1002, rank)]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_rank_seeds(tmp_path):
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mp.spawn(_rank, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    r0, r1 = np.load(tmp_path / "r0.npy"), np.load(tmp_path / "r1.npy")
+    assert r0[0] == r1[0] == 3.5          # the slowest rank's time, on every rank
+    assert r0[1] != r1[1]                 # independent batches per rank
+    assert bench.max_over_ranks(2.0, 1, "cpu") == 2.0

@@ -74,3 +74,20 @@ def test_decode_chain_matches_chunk_path():
     den = o_c.float().abs().amax(dim=(1, 3))
     assert float((num / den).max()) <= TOL_BF16_O
     assert err_s(S.cpu().numpy(), S_c.cpu().numpy()) <= 1e-2
+
+
+@pytest.mark.parametrize("N,H,D", [(303, 1, 128), (7, 45, 64), (1, 1, 128)])
+def test_decode_uneven_units(N, H, D):
+    """The persistent decode kernel gives CTAs different numbers of (n, h) units (303 units
+    over the resident CTAs), one unit, and the d = 64 bf16 shape; two chained steps."""
+    x = synth.make_inputs(N, 2, H, D, D, "bf16", seed=620 + N + D, s0_std=0.1)
+    S = x["S0"].cuda()
+    S_ref = x["S0"].numpy().astype(np.float64)
+    for t in range(2):
+        tok = {n: x[n][:, t].contiguous() for n in NAMES}
+        o = kda.kda_decode_step(*(tok[n].cuda() for n in NAMES), S, G_MIN)
+        torch.cuda.synchronize()
+        o_ref, S_ref = oracle.decode(*(synth.to_numpy32(tok[n]) for n in NAMES), S_ref, G_MIN)
+        assert _err_tok(o.float().cpu().numpy(), o_ref) <= TOL_BF16_O
+        assert err_s(S.cpu().numpy(), S_ref) <= 1e-5
+    assert kda.kda_device_status() == 0

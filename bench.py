@@ -205,9 +205,21 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(x, sample_tokens: int):
+def normwise_err(x, y, axes):
+    """Worst per-head normwise relative error max|x - y| / max|y| (the parity metric)."""
+    import numpy as np
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    num = np.max(np.abs(x - y), axis=axes)
+    den = np.maximum(np.max(np.abs(y), axis=axes), 1e-30)
+    return float(np.max(num / den))
+
+
+def cpu_baseline(x, sample_tokens: int, gpu_out=None):
     """The fp64 oracle, as it stands, on the first ``sample_tokens`` tokens of every head,
-    plus its chunked form (C = 16) on a shorter sample as a second CPU figure."""
+    plus its chunked form (C = 16) on a shorter sample as a second CPU figure.  When the
+    sample is the whole workload and ``gpu_out`` = (o, S_T) of the GPU on the same inputs, the
+    line also records their parity with the oracle."""
     import oracle
     from chunked_linear_attention_chunk_b200.synth import to_numpy32
     names = ("q", "k", "v", "a", "beta")
@@ -217,8 +229,16 @@ def cpu_baseline(x, sample_tokens: int):
     cores = min(os.cpu_count() or 1, B * H)
     oracle.recurrence(*(a[:, :16] for a in arrs), G_MIN, S0=S0)  # build/load outside timing
     t = time.perf_counter()
-    oracle.recurrence(*arrs, G_MIN, S0=S0, nthreads=cores)
+    o_ref, S_ref = oracle.recurrence(*arrs, G_MIN, S0=S0, nthreads=cores)
     dt = time.perf_counter() - t
+    parity = None
+    if gpu_out is not None and sample_tokens >= x["q"].shape[1]:
+        o_gpu, S_gpu = gpu_out
+        parity = {"o_max_rel": normwise_err(o_gpu.float().cpu().numpy(), o_ref, (1, 3)),
+                  "S_T_max_rel": normwise_err(S_gpu.cpu().numpy(), S_ref, (2, 3)),
+                  "metric": "worst per-head max|gpu - oracle| / max|oracle| over the full workload",
+                  "tolerance": {"o": 2e-2, "S_T": 1e-2}}
+    del o_ref, S_ref
     short = min(sample_tokens, 8192)
     t = time.perf_counter()
     oracle.chunked(16, *(a[:, :short] for a in arrs), G_MIN, S0=S0, nthreads=cores)
@@ -228,7 +248,8 @@ def cpu_baseline(x, sample_tokens: int):
             "sample": f"first {sample_tokens} of {x['q'].shape[1]} tokens, all {B * H} (batch, head) pairs "
                       f"of the 64K stage; fp64 token-by-token recurrence, {dt:.2f} s",
             "chunked_c16": {"value": B * short / dtc, "unit": UNIT,
-                            "sample": f"first {short} tokens, fp64 chunked form with C = 16, {dtc:.2f} s"}}
+                            "sample": f"first {short} tokens, fp64 chunked form with C = 16, {dtc:.2f} s"},
+            "parity": parity}
 
 
 def run_reference(args):
@@ -484,7 +505,7 @@ def run_libkda(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "gpu": torch.cuda.get_device_name(device),
         "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": D, "dv": D, "chunk": 64, "tile": 16,
                    "g_min": G_MIN, "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
                    "l2": "inputs exceed the 126 MB L2; no flush"},
@@ -519,7 +540,11 @@ def run_libkda(args):
     if spl is not None:
         line["sequence_parallel"] = spl
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
-        line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens)
+        # a fresh run of the main path on this exact input (later legs reuse o and S_T)
+        o_p, S_p = kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, workspace=ws)
+        torch.cuda.synchronize(device)
+        line["cpu_baseline"] = cpu_baseline(x, args.cpu_sample_tokens, gpu_out=(o_p, S_p))
+        del o_p, S_p
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -17,7 +17,8 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libkda.so")
+# KDA_DEBUG_CHECKS=1 selects the build with the kernels' index checks (libkda_debug.so)
+LIB_PATH = os.path.join(HERE, "libkda_debug.so" if os.environ.get("KDA_DEBUG_CHECKS") == "1" else "libkda.so")
 
 KDA_BF16 = 0
 KDA_F32 = 1
@@ -36,6 +37,7 @@ STATUS = {
     5: "KDA_ERR_CUDA",
     6: "KDA_ERR_DEVICE_TIMEOUT",
     7: "KDA_ERR_WORKSPACE",
+    8: "KDA_ERR_DEVICE_BOUNDS",
 }
 
 EXPORTS = (
@@ -76,8 +78,8 @@ def lib() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"libkda.so not found at {LIB_PATH}; build it with "
-            "`python -m chunked_linear_attention_chunk_b200.build`")
+            f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}; build it with "
+            "`python -m chunked_linear_attention_chunk_b200.build` (add --debug-checks for the debug build)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, L64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
     L.kda_gate_fwd.argtypes = [P, I, F, P, L64, P]

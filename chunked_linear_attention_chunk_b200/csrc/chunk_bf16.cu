@@ -82,6 +82,8 @@ struct SeqMap {
     int nseq = 0;                    // B or N
     int T = 0;                       // tokens per sequence (regular) or on the packed axis
     int NT = 0;                      // records per row
+    int64_t nrec = 0;                // records the workspace holds
+    int64_t ntok = 0;                // tokens on the flattened token axis (B * T, or T packed)
 };
 
 struct ChunkLoc {
@@ -338,6 +340,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const ChunkLoc loc = locate_chunk(map, H, blockIdx.x, blockIdx.y);
     if (!loc.live)  // packed batch: grid slots past the last chunk
         return;
+    if constexpr (kDebugChecks) {
+        if ((int64_t)loc.rec >= map.nrec || loc.n < 1 || loc.tok0 < 0 || loc.tok0 + loc.n > map.ntok ||
+            loc.h < 0 || loc.h >= H) {
+            if (threadIdx.x == 0)
+                report_device_error(status, KDA_ERR_DEVICE_BOUNDS);
+            return;
+        }
+    }
     const int n = loc.n, h = loc.h;
     unsigned char *rec = ws + loc.rec * R::Bytes;
     const int64_t rowstride = (int64_t)H * D;  // elements between consecutive tokens
@@ -963,6 +973,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const bool xfer = kAffine && blockIdx.x >= NB;
     const int blk = xfer ? blockIdx.x - NB : blockIdx.x, col0 = blk * kBV;
     const SeqLoc seq = locate_seq(map, H);
+    if constexpr (kDebugChecks) {
+        // the records this CTA reads and the token rows it can write (an invalid packed-batch
+        // table leaves nchunks = 0: nothing read or written, S_T still set)
+        const int64_t span = min((int64_t)seq.len, (int64_t)seq.nchunks * kC);
+        if (seq.nchunks < 0 || (int64_t)seq.rec0 + seq.nchunks > map.nrec || seq.sh >= map.nseq * H ||
+            (span > 0 && (seq.tok0 < 0 || seq.tok0 + span > map.ntok))) {
+            if (threadIdx.x == 0)
+                report_device_error(status, KDA_ERR_DEVICE_BOUNDS);
+            return;
+        }
+    }
     const int h = seq.h, NT = seq.nchunks, bh = seq.sh;
     const unsigned char *recs = ws + seq.rec0 * R::Bytes;
 
@@ -1179,12 +1200,14 @@ cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const flo
                    : launch_scan_d<128>(m, H, ws, S0, o, S_T, M_out, s);
 }
 
-SeqMap regular_map(int B, int T)
+SeqMap regular_map(int B, int T, int H)
 {
     SeqMap m;
     m.nseq = B;
     m.T = T;
     m.NT = (T + kC - 1) / kC;
+    m.nrec = (int64_t)B * H * m.NT;
+    m.ntok = (int64_t)B * T;
     return m;
 }
 
@@ -1248,20 +1271,20 @@ cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const vo
                              const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log,
                              void *workspace, cudaStream_t s)
 {
-    const SeqMap m = regular_map(B, T);
+    const SeqMap m = regular_map(B, T, H);
     return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, s);
 }
 
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
                              float *S_T, cudaStream_t s)
 {
-    return launch_scan(regular_map(B, T), H, D, workspace, S0, o, S_T, s);
+    return launch_scan(regular_map(B, T, H), H, D, workspace, S0, o, S_T, s);
 }
 
 cudaError_t launch_scan_affine_bf16(int B, int T, int H, int D, const void *workspace, float *S_zero, float *M,
                                     cudaStream_t s)
 {
-    return launch_scan(regular_map(B, T), H, D, workspace, nullptr, nullptr, S_zero, s, M);
+    return launch_scan(regular_map(B, T, H), H, D, workspace, nullptr, nullptr, S_zero, s, M);
 }
 
 // ------------------------------------------------------------------ segment combine
@@ -1349,6 +1372,8 @@ cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int
     m.nseq = N;
     m.T = T;
     m.NT = (int)varlen_records(N, T);
+    m.nrec = (int64_t)H * m.NT;
+    m.ntok = T;
     int32_t *choff = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + (size_t)H * m.NT * rec);
     m.choff = choff;
     seq_table_kernel<<<1, kTableThreads, 0, s>>>(cu, N, T, choff, status);

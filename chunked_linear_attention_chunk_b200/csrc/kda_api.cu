@@ -116,6 +116,7 @@ const char *kda_status_string(kda_status s)
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
     case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
     case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    case KDA_ERR_DEVICE_BOUNDS: return "KDA_ERR_DEVICE_BOUNDS";
     }
     return "KDA_ERR_UNKNOWN";
 }

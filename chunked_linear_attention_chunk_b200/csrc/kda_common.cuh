@@ -16,6 +16,15 @@ __device__ __forceinline__ void report_device_error(unsigned int *status, unsign
     atomicCAS(status, 0u, code);
 }
 
+// Debug builds (-DKDA_DEBUG_CHECKS, libkda_debug.so) check the ranges each CTA derives from
+// its grid coordinates against the buffers it was given; a failed check records
+// KDA_ERR_DEVICE_BOUNDS and the CTA returns before its first barrier.
+#ifdef KDA_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
 // ------------------------------------------------------------------ gate, fp64 exact
 // g = g_min * sigmoid(a), evaluated in float64 and rounded once to float32 (RN).
 __device__ __forceinline__ float gate_bounded_exact(float a, double g_min)

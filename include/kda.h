@@ -34,6 +34,10 @@
  *     invocations and may be made from several host threads.
  *   - Errors detected inside a kernel (a bounded wait that ran out) are recorded in a
  *     per-device status word and reported by kda_device_status().
+ *   - libkda_debug.so is the same library built with KDA_DEBUG_CHECKS: its prep and scan
+ *     CTAs check the record and token ranges they derive from their grid coordinates
+ *     against the buffers they were given and, on a mismatch, record KDA_ERR_DEVICE_BOUNDS
+ *     and return without touching memory.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -61,7 +65,8 @@ typedef enum {
     KDA_ERR_ALIAS = 4,          /* an output overlaps an input it must not overlap    */
     KDA_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed        */
     KDA_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out (kda_device_status) */
-    KDA_ERR_WORKSPACE = 7       /* workspace pointer missing or smaller than required */
+    KDA_ERR_WORKSPACE = 7,      /* workspace pointer missing or smaller than required */
+    KDA_ERR_DEVICE_BOUNDS = 8   /* debug build: a kernel's index check failed (kda_device_status) */
 } kda_status;
 
 /* The decay gate of the chunked forward. */
@@ -312,7 +317,8 @@ size_t kda_chunk_fwd_noalloc_max_scratch(void);
  * kda_device_status -- synchronise `stream`, then return and clear the current
  * device's kernel status word: KDA_OK; KDA_ERR_DEVICE_TIMEOUT if a kernel gave up on a
  * bounded wait since the last call; KDA_ERR_INVALID_ARG if kda_chunk_fwd_varlen found
- * its cu_seqlens invalid; KDA_ERR_CUDA if the synchronisation failed.  The first error
+ * its cu_seqlens invalid; KDA_ERR_DEVICE_BOUNDS if a debug-build index check failed;
+ * KDA_ERR_CUDA if the synchronisation failed.  The first error
  * recorded since the last call is the one reported.
  */
 kda_status kda_device_status(kda_stream_t stream);

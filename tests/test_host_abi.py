@@ -299,3 +299,11 @@ def test_beta_needs_only_its_element_size():
     beta = BASE + 4 * (n + 4096)
     assert _chunk(L, beta=beta + 2, ws_bytes=100) == WS
     assert _chunk(L, beta=beta + 1) == ALIGN
+
+
+def test_debug_build_exports_the_same_entry_points():
+    """libkda_debug.so (KDA_DEBUG_CHECKS) is the same ABI."""
+    path = build.build(debug_checks=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT\s+(kda_[a-z0-9_]+)$", out, re.M))
+    assert set(declared_functions()) <= exported

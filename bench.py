@@ -403,7 +403,7 @@ def run_libkda(args):
         spl = {"workload": f"one {T}-token sequence in {world} segment(s) of {seg}, H={H} d={D}",
                "ms_per_step": sp_ms, "value": tokens / (sp_ms * 1e-3), "unit": UNIT, "segments": world,
                "gpu_launches_per_step": 4, "collectives_per_step": 2 if world > 1 else 0}
-        del sd
+        del sd, xs
 
     # ---- end to end through the C ABI with pinned host buffers, pipelined across steps:
     # every step copies its inputs host -> device on one stream, runs kda_chunk_fwd on a

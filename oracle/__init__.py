@@ -13,6 +13,7 @@ passages of the pages each one follows):
 * ``recurrence(...)``           -- the token-by-token recurrence, fp64.
 * ``chunked(C, ...)``           -- the chunked form with pairwise exponentials, fp64.
 * ``decode(...)``               -- one decode step, state updated in place.
+* ``backward(...)``             -- gradients of the recurrence (reverse mode, by hand).
 * ``tile_factors_f32(...)``     -- counts of non-finite / subnormal values when a
   16-token tile's pairwise decay is factored densely in float32.
 
@@ -77,6 +78,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.oracle_tile_factors_f32.restype = _I
     lib.oracle_gate_heads_f32.argtypes = [_P, _L, _I, _I, _D, _P, _P]
     lib.oracle_gate_heads_f32.restype = None
+    lib.oracle_backward.argtypes = [_I] * 5 + [_P] * 5 + [_D, _I] + [_P] * 9 + [_I]
+    lib.oracle_backward.restype = _I
     return lib
 
 
@@ -163,6 +166,30 @@ def chunked(C, q, k, v, a, beta, g_min=-5.0, S0=None, kind=GATE_BOUNDED, nthread
     if st != 0:
         raise RuntimeError(f"oracle_chunked failed with status {st}")
     return o, ST
+
+
+def backward(q, k, v, a, beta, dO, g_min=-5.0, S0=None, dST=None, kind=GATE_BOUNDED, nthreads=0, lib=None):
+    """Gradients of a loss L given dO = dL/do [B,T,H,dv] and dST = dL/dS_T (None: zero).
+
+    Returns a dict of fp64 arrays: dq, dk, da [B,T,H,dk], dv [B,T,H,dv], dbeta [B,T,H],
+    dS0 [B,H,dk,dv] (the gradient with respect to the initial state, zero or not)."""
+    q, k, v, a, beta, S0, (B, T, H, dk, dv) = _seq_args(q, k, v, a, beta, S0)
+    dO = _f32(dO)
+    assert dO.shape == (B, T, H, dv), "dO must be [B,T,H,dv]"
+    if dST is not None:
+        dST = np.ascontiguousarray(dST, dtype=np.float64)
+        assert dST.shape == (B, H, dk, dv), "dST must be [B,H,dk,dv]"
+    out = {
+        "dq": np.zeros((B, T, H, dk)), "dk": np.zeros((B, T, H, dk)), "dv": np.zeros((B, T, H, dv)),
+        "da": np.zeros((B, T, H, dk)), "dbeta": np.zeros((B, T, H)), "dS0": np.zeros((B, H, dk, dv)),
+    }
+    st = _get(lib).oracle_backward(
+        B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), float(g_min), int(kind),
+        _ptr(S0), _ptr(dO), _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+        _ptr(out["da"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), int(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle_backward failed with status {st}")
+    return out
 
 
 def decode(q, k, v, a, beta, S, g_min=-5.0, kind=GATE_BOUNDED, nthreads=0, lib=None):

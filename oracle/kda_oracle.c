@@ -100,6 +100,10 @@ typedef struct {
     double *o, *ST;
     int nthreads, tid;
     int status;
+    /* backward only: upstream gradients in (dO, dST), input gradients out (g*) */
+    const float *dO;
+    const double *dST;
+    double *gq, *gk, *gv, *ga, *gbeta, *gS0;
 } job_t;
 
 static int resolve_threads(int nthreads, int units)
@@ -374,6 +378,211 @@ int oracle_chunked(int C, int B, int T, int H, int dk, int dv, const float *q, c
         return ORACLE_ERR_ARG;
     job_t J = {B, T, H, dk, dv, C, q, k, v, a, beta, g_min, kind, S0, o, ST, nthreads, 0, 0};
     return run_jobs(&J, chunked_worker);
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Backward of the recurrence (reverse-mode derivative, written out by hand).
+ *
+ * "Trillion-Parameter MoE Multimodal Models: Engineering ..." section 3.2 says long
+ * sequences are trained by recursing in chunks; training needs the gradients of a scalar
+ * loss L with respect to every input, given dL/do_t for every token and dL/dS_T.  The
+ * pages print no backward, so this is the derivative of the recurrence above and nothing
+ * else.  Per token, with S_prev = S_{t-1}:
+ *
+ *   Sd  = Diag(e^{g_t}) S_prev          (decayed state)
+ *   r   = v_t - Sd^T k_t,  u = beta_t r (delta correction)
+ *   S_t = Sd + k_t u^T,    o_t = S_t^T q_t
+ *
+ * and, walking t from T down to 1 with dS = dL/dS_t (dL/dS_T first):
+ *
+ *   dS      += q_t do_t^T               dq_t = S_t do_t
+ *   du       = dS^T k_t                 dk_t = dS u + Sd (-beta_t du)
+ *   dbeta_t  = du . r                   dv_t = beta_t du
+ *   dSd      = dS + k_t (-beta_t du)^T
+ *   dg_t[i]  = sum_j dSd[i,j] Sd[i,j]   da_t = dg_t * dg/da
+ *   dS_prev  = Diag(e^{g_t}) dSd
+ *
+ * dL/dS0 is the last dS_prev.  The states S_{t-1} are recomputed from checkpoints kept
+ * every BWD_SEG tokens, so memory stays O((T / BWD_SEG + BWD_SEG) dk dv) per sequence.  */
+#define BWD_SEG 64
+
+/* dg/da for the two gates: g_min * s (1 - s) (bounded) or 1 - s (log-sigmoid), with
+ * s = sigmoid(a).                                                                      */
+static double gate_grad_f64(double a, double g_min, int kind)
+{
+    const double s = 1.0 / (1.0 + exp(-a));
+    if (kind == ORACLE_GATE_BOUNDED)
+        return g_min * s * (1.0 - s);
+    return 1.0 - s;
+}
+
+/* One forward token: S_prev -> S (both dk x dv); decay and r are scratch.           */
+static void bwd_forward_token(const job_t *J, int b, int t, int h, const double *S_prev, double *S,
+                              double *decay, double *r)
+{
+    const int T = J->T, H = J->H, dk = J->dk, dv = J->dv;
+    const float *k = J->k + IDX_TOK(b, t, h, 0, T, H, dk);
+    const float *a = J->a + IDX_TOK(b, t, h, 0, T, H, dk);
+    const float *v = J->v + IDX_TOK(b, t, h, 0, T, H, dv);
+    const double beta = (double)J->beta[IDX_BETA(b, t, h, T, H)];
+    for (int i = 0; i < dk; ++i) {
+        decay[i] = exp(gate_f64((double)a[i], J->g_min, J->kind));
+        for (int j = 0; j < dv; ++j)
+            S[(int64_t)i * dv + j] = decay[i] * S_prev[(int64_t)i * dv + j];
+    }
+    for (int j = 0; j < dv; ++j) {
+        double kS = 0.0;
+        for (int i = 0; i < dk; ++i)
+            kS += (double)k[i] * S[(int64_t)i * dv + j];
+        r[j] = (double)v[j] - kS;
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j)
+            S[(int64_t)i * dv + j] += (double)k[i] * beta * r[j];
+}
+
+static void *backward_worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const int T = J->T, H = J->H, dk = J->dk, dv = J->dv;
+    const size_t SZ = (size_t)dk * dv;
+    const int nseg = (T + BWD_SEG - 1) / BWD_SEG;
+    double *ckpt = (double *)malloc(sizeof(double) * SZ * (size_t)(nseg > 0 ? nseg : 1));
+    double *seg = (double *)malloc(sizeof(double) * SZ * (BWD_SEG + 1));
+    double *Sd = (double *)malloc(sizeof(double) * SZ);
+    double *dS = (double *)malloc(sizeof(double) * SZ);
+    double *decay = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *r = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+    if (!ckpt || !seg || !Sd || !dS || !decay || !r || !du) {
+        J->status = ORACLE_ERR_NOMEM;
+        goto done;
+    }
+    for (int unit = J->tid; unit < J->B * H; unit += J->nthreads) {
+        const int b = unit / H, h = unit % H;
+        const int64_t s_off = IDX_S(b, h, H, dk, dv);
+        /* forward, keeping the state that enters every segment */
+        double *S = seg, *S_next = seg + SZ;
+        if (J->S0)
+            memcpy(S, J->S0 + s_off, sizeof(double) * SZ);
+        else
+            memset(S, 0, sizeof(double) * SZ);
+        for (int t = 0; t < T; ++t) {
+            if (t % BWD_SEG == 0)
+                memcpy(ckpt + (size_t)(t / BWD_SEG) * SZ, S, sizeof(double) * SZ);
+            bwd_forward_token(J, b, t, h, S, S_next, decay, r);
+            memcpy(S, S_next, sizeof(double) * SZ);
+        }
+        /* reverse sweep */
+        if (J->dST)
+            memcpy(dS, J->dST + s_off, sizeof(double) * SZ);
+        else
+            memset(dS, 0, sizeof(double) * SZ);
+        for (int sg = nseg - 1; sg >= 0; --sg) {
+            const int t0 = sg * BWD_SEG, t1 = (t0 + BWD_SEG < T) ? t0 + BWD_SEG : T;
+            /* seg[j] = S_{t0 + j - 1}: the state entering token t0 + j, j = 0 .. t1 - t0 */
+            memcpy(seg, ckpt + (size_t)sg * SZ, sizeof(double) * SZ);
+            for (int t = t0; t < t1; ++t)
+                bwd_forward_token(J, b, t, h, seg + (size_t)(t - t0) * SZ, seg + (size_t)(t - t0 + 1) * SZ,
+                                  decay, r);
+            for (int t = t1 - 1; t >= t0; --t) {
+                const double *S_prev = seg + (size_t)(t - t0) * SZ;
+                const double *S_t = seg + (size_t)(t - t0 + 1) * SZ;
+                const float *q = J->q + IDX_TOK(b, t, h, 0, T, H, dk);
+                const float *k = J->k + IDX_TOK(b, t, h, 0, T, H, dk);
+                const float *a = J->a + IDX_TOK(b, t, h, 0, T, H, dk);
+                const float *dO = J->dO + IDX_TOK(b, t, h, 0, T, H, dv);
+                const double beta = (double)J->beta[IDX_BETA(b, t, h, T, H)];
+                double *dq = J->gq + IDX_TOK(b, t, h, 0, T, H, dk);
+                double *dkk = J->gk + IDX_TOK(b, t, h, 0, T, H, dk);
+                double *dvv = J->gv + IDX_TOK(b, t, h, 0, T, H, dv);
+                double *da = J->ga + IDX_TOK(b, t, h, 0, T, H, dk);
+                /* this token's decayed state Sd and r = v - Sd^T k, again */
+                for (int i = 0; i < dk; ++i) {
+                    decay[i] = exp(gate_f64((double)a[i], J->g_min, J->kind));
+                    for (int j = 0; j < dv; ++j)
+                        Sd[(int64_t)i * dv + j] = decay[i] * S_prev[(int64_t)i * dv + j];
+                }
+                for (int j = 0; j < dv; ++j) {
+                    double kS = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        kS += (double)k[i] * Sd[(int64_t)i * dv + j];
+                    r[j] = (double)J->v[IDX_TOK(b, t, h, j, T, H, dv)] - kS;
+                }
+                /* o_t = S_t^T q_t */
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j)
+                        dS[(int64_t)i * dv + j] += (double)q[i] * (double)dO[j];
+                for (int i = 0; i < dk; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j)
+                        acc += S_t[(int64_t)i * dv + j] * (double)dO[j];
+                    dq[i] = acc;
+                }
+                /* S_t = Sd + k u^T, u = beta r */
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        acc += (double)k[i] * dS[(int64_t)i * dv + j];
+                    du[j] = acc;
+                }
+                double db = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    db += du[j] * r[j];
+                    dvv[j] = beta * du[j];
+                }
+                J->gbeta[IDX_BETA(b, t, h, T, H)] = db;
+                for (int i = 0; i < dk; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j)
+                        acc += dS[(int64_t)i * dv + j] * beta * r[j]          /* from k u^T        */
+                               - Sd[(int64_t)i * dv + j] * beta * du[j];      /* from r = v - Sd^T k */
+                    dkk[i] = acc;
+                }
+                /* dSd = dS - beta k du^T; dg; dS_prev */
+                for (int i = 0; i < dk; ++i) {
+                    double dg = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        const double d = dS[(int64_t)i * dv + j] - beta * (double)k[i] * du[j];
+                        dg += d * Sd[(int64_t)i * dv + j];
+                        dS[(int64_t)i * dv + j] = decay[i] * d;
+                    }
+                    da[i] = dg * gate_grad_f64((double)a[i], J->g_min, J->kind);
+                }
+            }
+        }
+        if (J->gS0)
+            memcpy(J->gS0 + s_off, dS, sizeof(double) * SZ);
+    }
+done:
+    free(ckpt);
+    free(seg);
+    free(Sd);
+    free(dS);
+    free(decay);
+    free(r);
+    free(du);
+    return NULL;
+}
+
+/* Gradients of L given dO = dL/do [B,T,H,dv] and dST = dL/dS_T [B,H,dk,dv] (NULL: zero).
+ * Outputs dq, dk, da [B,T,H,dk], dv [B,T,H,dv], dbeta [B,T,H], dS0 [B,H,dk,dv] (NULL:
+ * not stored), all fp64.  S0 NULL means a zero initial state.                          */
+int oracle_backward(int B, int T, int H, int dk, int dv, const float *q, const float *k,
+                    const float *v, const float *a, const float *beta, double g_min, int kind,
+                    const double *S0, const float *dO, const double *dST, double *dq, double *dk_,
+                    double *dv_, double *da, double *dbeta, double *dS0, int nthreads)
+{
+    int st = check_common(B, T, H, dk, dv, q, k, v, a, beta);
+    if (st != ORACLE_OK)
+        return st;
+    if (B * H == 0)
+        return ORACLE_OK;
+    if (T > 0 && (!dO || !dq || !dk_ || !dv_ || !da || !dbeta))
+        return ORACLE_ERR_ARG;
+    job_t J = {B, T, H, dk, dv, 0, q, k, v, a, beta, g_min, kind, S0, NULL, NULL, nthreads, 0, 0,
+               dO, dST, dq, dk_, dv_, da, dbeta, dS0};
+    return run_jobs(&J, backward_worker);
 }
 
 /* ------------------------------------------------------------------------------ */

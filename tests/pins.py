@@ -310,6 +310,97 @@ def pin_gate_head_scale(lib):
         "per-head scaled gate differs from g_min*expit(e^A a)"
 
 
+# ---------------------------------------------------------------------------- backward
+# The backward is the derivative of the recurrence: it is pinned by central finite
+# differences of the (separately pinned) forward, by the exact Euler identities of the
+# inputs the outputs are linear in, and by a hand-derived closed form at T = 1.
+
+
+def _grid_inputs(B, T, H, d, seed):
+    """Inputs on a 2^-8 grid (|x| < 4), so that x +- 2^-14 is exact in float32."""
+    rng = np.random.default_rng(seed)
+
+    def g8(x):
+        return (np.round(np.clip(x, -3.9, 3.9) * 256) / 256).astype(np.float32)
+
+    return dict(
+        q=g8(rng.normal(size=(B, T, H, d)) * 0.3), k=g8(rng.normal(size=(B, T, H, d)) * 0.3),
+        v=g8(rng.normal(size=(B, T, H, d))), a=g8(rng.normal(size=(B, T, H, d)) * 1.5),
+        beta=g8(rng.uniform(0.05, 0.95, size=(B, T, H))),
+        S0=g8(rng.normal(size=(B, H, d, d)) * 0.2).astype(np.float64),
+        dO=g8(rng.normal(size=(B, T, H, d))), dST=g8(rng.normal(size=(B, H, d, d))).astype(np.float64))
+
+
+def _loss(x, kind, lib):
+    o, ST = oracle.recurrence(x["q"], x["k"], x["v"], x["a"], x["beta"], G_MIN, S0=x["S0"], kind=kind, lib=lib)
+    return float(np.sum(o * x["dO"]) + np.sum(ST * x["dST"]))
+
+
+def pin_backward_finite_differences(lib):
+    """Every gradient against a central difference of L = <dO, o> + <dST, S_T>, at sampled
+    entries, for both gates; T = 70 spans the oracle's 64-token recompute segments."""
+    h = 2.0 ** -14
+    names = {"q": "dq", "k": "dk", "v": "dv", "a": "da", "beta": "dbeta", "S0": "dS0"}
+    for kind in (oracle.GATE_BOUNDED, oracle.GATE_LOGSIGMOID):
+        x = _grid_inputs(1, 70, 2, 8, seed=40 + kind)
+        grads = oracle.backward(x["q"], x["k"], x["v"], x["a"], x["beta"], x["dO"], G_MIN, S0=x["S0"],
+                                dST=x["dST"], kind=kind, lib=lib)
+        rng = np.random.default_rng(7 + kind)
+        for n, gname in names.items():
+            for _ in range(8):
+                idx = tuple(int(rng.integers(0, m)) for m in x[n].shape)
+                xp, xm = dict(x), dict(x)
+                xp[n] = x[n].copy()
+                xm[n] = x[n].copy()
+                xp[n][idx] += h
+                xm[n][idx] -= h
+                fd = (_loss(xp, kind, lib) - _loss(xm, kind, lib)) / (2 * h)
+                got = grads[gname][idx]
+                assert abs(got - fd) <= 1e-6 * max(abs(fd), 1e-3), f"d{n}{idx} (kind {kind}): {got} vs {fd}"
+
+
+def pin_backward_linear_inputs(lib):
+    """o and S_T are linear in (v, S0) jointly and o is linear in q, so (Euler) the loss
+    equals <dv, v> + <dS0, S0> exactly, and with dST = 0 it equals <dq, q>."""
+    x = _inputs(2, 45, 2, 16, seed=41)
+    rng = np.random.default_rng(42)
+    dO = rng.normal(size=x["v"].shape).astype(np.float32)
+    dST = rng.normal(size=x["S0"].shape)
+    o, ST = oracle.recurrence(x["q"], x["k"], x["v"], x["a"], x["beta"], G_MIN, S0=x["S0"], lib=lib)
+    g = oracle.backward(x["q"], x["k"], x["v"], x["a"], x["beta"], dO, G_MIN, S0=x["S0"], dST=dST, lib=lib)
+    L = np.sum(o * dO) + np.sum(ST * dST)
+    euler_vs = np.sum(g["dv"] * x["v"]) + np.sum(g["dS0"] * x["S0"])
+    assert abs(L - euler_vs) <= 1e-10 * max(abs(L), 1.0), (L, euler_vs)
+    g0 = oracle.backward(x["q"], x["k"], x["v"], x["a"], x["beta"], dO, G_MIN, S0=x["S0"], lib=lib)
+    Lo = np.sum(o * dO)
+    assert abs(Lo - np.sum(g0["dq"] * x["q"])) <= 1e-10 * max(abs(Lo), 1.0)
+
+
+def pin_backward_single_token_closed_form(lib):
+    """T = 1 from a zero state, by hand: o = b (k.q) v and S_T = b k v^T, so with weights
+    w = dO, W = dST the gradients are dq = b (v.w) k, dk = b (v.w) q + b W v,
+    dv = b (k.q) w + b W^T k, dbeta = (k.q)(v.w) + k^T W v and da = 0; and since
+    S_T = (I - b k k^T) D S0 + b k v^T, dS0 = D (I - b k k^T) (q w^T + W), D = Diag(e^g)."""
+    rng = np.random.default_rng(43)
+    d = 5
+    q, k, v, a, w = (rng.normal(size=(1, 1, 1, d)).astype(np.float32) for _ in range(5))
+    beta = np.array([[[0.625]]], np.float32)
+    W = rng.normal(size=(1, 1, d, d))
+    g = oracle.backward(q, k, v, a, beta, w, G_MIN, dST=W, lib=lib)
+    qq, kk, vv, ww = (np.asarray(x, np.float64).reshape(-1) for x in (q, k, v, w))
+    WW = W[0, 0]
+    b = 0.625
+    kq, vw = kk @ qq, vv @ ww
+    assert np.allclose(g["dq"].reshape(-1), b * vw * kk, rtol=1e-12, atol=1e-14)
+    assert np.allclose(g["dk"].reshape(-1), b * vw * qq + b * WW @ vv, rtol=1e-12, atol=1e-14)
+    assert np.allclose(g["dv"].reshape(-1), b * kq * ww + b * WW.T @ kk, rtol=1e-12, atol=1e-14)
+    assert np.isclose(g["dbeta"].reshape(()), kq * vw + kk @ WW @ vv, rtol=1e-12, atol=1e-14)
+    assert np.all(g["da"] == 0.0)
+    D = np.exp(G_MIN * scipy.special.expit(np.asarray(a, np.float64).reshape(-1)))
+    ref = D[:, None] * ((np.eye(d) - b * np.outer(kk, kk)) @ (np.outer(qq, ww) + WW))
+    assert np.allclose(g["dS0"][0, 0], ref, rtol=1e-12, atol=1e-14)
+
+
 ALL_PINS = [
     pin_gate_special_values,
     pin_gate_vs_library,
@@ -326,4 +417,7 @@ ALL_PINS = [
     pin_decode_step,
     pin_range_claim,
     pin_gate_head_scale,
+    pin_backward_finite_differences,
+    pin_backward_linear_inputs,
+    pin_backward_single_token_closed_form,
 ]

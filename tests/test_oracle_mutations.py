@@ -41,6 +41,15 @@ MUTATIONS = [
                                 "exp(G[(int64_t)s * dk + c] - G[(int64_t)r * dk + c]);\n                    A_rs", 0)]),
     ("tile_col_factor_sign", [("expf(Gf - Gr);", "expf(Gr - Gf);", 0)]),
     ("head_scale_ignored", [("const double scale = exp((double)A_log[h]);", "const double scale = 1.0;", 0)]),
+    ("bwd_erase_path_dropped", [("                               - Sd[(int64_t)i * dv + j] * beta * du[j];", "                               ;", 0)]),
+    ("bwd_dq_from_previous_state", [("acc += S_t[(int64_t)i * dv + j] * (double)dO[j];", "acc += S_prev[(int64_t)i * dv + j] * (double)dO[j];", 0)]),
+    ("bwd_state_grad_undecayed", [("dS[(int64_t)i * dv + j] = decay[i] * d;", "dS[(int64_t)i * dv + j] = d;", 0)]),
+    ("bwd_dg_uses_dS", [("dg += d * Sd[(int64_t)i * dv + j];", "dg += dS[(int64_t)i * dv + j] * Sd[(int64_t)i * dv + j];", 0)]),
+    ("bwd_dbeta_sign", [("db += du[j] * r[j];", "db -= du[j] * r[j];", 0)]),
+    ("bwd_dv_without_beta", [("dvv[j] = beta * du[j];", "dvv[j] = du[j];", 0)]),
+    ("bwd_gate_grad_missing_factor", [("return g_min * s * (1.0 - s);", "return g_min * s;", 0)]),
+    ("bwd_logsig_grad", [("    return 1.0 - s;\n}", "    return s;\n}", 0)]),
+    ("bwd_output_grad_transposed", [("dS[(int64_t)i * dv + j] += (double)q[i] * (double)dO[j];", "dS[(int64_t)i * dv + j] += (double)q[j] * (double)dO[i];", 0)]),
     ("head_scale_wrong_head", [("const double scale = exp((double)A_log[h]);",
                                 "const double scale = exp((double)A_log[0]);", 0)]),
 ]

@@ -59,6 +59,9 @@ EXPORTS = (
     "kda_gate_fwd_heads",
     "kda_chunk_fwd_scan_affine",
     "kda_state_combine",
+    "kda_chunk_bwd_workspace",
+    "kda_chunk_bwd_offsets",
+    "kda_chunk_bwd",
 )
 
 
@@ -118,6 +121,12 @@ def lib() -> ctypes.CDLL:
     L.kda_state_combine.argtypes = [I, I, I, I, I, P, P, P, P, P]
     L.kda_state_combine.restype = I
     L.kda_chunk_fwd_varlen.restype = I
+    L.kda_chunk_bwd_workspace.argtypes = [I, I, I, I, I, I]
+    L.kda_chunk_bwd_workspace.restype = S
+    L.kda_chunk_bwd_offsets.argtypes = [I, I, I, I, I, P, P]
+    L.kda_chunk_bwd_offsets.restype = I
+    L.kda_chunk_bwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_bwd.restype = I
     _lib = L
     return L
 
@@ -207,6 +216,55 @@ def kda_chunk_fwd(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=No
                              _stream(q.device))
     _raise(st, "kda_chunk_fwd")
     return o, S_T
+
+
+def kda_chunk_bwd_workspace(B: int, T: int, H: int, dk: int, dv: int, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(lib().kda_chunk_bwd_workspace(B, T, H, dk, dv, code))
+
+
+def kda_chunk_bwd_offsets(B: int, T: int, H: int, dk: int, dv: int):
+    """Byte offsets in the backward workspace of the saved chunk states and of the state
+    gradients (float32 [B, H, NT, dk, dv] each, NT = ceil(T / 64))."""
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = lib().kda_chunk_bwd_offsets(B, T, H, dk, dv, ctypes.byref(a), ctypes.byref(b))
+    _raise(st, "kda_chunk_bwd_offsets")
+    return int(a.value), int(b.value)
+
+
+def kda_chunk_bwd(q, k, v, a, beta, dO, g_min: float = -5.0, S0=None, dS_T=None, workspace=None,
+                  return_dS0: bool = True, out=None):
+    """Gradients of the bf16 chunked forward.  q, k, a [B,T,H,dk], v and dO [B,T,H,dv],
+    beta [B,T,H] (bfloat16); S0 and dS_T [B,H,dk,dv] float32 or None (zeros).  Returns a
+    dict of float32 tensors dq, dk, dv, da, dbeta and dS0 (None unless ``return_dS0``);
+    ``out`` may supply some of those tensors."""
+    _check_cuda(q, k, v, a, beta, dO, S0, dS_T, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, a, beta, dO)):
+        raise TypeError("kda_chunk_bwd takes bfloat16 q, k, v, a, beta, dO")
+    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or dO.shape != v.shape \
+            or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v,dO [B,T,H,dv], beta [B,T,H]")
+    dev = q.device
+    shapes = {"dq": q.shape, "dk": q.shape, "dv": v.shape, "da": q.shape, "dbeta": beta.shape,
+              "dS0": (B, H, dk, dv)}
+    g = dict(out or {})
+    for name, shp in shapes.items():
+        if name not in g and (name != "dS0" or return_dS0):
+            g[name] = torch.empty(shp, dtype=torch.float32, device=dev)
+    g.setdefault("dS0", None)
+    _check_cuda(*g.values())
+    need = int(lib().kda_chunk_bwd_workspace(B, T, H, dk, dv, KDA_BF16))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_bwd(B, T, H, dk, dv, KDA_BF16, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
+                             float(g_min), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]),
+                             _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), _ptr(workspace),
+                             ws_bytes, _stream(dev))
+    _raise(st, "kda_chunk_bwd")
+    return g
 
 
 def kda_chunk_fwd_logsigmoid(q, k, v, a, beta, S0=None, o=None, S_T=None, workspace=None,

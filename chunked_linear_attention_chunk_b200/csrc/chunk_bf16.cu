@@ -32,6 +32,8 @@
 // warp streams the records through a 3-stage mbarrier pipeline with bulk copies, and per
 // chunk one tcgen05 round computes [N S, Q' S] while four consumer warps, one TMEM lane
 // (= one state row or chunk row) per thread, keep the fp32 state block in registers.
+#include <algorithm>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "tcgen05.cuh"
@@ -955,11 +957,13 @@ __device__ __forceinline__ void store_state(unsigned char *sbuf, int row, const 
                        pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
 }
 
-template <int D, bool kAffine>
+// kSave: also write the fp32 state entering every chunk to Hs (one D x D block per record,
+// indexed like the records), for the backward.
+template <int D, bool kAffine, bool kSave>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, float *__restrict__ M_out,
-                unsigned int *status)
+                float *__restrict__ Hs, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char scan_smem[];
     using SM = ScanSmem<D>;
@@ -1051,6 +1055,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         uint32_t mma_phase = 0;
         for (int c = 0; c < NT; ++c) {
             const int s = c % kStages;
+            if constexpr (kSave) {
+                if (srow) {
+                    float4 *hp = reinterpret_cast<float4 *>(Hs + ((seq.rec0 + c) * D + row) * D + col0);
+#pragma unroll
+                    for (int j = 0; j < kBV; j += 4)
+                        hp[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                }
+            }
             mbar_wait_bounded(&sm.full[s], (c / kStages) & 1, status);
             const unsigned char *st = sm.stage[s];
             const uint32_t st_a = smem_u32(st);
@@ -1146,6 +1158,762 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ================================================================== backward
+// The chunked backward, derived from the chunked form above.  With dS' = dL/d(state after
+// the chunk) and dO = dL/dO (per chunk, entering state S):
+//   dU = Khat dS' + P^T dO,   dKhat = U dS'^T,   dQbar = dO S^T,   dP = lower_incl(dO U^T)
+//   dW = -dU S^T,   dGamma = rowsum(dS' * S),   dS = Diag(Gamma) dS' + Qbar^T dO - W^T dU
+// and, substituting dU, the state gradient walks the chunks backwards with the records the
+// forward wrote:
+//   dS = (Diag(Gamma) - N)^T dS' + Q'^T dO.
+// Through the WY form (W = T Bk, Utilde = T Bv, Bk = diag(beta) Kbar, Bv = diag(beta) V,
+// T = (I + A)^{-1}):  dBk = T^T dW,  dBv = T^T dU,  dT = dW Bk^T + dU Bv^T,
+// dA = -strict_lower(T^T dT T^T); then the pairwise decay products A and P hand their
+// gradients to q, k and the cumulative log-decay G, and dg is the reverse cumulative sum
+// of dG inside the chunk.
+//
+// Three launches after the forward prep: the scan again with the entering state of every
+// chunk saved (scan_kernel<.., kSave>), the reverse state-gradient scan (dscan_kernel,
+// tcgen05), and the per-chunk gradients (bwd_chunk_kernel).
+
+// ------------------------------------------------------------------ reverse state-gradient scan
+// One CTA per (32-column block of dv, sequence*head), chunks in reverse order.  Per chunk one
+// tcgen05 round computes [N^T dS' | Q'^T dO]: N and Q' are the record's K-major operands,
+// read here as MN-major (transposed) A operands; dS' (bf16 copy) and the chunk's dO block
+// are MN-major B operands.  The fp32 gradient block stays in registers, one row per thread.
+template <int D>
+struct DScanSmem {
+    // An M = 128 MN-major read of Q' (and of N when D = 64) covers two 64-row MN blocks; past
+    // the operand those bytes only feed accumulator lanes that are never read.
+    static constexpr uint32_t kRead = Rec<D>::Qp + 2u * kC * 128u > Rec<D>::Shared ? Rec<D>::Qp + 2u * kC * 128u
+                                                                                   : Rec<D>::Shared;
+    static constexpr uint32_t kStageStride = (kRead + 1023) / 1024 * 1024;
+    alignas(1024) unsigned char stage[kStages][kStageStride];
+    alignas(1024) unsigned char sbuf[D * kBV * 2];   // dS' block, bf16, MN-major 64-byte swizzle
+    alignas(1024) unsigned char obuf[kC * kBV * 2];  // dO block of the chunk, same layout (row = token)
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t mma_bar;
+    uint32_t tmem_slot;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kScanThreads, 1)
+    dscan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const __nv_bfloat16 *__restrict__ dO,
+                 const float *__restrict__ dS_T, float *__restrict__ dHs, float *__restrict__ dS0,
+                 unsigned int *status)
+{
+    extern __shared__ __align__(1024) unsigned char dscan_smem[];
+    using SM = DScanSmem<D>;
+    using R = Rec<D>;
+    SM &sm = *reinterpret_cast<SM *>(dscan_smem + ((1024u - (smem_u32(dscan_smem) & 1023u)) & 1023u));
+    constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N^T dS'; [kBV, 2 kBV): Q'^T dO
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int blk = blockIdx.x, col0 = blk * kBV;
+    const SeqLoc seq = locate_seq(map, H);
+    if constexpr (kDebugChecks) {
+        const int64_t span = min((int64_t)seq.len, (int64_t)seq.nchunks * kC);
+        if (seq.nchunks < 0 || (int64_t)seq.rec0 + seq.nchunks > map.nrec || seq.sh >= map.nseq * H ||
+            (span > 0 && (seq.tok0 < 0 || seq.tok0 + span > map.ntok))) {
+            if (threadIdx.x == 0)
+                report_device_error(status, KDA_ERR_DEVICE_BOUNDS);
+            return;
+        }
+    }
+    const int h = seq.h, NT = seq.nchunks, bh = seq.sh;
+    const unsigned char *recs = ws + seq.rec0 * R::Bytes;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.mma_bar, 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 0)
+        tc::tmem_alloc(&sm.tmem_slot, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_slot;
+
+    if (warp == kScanWarps) {
+        // ---------------- producer: the records' shared part, last chunk first
+        if (lane == 0) {
+            for (int i = 0; i < NT; ++i) {
+                const int c = NT - 1 - i, s = i % kStages;
+                if (i >= kStages)
+                    mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, status);
+                mbar_arrive_expect_tx(&sm.full[s], R::Shared);
+                bulk_g2s(sm.stage[s], recs + (size_t)c * R::Bytes, R::Shared, &sm.full[s]);
+            }
+        }
+        __syncwarp();
+    } else {
+        const int row = warp * 32 + lane;
+        const bool srow = row < D;    // owns gradient row `row` (key channel)
+        const bool trow = row < kC;   // loads token row `row` of the chunk's dO block
+        const uint32_t lane_addr = tc::taddr(tmem, (uint32_t)warp * 32, 0);
+        float S[kBV];
+#pragma unroll
+        for (int j = 0; j < kBV; ++j)
+            S[j] = 0.f;
+        if (srow && dS_T) {
+#pragma unroll
+            for (int j = 0; j < kBV; j += 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(&dS_T[((size_t)bh * D + row) * D + col0 + j]);
+                S[j] = v.x;
+                S[j + 1] = v.y;
+                S[j + 2] = v.z;
+                S[j + 3] = v.w;
+            }
+        }
+        // dO row of chunk c (zero past the sequence)
+        auto load_do = [&](int c, uint4 (&r)[4]) {
+            const int t = c * kC + row;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                r[q] = make_uint4(0u, 0u, 0u, 0u);
+            if (trow && t < seq.len) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(dO + ((seq.tok0 + t) * H + h) * D + col0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    r[q] = p[q];
+            }
+        };
+        uint4 cur[4];
+        if (NT > 0)
+            load_do(NT - 1, cur);
+
+        const uint32_t id_t = tc::idesc_bf16(128, kBV, true, true);  // A MN-major, B MN-major
+        const uint32_t sbuf_a = smem_u32(sm.sbuf), obuf_a = smem_u32(sm.obuf);
+        uint32_t mma_phase = 0;
+        for (int i = 0; i < NT; ++i) {
+            const int c = NT - 1 - i, s = i % kStages;
+            // dS' of chunk c (the gradient of the state after it) is what the rows hold now
+            if (srow) {
+                float4 *hp = reinterpret_cast<float4 *>(dHs + ((seq.rec0 + c) * D + row) * D + col0);
+#pragma unroll
+                for (int j = 0; j < kBV; j += 4)
+                    hp[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                store_state(sm.sbuf, row, S);
+            }
+            if (trow) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(sm.obuf + tc::mnmaj_sw64(row, q * 8)) = cur[q];
+                if (c > 0)
+                    load_do(c - 1, cur);
+            }
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            consumer_sync();
+            tc::fence_after_sync();
+            mbar_wait_bounded(&sm.full[s], (i / kStages) & 1, status);
+            const unsigned char *st = sm.stage[s];
+            const uint32_t st_a = smem_u32(st);
+            if (tid == 0) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t an = tc::smem_desc(st_a + R::Nm + ks * 2048, D * 128, 1024, tc::kSw128);
+                    const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
+                    tc::mma_bf16(tmem, an, bd, id_t, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks) {
+                    const uint64_t aq = tc::smem_desc(st_a + R::Qp + ks * 2048, kC * 128, 1024, tc::kSw128);
+                    const uint64_t bo = tc::smem_desc(obuf_a + ks * 1024, 0, 512, tc::kSw64);
+                    tc::mma_bf16(tmem + kBV, aq, bo, id_t, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(&sm.mma_bar);
+            }
+            if (srow) {
+                const float g = reinterpret_cast<const float *>(st + R::Gam)[row];
+#pragma unroll
+                for (int j = 0; j < kBV; ++j)
+                    S[j] *= g;
+            }
+            mbar_wait_bounded(&sm.mma_bar, mma_phase, status);
+            mma_phase ^= 1;
+            tc::fence_after_sync();
+            if (srow) {
+                uint32_t d[kBV], y[kBV];
+                tc::ld_32x32b_x32(lane_addr, d);
+                tc::ld_32x32b_x32(lane_addr + kBV, y);
+                tc::wait_ld();
+#pragma unroll
+                for (int j = 0; j < kBV; ++j)
+                    S[j] += __uint_as_float(y[j]) - __uint_as_float(d[j]);
+            }
+            tc::fence_before_sync();
+            consumer_sync();
+            tc::fence_after_sync();
+            if (tid == 0)
+                mbar_arrive_local(&sm.empty[s]);
+        }
+        if (dS0 && srow)
+#pragma unroll
+            for (int j = 0; j < kBV; j += 4)
+                *reinterpret_cast<float4 *>(&dS0[((size_t)bh * D + row) * D + col0 + j]) =
+                    make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ per-chunk gradients
+// Persistent: kBwdSlots CTAs of 512 threads walk the chunks.  q, k, G and the chunk's 64 x 64
+// matrices stay in shared memory; the 64 x D intermediates live in a float32 scratch slot of
+// the workspace per CTA (small enough to stay in L2).  Dense contractions go through
+// cta_gemm (TF32 mma.sync, fp32 accumulation).  The pairwise decay products are 16 x 16
+// tile pairs on the same mma, with the decay factored through a reference token of the row
+// tile, exactly as in the forward: the tile's first token for tiles below the diagonal
+// (both factors <= 1), its middle token on the diagonal (factors <= e^{8 |g_min|}).
+constexpr int kBwdThreads = 512;
+constexpr int kBwdWarps = kBwdThreads / 32;
+constexpr int kBwdSlots = 148;  // one CTA per SM of a 148-SM part
+
+template <int D>
+struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blocks
+    static constexpr int CD = kC * D;
+    static constexpr int Kb = 0, Kh = Kb + CD, Qb = Kh + CD;
+    static constexpr int Bk = Qb + CD;   // diag(beta) Kbar, later dBk
+    static constexpr int Bv = Bk + CD;   // diag(beta) V, later dBv
+    static constexpr int W = Bv + CD;    // W, then dW, then the pairwise dq
+    static constexpr int U = W + CD;     // Utilde, U, then dk
+    static constexpr int dO = U + CD;    // dO, then the pairwise dG
+    static constexpr int dU = dO + CD;
+    static constexpr int dKh = dU + CD;
+    static constexpr int dQb = dKh + CD;
+    static constexpr int Gp = dQb + CD;  // dg/da = g_min sigma(a) (1 - sigma(a))
+    static constexpr int floats = Gp + CD;
+};
+
+constexpr int kGTM = 64, kGTN = 64, kGTK = 32;
+constexpr int kGLDA = kGTK + 4, kGLDB = kGTN + 8;  // conflict-free fragment reads
+constexpr int kGStage = kGTM * kGLDA + kGTK * kGLDB;
+constexpr int kGPA = kGTM * kGTK / kBwdThreads, kGPB = kGTK * kGTN / kBwdThreads;
+
+template <int D>
+struct BwdSmem {  // float offsets in shared memory
+    static constexpr int LDD = D + 4;    // conflict-free mma fragment reads
+    static constexpr int LDC = kC + 4;
+    static constexpr int q = 0, k = q + kC * LDD, G = k + kC * LDD;  // q later holds dG
+    static constexpr int Ap = G + kC * LDD, P = Ap + kC * LDC, T = P + kC * LDC;
+    static constexpr int dT = T + kC * LDC;  // dT, then dP
+    static constexpr int X = dT + kC * LDC, dA = X + kC * LDC;
+    static constexpr int stage = dA + kC * LDC;
+    static constexpr int beta = stage + kGStage;
+    static constexpr int dGam = beta + kC;
+    static constexpr int seg = dGam + D;  // row-segment sums: of dG, then of dKhat * Khat
+    static constexpr int floats = seg + 2 * kBwdThreads;
+    static constexpr size_t bytes = (size_t)floats * 4;
+    static_assert(bytes <= 232448, "shared memory per block");
+};
+
+// Strided fp32 matrix view: element (i, j) at p[i * rs + j * cs] (shared or global memory).
+struct MatV {
+    const float *p;
+    int rs, cs;
+    __device__ __forceinline__ float at(int i, int j) const { return p[(int64_t)i * rs + (int64_t)j * cs]; }
+};
+
+// C[M x N] = A[M x K] B[K x N] on the whole CTA (M, N, K multiples of 64, 64, 32); every
+// output element goes to epi(i, j, value) exactly once, from a thread fixed by (M, N).
+// Operands are staged through shared memory as TF32 in 64 x 32 / 32 x 64 tiles, the next
+// tile fetched into registers while the tensor cores work on the current one; warp w
+// computes rows 16 (w / 4) .. + 16 and columns 16 (w % 4) .. + 16 of each 64 x 64 tile.
+template <class Epi>
+__device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, Epi epi)
+{
+    uint32_t *sA = stage, *sB = stage + kGTM * kGLDA;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int wm = (warp >> 2) * 16, wn = (warp & 3) * 16;
+    float ra[kGPA], rb[kGPB];
+    auto fetch = [&](int m0, int n0, int k0) {
+#pragma unroll
+        for (int p = 0; p < kGPA; ++p) {
+            const int e = tid + p * kBwdThreads;
+            const int i = A.cs == 1 ? e / kGTK : e % kGTM, kk = A.cs == 1 ? e % kGTK : e / kGTM;
+            ra[p] = A.at(m0 + i, k0 + kk);
+        }
+#pragma unroll
+        for (int p = 0; p < kGPB; ++p) {
+            const int e = tid + p * kBwdThreads;
+            const int kk = B.cs == 1 ? e / kGTN : e % kGTK, j = B.cs == 1 ? e % kGTN : e / kGTK;
+            rb[p] = B.at(k0 + kk, n0 + j);
+        }
+    };
+    fetch(0, 0, 0);
+    for (int m0 = 0; m0 < M; m0 += kGTM)
+        for (int n0 = 0; n0 < N; n0 += kGTN) {
+            float acc[2][4] = {};
+            for (int k0 = 0; k0 < K; k0 += kGTK) {
+                __syncthreads();  // the previous tile's readers are done
+#pragma unroll
+                for (int p = 0; p < kGPA; ++p) {
+                    const int e = tid + p * kBwdThreads;
+                    const int i = A.cs == 1 ? e / kGTK : e % kGTM, kk = A.cs == 1 ? e % kGTK : e / kGTM;
+                    sA[i * kGLDA + kk] = to_tf32(ra[p]);
+                }
+#pragma unroll
+                for (int p = 0; p < kGPB; ++p) {
+                    const int e = tid + p * kBwdThreads;
+                    const int kk = B.cs == 1 ? e / kGTN : e % kGTK, j = B.cs == 1 ? e % kGTN : e / kGTK;
+                    sB[kk * kGLDB + j] = to_tf32(rb[p]);
+                }
+                __syncthreads();
+                // the next tile, in this output tile or the next one
+                if (k0 + kGTK < K)
+                    fetch(m0, n0, k0 + kGTK);
+                else if (n0 + kGTN < N)
+                    fetch(m0, n0 + kGTN, 0);
+                else if (m0 + kGTM < M)
+                    fetch(m0 + kGTM, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < kGTK; kk += 8) {
+                    uint32_t af[4];
+                    af[0] = sA[(wm + g) * kGLDA + kk + t];
+                    af[1] = sA[(wm + g + 8) * kGLDA + kk + t];
+                    af[2] = sA[(wm + g) * kGLDA + kk + t + 4];
+                    af[3] = sA[(wm + g + 8) * kGLDA + kk + t + 4];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        uint32_t bf[2];
+                        bf[0] = sB[(kk + t) * kGLDB + wn + nt * 8 + g];
+                        bf[1] = sB[(kk + t + 4) * kGLDB + wn + nt * 8 + g];
+                        mma_tf32_1688(acc[nt], af, bf);
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int i = m0 + wm + g, j = n0 + wn + nt * 8 + 2 * t;
+                epi(i, j, acc[nt][0]);
+                epi(i, j + 1, acc[nt][1]);
+                epi(i + 8, j, acc[nt][2]);
+                epi(i + 8, j + 1, acc[nt][3]);
+            }
+        }
+    __syncthreads();
+}
+
+// One tile pair (I, J), J <= I, of the forward pairwise products on one warp:
+//   A'_rs = sum_c k_rc k_sc e^{G_rc - G_sc} (s < r),  P_rs = sum_c q_rc k_sc e^{..} (s <= r)
+// with e^{G_r - G_s} = e^{G_r - G_m} e^{G_m - G_s}, m the reference token of tile I.
+template <int D>
+__device__ void pair_fwd_tile(const float *sq, const float *sk, const float *sG, float *Ap, float *P, int I, int J,
+                              int lane)
+{
+    using SL = BwdSmem<D>;
+    constexpr int LDD = SL::LDD, LDC = SL::LDC;
+    const int g = lane >> 2, t = lane & 3;
+    const int m = J < I ? I * kTile : I * kTile + kRef;
+    const int r0 = I * kTile, s0 = J * kTile;
+    float aA[2][4] = {}, aP[2][4] = {};
+#pragma unroll 2
+    for (int kk = 0; kk < D; kk += 8) {
+        uint32_t fk[4], fq[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int r = r0 + g + (x & 1) * 8, c = kk + t + (x >> 1) * 4;
+            const float f = __expf(sG[r * LDD + c] - sG[m * LDD + c]);
+            fk[x] = to_tf32(sk[r * LDD + c] * f);
+            fq[x] = to_tf32(sq[r * LDD + c] * f);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t b[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int c = kk + t + x * 4, s = s0 + nt * 8 + g;
+                b[x] = to_tf32(sk[s * LDD + c] * __expf(sG[m * LDD + c] - sG[s * LDD + c]));
+            }
+            mma_tf32_1688(aA[nt], fk, b);
+            mma_tf32_1688(aP[nt], fq, b);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int r = r0 + g + (x >> 1) * 8, s = s0 + nt * 8 + 2 * t + (x & 1);
+            Ap[r * LDC + s] = s < r ? aA[nt][x] : 0.f;
+            P[r * LDC + s] = s <= r ? aP[nt][x] : 0.f;
+        }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_chunk_kernel(SeqMap map, int H, int nunits, const __nv_bfloat16 *__restrict__ qg,
+                     const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ vg,
+                     const __nv_bfloat16 *__restrict__ ag, const __nv_bfloat16 *__restrict__ betag, float g_min,
+                     const __nv_bfloat16 *__restrict__ dOg, const float *__restrict__ Hs,
+                     const float *__restrict__ dHs, float *scratch, float *__restrict__ dq, float *__restrict__ dk,
+                     float *__restrict__ dv, float *__restrict__ da, float *__restrict__ dbeta, unsigned int *status)
+{
+    using L = BwdSlot<D>;
+    using SL = BwdSmem<D>;
+    constexpr int CD = kC * D, LDD = SL::LDD, LDC = SL::LDC;
+    constexpr int NH = D / 64;  // 64-channel halves handled per warp in the pairwise backward
+    extern __shared__ __align__(16) float bsm[];
+    float *const sq = bsm + SL::q, *const sk = bsm + SL::k, *const sG = bsm + SL::G;
+    float *const sAp = bsm + SL::Ap, *const sP = bsm + SL::P, *const sT = bsm + SL::T;
+    float *const sdT = bsm + SL::dT, *const sX = bsm + SL::X, *const sdA = bsm + SL::dA;
+    uint32_t *const stage = reinterpret_cast<uint32_t *>(bsm + SL::stage);
+    float *const sbeta = bsm + SL::beta, *const sdGam = bsm + SL::dGam;
+    float *const sseg = bsm + SL::seg;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *sl = scratch + (size_t)blockIdx.x * L::floats;
+    float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Qb = sl + L::Qb, *const Bk = sl + L::Bk;
+    float *const Bv = sl + L::Bv, *const W = sl + L::W, *const U = sl + L::U, *const dOs = sl + L::dO;
+    float *const dU = sl + L::dU, *const dKh = sl + L::dKh, *const dQb = sl + L::dQb, *const Gp = sl + L::Gp;
+
+    for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
+        // regular batch: unit = (b*H + h) * NT + chunk; packed batch: unit = h * NT + chunk slot
+        const ChunkLoc loc = locate_chunk(map, H, unit % map.NT, unit / map.NT);
+        if (!loc.live)
+            continue;
+        if constexpr (kDebugChecks) {
+            if (loc.n < 1 || loc.n > kC || (int64_t)loc.rec >= map.nrec || loc.tok0 < 0 ||
+                loc.tok0 + loc.n > map.ntok) {
+                if (tid == 0)
+                    report_device_error(status, KDA_ERR_DEVICE_BOUNDS);
+                return;
+            }
+        }
+        const int n = loc.n, h = loc.h;
+        const int64_t tok0 = loc.tok0;
+        const float *S = Hs + loc.rec * (size_t)D * D;
+        const float *dSn = dHs + loc.rec * (size_t)D * D;
+        auto tix = [&](int r) { return (tok0 + r) * H + h; };  // token-head row index
+
+        // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da
+#pragma unroll 4
+        for (int e = tid; e < CD; e += kBwdThreads) {
+            const int r = e / D, c = e % D;
+            const bool ok = r < n;
+            const size_t gi = (size_t)tix(ok ? r : 0) * D + c;
+            const float av = __bfloat162float(ag[gi]);
+            const float sg = __fdividef(1.f, 1.f + __expf(-av));
+            sq[r * LDD + c] = ok ? __bfloat162float(qg[gi]) : 0.f;
+            sk[r * LDD + c] = ok ? __bfloat162float(kg[gi]) : 0.f;
+            sG[r * LDD + c] = ok ? gate_bounded_fast(av, g_min) : 0.f;
+            Gp[e] = g_min * sg * (1.f - sg);
+            Bv[e] = ok ? __bfloat162float(vg[gi]) : 0.f;
+            dOs[e] = ok ? __bfloat162float(dOg[gi]) : 0.f;
+        }
+        for (int r = tid; r < kC; r += kBwdThreads)
+            sbeta[r] = r < n ? __bfloat162float(betag[tix(r)]) : 0.f;
+        __syncthreads();
+        // 2. G = inclusive cumulative sum over the chunk, per channel
+        for (int c = tid; c < D; c += kBwdThreads) {
+            float acc = 0.f;
+            for (int r = 0; r < kC; ++r) {
+                acc += sG[r * LDD + c];
+                sG[r * LDD + c] = acc;
+            }
+        }
+        __syncthreads();
+        // 3. decay-scaled operands (scratch) and 4. the pairwise products A', P (warps 0..9)
+        for (int e = tid; e < CD; e += kBwdThreads) {
+            const int r = e / D, c = e % D;
+            const float Gv = sG[r * LDD + c], e1 = __expf(Gv), eh = __expf(sG[(kC - 1) * LDD + c] - Gv);
+            const float kv = sk[r * LDD + c];
+            Kb[e] = kv * e1;
+            Kh[e] = kv * eh;
+            Qb[e] = sq[r * LDD + c] * e1;
+            Bk[e] = sbeta[r] * kv * e1;
+            Bv[e] *= sbeta[r];
+        }
+        if (warp < kTiles * (kTiles + 1) / 2) {
+            int I = 0, J = warp;  // warp -> (I, J), J <= I, row by row
+            while (J > I) {
+                J -= I + 1;
+                ++I;
+            }
+            pair_fwd_tile<D>(sq, sk, sG, sAp, sP, I, J, lane);
+        }
+        for (int e = tid; e < kC * kC; e += kBwdThreads) {
+            const int r = e / kC, s = e % kC;
+            sT[r * LDC + s] = r == s ? 1.f : 0.f;
+            if (s / kTile > r / kTile)  // tiles above the diagonal (the pairwise tiles write the rest)
+                sAp[r * LDC + s] = sP[r * LDC + s] = 0.f;
+        }
+        __syncthreads();
+        // 5. T = (I + A)^{-1}, A = diag(beta) A', unit lower triangular, by 16 x 16 blocks: the
+        //    diagonal blocks by forward substitution (one warp each), then block rows by level,
+        //    T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
+        if (warp < kTiles) {
+            const int b0 = warp * kTile, j = lane & 15;
+            for (int rr = 1; rr < kTile; ++rr) {
+                const int r = b0 + rr;
+                float acc = 0.f;
+                if (lane < kTile && j < rr)
+                    for (int s = j; s < rr; ++s)
+                        acc = fmaf(sAp[r * LDC + b0 + s], sT[(b0 + s) * LDC + b0 + j], acc);
+                __syncwarp();
+                if (lane < kTile && j < rr)
+                    sT[r * LDC + b0 + j] = -sbeta[r] * acc;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        for (int lvl = 1; lvl < kTiles; ++lvl) {
+            if (warp < kTiles - lvl) {
+                const int J = warp, I = warp + lvl;
+                const int rr = lane >> 1, j0 = (lane & 1) * 8, r = I * kTile + rr;
+                float x[8] = {};
+                for (int K = J; K < I; ++K)
+                    for (int s = 0; s < kTile; ++s) {
+                        const float av = sAp[r * LDC + K * kTile + s];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            x[u] = fmaf(av, sT[(K * kTile + s) * LDC + J * kTile + j0 + u], x[u]);
+                    }
+                float *Xs = sX + warp * kTile * LDC;  // 16 x 16 per warp (sX is free until step 6)
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    Xs[rr * LDC + j0 + u] = sbeta[r] * x[u];
+                __syncwarp();
+                float y[8] = {};
+                for (int uu = 0; uu < kTile; ++uu) {
+                    const float tv = sT[r * LDC + I * kTile + uu];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        y[u] = fmaf(tv, Xs[uu * LDC + j0 + u], y[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    sT[r * LDC + J * kTile + j0 + u] = -y[u];
+            }
+            __syncthreads();
+        }
+        // 6. dense contractions
+        const MatV Tn{sT, LDC, 1}, Tt{sT, 1, LDC};
+        cta_gemm(kC, D, kC, Tn, MatV{Bk, D, 1}, stage, [&](int i, int j, float x) { W[i * D + j] = x; });
+        cta_gemm(kC, D, kC, Tn, MatV{Bv, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] = x; });
+        cta_gemm(kC, D, D, MatV{W, D, 1}, MatV{S, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] -= x; });
+        cta_gemm(kC, D, D, MatV{Kh, D, 1}, MatV{dSn, D, 1}, stage, [&](int i, int j, float x) { dU[i * D + j] = x; });
+        cta_gemm(kC, D, kC, MatV{sP, 1, LDC}, MatV{dOs, D, 1}, stage,
+                 [&](int i, int j, float x) { dU[i * D + j] += x; });
+        cta_gemm(kC, D, D, MatV{U, D, 1}, MatV{dSn, 1, D}, stage, [&](int i, int j, float x) { dKh[i * D + j] = x; });
+        cta_gemm(kC, D, D, MatV{dOs, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { dQb[i * D + j] = x; });
+        cta_gemm(kC, D, D, MatV{dU, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { W[i * D + j] = -x; });
+        float *const dW = W;
+        // dGamma_i = sum_j dS'_ij S_ij, warp per row
+#pragma unroll
+        for (int ii = 0; ii < D / kBwdWarps; ++ii) {
+            const int i = warp + ii * kBwdWarps;
+            float acc = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < D / 32; ++jj)
+                acc = fmaf(dSn[(size_t)i * D + lane + 32 * jj], S[(size_t)i * D + lane + 32 * jj], acc);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0)
+                sdGam[i] = acc;
+        }
+        cta_gemm(kC, kC, D, MatV{dW, D, 1}, MatV{Bk, 1, D}, stage,
+                 [&](int i, int j, float x) { sdT[i * LDC + j] = x; });
+        cta_gemm(kC, kC, D, MatV{dU, D, 1}, MatV{Bv, 1, D}, stage,
+                 [&](int i, int j, float x) { sdT[i * LDC + j] += x; });
+        cta_gemm(kC, D, kC, Tt, MatV{dW, D, 1}, stage, [&](int i, int j, float x) { Bk[i * D + j] = x; });
+        cta_gemm(kC, D, kC, Tt, MatV{dU, D, 1}, stage, [&](int i, int j, float x) { Bv[i * D + j] = x; });
+        cta_gemm(kC, kC, kC, MatV{sdT, LDC, 1}, Tt, stage, [&](int i, int j, float x) { sX[i * LDC + j] = x; });
+        cta_gemm(kC, kC, kC, Tt, MatV{sX, LDC, 1}, stage,
+                 [&](int i, int j, float x) { sdA[i * LDC + j] = j < i ? -x : 0.f; });
+        cta_gemm(kC, kC, D, MatV{dOs, D, 1}, MatV{U, 1, D}, stage,
+                 [&](int i, int j, float x) { sdT[i * LDC + j] = j <= i ? x : 0.f; });
+        float *const dBk = Bk, *const dBv = Bv, *const sdP = sdT;  // dA' = diag(beta) dA
+        // 7. pairwise products backward, rows: for r in tile I, channels of one 64-wide half,
+        //    dq_r = sum_{s<=r} dP_rs k_s E_rs,  dk_r = sum_{s<r} dA'_rs k_s E_rs,  dG_r = q_r dq_r + k_r dk_r
+        //    (E_rs = e^{G_r - G_s} per channel), one warp per (I, half).  dq -> W, dk -> U, dG -> dO.
+        if (warp < kTiles * NH) {
+            const int I = warp / NH, c0 = (warp % NH) * 64, g = lane >> 2, t = lane & 3;
+            for (int pass = 0; pass < 2; ++pass) {  // 0: tiles J < I (reference 16 I), 1: J = I (middle)
+                const int m = pass == 0 ? I * kTile : I * kTile + kRef;
+                float aq[8][4] = {}, ak[8][4] = {};
+                const int J0 = pass == 0 ? 0 : I, J1 = pass == 0 ? I : I + 1;
+                for (int J = J0; J < J1; ++J) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t fp[4], fa[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const int r = I * kTile + g + (x & 1) * 8, s = J * kTile + ks * 8 + t + (x >> 1) * 4;
+                            fp[x] = to_tf32(sdP[r * LDC + s]);
+                            fa[x] = to_tf32(sbeta[r] * sdA[r * LDC + s]);
+                        }
+#pragma unroll
+                        for (int nf = 0; nf < 8; ++nf) {
+                            uint32_t b[2];
+#pragma unroll
+                            for (int x = 0; x < 2; ++x) {
+                                const int s = J * kTile + ks * 8 + t + x * 4, c = c0 + nf * 8 + g;
+                                b[x] = to_tf32(sk[s * LDD + c] * __expf(sG[m * LDD + c] - sG[s * LDD + c]));
+                            }
+                            mma_tf32_1688(aq[nf], fp, b);
+                            mma_tf32_1688(ak[nf], fa, b);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int r = I * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
+                        const float f = __expf(sG[r * LDD + c] - sG[m * LDD + c]);
+                        const float vq = aq[nf][x] * f, vk = ak[nf][x] * f;
+                        const float dg = sq[r * LDD + c] * vq + sk[r * LDD + c] * vk;
+                        if (pass == 0) {
+                            W[r * D + c] = vq;
+                            U[r * D + c] = vk;
+                            dOs[r * D + c] = dg;
+                        } else {
+                            W[r * D + c] += vq;
+                            U[r * D + c] += vk;
+                            dOs[r * D + c] += dg;
+                        }
+                    }
+            }
+        }
+        __syncthreads();
+        //    columns: dk_s += sum_{r>=s} (dP_rs q_r + dA'_rs k_r) E_rs and dG_s -= k_s (that sum), one
+        //    warp per (column tile J, half); each row tile I >= J has its own reference.
+        if (warp < kTiles * NH) {
+            const int J = warp / NH, c0 = (warp % NH) * 64, g = lane >> 2, t = lane & 3;
+            float tot[8][4] = {};
+            for (int I = J; I < kTiles; ++I) {
+                const int m = I > J ? I * kTile : I * kTile + kRef;
+                float acc[8][4] = {};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t fp[4], fa[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {  // A(s, r) = dP_rs: s = row of the product
+                        const int s = J * kTile + g + (x & 1) * 8, r = I * kTile + ks * 8 + t + (x >> 1) * 4;
+                        fp[x] = to_tf32(sdP[r * LDC + s]);
+                        fa[x] = to_tf32(sbeta[r] * sdA[r * LDC + s]);
+                    }
+#pragma unroll
+                    for (int nf = 0; nf < 8; ++nf) {
+                        uint32_t bq[2], bk[2];
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            const int r = I * kTile + ks * 8 + t + x * 4, c = c0 + nf * 8 + g;
+                            const float f = __expf(sG[r * LDD + c] - sG[m * LDD + c]);
+                            bq[x] = to_tf32(sq[r * LDD + c] * f);
+                            bk[x] = to_tf32(sk[r * LDD + c] * f);
+                        }
+                        mma_tf32_1688(acc[nf], fp, bq);
+                        mma_tf32_1688(acc[nf], fa, bk);
+                    }
+                }
+#pragma unroll
+                for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int s = J * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
+                        tot[nf][x] = fmaf(acc[nf][x], __expf(sG[m * LDD + c] - sG[s * LDD + c]), tot[nf][x]);
+                    }
+            }
+#pragma unroll
+            for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int s = J * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
+                    U[s * D + c] += tot[nf][x];
+                    dOs[s * D + c] -= sk[s * LDD + c] * tot[nf][x];
+                }
+        }
+        __syncthreads();
+        // 8. the decay-scaled operands' gradients; outputs dq, dk, dv; dG -> sq
+#pragma unroll 2
+        for (int e = tid; e < CD; e += kBwdThreads) {
+            const int r = e / D, c = e % D;
+            const float Gv = sG[r * LDD + c], e1 = __expf(Gv), eh = __expf(sG[(kC - 1) * LDD + c] - Gv);
+            const float kv = sk[r * LDD + c];
+            const float dkb = sbeta[r] * dBk[e];
+            const float dqv = W[e] + dQb[e] * e1;
+            const float dkv = U[e] + dkb * e1 + dKh[e] * eh;
+            sq[r * LDD + c] = dOs[e] + (dQb[e] * sq[r * LDD + c] + dkb * kv) * e1 - dKh[e] * kv * eh;
+            if (r < n) {
+                const size_t gi = (size_t)tix(r) * D + c;
+                dq[gi] = dqv;
+                dk[gi] = dkv;
+                dv[gi] = sbeta[r] * dBv[e];
+            }
+        }
+        __syncthreads();
+        // 9. dg = reverse cumulative sum of dG (G_last also carries Gamma and Khat); da = dg g'(a).
+        //    Thread (segment, channel): sums of row segments first, then each segment's scan.
+        constexpr int NSEG = kBwdThreads / D, SR = kC / NSEG;
+        {
+            const int c = tid % D, sgi = tid / D, r0 = sgi * SR;
+            const float Gl = sG[(kC - 1) * LDD + c];
+            float loc = 0.f, lkh = 0.f;  // dG, and dKhat * Khat (G_last's share), over the segment
+#pragma unroll
+            for (int u = 0; u < SR; ++u) {
+                const int r = r0 + u;
+                loc += sq[r * LDD + c];
+                lkh = fmaf(dKh[r * D + c] * sk[r * LDD + c], __expf(Gl - sG[r * LDD + c]), lkh);
+            }
+            sseg[sgi * D + c] = loc;
+            sseg[kBwdThreads + sgi * D + c] = lkh;
+        }
+        __syncthreads();
+        {
+            const int c = tid % D, sgi = tid / D, r0 = sgi * SR;
+            float gp[SR];
+#pragma unroll
+            for (int u = 0; u < SR; ++u)
+                gp[u] = Gp[(r0 + u) * D + c];
+            float acc = sdGam[c] * __expf(sG[(kC - 1) * LDD + c]);
+            for (int s2 = 0; s2 < NSEG; ++s2)
+                acc += sseg[kBwdThreads + s2 * D + c];
+            for (int s2 = sgi + 1; s2 < NSEG; ++s2)
+                acc += sseg[s2 * D + c];
+#pragma unroll
+            for (int u = SR - 1; u >= 0; --u) {
+                const int r = r0 + u;
+                acc += sq[r * LDD + c];
+                if (r < n)
+                    da[(size_t)tix(r) * D + c] = acc * gp[u];
+            }
+        }
+        // 10. dbeta_r = sum_c dBk_rc Kbar_rc + sum_c dBv_rc v_rc + sum_s dA_rs A'_rs; warp per row
+#pragma unroll
+        for (int rr = 0; rr < kC / kBwdWarps; ++rr) {
+            const int r = warp + rr * kBwdWarps;
+            if (r >= n)
+                break;
+            float acc = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                const int c = lane + 32 * cc;
+                acc += dBk[r * D + c] * Kb[r * D + c] +
+                       dBv[r * D + c] * __bfloat162float(vg[(size_t)tix(r) * D + c]);
+            }
+#pragma unroll
+            for (int ss = 0; ss < kC / 32; ++ss)
+                acc += sdA[r * LDC + lane + 32 * ss] * sAp[r * LDC + lane + 32 * ss];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0)
+                dbeta[tix(r)] = acc;
+        }
+        __syncthreads();  // shared memory and the slot are reused by the next chunk
+    }
+}
+
 template <int D, bool kLogSig>
 cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, const void *k, const void *v,
                           const void *a, const void *beta, float g_min, const float *A_log, void *ws, cudaStream_t s)
@@ -1166,19 +1934,19 @@ cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, cons
 
 template <int D>
 cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S0, void *o, float *S_T,
-                          float *M_out, cudaStream_t s)
+                          float *M_out, cudaStream_t s, float *Hs = nullptr)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
     const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
     // with M_out: the state blocks and, after them, as many transfer-map blocks
-    auto kernel = M_out ? scan_kernel<D, true> : scan_kernel<D, false>;
+    auto kernel = Hs ? scan_kernel<D, false, true> : M_out ? scan_kernel<D, true, false> : scan_kernel<D, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     kernel<<<dim3((M_out ? 2 : 1) * (D / kBV), m.nseq * H), kScanThreads, smem, s>>>(
-        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, M_out, status);
+        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, M_out, Hs, status);
     return cudaGetLastError();
 }
 
@@ -1198,6 +1966,65 @@ cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const flo
 {
     return D == 64 ? launch_scan_d<64>(m, H, ws, S0, o, S_T, M_out, s)
                    : launch_scan_d<128>(m, H, ws, S0, o, S_T, M_out, s);
+}
+
+// Backward workspace: the forward records, then the entering state of every chunk and the
+// gradient of the state after it (fp32, D x D per record, in record order), then the
+// per-CTA scratch slots of bwd_chunk_kernel.
+struct BwdLayout {
+    size_t states, dstates, scratch, total;
+};
+
+BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D)
+{
+    const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
+    const size_t blk = (size_t)D * D * 4;
+    const size_t slot = (size_t)(D == 64 ? BwdSlot<64>::floats : BwdSlot<128>::floats) * 4;
+    BwdLayout l;
+    l.states = ((size_t)nrec * rec + 255) / 256 * 256;
+    l.dstates = l.states + (size_t)nrec * blk;
+    l.scratch = l.dstates + (size_t)nrec * blk;
+    l.total = l.scratch + (size_t)std::min<int64_t>(nunits, kBwdSlots) * slot;
+    return l;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
+                         const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da, float *dbeta,
+                         float *dS0, void *ws, cudaStream_t s)
+{
+    unsigned int *status = device_status_ptr();
+    if (!status)
+        return cudaErrorInvalidDevice;
+    const BwdLayout l = bwd_layout(m.nrec, nunits, D);
+    unsigned char *base = static_cast<unsigned char *>(ws);
+    float *Hs = reinterpret_cast<float *>(base + l.states), *dHs = reinterpret_cast<float *>(base + l.dstates);
+    float *scratch = reinterpret_cast<float *>(base + l.scratch);
+    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, nullptr, ws, s);
+    if (e == cudaSuccess)
+        e = launch_scan_d<D>(m, H, ws, S0, nullptr, nullptr, nullptr, s, Hs);
+    if (e != cudaSuccess)
+        return e;
+    const size_t smem = sizeof(DScanSmem<D>) + 1024;
+    e = cudaFuncSetAttribute(dscan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    dscan_kernel<D><<<dim3(D / kBV, m.nseq * H), kScanThreads, smem, s>>>(
+        m, H, static_cast<const unsigned char *>(ws), static_cast<const __nv_bfloat16 *>(dO), dS_T, dHs, dS0, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const int grid = (int)std::min<int64_t>(nunits, kBwdSlots);
+    e = cudaFuncSetAttribute(bwd_chunk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdSmem<D>::bytes);
+    if (e != cudaSuccess)
+        return e;
+    bwd_chunk_kernel<D><<<grid, kBwdThreads, BwdSmem<D>::bytes, s>>>(
+        m, H, (int)nunits, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
+        static_cast<const __nv_bfloat16 *>(beta), g_min, static_cast<const __nv_bfloat16 *>(dO), Hs, dHs, scratch,
+        dq, dk, dv, da, dbeta, status);
+    return cudaGetLastError();
 }
 
 SeqMap regular_map(int B, int T, int H)
@@ -1285,6 +2112,33 @@ cudaError_t launch_scan_affine_bf16(int B, int T, int H, int D, const void *work
                                     cudaStream_t s)
 {
     return launch_scan(regular_map(B, T, H), H, D, workspace, nullptr, nullptr, S_zero, s, M);
+}
+
+size_t chunk_bf16_bwd_workspace(int B, int T, int H, int D)
+{
+    const SeqMap m = regular_map(B, T, H);
+    return bwd_layout(m.nrec, m.nrec, D).total;
+}
+
+void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *dstates)
+{
+    const SeqMap m = regular_map(B, T, H);
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D);
+    *states = l.states;
+    *dstates = l.dstates;
+}
+
+cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                                  const void *a, const void *beta, float g_min, const float *S0, const void *dO,
+                                  const float *dS_T, float *dq, float *dk, float *dv, float *da, float *dbeta,
+                                  float *dS0, void *workspace, cudaStream_t s)
+{
+    const SeqMap m = regular_map(B, T, H);
+    const dim3 grid(m.NT, B * H);
+    return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk, dv, da,
+                                      dbeta, dS0, workspace, s)
+                   : launch_bwd_d<128>(m, H, grid, m.nrec, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk, dv, da,
+                                       dbeta, dS0, workspace, s);
 }
 
 // ------------------------------------------------------------------ segment combine

@@ -500,6 +500,81 @@ kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const 
     return from_cuda(launch_decode(N, H, dk, dtype, q, k, v, a, beta, g_min, S, o, (cudaStream_t)stream));
 }
 
+size_t kda_chunk_bwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (B < 1 || H < 1 || T <= 0 || dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16)
+        return 0;
+    return chunk_bf16_bwd_workspace(B, T, H, dk);
+}
+
+kda_status kda_chunk_bwd_offsets(int B, int T, int H, int dk, int dv, size_t *states_offset,
+                                 size_t *dstates_offset)
+{
+    if (!states_offset || !dstates_offset)
+        return KDA_ERR_INVALID_ARG;
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, KDA_BF16, sh);
+    if (st != KDA_OK)
+        return st;
+    if (T == 0) {
+        *states_offset = *dstates_offset = 0;
+        return KDA_OK;
+    }
+    chunk_bf16_bwd_offsets(B, T, H, dk, states_offset, dstates_offset);
+    return KDA_OK;
+}
+
+kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
+                         const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_, float *da,
+                         float *dbeta, float *dS0, void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
+    if (st != KDA_OK)
+        return st;
+    if (dtype != KDA_BF16 || (int64_t)B * H * (((int64_t)T + 63) / 64) > 0x7fffffff)
+        return KDA_ERR_UNSUPPORTED;
+    st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!all_aligned({S0, dS_T, dS0}))
+        return KDA_ERR_ALIGNMENT;
+    const Range rS0(S0, sh.ns * 4), rdST(dS_T, sh.ns * 4), rdS0(dS0, sh.ns * 4);
+    if (overlaps(rdS0, rS0) || overlaps(rdS0, rdST))
+        return KDA_ERR_ALIAS;
+    if (T == 0) {
+        if (!dS0)
+            return KDA_OK;
+        if (dS_T)
+            return from_cuda(cudaMemcpyAsync(dS0, dS_T, (size_t)sh.ns * 4, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(dS0, 0, (size_t)sh.ns * 4, s));
+    }
+    if (!q || !k || !v || !a || !beta || !dO || !dq || !dk_ || !dv_ || !da || !dbeta)
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, a, dO, dq, dk_, dv_, da, dbeta, workspace}) || !beta_aligned(beta, 2))
+        return KDA_ERR_ALIGNMENT;
+    const size_t need = chunk_bf16_bwd_workspace(B, T, H, dk);
+    if (!workspace || ws_bytes < need)
+        return KDA_ERR_WORKSPACE;
+    const int64_t es = 2;
+    const Range ins[] = {Range(q, sh.nk * es), Range(k, sh.nk * es), Range(v, sh.nv * es), Range(a, sh.nk * es),
+                         Range(beta, sh.ntok * es), Range(dO, sh.nv * es), rS0, rdST};
+    const Range outs[] = {Range(dq, sh.nk * 4), Range(dk_, sh.nk * 4), Range(dv_, sh.nv * 4), Range(da, sh.nk * 4),
+                          Range(dbeta, sh.ntok * 4), rdS0, Range(workspace, (int64_t)need)};
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+        for (const Range &in : ins)
+            if (overlaps(outs[i], in))
+                return KDA_ERR_ALIAS;
+        for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+            if (overlaps(outs[i], outs[j]))
+                return KDA_ERR_ALIAS;
+    }
+    return from_cuda(launch_chunk_bwd_bf16(B, T, H, dk, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk_, dv_, da,
+                                           dbeta, dS0, workspace, s));
+}
+
 kda_status kda_device_status(kda_stream_t stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)

@@ -270,6 +270,40 @@ kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M
                              const float *S0, float *S_in, kda_stream_t stream);
 
 /*
+ * kda_chunk_bwd -- gradients of the bfloat16 chunked forward (bounded gate) with respect
+ * to every input, given the gradient of the loss with respect to o and to the final
+ * state.  Passage: long sequences are trained by recursing in chunks ("Trillion-Parameter
+ * MoE ... Engineering" section 3.2); the pages print no backward, so this is the
+ * derivative of kda_chunk_fwd's recurrence, computed in the same chunked form:
+ *     dS = (Diag(Gamma) - N)^T dS' + Q'^T dO        (state gradient, chunks in reverse)
+ * and, inside each chunk, the reverse of the chunk's products (see chunk_bf16.cu).  It
+ * recomputes the forward (prep and scan) inside the call; nothing of a forward call is
+ * needed.  All gradients are float32.
+ *   B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, S0: exactly as in kda_chunk_fwd
+ *                (dtype must be KDA_BF16; S0 may be NULL for zeros).
+ *   dO           [B, T, H, dv] bfloat16: dL/do.
+ *   dS_T         [B, H, dk, dv] float32 or NULL (zero): dL/dS_T.
+ *   dq, dk_, da  [B, T, H, dk] float32 out;  dv_: [B, T, H, dv] float32 out;
+ *   dbeta        [B, T, H] float32 out;  dS0: [B, H, dk, dv] float32 out or NULL.
+ *                da is the gradient with respect to the gate's pre-activation a.
+ *   workspace    >= kda_chunk_bwd_workspace(B, T, H, dk, dv, dtype) bytes, 16-byte
+ *                aligned: the forward's records, the state entering every chunk and the
+ *                gradient of the state after it (float32, dk x dv per (b, h, chunk), in
+ *                that order, from the byte offsets kda_chunk_bwd_offsets gives), then the
+ *                gradient kernel's scratch.
+ * The outputs must not overlap each other, an input or the workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.  T == 0 writes dS0 =
+ * dS_T (or zeros) and nothing else.
+ */
+size_t kda_chunk_bwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype);
+kda_status kda_chunk_bwd_offsets(int B, int T, int H, int dk, int dv, size_t *states_offset,
+                                 size_t *dstates_offset);
+kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
+                         const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_, float *da,
+                         float *dbeta, float *dS0, void *workspace, size_t ws_bytes, kda_stream_t stream);
+
+/*
  * kda_decode_step -- one token for N independent sequences, state updated in place.
  * Passage: the incremental state of constant size used at inference ("Trillion-
  * Parameter MoE ... Engineering" section 3.2).  Per (n, h):

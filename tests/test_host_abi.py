@@ -307,3 +307,48 @@ def test_debug_build_exports_the_same_entry_points():
     out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
     exported = set(re.findall(r"\bT\s+(kda_[a-z0-9_]+)$", out, re.M))
     assert set(declared_functions()) <= exported
+
+
+def test_chunk_bwd_entry_validates(L):
+    """kda_chunk_bwd rejects every bad argument before a launch (fake pointers: none of
+    these calls may pass validation)."""
+    P = ctypes.c_void_p
+    B, T, H, D = 1, 64, 1, 128
+    nb = B * T * H * D * 2
+    need = L.kda_chunk_bwd_workspace(B, T, H, D, D, kda.KDA_BF16)
+    assert need > L.kda_chunk_fwd_workspace(B, T, H, D, D, kda.KDA_BF16)
+    assert L.kda_chunk_bwd_workspace(B, T, H, D, D, kda.KDA_F32) == 0
+    assert L.kda_chunk_bwd_workspace(B, T, H, 96, 96, kda.KDA_BF16) == 0
+    step = nb * 2 + 4096
+    ins = [BASE + i * step for i in range(6)]          # q, k, v, a, beta, dO
+    outs = [BASE + (6 + i) * step for i in range(5)]   # dq, dk, dv, da, dbeta
+    ws = BASE + 12 * step
+
+    def bwd(dtype=kda.KDA_BF16, g_min=-5.0, q=ins[0], dO=ins[5], dq=outs[0], dbeta=outs[4], w=ws, wb=need,
+            S0=None, dST=None, dS0=None, dk=D):
+        return L.kda_chunk_bwd(B, T, H, dk, dk, dtype, P(q), P(ins[1]), P(ins[2]), P(ins[3]), P(ins[4]),
+                               ctypes.c_float(g_min), P(S0), P(dO), P(dST), P(dq), P(outs[1]), P(outs[2]),
+                               P(outs[3]), P(dbeta), P(dS0), P(w), wb, None)
+
+    assert bwd(dtype=kda.KDA_F32) == UNSUPPORTED
+    assert bwd(dk=96) == UNSUPPORTED
+    assert bwd(g_min=0.0) == INVALID
+    assert bwd(q=0) == INVALID
+    assert bwd(dO=0) == INVALID
+    assert bwd(dq=0) == INVALID
+    assert bwd(q=BASE + 8) == ALIGN
+    assert bwd(dq=outs[0] + 4) == ALIGN
+    assert bwd(dbeta=outs[4] + 2) == ALIGN
+    assert bwd(w=0) == WS
+    assert bwd(wb=need - 1) == WS
+    assert bwd(dq=ins[2]) == ALIAS                        # an output over v
+    assert bwd(dq=outs[1]) == ALIAS                       # two outputs on one buffer
+    assert bwd(w=outs[3] - 1024) == ALIAS                 # workspace over da
+    S = BASE * 2
+    assert bwd(S0=S, dS0=S) == ALIAS
+    assert bwd(dST=S, dS0=S + 4096) == ALIAS
+    sa, sb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert L.kda_chunk_bwd_offsets(B, T, H, D, D, ctypes.byref(sa), ctypes.byref(sb)) == OK
+    assert sa.value >= L.kda_chunk_fwd_workspace(B, T, H, D, D, kda.KDA_BF16) and sa.value % 16 == 0
+    assert sb.value == sa.value + B * H * D * D * 4
+    assert L.kda_chunk_bwd_offsets(B, T, H, D, D, None, ctypes.byref(sb)) == INVALID

@@ -49,6 +49,12 @@ BYTES_PER_TOKEN_HEAD = 4 * 256 + 2 + 256
 # The prep kernel's share of them (it reads the inputs; the scan writes o and the states).
 # The workspace records between the two kernels are the implementation's own traffic.
 PREP_BYTES_PER_TOKEN_HEAD = 4 * 256 + 2
+# Backward, per token-head at d = 128: q, k, v, a, dO read (bf16) and beta; dq, dk, dv, da
+# written (float32) and dbeta.
+BWD_BYTES_PER_TOKEN_HEAD = 5 * 256 + 2 + 4 * 512 + 4
+# The per-chunk gradient kernel also reads the chunk's saved state and state gradient
+# (2 x dk dv x 4 B per 64 tokens).
+BWD_CHUNK_BYTES_PER_TOKEN_HEAD = BWD_BYTES_PER_TOKEN_HEAD + 2 * 128 * 128 * 4 // 64
 # Triangle-aware flops per token-head at the 16-token tile (state products W S, Qbar S,
 # Khat^T U: 6 dk dv; tile products and W: dk (3C - 1); Utilde and P U: 2 C dv; solve
 # C^2/3; Gamma scaling dk dv / C), C = 16.
@@ -78,8 +84,9 @@ def kernel_source_hash() -> str:
 
 
 def measured_traffic_per_token_head(kernel: str):
-    """DRAM bytes (read + write) per token-head of one launch of ``kernel`` ("prep" or
-    "scan") from the committed ncu summary, or None when the kernels changed since."""
+    """DRAM bytes (read + write) per token-head of one launch of ``kernel`` ("prep", "scan",
+    "bwd_chunk" or "dscan") from the committed ncu summary, or None when the kernels changed
+    since."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     d = json.load(open(PROFILE_TRAFFIC))
@@ -405,6 +412,37 @@ def run_libkda(args):
                "gpu_launches_per_step": 4, "collectives_per_step": 2 if world > 1 else 0}
         del sd, xs
 
+    # ---- backward: the gradients of every input for the same workload and inputs, one
+    # kda_chunk_bwd per step (prep, state-saving scan, reverse state-gradient scan, per-chunk
+    # gradients: four launches), dL/do seeded normal, no gradient on the final state
+    bwd = None
+    if args.only != "decode" and not args.no_bwd:
+        gen = torch.Generator().manual_seed(rank_seed(w.seed + 17, rank))
+        dO = torch.randn((B, T, H, D), generator=gen).to(torch.bfloat16).to(device)
+        ws_b = torch.empty(kda.kda_chunk_bwd_workspace(B, T, H, D, D), dtype=torch.uint8, device=device)
+        gout = {}
+
+        def bwd_step():
+            gout.update(kda.kda_chunk_bwd(*(d[n] for n in names), dO, G_MIN, S0=S0, workspace=ws_b,
+                                          out=gout or None))
+
+        bwd_ms = time_steps(bwd_step, max(3, min(args.steps, 5)), 3, world, device)
+        assert kda.kda_device_status(device) == 0
+        bwd_bytes = token_heads * BWD_BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+        bwd_traffic = measured_traffic_per_token_head("bwd_chunk")
+        bwd_gbs = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+        bwd = {"what": "kda_chunk_bwd: dq, dk, dv, da, dbeta, dS0 (float32) from dL/do",
+               "ms_per_step": bwd_ms, "value": world * tokens / (bwd_ms * 1e-3), "unit": UNIT,
+               "gpu_launches_per_step": 4, "vs_forward_time": bwd_ms / ms, "workspace_bytes": ws_b.numel(),
+               "roofline": {"bound": "hbm", "achieved": bwd_gbs, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": bwd_gbs / hbm_peak, "peak_kind": peak_kind,
+                            "kernels": "the whole backward path (four launches)",
+                            "algorithmic_bytes_per_step": bwd_bytes},
+               "dominant_kernel": {"kernel": "bwd_chunk_kernel (per-chunk gradients)",
+                                   "algorithmic_bytes_per_token_head": BWD_CHUNK_BYTES_PER_TOKEN_HEAD,
+                                   "traffic": None if bwd_traffic is None else bwd_traffic * token_heads}}
+        del ws_b, gout, dO
+
     # ---- end to end through the C ABI with pinned host buffers, pipelined across steps:
     # every step copies its inputs host -> device on one stream, runs kda_chunk_fwd on a
     # second, and reads o and S_T back on a third; device and host buffers are double-
@@ -539,6 +577,8 @@ def run_libkda(args):
         line["varlen"] = vl
     if spl is not None:
         line["sequence_parallel"] = spl
+    if bwd is not None:
+        line["backward"] = bwd
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.only != "decode":
         # a fresh run of the main path on this exact input (later legs reuse o and S_T)
         o_p, S_p = kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, workspace=ws)
@@ -568,6 +608,7 @@ def main(argv=None):
     ap.add_argument("--no-ablation", action="store_true", help="skip timing the log-sigmoid ablation path")
     ap.add_argument("--no-varlen", action="store_true", help="skip timing the packed variable-length batch")
     ap.add_argument("--no-sp", action="store_true", help="skip timing the sequence-parallel leg")
+    ap.add_argument("--no-bwd", action="store_true", help="skip timing the backward leg")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

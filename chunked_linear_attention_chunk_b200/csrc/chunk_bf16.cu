@@ -1391,13 +1391,14 @@ struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blo
     static constexpr int dKh = dU + CD;
     static constexpr int dQb = dKh + CD;
     static constexpr int Gp = dQb + CD;  // dg/da = g_min sigma(a) (1 - sigma(a))
-    static constexpr int floats = Gp + CD;
+    static constexpr int X = Gp + CD;    // dT T^T, 64 x 64
+    static constexpr int floats = X + kC * kC;
 };
 
-constexpr int kGTM = 64, kGTN = 64, kGTK = 32;
-constexpr int kGLDA = kGTK + 4, kGLDB = kGTN + 8;  // conflict-free fragment reads
-constexpr int kGStage = kGTM * kGLDA + kGTK * kGLDB;
-constexpr int kGPA = kGTM * kGTK / kBwdThreads, kGPB = kGTK * kGTN / kBwdThreads;
+constexpr int kGTM = 64, kGTK = 32;  // output tiles of 64 x TN (TN = 64 or 128), K steps of 32
+constexpr int kGLDA = kGTK + 4;       // conflict-free fragment reads (B: TN + 8)
+constexpr int kGStage = kGTM * kGLDA + kGTK * (128 + 8);
+constexpr int kGPA = kGTM * kGTK / kBwdThreads;
 
 template <int D>
 struct BwdSmem {  // float offsets in shared memory
@@ -1405,8 +1406,8 @@ struct BwdSmem {  // float offsets in shared memory
     static constexpr int LDC = kC + 4;
     static constexpr int q = 0, k = q + kC * LDD, G = k + kC * LDD;  // q later holds dG
     static constexpr int Ap = G + kC * LDD, P = Ap + kC * LDC, T = P + kC * LDC;
-    static constexpr int dT = T + kC * LDC;  // dT, then dP
-    static constexpr int X = dT + kC * LDC, dA = X + kC * LDC;
+    static constexpr int dT = T + kC * LDC;  // scratch of the block solve, then dT, then dP
+    static constexpr int dA = dT + kC * LDC;
     static constexpr int stage = dA + kC * LDC;
     static constexpr int beta = stage + kGStage;
     static constexpr int dGam = beta + kC;
@@ -1423,17 +1424,18 @@ struct MatV {
     __device__ __forceinline__ float at(int i, int j) const { return p[(int64_t)i * rs + (int64_t)j * cs]; }
 };
 
-// C[M x N] = A[M x K] B[K x N] on the whole CTA (M, N, K multiples of 64, 64, 32); every
+// C[M x N] = A[M x K] B[K x N] on the whole CTA (M, N, K multiples of 64, TN, 32); every
 // output element goes to epi(i, j, value) exactly once, from a thread fixed by (M, N).
-// Operands are staged through shared memory as TF32 in 64 x 32 / 32 x 64 tiles, the next
+// Operands are staged through shared memory as TF32 in 64 x 32 / 32 x TN tiles, the next
 // tile fetched into registers while the tensor cores work on the current one; warp w
-// computes rows 16 (w / 4) .. + 16 and columns 16 (w % 4) .. + 16 of each 64 x 64 tile.
-template <class Epi>
+// computes rows 16 (w / 4) .. + 16 and columns TN/4 (w % 4) .. + TN/4 of each 64 x TN tile.
+template <int TN, class Epi>
 __device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, Epi epi)
 {
+    constexpr int kGTN = TN, kGLDB = TN + 8, kGPB = kGTK * TN / kBwdThreads, NF = TN / 32;
     uint32_t *sA = stage, *sB = stage + kGTM * kGLDA;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int wm = (warp >> 2) * 16, wn = (warp & 3) * 16;
+    const int wm = (warp >> 2) * 16, wn = (warp & 3) * (TN / 4);
     float ra[kGPA], rb[kGPB];
     auto fetch = [&](int m0, int n0, int k0) {
 #pragma unroll
@@ -1452,7 +1454,7 @@ __device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, E
     fetch(0, 0, 0);
     for (int m0 = 0; m0 < M; m0 += kGTM)
         for (int n0 = 0; n0 < N; n0 += kGTN) {
-            float acc[2][4] = {};
+            float acc[NF][4] = {};
             for (int k0 = 0; k0 < K; k0 += kGTK) {
                 __syncthreads();  // the previous tile's readers are done
 #pragma unroll
@@ -1483,7 +1485,7 @@ __device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, E
                     af[2] = sA[(wm + g) * kGLDA + kk + t + 4];
                     af[3] = sA[(wm + g + 8) * kGLDA + kk + t + 4];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
+                    for (int nt = 0; nt < NF; ++nt) {
                         uint32_t bf[2];
                         bf[0] = sB[(kk + t) * kGLDB + wn + nt * 8 + g];
                         bf[1] = sB[(kk + t + 4) * kGLDB + wn + nt * 8 + g];
@@ -1492,7 +1494,7 @@ __device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, E
                 }
             }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < NF; ++nt) {
                 const int i = m0 + wm + g, j = n0 + wn + nt * 8 + 2 * t;
                 epi(i, j, acc[nt][0]);
                 epi(i, j + 1, acc[nt][1]);
@@ -1560,11 +1562,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     using L = BwdSlot<D>;
     using SL = BwdSmem<D>;
     constexpr int CD = kC * D, LDD = SL::LDD, LDC = SL::LDC;
-    constexpr int NH = D / 64;  // 64-channel halves handled per warp in the pairwise backward
+    constexpr int NQ = D / 32;  // 32-channel quarters (per warp) of the pairwise backward
     extern __shared__ __align__(16) float bsm[];
     float *const sq = bsm + SL::q, *const sk = bsm + SL::k, *const sG = bsm + SL::G;
     float *const sAp = bsm + SL::Ap, *const sP = bsm + SL::P, *const sT = bsm + SL::T;
-    float *const sdT = bsm + SL::dT, *const sX = bsm + SL::X, *const sdA = bsm + SL::dA;
+    float *const sdT = bsm + SL::dT, *const sdA = bsm + SL::dA;
     uint32_t *const stage = reinterpret_cast<uint32_t *>(bsm + SL::stage);
     float *const sbeta = bsm + SL::beta, *const sdGam = bsm + SL::dGam;
     float *const sseg = bsm + SL::seg;
@@ -1573,6 +1575,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Qb = sl + L::Qb, *const Bk = sl + L::Bk;
     float *const Bv = sl + L::Bv, *const W = sl + L::W, *const U = sl + L::U, *const dOs = sl + L::dO;
     float *const dU = sl + L::dU, *const dKh = sl + L::dKh, *const dQb = sl + L::dQb, *const Gp = sl + L::Gp;
+    float *const Xg = sl + L::X;
 
     for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
         // regular batch: unit = (b*H + h) * NT + chunk; packed batch: unit = h * NT + chunk slot
@@ -1654,8 +1657,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int rr = 1; rr < kTile; ++rr) {
                 const int r = b0 + rr;
                 float acc = 0.f;
-                if (lane < kTile && j < rr)
-                    for (int s = j; s < rr; ++s)
+#pragma unroll
+                for (int s = 0; s < kTile - 1; ++s)
+                    if (s >= j && s < rr)
                         acc = fmaf(sAp[r * LDC + b0 + s], sT[(b0 + s) * LDC + b0 + j], acc);
                 __syncwarp();
                 if (lane < kTile && j < rr)
@@ -1670,18 +1674,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int rr = lane >> 1, j0 = (lane & 1) * 8, r = I * kTile + rr;
                 float x[8] = {};
                 for (int K = J; K < I; ++K)
+#pragma unroll
                     for (int s = 0; s < kTile; ++s) {
                         const float av = sAp[r * LDC + K * kTile + s];
 #pragma unroll
                         for (int u = 0; u < 8; ++u)
                             x[u] = fmaf(av, sT[(K * kTile + s) * LDC + J * kTile + j0 + u], x[u]);
                     }
-                float *Xs = sX + warp * kTile * LDC;  // 16 x 16 per warp (sX is free until step 6)
+                float *Xs = sdT + warp * kTile * LDC;  // 16 x 16 per warp (sdT is free until step 6)
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     Xs[rr * LDC + j0 + u] = sbeta[r] * x[u];
                 __syncwarp();
                 float y[8] = {};
+#pragma unroll
                 for (int uu = 0; uu < kTile; ++uu) {
                     const float tv = sT[r * LDC + I * kTile + uu];
 #pragma unroll
@@ -1696,15 +1702,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // 6. dense contractions
         const MatV Tn{sT, LDC, 1}, Tt{sT, 1, LDC};
-        cta_gemm(kC, D, kC, Tn, MatV{Bk, D, 1}, stage, [&](int i, int j, float x) { W[i * D + j] = x; });
-        cta_gemm(kC, D, kC, Tn, MatV{Bv, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] = x; });
-        cta_gemm(kC, D, D, MatV{W, D, 1}, MatV{S, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] -= x; });
-        cta_gemm(kC, D, D, MatV{Kh, D, 1}, MatV{dSn, D, 1}, stage, [&](int i, int j, float x) { dU[i * D + j] = x; });
-        cta_gemm(kC, D, kC, MatV{sP, 1, LDC}, MatV{dOs, D, 1}, stage,
+        cta_gemm<D>(kC, D, kC, Tn, MatV{Bk, D, 1}, stage, [&](int i, int j, float x) { W[i * D + j] = x; });
+        cta_gemm<D>(kC, D, kC, Tn, MatV{Bv, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] = x; });
+        cta_gemm<D>(kC, D, D, MatV{W, D, 1}, MatV{S, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] -= x; });
+        cta_gemm<D>(kC, D, D, MatV{Kh, D, 1}, MatV{dSn, D, 1}, stage, [&](int i, int j, float x) { dU[i * D + j] = x; });
+        cta_gemm<D>(kC, D, kC, MatV{sP, 1, LDC}, MatV{dOs, D, 1}, stage,
                  [&](int i, int j, float x) { dU[i * D + j] += x; });
-        cta_gemm(kC, D, D, MatV{U, D, 1}, MatV{dSn, 1, D}, stage, [&](int i, int j, float x) { dKh[i * D + j] = x; });
-        cta_gemm(kC, D, D, MatV{dOs, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { dQb[i * D + j] = x; });
-        cta_gemm(kC, D, D, MatV{dU, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { W[i * D + j] = -x; });
+        cta_gemm<D>(kC, D, D, MatV{U, D, 1}, MatV{dSn, 1, D}, stage, [&](int i, int j, float x) { dKh[i * D + j] = x; });
+        cta_gemm<D>(kC, D, D, MatV{dOs, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { dQb[i * D + j] = x; });
+        cta_gemm<D>(kC, D, D, MatV{dU, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { W[i * D + j] = -x; });
         float *const dW = W;
         // dGamma_i = sum_j dS'_ij S_ij, warp per row
 #pragma unroll
@@ -1720,26 +1726,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0)
                 sdGam[i] = acc;
         }
-        cta_gemm(kC, kC, D, MatV{dW, D, 1}, MatV{Bk, 1, D}, stage,
+        cta_gemm<64>(kC, kC, D, MatV{dW, D, 1}, MatV{Bk, 1, D}, stage,
                  [&](int i, int j, float x) { sdT[i * LDC + j] = x; });
-        cta_gemm(kC, kC, D, MatV{dU, D, 1}, MatV{Bv, 1, D}, stage,
+        cta_gemm<64>(kC, kC, D, MatV{dU, D, 1}, MatV{Bv, 1, D}, stage,
                  [&](int i, int j, float x) { sdT[i * LDC + j] += x; });
-        cta_gemm(kC, D, kC, Tt, MatV{dW, D, 1}, stage, [&](int i, int j, float x) { Bk[i * D + j] = x; });
-        cta_gemm(kC, D, kC, Tt, MatV{dU, D, 1}, stage, [&](int i, int j, float x) { Bv[i * D + j] = x; });
-        cta_gemm(kC, kC, kC, MatV{sdT, LDC, 1}, Tt, stage, [&](int i, int j, float x) { sX[i * LDC + j] = x; });
-        cta_gemm(kC, kC, kC, Tt, MatV{sX, LDC, 1}, stage,
+        cta_gemm<D>(kC, D, kC, Tt, MatV{dW, D, 1}, stage, [&](int i, int j, float x) { Bk[i * D + j] = x; });
+        cta_gemm<D>(kC, D, kC, Tt, MatV{dU, D, 1}, stage, [&](int i, int j, float x) { Bv[i * D + j] = x; });
+        cta_gemm<64>(kC, kC, kC, MatV{sdT, LDC, 1}, Tt, stage, [&](int i, int j, float x) { Xg[i * kC + j] = x; });
+        cta_gemm<64>(kC, kC, kC, Tt, MatV{Xg, kC, 1}, stage,
                  [&](int i, int j, float x) { sdA[i * LDC + j] = j < i ? -x : 0.f; });
-        cta_gemm(kC, kC, D, MatV{dOs, D, 1}, MatV{U, 1, D}, stage,
+        cta_gemm<64>(kC, kC, D, MatV{dOs, D, 1}, MatV{U, 1, D}, stage,
                  [&](int i, int j, float x) { sdT[i * LDC + j] = j <= i ? x : 0.f; });
         float *const dBk = Bk, *const dBv = Bv, *const sdP = sdT;  // dA' = diag(beta) dA
-        // 7. pairwise products backward, rows: for r in tile I, channels of one 64-wide half,
+        // 7. pairwise products backward, rows: for r in tile I, channels of one 32-wide quarter,
         //    dq_r = sum_{s<=r} dP_rs k_s E_rs,  dk_r = sum_{s<r} dA'_rs k_s E_rs,  dG_r = q_r dq_r + k_r dk_r
-        //    (E_rs = e^{G_r - G_s} per channel), one warp per (I, half).  dq -> W, dk -> U, dG -> dO.
-        if (warp < kTiles * NH) {
-            const int I = warp / NH, c0 = (warp % NH) * 64, g = lane >> 2, t = lane & 3;
+        //    (E_rs = e^{G_r - G_s} per channel), one warp per (I, 32-channel quarter).  dq -> W, dk -> U, dG -> dO.
+        if (warp < kTiles * NQ) {
+            const int I = warp / NQ, c0 = (warp % NQ) * 32, g = lane >> 2, t = lane & 3;
             for (int pass = 0; pass < 2; ++pass) {  // 0: tiles J < I (reference 16 I), 1: J = I (middle)
                 const int m = pass == 0 ? I * kTile : I * kTile + kRef;
-                float aq[8][4] = {}, ak[8][4] = {};
+                float aq[4][4] = {}, ak[4][4] = {};
                 const int J0 = pass == 0 ? 0 : I, J1 = pass == 0 ? I : I + 1;
                 for (int J = J0; J < J1; ++J) {
 #pragma unroll
@@ -1752,7 +1758,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             fa[x] = to_tf32(sbeta[r] * sdA[r * LDC + s]);
                         }
 #pragma unroll
-                        for (int nf = 0; nf < 8; ++nf) {
+                        for (int nf = 0; nf < 4; ++nf) {
                             uint32_t b[2];
 #pragma unroll
                             for (int x = 0; x < 2; ++x) {
@@ -1765,7 +1771,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 }
 #pragma unroll
-                for (int nf = 0; nf < 8; ++nf)
+                for (int nf = 0; nf < 4; ++nf)
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         const int r = I * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
@@ -1786,13 +1792,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncthreads();
         //    columns: dk_s += sum_{r>=s} (dP_rs q_r + dA'_rs k_r) E_rs and dG_s -= k_s (that sum), one
-        //    warp per (column tile J, half); each row tile I >= J has its own reference.
-        if (warp < kTiles * NH) {
-            const int J = warp / NH, c0 = (warp % NH) * 64, g = lane >> 2, t = lane & 3;
-            float tot[8][4] = {};
+        //    warp per (column tile J, quarter); each row tile I >= J has its own reference.
+        if (warp < kTiles * NQ) {
+            const int J = warp / NQ, c0 = (warp % NQ) * 32, g = lane >> 2, t = lane & 3;
+            float tot[4][4] = {};
             for (int I = J; I < kTiles; ++I) {
                 const int m = I > J ? I * kTile : I * kTile + kRef;
-                float acc[8][4] = {};
+                float acc[4][4] = {};
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                     uint32_t fp[4], fa[4];
@@ -1803,7 +1809,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         fa[x] = to_tf32(sbeta[r] * sdA[r * LDC + s]);
                     }
 #pragma unroll
-                    for (int nf = 0; nf < 8; ++nf) {
+                    for (int nf = 0; nf < 4; ++nf) {
                         uint32_t bq[2], bk[2];
 #pragma unroll
                         for (int x = 0; x < 2; ++x) {
@@ -1817,7 +1823,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 }
 #pragma unroll
-                for (int nf = 0; nf < 8; ++nf)
+                for (int nf = 0; nf < 4; ++nf)
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         const int s = J * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
@@ -1825,7 +1831,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
             }
 #pragma unroll
-            for (int nf = 0; nf < 8; ++nf)
+            for (int nf = 0; nf < 4; ++nf)
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     const int s = J * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
@@ -1835,7 +1841,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncthreads();
         // 8. the decay-scaled operands' gradients; outputs dq, dk, dv; dG -> sq
-#pragma unroll 2
+#pragma unroll 4
         for (int e = tid; e < CD; e += kBwdThreads) {
             const int r = e / D, c = e % D;
             const float Gv = sG[r * LDD + c], e1 = __expf(Gv), eh = __expf(sG[(kC - 1) * LDD + c] - Gv);

@@ -62,6 +62,8 @@ EXPORTS = (
     "kda_chunk_bwd_workspace",
     "kda_chunk_bwd_offsets",
     "kda_chunk_bwd",
+    "kda_chunk_bwd_varlen_workspace",
+    "kda_chunk_bwd_varlen",
 )
 
 
@@ -125,8 +127,12 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_bwd_workspace.restype = S
     L.kda_chunk_bwd_offsets.argtypes = [I, I, I, I, I, P, P]
     L.kda_chunk_bwd_offsets.restype = I
-    L.kda_chunk_bwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_bwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     L.kda_chunk_bwd.restype = I
+    L.kda_chunk_bwd_varlen_workspace.argtypes = [I, I, I, I, I, I]
+    L.kda_chunk_bwd_varlen_workspace.restype = S
+    L.kda_chunk_bwd_varlen.argtypes = [I, P, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.kda_chunk_bwd_varlen.restype = I
     _lib = L
     return L
 
@@ -232,38 +238,82 @@ def kda_chunk_bwd_offsets(B: int, T: int, H: int, dk: int, dv: int):
     return int(a.value), int(b.value)
 
 
-def kda_chunk_bwd(q, k, v, a, beta, dO, g_min: float = -5.0, S0=None, dS_T=None, workspace=None,
-                  return_dS0: bool = True, out=None):
-    """Gradients of the bf16 chunked forward.  q, k, a [B,T,H,dk], v and dO [B,T,H,dv],
-    beta [B,T,H] (bfloat16); S0 and dS_T [B,H,dk,dv] float32 or None (zeros).  Returns a
-    dict of float32 tensors dq, dk, dv, da, dbeta and dS0 (None unless ``return_dS0``);
-    ``out`` may supply some of those tensors."""
-    _check_cuda(q, k, v, a, beta, dO, S0, dS_T, workspace)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    if any(t.dtype != torch.bfloat16 for t in (q, k, v, a, beta, dO)):
-        raise TypeError("kda_chunk_bwd takes bfloat16 q, k, v, a, beta, dO")
-    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or dO.shape != v.shape \
-            or beta.shape != (B, T, H):
-        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v,dO [B,T,H,dv], beta [B,T,H]")
+def _bwd_outputs(q, v, beta, n_state, H, dk, dv, return_dS0, A_log, out):
     dev = q.device
     shapes = {"dq": q.shape, "dk": q.shape, "dv": v.shape, "da": q.shape, "dbeta": beta.shape,
-              "dS0": (B, H, dk, dv)}
+              "dS0": (n_state, H, dk, dv), "dA_log": (H,)}
     g = dict(out or {})
     for name, shp in shapes.items():
-        if name not in g and (name != "dS0" or return_dS0):
+        if name in g:
+            continue
+        if (name == "dS0" and not return_dS0) or (name == "dA_log" and A_log is None):
+            g[name] = None
+        else:
             g[name] = torch.empty(shp, dtype=torch.float32, device=dev)
-    g.setdefault("dS0", None)
     _check_cuda(*g.values())
+    return g
+
+
+def _bwd_checks(q, k, v, a, beta, dO, A_log, token_dims):
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, a, beta, dO)):
+        raise TypeError("the backward takes bfloat16 q, k, v, a, beta, dO")
+    if k.shape != q.shape or a.shape != q.shape or dO.shape != v.shape or \
+            v.shape[:token_dims] != q.shape[:token_dims] or beta.shape != q.shape[:token_dims + 1]:
+        raise ValueError("shape mismatch: q, k, a [.., H, dk], v, dO [.., H, dv], beta [.., H]")
+    if A_log is not None and (A_log.dtype != torch.float32 or A_log.shape != (q.shape[-2],)):
+        raise ValueError("A_log must be float32 [H]")
+
+
+def kda_chunk_bwd(q, k, v, a, beta, dO, g_min: float = -5.0, S0=None, dS_T=None, workspace=None,
+                  return_dS0: bool = True, out=None, A_log=None):
+    """Gradients of the bf16 chunked forward.  q, k, a [B,T,H,dk], v and dO [B,T,H,dv],
+    beta [B,T,H] (bfloat16); S0 and dS_T [B,H,dk,dv] float32 or None (zeros); A_log float32
+    [H] or None (the gate's per-head scale e^{A_log[h]}).  Returns a dict of float32 tensors
+    dq, dk, dv, da, dbeta, dS0 (None unless ``return_dS0``) and dA_log (None without
+    A_log); ``out`` may supply some of those tensors."""
+    _check_cuda(q, k, v, a, beta, dO, S0, dS_T, workspace, A_log)
+    _bwd_checks(q, k, v, a, beta, dO, A_log, 2)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g = _bwd_outputs(q, v, beta, B, H, dk, dv, return_dS0, A_log, out)
     need = int(lib().kda_chunk_bwd_workspace(B, T, H, dk, dv, KDA_BF16))
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().kda_chunk_bwd(B, T, H, dk, dv, KDA_BF16, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
-                             float(g_min), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]),
-                             _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), _ptr(workspace),
-                             ws_bytes, _stream(dev))
+                             float(g_min), _ptr(A_log), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]),
+                             _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), _ptr(g["dA_log"]),
+                             _ptr(workspace), ws_bytes, _stream(q.device))
     _raise(st, "kda_chunk_bwd")
+    return g
+
+
+def kda_chunk_bwd_varlen_workspace(N: int, T: int, H: int, dk: int, dv: int) -> int:
+    return int(lib().kda_chunk_bwd_varlen_workspace(N, T, H, dk, dv, KDA_BF16))
+
+
+def kda_chunk_bwd_varlen(q, k, v, a, beta, dO, cu_seqlens, g_min: float = -5.0, S0=None, dS_T=None,
+                         workspace=None, return_dS0: bool = True, out=None, A_log=None):
+    """Backward over a packed batch: q, k, a [T,H,dk], v and dO [T,H,dv], beta [T,H]
+    (bfloat16); cu_seqlens int32 [N+1] on the device; S0, dS_T [N,H,dk,dv] float32 or None.
+    Returns the dict of ``kda_chunk_bwd`` with token gradients [T,H,.] and dS0 [N,H,dk,dv]."""
+    _check_cuda(q, k, v, a, beta, dO, cu_seqlens, S0, dS_T, workspace, A_log)
+    _bwd_checks(q, k, v, a, beta, dO, A_log, 1)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    g = _bwd_outputs(q, v, beta, N, H, dk, dv, return_dS0, A_log, out)
+    need = int(lib().kda_chunk_bwd_varlen_workspace(N, T, H, dk, dv, KDA_BF16))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_bwd_varlen(N, _ptr(cu_seqlens), T, H, dk, dv, KDA_BF16, float(g_min), _ptr(A_log),
+                                    _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                    _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]),
+                                    _ptr(g["dS0"]), _ptr(g["dA_log"]), _ptr(workspace), ws_bytes, _stream(q.device))
+    _raise(st, "kda_chunk_bwd_varlen")
     return g
 
 

@@ -1412,7 +1412,8 @@ struct BwdSmem {  // float offsets in shared memory
     static constexpr int beta = stage + kGStage;
     static constexpr int dGam = beta + kC;
     static constexpr int seg = dGam + D;  // row-segment sums: of dG, then of dKhat * Khat
-    static constexpr int floats = seg + 2 * kBwdThreads;
+    static constexpr int red = seg + 2 * kBwdThreads;  // per-warp partial sums of dA_log
+    static constexpr int floats = red + kBwdWarps;
     static constexpr size_t bytes = (size_t)floats * 4;
     static_assert(bytes <= 232448, "shared memory per block");
 };
@@ -1555,9 +1556,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_chunk_kernel(SeqMap map, int H, int nunits, const __nv_bfloat16 *__restrict__ qg,
                      const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ vg,
                      const __nv_bfloat16 *__restrict__ ag, const __nv_bfloat16 *__restrict__ betag, float g_min,
-                     const __nv_bfloat16 *__restrict__ dOg, const float *__restrict__ Hs,
-                     const float *__restrict__ dHs, float *scratch, float *__restrict__ dq, float *__restrict__ dk,
-                     float *__restrict__ dv, float *__restrict__ da, float *__restrict__ dbeta, unsigned int *status)
+                     const float *__restrict__ A_log, const __nv_bfloat16 *__restrict__ dOg,
+                     const float *__restrict__ Hs, const float *__restrict__ dHs, float *scratch,
+                     float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ da,
+                     float *__restrict__ dbeta, float *__restrict__ dA_part, unsigned int *status)
 {
     using L = BwdSlot<D>;
     using SL = BwdSmem<D>;
@@ -1569,7 +1571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *const sdT = bsm + SL::dT, *const sdA = bsm + SL::dA;
     uint32_t *const stage = reinterpret_cast<uint32_t *>(bsm + SL::stage);
     float *const sbeta = bsm + SL::beta, *const sdGam = bsm + SL::dGam;
-    float *const sseg = bsm + SL::seg;
+    float *const sseg = bsm + SL::seg, *const sred = bsm + SL::red;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *sl = scratch + (size_t)blockIdx.x * L::floats;
     float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Qb = sl + L::Qb, *const Bk = sl + L::Bk;
@@ -1595,6 +1597,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float *S = Hs + loc.rec * (size_t)D * D;
         const float *dSn = dHs + loc.rec * (size_t)D * D;
         auto tix = [&](int r) { return (tok0 + r) * H + h; };  // token-head row index
+        // the gate's argument is scale * a (scale = e^{A_log[h]}, or 1)
+        const float scale = A_log ? __expf(A_log[h]) : 1.0f;
 
         // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da
 #pragma unroll 4
@@ -1602,12 +1606,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int r = e / D, c = e % D;
             const bool ok = r < n;
             const size_t gi = (size_t)tix(ok ? r : 0) * D + c;
-            const float av = __bfloat162float(ag[gi]);
+            const float av = scale * __bfloat162float(ag[gi]);
             const float sg = __fdividef(1.f, 1.f + __expf(-av));
             sq[r * LDD + c] = ok ? __bfloat162float(qg[gi]) : 0.f;
             sk[r * LDD + c] = ok ? __bfloat162float(kg[gi]) : 0.f;
             sG[r * LDD + c] = ok ? gate_bounded_fast(av, g_min) : 0.f;
-            Gp[e] = g_min * sg * (1.f - sg);
+            Gp[e] = g_min * sg * (1.f - sg) * scale;
             Bv[e] = ok ? __bfloat162float(vg[gi]) : 0.f;
             dOs[e] = ok ? __bfloat162float(dOg[gi]) : 0.f;
         }
@@ -1886,12 +1890,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 acc += sseg[kBwdThreads + s2 * D + c];
             for (int s2 = sgi + 1; s2 < NSEG; ++s2)
                 acc += sseg[s2 * D + c];
+            float dal = 0.f;  // sum of da * a over the segment: this chunk's share of dL/dA_log
 #pragma unroll
             for (int u = SR - 1; u >= 0; --u) {
                 const int r = r0 + u;
                 acc += sq[r * LDD + c];
-                if (r < n)
-                    da[(size_t)tix(r) * D + c] = acc * gp[u];
+                if (r < n) {
+                    const size_t gi = (size_t)tix(r) * D + c;
+                    const float dav = acc * gp[u];
+                    da[gi] = dav;
+                    if (dA_part)
+                        dal = fmaf(dav, __bfloat162float(ag[gi]), dal);
+                }
+            }
+            if (dA_part) {  // dL/dA_log = sum over the head's tokens and channels of da * a
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    dal += __shfl_xor_sync(0xffffffffu, dal, o);
+                if (lane == 0)
+                    sred[warp] = dal;
             }
         }
         // 10. dbeta_r = sum_c dBk_rc Kbar_rc + sum_c dBv_rc v_rc + sum_s dA_rs A'_rs; warp per row
@@ -1917,7 +1934,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 dbeta[tix(r)] = acc;
         }
         __syncthreads();  // shared memory and the slot are reused by the next chunk
+        if (dA_part && tid == 0) {
+            float sum = 0.f;
+            for (int w = 0; w < kBwdWarps; ++w)
+                sum += sred[w];
+            dA_part[loc.rec] = sum;
+        }
     }
+}
+
+// dL/dA_log[h]: the sum of the per-chunk partials of head h, in a fixed order.  One CTA per
+// head; regular batch: records (b H + h) NT + n; packed batch: records h NT + g, g < chunks.
+constexpr int kRedThreads = 256;
+
+__global__ void __launch_bounds__(kRedThreads)
+    dalog_reduce_kernel(SeqMap map, int H, const float *__restrict__ part, float *__restrict__ dA_log)
+{
+    __shared__ float buf[kRedThreads];
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const int64_t per = map.cu ? (int64_t)map.choff[map.nseq] : (int64_t)map.nseq * map.NT;
+    float acc = 0.f;
+    for (int64_t i = tid; i < per; i += kRedThreads) {
+        const int64_t rec = map.cu ? (int64_t)h * map.NT + i
+                                   : ((i / map.NT) * H + h) * (int64_t)map.NT + i % map.NT;
+        acc += part[rec];
+    }
+    buf[tid] = acc;
+    __syncthreads();
+    for (int s2 = kRedThreads / 2; s2 > 0; s2 >>= 1) {
+        if (tid < s2)
+            buf[tid] += buf[tid + s2];
+        __syncthreads();
+    }
+    if (tid == 0)
+        dA_log[h] = buf[0];
 }
 
 template <int D, bool kLogSig>
@@ -1974,40 +2024,45 @@ cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const flo
                    : launch_scan_d<128>(m, H, ws, S0, o, S_T, M_out, s);
 }
 
-// Backward workspace: the forward records, then the entering state of every chunk and the
-// gradient of the state after it (fp32, D x D per record, in record order), then the
-// per-CTA scratch slots of bwd_chunk_kernel.
+// Backward workspace: the forward records (and, for a packed batch, the chunk table), then the
+// entering state of every chunk and the gradient of the state after it (fp32, D x D per
+// record, in record order), the per-chunk partials of dL/dA_log, and the per-CTA scratch slots
+// of bwd_chunk_kernel.
 struct BwdLayout {
-    size_t states, dstates, scratch, total;
+    size_t table, states, dstates, parts, scratch, total;
 };
 
-BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D)
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D, int nseq_packed = 0)
 {
     const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
     const size_t blk = (size_t)D * D * 4;
     const size_t slot = (size_t)(D == 64 ? BwdSlot<64>::floats : BwdSlot<128>::floats) * 4;
     BwdLayout l;
-    l.states = ((size_t)nrec * rec + 255) / 256 * 256;
+    l.table = (size_t)nrec * rec;
+    l.states = round256(l.table + (nseq_packed ? (size_t)(nseq_packed + 1) * 4 : 0));
     l.dstates = l.states + (size_t)nrec * blk;
-    l.scratch = l.dstates + (size_t)nrec * blk;
+    l.parts = l.dstates + (size_t)nrec * blk;
+    l.scratch = round256(l.parts + (size_t)nrec * 4);
     l.total = l.scratch + (size_t)std::min<int64_t>(nunits, kBwdSlots) * slot;
     return l;
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits, const void *q, const void *k,
-                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
-                         const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da, float *dbeta,
-                         float *dS0, void *ws, cudaStream_t s)
+cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits, const BwdLayout &l,
+                         const void *q, const void *k, const void *v, const void *a, const void *beta, float g_min,
+                         const float *A_log, const float *S0, const void *dO, const float *dS_T, float *dq, float *dk,
+                         float *dv, float *da, float *dbeta, float *dS0, float *dA_log, void *ws, cudaStream_t s)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
-    const BwdLayout l = bwd_layout(m.nrec, nunits, D);
     unsigned char *base = static_cast<unsigned char *>(ws);
     float *Hs = reinterpret_cast<float *>(base + l.states), *dHs = reinterpret_cast<float *>(base + l.dstates);
+    float *parts = dA_log ? reinterpret_cast<float *>(base + l.parts) : nullptr;
     float *scratch = reinterpret_cast<float *>(base + l.scratch);
-    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, nullptr, ws, s);
+    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, A_log, ws, s);
     if (e == cudaSuccess)
         e = launch_scan_d<D>(m, H, ws, S0, nullptr, nullptr, nullptr, s, Hs);
     if (e != cudaSuccess)
@@ -2028,8 +2083,12 @@ cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits,
     bwd_chunk_kernel<D><<<grid, kBwdThreads, BwdSmem<D>::bytes, s>>>(
         m, H, (int)nunits, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-        static_cast<const __nv_bfloat16 *>(beta), g_min, static_cast<const __nv_bfloat16 *>(dO), Hs, dHs, scratch,
-        dq, dk, dv, da, dbeta, status);
+        static_cast<const __nv_bfloat16 *>(beta), g_min, A_log, static_cast<const __nv_bfloat16 *>(dO), Hs, dHs,
+        scratch, dq, dk, dv, da, dbeta, parts, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !dA_log)
+        return e;
+    dalog_reduce_kernel<<<H, kRedThreads, 0, s>>>(m, H, parts, dA_log);
     return cudaGetLastError();
 }
 
@@ -2135,16 +2194,53 @@ void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *
 }
 
 cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                                  const void *a, const void *beta, float g_min, const float *S0, const void *dO,
-                                  const float *dS_T, float *dq, float *dk, float *dv, float *da, float *dbeta,
-                                  float *dS0, void *workspace, cudaStream_t s)
+                                  const void *a, const void *beta, float g_min, const float *A_log, const float *S0,
+                                  const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da,
+                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s)
 {
     const SeqMap m = regular_map(B, T, H);
     const dim3 grid(m.NT, B * H);
-    return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk, dv, da,
-                                      dbeta, dS0, workspace, s)
-                   : launch_bwd_d<128>(m, H, grid, m.nrec, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk, dv, da,
-                                       dbeta, dS0, workspace, s);
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D);
+    return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk, dv,
+                                      da, dbeta, dS0, dA_log, workspace, s)
+                   : launch_bwd_d<128>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk,
+                                       dv, da, dbeta, dS0, dA_log, workspace, s);
+}
+
+size_t chunk_bf16_bwd_varlen_workspace(int N, int T, int H, int D)
+{
+    const int64_t nrec = (int64_t)H * (int64_t)varlen_records(N, T);
+    return bwd_layout(nrec, nrec, D, N).total;
+}
+
+cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
+                                         const void *v, const void *a, const void *beta, float g_min,
+                                         const float *A_log, const float *S0, const void *dO, const float *dS_T,
+                                         float *dq, float *dk, float *dv, float *da, float *dbeta, float *dS0,
+                                         float *dA_log, void *workspace, cudaStream_t s)
+{
+    unsigned int *status = device_status_ptr();
+    if (!status)
+        return cudaErrorInvalidDevice;
+    SeqMap m;
+    m.cu = cu;
+    m.nseq = N;
+    m.T = T;
+    m.NT = (int)varlen_records(N, T);
+    m.nrec = (int64_t)H * m.NT;
+    m.ntok = T;
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, N);
+    int32_t *choff = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + l.table);
+    m.choff = choff;
+    seq_table_kernel<<<1, kTableThreads, 0, s>>>(cu, N, T, choff, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const dim3 grid(m.NT, H);
+    return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk, dv,
+                                      da, dbeta, dS0, dA_log, workspace, s)
+                   : launch_bwd_d<128>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk,
+                                       dv, da, dbeta, dS0, dA_log, workspace, s);
 }
 
 // ------------------------------------------------------------------ segment combine

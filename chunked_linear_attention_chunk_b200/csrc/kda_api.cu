@@ -525,9 +525,10 @@ kda_status kda_chunk_bwd_offsets(int B, int T, int H, int dk, int dv, size_t *st
 }
 
 kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
-                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
-                         const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_, float *da,
-                         float *dbeta, float *dS0, void *workspace, size_t ws_bytes, kda_stream_t stream)
+                         const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                         const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
+                         float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
+                         kda_stream_t stream)
 {
     ChunkShape sh;
     kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
@@ -539,12 +540,21 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
     if (st != KDA_OK)
         return st;
     cudaStream_t s = (cudaStream_t)stream;
-    if (!all_aligned({S0, dS_T, dS0}))
+    if (dA_log && !A_log)
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({S0, dS_T, dS0}) || ((uintptr_t)A_log & 3u) || ((uintptr_t)dA_log & 3u))
         return KDA_ERR_ALIGNMENT;
-    const Range rS0(S0, sh.ns * 4), rdST(dS_T, sh.ns * 4), rdS0(dS0, sh.ns * 4);
-    if (overlaps(rdS0, rS0) || overlaps(rdS0, rdST))
+    const Range rS0(S0, sh.ns * 4), rdST(dS_T, sh.ns * 4), rdS0(dS0, sh.ns * 4), rA(A_log, (int64_t)H * 4),
+        rdA(dA_log, (int64_t)H * 4);
+    if (overlaps(rdS0, rS0) || overlaps(rdS0, rdST) || overlaps(rdS0, rA) || overlaps(rdA, rA) ||
+        overlaps(rdA, rS0) || overlaps(rdA, rdST) || overlaps(rdA, rdS0))
         return KDA_ERR_ALIAS;
     if (T == 0) {
+        if (dA_log) {
+            const kda_status z = from_cuda(cudaMemsetAsync(dA_log, 0, (size_t)H * 4, s));
+            if (z != KDA_OK)
+                return z;
+        }
         if (!dS0)
             return KDA_OK;
         if (dS_T)
@@ -560,9 +570,9 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
         return KDA_ERR_WORKSPACE;
     const int64_t es = 2;
     const Range ins[] = {Range(q, sh.nk * es), Range(k, sh.nk * es), Range(v, sh.nv * es), Range(a, sh.nk * es),
-                         Range(beta, sh.ntok * es), Range(dO, sh.nv * es), rS0, rdST};
+                         Range(beta, sh.ntok * es), Range(dO, sh.nv * es), rS0, rdST, rA};
     const Range outs[] = {Range(dq, sh.nk * 4), Range(dk_, sh.nk * 4), Range(dv_, sh.nv * 4), Range(da, sh.nk * 4),
-                          Range(dbeta, sh.ntok * 4), rdS0, Range(workspace, (int64_t)need)};
+                          Range(dbeta, sh.ntok * 4), rdS0, rdA, Range(workspace, (int64_t)need)};
     for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
         for (const Range &in : ins)
             if (overlaps(outs[i], in))
@@ -571,8 +581,76 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
             if (overlaps(outs[i], outs[j]))
                 return KDA_ERR_ALIAS;
     }
-    return from_cuda(launch_chunk_bwd_bf16(B, T, H, dk, q, k, v, a, beta, g_min, S0, dO, dS_T, dq, dk_, dv_, da,
-                                           dbeta, dS0, workspace, s));
+    return from_cuda(launch_chunk_bwd_bf16(B, T, H, dk, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk_, dv_,
+                                           da, dbeta, dS0, dA_log, workspace, s));
+}
+
+size_t kda_chunk_bwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (N < 1 || T < 1 || T > kMaxPackedTokens || H < 1 || dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16)
+        return 0;
+    return chunk_bf16_bwd_varlen_workspace(N, T, H, dk);
+}
+
+kda_status kda_chunk_bwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
+                                float g_min, const float *A_log, const void *q, const void *k, const void *v,
+                                const void *a, const void *beta, const float *S0, const void *dO, const float *dS_T,
+                                float *dq, float *dk_, float *dv_, float *da, float *dbeta, float *dS0,
+                                float *dA_log, void *workspace, size_t ws_bytes, kda_stream_t stream)
+{
+    if (!dtype_ok(dtype) || N < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = check_gmin(g_min);
+    if (st != KDA_OK)
+        return st;
+    if (dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16 || T > kMaxPackedTokens || (int64_t)N * H > 65535 ||
+        (int64_t)H * (((int64_t)T + 63) / 64 + N) > 0x7fffffff)
+        return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || (dA_log && !A_log))
+        return KDA_ERR_INVALID_ARG;
+    const int64_t nk = (int64_t)T * H * dk, ntok = (int64_t)T * H, ns = (int64_t)N * H * dk * dv;
+    if (!all_aligned({S0, dS_T, dS0}) || ((uintptr_t)cu_seqlens & 3u) || ((uintptr_t)A_log & 3u) ||
+        ((uintptr_t)dA_log & 3u))
+        return KDA_ERR_ALIGNMENT;
+    const Range rcu(cu_seqlens, (int64_t)(N + 1) * 4), rS0(S0, ns * 4), rdST(dS_T, ns * 4), rdS0(dS0, ns * 4),
+        rA(A_log, (int64_t)H * 4), rdA(dA_log, (int64_t)H * 4);
+    if (T == 0) {
+        // nothing to differentiate through; the state gradient passes unchanged (cu is not read)
+        if (overlaps(rdS0, rS0) || overlaps(rdS0, rdST) || overlaps(rdS0, rA) || overlaps(rdA, rA) ||
+            overlaps(rdA, rdS0) || overlaps(rdA, rdST) || overlaps(rdA, rS0) || overlaps(rdS0, rcu) ||
+            overlaps(rdA, rcu))
+            return KDA_ERR_ALIAS;
+        cudaStream_t s = (cudaStream_t)stream;
+        if (dA_log && (st = from_cuda(cudaMemsetAsync(dA_log, 0, (size_t)H * 4, s))) != KDA_OK)
+            return st;
+        if (!dS0)
+            return KDA_OK;
+        if (dS_T)
+            return from_cuda(cudaMemcpyAsync(dS0, dS_T, (size_t)ns * 4, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(dS0, 0, (size_t)ns * 4, s));
+    }
+    if (!q || !k || !v || !a || !beta || !dO || !dq || !dk_ || !dv_ || !da || !dbeta)
+        return KDA_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, a, dO, dq, dk_, dv_, da, dbeta, workspace}) || !beta_aligned(beta, 2))
+        return KDA_ERR_ALIGNMENT;
+    const size_t need = chunk_bf16_bwd_varlen_workspace(N, T, H, dk);
+    if (!workspace || ws_bytes < need)
+        return KDA_ERR_WORKSPACE;
+    const Range ins[] = {Range(q, nk * 2), Range(k, nk * 2), Range(v, nk * 2), Range(a, nk * 2), Range(beta, ntok * 2),
+                         Range(dO, nk * 2), rS0, rdST, rA, rcu};
+    const Range outs[] = {Range(dq, nk * 4), Range(dk_, nk * 4), Range(dv_, nk * 4), Range(da, nk * 4),
+                          Range(dbeta, ntok * 4), rdS0, rdA, Range(workspace, (int64_t)need)};
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+        for (const Range &in : ins)
+            if (overlaps(outs[i], in))
+                return KDA_ERR_ALIAS;
+        for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+            if (overlaps(outs[i], outs[j]))
+                return KDA_ERR_ALIAS;
+    }
+    return from_cuda(launch_chunk_bwd_bf16_varlen(N, cu_seqlens, T, H, dk, q, k, v, a, beta, g_min, A_log, S0, dO,
+                                                  dS_T, dq, dk_, dv_, da, dbeta, dS0, dA_log, workspace,
+                                                  (cudaStream_t)stream));
 }
 
 kda_status kda_device_status(kda_stream_t stream)

@@ -52,15 +52,23 @@ cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int
                                      const float *A_log, const float *S0, void *o, float *S_T, void *workspace,
                                      cudaStream_t s);
 
-// Backward of the bf16 chunked forward (bounded gate): prep, the scan saving every chunk's
-// entering state, the reverse state-gradient scan and the per-chunk gradients.  Gradients
-// are float32; S0, dS_T and dS0 are nullable.
+// Backward of the bf16 chunked forward (bounded gate, optional per-head scale A_log): prep,
+// the scan saving every chunk's entering state, the reverse state-gradient scan, the
+// per-chunk gradients and (with dA_log) the per-head reduction of dL/dA_log.  Gradients are
+// float32; A_log, S0, dS_T, dS0 and dA_log are nullable.
 size_t chunk_bf16_bwd_workspace(int B, int T, int H, int D);
 void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *dstates);
 cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
-                                  const void *a, const void *beta, float g_min, const float *S0, const void *dO,
-                                  const float *dS_T, float *dq, float *dk, float *dv, float *da, float *dbeta,
-                                  float *dS0, void *workspace, cudaStream_t s);
+                                  const void *a, const void *beta, float g_min, const float *A_log, const float *S0,
+                                  const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da,
+                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s);
+// The same over a packed batch (cu on the device, checked on the device as in the forward).
+size_t chunk_bf16_bwd_varlen_workspace(int N, int T, int H, int D);
+cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
+                                         const void *v, const void *a, const void *beta, float g_min,
+                                         const float *A_log, const float *S0, const void *dO, const float *dS_T,
+                                         float *dq, float *dk, float *dv, float *da, float *dbeta, float *dS0,
+                                         float *dA_log, void *workspace, cudaStream_t s);
 // K4: single-token decode step.
 cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,
                           const void *a, const void *beta, float g_min, float *S, void *o, cudaStream_t s);

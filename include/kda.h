@@ -270,22 +270,27 @@ kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M
                              const float *S0, float *S_in, kda_stream_t stream);
 
 /*
- * kda_chunk_bwd -- gradients of the bfloat16 chunked forward (bounded gate) with respect
- * to every input, given the gradient of the loss with respect to o and to the final
- * state.  Passage: long sequences are trained by recursing in chunks ("Trillion-Parameter
- * MoE ... Engineering" section 3.2); the pages print no backward, so this is the
- * derivative of kda_chunk_fwd's recurrence, computed in the same chunked form:
+ * kda_chunk_bwd -- gradients of the bfloat16 chunked forward (bounded gate, optionally with
+ * the per-head scale e^{A_log[h]} on the gate's argument) with respect to every input,
+ * given the gradient of the loss with respect to o and to the final state.  Passage: long
+ * sequences are trained by recursing in chunks ("Trillion-Parameter MoE ... Engineering"
+ * section 3.2); the pages print no backward, so this is the derivative of kda_chunk_fwd's
+ * recurrence, computed in the same chunked form:
  *     dS = (Diag(Gamma) - N)^T dS' + Q'^T dO        (state gradient, chunks in reverse)
  * and, inside each chunk, the reverse of the chunk's products (see chunk_bf16.cu).  It
  * recomputes the forward (prep and scan) inside the call; nothing of a forward call is
  * needed.  All gradients are float32.
  *   B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, S0: exactly as in kda_chunk_fwd
  *                (dtype must be KDA_BF16; S0 may be NULL for zeros).
+ *   A_log        NULL, or a DEVICE array of H float32 values (4-byte aligned): the gate is
+ *                g = g_min * sigmoid(e^{A_log[h]} a), as in kda_chunk_fwd_prep.
  *   dO           [B, T, H, dv] bfloat16: dL/do.
  *   dS_T         [B, H, dk, dv] float32 or NULL (zero): dL/dS_T.
  *   dq, dk_, da  [B, T, H, dk] float32 out;  dv_: [B, T, H, dv] float32 out;
  *   dbeta        [B, T, H] float32 out;  dS0: [B, H, dk, dv] float32 out or NULL.
- *                da is the gradient with respect to the gate's pre-activation a.
+ *                da is the gradient with respect to the gate's input a.
+ *   dA_log       [H] float32 out, or NULL (needs A_log): dL/dA_log, the sum over the head's
+ *                tokens and channels of da * a, reduced in a fixed order.
  *   workspace    >= kda_chunk_bwd_workspace(B, T, H, dk, dv, dtype) bytes, 16-byte
  *                aligned: the forward's records, the state entering every chunk and the
  *                gradient of the state after it (float32, dk x dv per (b, h, chunk), in
@@ -293,15 +298,29 @@ kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M
  *                gradient kernel's scratch.
  * The outputs must not overlap each other, an input or the workspace.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.  T == 0 writes dS0 =
- * dS_T (or zeros) and nothing else.
+ * dS_T (or zeros), dA_log = 0, and nothing else.
+ *
+ * kda_chunk_bwd_varlen -- the same over a packed batch of N sequences on one token axis, as
+ * kda_chunk_fwd_varlen lays it out (cu_seqlens on the device and checked there; each
+ * sequence starts from S0[s] and ends with the gradient dS_T[s]).  Token tensors and their
+ * gradients are [T, H, .], states [N, H, dk, dv].  Workspace: kda_chunk_bwd_varlen_workspace.
+ * An invalid cu_seqlens records KDA_ERR_INVALID_ARG in the device status word; the
+ * gradients are then unspecified but nothing outside the buffers is touched.
  */
 size_t kda_chunk_bwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 kda_status kda_chunk_bwd_offsets(int B, int T, int H, int dk, int dv, size_t *states_offset,
                                  size_t *dstates_offset);
 kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
-                         const void *v, const void *a, const void *beta, float g_min, const float *S0,
-                         const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_, float *da,
-                         float *dbeta, float *dS0, void *workspace, size_t ws_bytes, kda_stream_t stream);
+                         const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                         const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
+                         float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
+                         kda_stream_t stream);
+size_t kda_chunk_bwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype);
+kda_status kda_chunk_bwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
+                                float g_min, const float *A_log, const void *q, const void *k, const void *v,
+                                const void *a, const void *beta, const float *S0, const void *dO, const float *dS_T,
+                                float *dq, float *dk_, float *dv_, float *da, float *dbeta, float *dS0,
+                                float *dA_log, void *workspace, size_t ws_bytes, kda_stream_t stream);
 
 /*
  * kda_decode_step -- one token for N independent sequences, state updated in place.

@@ -62,7 +62,7 @@ def _gpu(x, dO, dST, S0, workspace=None):
                           workspace=workspace)
     torch.cuda.synchronize()
     assert kda.kda_device_status() == 0
-    return {n: t.cpu().numpy() for n, t in g.items()}
+    return {n: t.cpu().numpy() for n, t in g.items() if t is not None}
 
 
 def _check(got, ref):
@@ -152,3 +152,98 @@ def test_bwd_full_size_sampled_heads():
             gh = got[n][:, h:h + 1] if n == "dS0" else got[n][:, :, h:h + 1]
             e = _err_state(gh, ref[n]) if n == "dS0" else _err(gh, ref[n])
             assert e <= TOL_BWD, f"head {h} {n}: {e:.3e}"
+
+
+def _oracle_scaled(x, dO, dST, S0, A_log):
+    """The oracle on the gate's scaled argument: g = g_min sigma(e^{A_h} a) is the bounded gate
+    of a' = e^{A_h} a, so da = e^{A_h} da' and dL/dA_log[h] = sum over the head of da' a'."""
+    scale = np.exp(A_log.astype(np.float64))
+    a_s = (synth.to_numpy32(x["a"]).astype(np.float64) * scale[None, None, :, None]).astype(np.float32)
+    xs = dict(x)
+    xs["a"] = torch.from_numpy(a_s)
+    ref = _oracle(xs, dO, dST, S0)
+    dA = np.einsum("bthc,bthc->h", ref["da"], a_s.astype(np.float64))
+    terms = np.einsum("bthc->h", np.abs(ref["da"] * a_s.astype(np.float64)))
+    ref["da"] = ref["da"] * scale[None, None, :, None]
+    return ref, dA, terms
+
+
+@pytest.mark.parametrize("B,T,H,D", [(2, 150, 3, 64), (1, 200, 2, 128)])
+def test_bwd_head_scaled_gate(B, T, H, D):
+    """A_log given: every gradient against the oracle run on e^{A_h} a, and dL/dA_log against
+    the chain rule (the sum of da' a' over the head), within 2e-2 of the sum of |da' a'|."""
+    x, dO, dST, S0 = _case(B, T, H, D, seed=750 + T)
+    A_log = (np.random.default_rng(751).normal(size=H) * 0.5).astype(np.float32)
+    d = {n: x[n].cuda() for n in NAMES}
+    g = kda.kda_chunk_bwd(*(d[n] for n in NAMES), dO.cuda(), G_MIN, S0=S0.cuda(), dS_T=dST.cuda(),
+                          A_log=torch.from_numpy(A_log).cuda())
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    got = {n: t.cpu().numpy() for n, t in g.items()}
+    ref, dA, terms = _oracle_scaled(x, dO, dST, S0, A_log)
+    _check(got, ref)
+    assert np.all(np.abs(got["dA_log"] - dA) <= TOL_BWD * terms), (got["dA_log"], dA, terms)
+    # the reduction is the sum of the kernel's own da * a
+    own = np.einsum("bthc,bthc->h", got["da"].astype(np.float64), synth.to_numpy32(x["a"]).astype(np.float64))
+    assert np.all(np.abs(got["dA_log"] - own) <= 1e-4 * np.abs(got["da"] * synth.to_numpy32(x["a"])).sum((0, 1, 3)))
+
+
+def _packed(lengths, H, D, seed):
+    T = int(sum(lengths))
+    x = synth.make_inputs(1, T, H, D, D, "bf16", seed=seed, s0_std=0.1)
+    N = len(lengths)
+    rng = np.random.default_rng(seed)
+    S0 = torch.from_numpy((rng.normal(size=(N, H, D, D)) * 0.1).astype(np.float32))
+    dST = torch.from_numpy((rng.normal(size=(N, H, D, D)) * 0.5).astype(np.float32))
+    dO = torch.from_numpy(rng.normal(size=(1, T, H, D)).astype(np.float32)).to(torch.bfloat16)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    return x, dO, dST, S0, cu
+
+
+@pytest.mark.parametrize("lengths,H,D,with_A", [([70, 0, 129, 64], 2, 64, False), ([1, 200, 63], 2, 128, True)])
+def test_bwd_varlen_matches_oracle(lengths, H, D, with_A):
+    """Packed sequences (one empty, a single token, tails, exact chunks): each sequence against
+    the oracle on its own slice with its own S0 and dS_T."""
+    x, dO, dST, S0, cu = _packed(lengths, H, D, seed=760 + D)
+    A_log = (np.random.default_rng(761).normal(size=H) * 0.5).astype(np.float32) if with_A else None
+    pk = {n: x[n][0].cuda() for n in NAMES}
+    g = kda.kda_chunk_bwd_varlen(*(pk[n] for n in NAMES), dO[0].cuda(), torch.from_numpy(cu).cuda(), G_MIN,
+                                 S0=S0.cuda(), dS_T=dST.cuda(),
+                                 A_log=None if A_log is None else torch.from_numpy(A_log).cuda())
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    got = {n: (None if t is None else t.cpu().numpy()) for n, t in g.items()}
+    dA_tot, terms_tot = np.zeros(H), np.zeros(H)
+    for s in range(len(lengths)):
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        if t1 == t0:
+            assert np.array_equal(got["dS0"][s], dST[s].numpy()), "empty sequence passes dS_T through"
+            continue
+        xs = {n: x[n][:, t0:t1] for n in NAMES}
+        if with_A:
+            ref, dA, terms = _oracle_scaled(xs, dO[:, t0:t1], dST[s:s + 1], S0[s:s + 1], A_log)
+            dA_tot += dA
+            terms_tot += terms
+        else:
+            ref = _oracle(xs, dO[:, t0:t1], dST[s:s + 1], S0[s:s + 1])
+        gs = {n: got[n][None, t0:t1] for n in ("dq", "dk", "dv", "da", "dbeta")}
+        gs["dS0"] = got["dS0"][s:s + 1]
+        _check(gs, ref)
+    if with_A:
+        assert np.all(np.abs(got["dA_log"] - dA_tot) <= TOL_BWD * terms_tot)
+
+
+def test_bwd_varlen_equal_lengths_equals_regular_batch():
+    """B equal-length sequences packed give exactly the regular batch's gradients."""
+    B, T, H, D = 3, 130, 2, 128
+    x, dO, dST, S0 = _case(B, T, H, D, seed=770)
+    reg = _gpu(x, dO, dST, S0)
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32).cuda()
+    pk = {n: x[n].reshape(B * T, *x[n].shape[2:]).cuda() for n in NAMES}
+    g = kda.kda_chunk_bwd_varlen(*(pk[n] for n in NAMES), dO.reshape(B * T, H, D).cuda(), cu, G_MIN,
+                                 S0=S0.cuda(), dS_T=dST.cuda())
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    for n in ("dq", "dk", "dv", "da", "dbeta"):
+        assert np.array_equal(g[n].cpu().numpy().reshape(reg[n].shape), reg[n]), n
+    assert np.array_equal(g["dS0"].cpu().numpy(), reg["dS0"])

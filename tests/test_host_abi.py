@@ -325,10 +325,10 @@ def test_chunk_bwd_entry_validates(L):
     ws = BASE + 12 * step
 
     def bwd(dtype=kda.KDA_BF16, g_min=-5.0, q=ins[0], dO=ins[5], dq=outs[0], dbeta=outs[4], w=ws, wb=need,
-            S0=None, dST=None, dS0=None, dk=D):
+            S0=None, dST=None, dS0=None, dk=D, A=None, dA=None):
         return L.kda_chunk_bwd(B, T, H, dk, dk, dtype, P(q), P(ins[1]), P(ins[2]), P(ins[3]), P(ins[4]),
-                               ctypes.c_float(g_min), P(S0), P(dO), P(dST), P(dq), P(outs[1]), P(outs[2]),
-                               P(outs[3]), P(dbeta), P(dS0), P(w), wb, None)
+                               ctypes.c_float(g_min), P(A), P(S0), P(dO), P(dST), P(dq), P(outs[1]), P(outs[2]),
+                               P(outs[3]), P(dbeta), P(dS0), P(dA), P(w), wb, None)
 
     assert bwd(dtype=kda.KDA_F32) == UNSUPPORTED
     assert bwd(dk=96) == UNSUPPORTED
@@ -347,8 +347,45 @@ def test_chunk_bwd_entry_validates(L):
     S = BASE * 2
     assert bwd(S0=S, dS0=S) == ALIAS
     assert bwd(dST=S, dS0=S + 4096) == ALIAS
+    assert bwd(dA=BASE * 3) == INVALID                    # dA_log needs A_log
+    assert bwd(A=BASE * 3 + 2) == ALIGN
+    assert bwd(A=BASE * 3, dA=BASE * 3) == ALIAS
+    assert bwd(A=BASE * 3, dA=outs[0]) == ALIAS           # dA_log inside dq
     sa, sb = ctypes.c_size_t(0), ctypes.c_size_t(0)
     assert L.kda_chunk_bwd_offsets(B, T, H, D, D, ctypes.byref(sa), ctypes.byref(sb)) == OK
     assert sa.value >= L.kda_chunk_fwd_workspace(B, T, H, D, D, kda.KDA_BF16) and sa.value % 16 == 0
     assert sb.value == sa.value + B * H * D * D * 4
     assert L.kda_chunk_bwd_offsets(B, T, H, D, D, None, ctypes.byref(sb)) == INVALID
+
+
+def test_chunk_bwd_varlen_entry_validates(L):
+    """kda_chunk_bwd_varlen rejects bad arguments before a launch (fake pointers)."""
+    P = ctypes.c_void_p
+    N, T, H, D = 3, 200, 2, 64
+    nb = T * H * D * 2
+    need = L.kda_chunk_bwd_varlen_workspace(N, T, H, D, D, kda.KDA_BF16)
+    assert need > L.kda_chunk_bwd_workspace(1, T, H, D, D, kda.KDA_BF16)
+    assert L.kda_chunk_bwd_varlen_workspace(0, T, H, D, D, kda.KDA_BF16) == 0
+    step = nb * 2 + 4096
+    ins = [BASE + i * step for i in range(6)]
+    outs = [BASE + (6 + i) * step for i in range(5)]
+    ws = BASE + 12 * step
+    cu = BASE + 13 * step
+
+    def bwd(n=N, cu_=cu, q=ins[0], dq=outs[0], w=ws, wb=need, g_min=-5.0, dk=D, A=None, dA=None):
+        return L.kda_chunk_bwd_varlen(n, P(cu_), T, H, dk, dk, kda.KDA_BF16, ctypes.c_float(g_min), P(A), P(q),
+                                      P(ins[1]), P(ins[2]), P(ins[3]), P(ins[4]), None, P(ins[5]), None, P(dq),
+                                      P(outs[1]), P(outs[2]), P(outs[3]), P(outs[4]), None, P(dA), P(w), wb, None)
+
+    assert bwd(n=0) == INVALID
+    assert bwd(cu_=0) == INVALID
+    assert bwd(cu_=cu + 2) == ALIGN
+    assert bwd(g_min=0.0) == INVALID
+    assert bwd(dk=96) == UNSUPPORTED
+    assert bwd(q=0) == INVALID
+    assert bwd(dq=outs[0] + 4) == ALIGN
+    assert bwd(w=0) == WS
+    assert bwd(wb=need - 1) == WS
+    assert bwd(dq=ins[1]) == ALIAS
+    assert bwd(w=cu) == ALIAS                             # workspace over cu_seqlens
+    assert bwd(dA=BASE * 3) == INVALID

@@ -441,7 +441,26 @@ def run_libkda(args):
                "dominant_kernel": {"kernel": "bwd_chunk_kernel (per-chunk gradients)",
                                    "algorithmic_bytes_per_token_head": BWD_CHUNK_BYTES_PER_TOKEN_HEAD,
                                    "traffic": None if bwd_traffic is None else bwd_traffic * token_heads}}
-        del ws_b, gout, dO
+        del ws_b, gout
+        # the same over the packed batch of the varlen leg (documents of mixed length)
+        if (B, T, H) == (1, synth.VARLEN_64K_T, synth.VARLEN_64K_H):
+            lengths = synth.document_lengths(T)
+            cu_b = torch.from_numpy(synth.cu_seqlens(lengths)).to(device)
+            ws_vb = torch.empty(kda.kda_chunk_bwd_varlen_workspace(len(lengths), T, H, D, D), dtype=torch.uint8,
+                                device=device)
+            packed = [d[n][0] for n in names]
+            gv = {}
+
+            def bwd_vl_step():
+                gv.update(kda.kda_chunk_bwd_varlen(*packed, dO[0], cu_b, G_MIN, workspace=ws_vb, out=gv or None))
+
+            bvl_ms = time_steps(bwd_vl_step, max(3, min(args.steps, 5)), 3, world, device)
+            assert kda.kda_device_status(device) == 0
+            bwd["packed"] = {"workload": f"the varlen leg's {len(lengths)} documents on the 64K axis",
+                             "ms_per_step": bvl_ms, "value": world * tokens / (bvl_ms * 1e-3), "unit": UNIT,
+                             "gpu_launches_per_step": 5}
+            del ws_vb, gv
+        del dO
 
     # ---- end to end through the C ABI with pinned host buffers, pipelined across steps:
     # every step copies its inputs host -> device on one stream, runs kda_chunk_fwd on a

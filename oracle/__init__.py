@@ -14,6 +14,9 @@ passages of the pages each one follows):
 * ``chunked(C, ...)``           -- the chunked form with pairwise exponentials, fp64.
 * ``decode(...)``               -- one decode step, state updated in place.
 * ``backward(...)``             -- gradients of the recurrence (reverse mode, by hand).
+
+``oracle.chunked_backward`` (fp64 numpy) writes the same gradients out in the chunked form,
+chunk by chunk in reverse; it is pinned equal to ``backward``.
 * ``tile_factors_f32(...)``     -- counts of non-finite / subnormal values when a
   16-token tile's pairwise decay is factored densely in float32.
 

@@ -401,6 +401,24 @@ def pin_backward_single_token_closed_form(lib):
     assert np.allclose(g["dS0"][0, 0], ref, rtol=1e-12, atol=1e-14)
 
 
+def pin_backward_chunked_equals_recurrence(lib):
+    """The chunked form of the backward (fp64 numpy, chunk algebra written out) equals the
+    token-level derivative at every chunk size, both gates, ragged tails included."""
+    from oracle.chunked_backward import chunked_backward
+    for kind in (oracle.GATE_BOUNDED, oracle.GATE_LOGSIGMOID):
+        for C, T in ((1, 5), (7, 64), (16, 37), (64, 150)):
+            x = _inputs(2, T, 2, 8, seed=80 + C + T, s0_std=0.2)
+            rng = np.random.default_rng(C + T)
+            dO = rng.normal(size=x["v"].shape).astype(np.float32)
+            dST = rng.normal(size=x["S0"].shape)
+            ref = oracle.backward(x["q"], x["k"], x["v"], x["a"], x["beta"], dO, G_MIN, S0=x["S0"], dST=dST,
+                                  kind=kind, lib=lib)
+            got = chunked_backward(C, x["q"], x["k"], x["v"], x["a"], x["beta"], dO, G_MIN, S0=x["S0"], dST=dST,
+                                   kind=kind)
+            for n in ref:
+                assert _rel(got[n], ref[n]) < 1e-11, (kind, C, T, n, _rel(got[n], ref[n]))
+
+
 ALL_PINS = [
     pin_gate_special_values,
     pin_gate_vs_library,
@@ -420,4 +438,5 @@ ALL_PINS = [
     pin_backward_finite_differences,
     pin_backward_linear_inputs,
     pin_backward_single_token_closed_form,
+    pin_backward_chunked_equals_recurrence,
 ]

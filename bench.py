@@ -31,6 +31,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -109,8 +110,11 @@ class ClockSampler:
         self.path = None
 
     def __enter__(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{self.gpu}_{os.getpid()}.csv")
+        # raw samples go to KDA_BENCH_OUT (default: the system temp directory); their summary
+        # goes into the JSON line
+        out = os.environ.get("KDA_BENCH_OUT") or tempfile.gettempdir()
+        os.makedirs(out, exist_ok=True)
+        self.path = os.path.join(out, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",

@@ -75,12 +75,38 @@ def peaks():
 KERNEL_SOURCES = ("chunk_bf16.cu", "kda_common.cuh", "tcgen05.cuh")
 
 
+def strip_comments(src: str) -> str:
+    """C/C++/CUDA source without its // and /* */ comments (string and character literals
+    kept as they are), so that a comment edit leaves the hash of the code unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_hash() -> str:
-    """Hash of the chunk kernels' sources: a traffic figure is valid only for these."""
+    """Hash of the chunk kernels' code (comments removed, whitespace collapsed): a traffic
+    figure is valid only for this code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_linear_attention_chunk_b200", "csrc")
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        code = " ".join(strip_comments(open(os.path.join(csrc, f)).read()).split())  # layout-free
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

@@ -1369,11 +1369,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 // ------------------------------------------------------------------ per-chunk gradients
 // Persistent: kBwdSlots CTAs of 512 threads walk the chunks.  q, k, G and the chunk's 64 x 64
 // matrices stay in shared memory; the 64 x D intermediates live in a float32 scratch slot of
-// the workspace per CTA (small enough to stay in L2).  Dense contractions go through
-// cta_gemm (TF32 mma.sync, fp32 accumulation).  The pairwise decay products are 16 x 16
-// tile pairs on the same mma, with the decay factored through a reference token of the row
-// tile, exactly as in the forward: the tile's first token for tiles below the diagonal
-// (both factors <= 1), its middle token on the diagonal (factors <= e^{8 |g_min|}).
+// the workspace per CTA (written and read back by the same CTA; L2 holds part of it).  Dense
+// contractions go through cta_gemm (TF32 mma.sync, fp32 accumulation).  The pairwise decay
+// products are 16 x 16 tile pairs on the same mma, with the decay factored through a
+// reference token of the ROW tile (the forward's prep uses the column tile's middle token;
+// either factoring is exact): the row tile's first token for tiles below the diagonal (both
+// factors <= 1), its middle token on the diagonal (factors <= e^{8 |g_min|}).
 constexpr int kBwdThreads = 512;
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kBwdSlots = 148;  // one CTA per SM of a 148-SM part

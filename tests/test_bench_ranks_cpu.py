@@ -30,3 +30,22 @@ def test_max_over_ranks_and_rank_seeds(tmp_path):
     assert r0[0] == r1[0] == 3.5          # the slowest rank's time, on every rank
     assert r0[1] != r1[1]                 # independent batches per rank
     assert bench.max_over_ranks(2.0, 1, "cpu") == 2.0
+
+
+def test_kernel_hash_ignores_comments_not_code():
+    """The traffic figures are keyed to the kernels' code: comment and layout edits keep the
+    hash, a code edit changes it, and comment markers inside literals are code."""
+    import bench
+
+    base = 'int f(int x) { return x + 1; } // one\n/* two */ const char *s = "a // b /* c */";\n'
+    same = '/* lead */\nint f(int x)   {\n  return x + 1;  // changed comment\n}\nconst char *s = "a // b /* c */";'
+    other = 'int f(int x) { return x + 2; }\nconst char *s = "a // b /* c */";'
+    lit = 'int f(int x) { return x + 1; }\nconst char *s = "a // b";'
+
+    def norm(src):
+        return " ".join(bench.strip_comments(src).split())
+
+    assert norm(base) == norm(same)
+    assert norm(base) != norm(other)
+    assert norm(base) != norm(lit)
+    assert "'/'" in bench.strip_comments("char c = '/'; // x")

@@ -161,6 +161,16 @@ def test_python_binding_has_no_cpu_fallback():
     x = torch.zeros(16, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         kda.kda_gate_fwd(x)
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    beta = torch.zeros(1, 8, 1, dtype=torch.bfloat16)
+    for call in (lambda: kda.kda_chunk_fwd(q, q, q, q, beta),
+                 lambda: kda.kda_chunk_bwd(q, q, q, q, beta, q),
+                 lambda: kda.kda_chunk_bwd_varlen(q[0], q[0], q[0], q[0], beta[0], q[0],
+                                                  torch.tensor([0, 8], dtype=torch.int32)),
+                 lambda: kda.kda_decode_step(q[:, 0], q[:, 0], q[:, 0], q[:, 0], beta[:, 0],
+                                             torch.zeros(1, 1, 64, 64))):
+        with pytest.raises(ValueError):
+            call()
 
 
 def _chunk_logsig(L, B=1, T=64, H=1, dk=128, dv=128, dt=kda.KDA_BF16, q=None, o=None, S0=None, ST=None, ws=None,

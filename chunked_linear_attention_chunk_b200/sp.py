@@ -11,9 +11,19 @@ Over a segment the state map is affine, S_out = M S_in + S_zero.  Every rank
 The exchanged maps are tiny next to the tokens (2 d^2 floats per head per rank), so a
 plain NCCL all-gather over NVLink is the whole collective.
 
-The per-segment steps are an object with three methods, so the same orchestration runs
-with the CUDA library (``LibkdaSegmentOps``) or, in CPU tests, with any other
-implementation of the steps.  This module holds no arithmetic of the method.
+The backward (``sp_chunk_bwd``) runs on the same maps.  The gradient of a segment's
+incoming state is affine in the gradient of its outgoing one, dS_in = M^T dS_out + dZ, where
+dZ is the segment's backward from a zero outgoing gradient.  Every rank
+  1. forms its incoming state as in the forward (maps, all-gather, prefix),
+  2. runs its segment's backward from a zero outgoing gradient and keeps dZ   -- libkda,
+  3. all-gathers dZ                                                            -- exchange,
+  4. forms every segment's outgoing gradient by the suffix
+     dS_out[r] = M[r+1]^T dS_out[r+1] + dZ[r+1], dS_out[R-1] = dS_T           -- libkda,
+  5. runs its segment's backward again with dS_out[rank]: the token gradients -- libkda.
+
+The per-segment steps are an object with a few methods, so the same orchestration runs with
+the CUDA library (``LibkdaSegmentOps``) or, in CPU tests, with any other implementation of
+the steps.  This module holds no arithmetic of the method.
 """
 from __future__ import annotations
 
@@ -45,6 +55,13 @@ class LibkdaSegmentOps:
         ws, (B, T, H, dk, dv) = handle
         return kda.kda_chunk_fwd_scan(ws, B, T, H, dk, dv, S0=S_in.contiguous())
 
+    def backward(self, tokens, S_in, dO, dS_T):
+        """The segment's gradients (dict of kda_chunk_bwd) from S_in, given dO and dS_T."""
+        if self.gate != kda.KDA_GATE_BOUNDED:
+            raise ValueError("the backward supports the bounded gate only")
+        return kda.kda_chunk_bwd(*tokens, dO, self.g_min, S0=S_in.contiguous(),
+                                 dS_T=None if dS_T is None else dS_T.contiguous(), A_log=self.A_log)
+
 
 def sp_chunk_fwd(q, k, v, a, beta, S0=None, group=None, ops=None):
     """This rank's segment of a sequence-parallel chunked forward.
@@ -68,3 +85,36 @@ def sp_chunk_fwd(q, k, v, a, beta, S0=None, group=None, ops=None):
     S_in = ops.combine(torch.stack(Ms), torch.stack(Zs), S0)
     o, _ = ops.forward(handle, S_in[rank])
     return o, S_in[world]
+
+
+def _gather(x, world, group):
+    if world == 1:
+        return [x]
+    xs = [torch.empty_like(x) for _ in range(world)]
+    dist.all_gather(xs, x.contiguous(), group=group)
+    return xs
+
+
+def sp_chunk_bwd(q, k, v, a, beta, dO, S0=None, dS_T=None, group=None, ops=None):
+    """This rank's segment of a sequence-parallel backward (the segments as in
+    ``sp_chunk_fwd``; dO is this segment's dL/do, dS_T the gradient of the whole sequence's
+    final state, the same on every rank, or None).  Returns the ``kda_chunk_bwd`` dict of
+    this segment's token gradients, with dS0 the gradient of the sequence's initial state
+    (identical on every rank) and, given A_log, dA_log summed over all segments."""
+    ops = ops if ops is not None else LibkdaSegmentOps()
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    tokens = (q, k, v, a, beta)
+    _, S_zero, M = ops.maps(*tokens)
+    Ms = _gather(M, world, group)
+    S_in = ops.combine(torch.stack(Ms), torch.stack(_gather(S_zero, world, group)), S0)
+    dZ = ops.backward(tokens, S_in[rank], dO, None)["dS0"]
+    dZs = _gather(dZ, world, group)
+    # suffix over the segments in reverse order: X[j + 1] = M[R-1-j]^T X[j] + dZ[R-1-j], X[0] = dS_T
+    Mt = torch.stack([Ms[world - 1 - j].transpose(-1, -2) for j in range(world)])
+    X = ops.combine(Mt, torch.stack([dZs[world - 1 - j] for j in range(world)]), dS_T)
+    g = ops.backward(tokens, S_in[rank], dO, X[world - 1 - rank])
+    g["dS0"] = X[world]
+    if g.get("dA_log") is not None and world > 1:
+        dist.all_reduce(g["dA_log"], group=group)
+    return g

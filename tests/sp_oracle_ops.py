@@ -40,3 +40,9 @@ class OracleSegmentOps:
     def forward(self, x, S_in):
         o, S_T = oracle.recurrence(*x, self.g_min, S0=S_in.numpy())
         return torch.from_numpy(o), torch.from_numpy(S_T)
+
+    def backward(self, tokens, S_in, dO, dS_T):
+        x = [_np(t) for t in tokens]
+        r = oracle.backward(*x, _np(dO), self.g_min, S0=S_in.numpy(),
+                            dST=None if dS_T is None else dS_T.to(torch.float64).numpy())
+        return {n: torch.from_numpy(v) for n, v in r.items()}

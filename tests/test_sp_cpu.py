@@ -50,3 +50,53 @@ def test_two_ranks_match_one_sequence(tmp_path):
         o = np.load(tmp_path / f"o{r}.npy")
         assert np.allclose(o, o_ref[:, CUT[r]:CUT[r + 1]], rtol=1e-9, atol=1e-12), r
         assert np.allclose(np.load(tmp_path / f"s{r}.npy"), S_ref, rtol=1e-9, atol=1e-12), r
+
+
+def _rank_bwd(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from chunked_linear_attention_chunk_b200.sp import sp_chunk_bwd
+        x = _inputs()
+        dO, dST = _grads()
+        seg = [x[n][:, CUT[rank]:CUT[rank + 1]] for n in NAMES]
+        g = sp_chunk_bwd(*seg, dO[:, CUT[rank]:CUT[rank + 1]], S0=x["S0"].double(), dS_T=dST,
+                         ops=OracleSegmentOps())
+        for n, t in g.items():
+            if t is not None:
+                np.save(os.path.join(out_dir, f"{n}{rank}.npy"), t.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _grads():
+    rng = np.random.default_rng(1301)
+    dO = torch.from_numpy(rng.normal(size=(B, T, H, D)).astype(np.float32))
+    dST = torch.from_numpy(rng.normal(size=(B, H, D, D)))
+    return dO, dST
+
+
+def test_two_ranks_backward_match_one_sequence(tmp_path):
+    """The sequence-parallel backward: each rank's token gradients equal the slice of one
+    backward over the whole sequence, and every rank returns the whole sequence's dS0."""
+    mp.spawn(_rank_bwd, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True)
+    x = _inputs()
+    dO, dST = _grads()
+    ref = oracle.backward(*(x[n].numpy() for n in NAMES), dO.numpy(), -5.0, S0=x["S0"].numpy().astype(np.float64),
+                          dST=dST.numpy())
+    for r in range(2):
+        for n in ("dq", "dk", "dv", "da", "dbeta"):
+            got = np.load(tmp_path / f"{n}{r}.npy")
+            assert np.allclose(got, ref[n][:, CUT[r]:CUT[r + 1]], rtol=1e-8, atol=1e-11), (r, n)
+        assert np.allclose(np.load(tmp_path / f"dS0{r}.npy"), ref["dS0"], rtol=1e-8, atol=1e-11), r
+
+
+def test_one_rank_backward_is_the_plain_backward():
+    from chunked_linear_attention_chunk_b200.sp import sp_chunk_bwd
+    x = _inputs()
+    dO, dST = _grads()
+    g = sp_chunk_bwd(*(x[n] for n in NAMES), dO, S0=x["S0"].double(), dS_T=dST, ops=OracleSegmentOps())
+    ref = oracle.backward(*(x[n].numpy() for n in NAMES), dO.numpy(), -5.0, S0=x["S0"].numpy().astype(np.float64),
+                          dST=dST.numpy())
+    for n in ref:
+        assert np.allclose(g[n].numpy(), ref[n], rtol=1e-9, atol=1e-12), n

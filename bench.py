@@ -289,6 +289,26 @@ def cpu_baseline(x, sample_tokens: int, gpu_out=None):
             "parity": parity}
 
 
+def cpu_baseline_bwd(x, dO, sample_tokens: int):
+    """The fp64 oracle's backward, as it stands, on the first ``sample_tokens`` tokens of every
+    (batch, head) pair of the same inputs and dL/do (dL/dS_T = 0), on the host's cores."""
+    import oracle
+    from chunked_linear_attention_chunk_b200.synth import to_numpy32
+    names = ("q", "k", "v", "a", "beta")
+    arrs = [to_numpy32(x[n][:, :sample_tokens].cpu()) for n in names]
+    dOs = to_numpy32(dO[:, :sample_tokens].cpu())
+    S0 = x["S0"].cpu().numpy().astype("float64")
+    B, Ts, H, _ = arrs[0].shape
+    cores = min(os.cpu_count() or 1, B * H)
+    oracle.backward(*(a[:, :4] for a in arrs), dOs[:, :4], G_MIN, S0=S0)  # build/load outside timing
+    t = time.perf_counter()
+    oracle.backward(*arrs, dOs, G_MIN, S0=S0, nthreads=cores)
+    dt = time.perf_counter() - t
+    return {"value": B * Ts / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {Ts} of {x['q'].shape[1]} tokens, all {B * H} (batch, head) pairs; fp64 "
+                      f"token-by-token backward with 64-token recompute, {dt:.2f} s"}
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -461,7 +481,11 @@ def run_libkda(args):
         bwd_bytes = token_heads * BWD_BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
         bwd_traffic = measured_traffic_per_token_head("bwd_chunk")
         bwd_gbs = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+        bwd_cpu = None
+        if world == 1 and rank == 0 and not args.no_cpu_baseline:
+            bwd_cpu = cpu_baseline_bwd(x, dO, min(T, 8192))
         bwd = {"what": "kda_chunk_bwd: dq, dk, dv, da, dbeta, dS0 (float32) from dL/do",
+               "cpu_baseline": bwd_cpu,
                "ms_per_step": bwd_ms, "value": world * tokens / (bwd_ms * 1e-3), "unit": UNIT,
                "gpu_launches_per_step": 4, "vs_forward_time": bwd_ms / ms, "workspace_bytes": ws_b.numel(),
                "roofline": {"bound": "hbm", "achieved": bwd_gbs, "peak": hbm_peak, "unit": "GB/s",

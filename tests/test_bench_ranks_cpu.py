@@ -49,3 +49,18 @@ def test_kernel_hash_ignores_comments_not_code():
     assert norm(base) != norm(other)
     assert norm(base) != norm(lit)
     assert "'/'" in bench.strip_comments("char c = '/'; // x")
+
+
+def test_backward_cpu_baseline_runs_on_a_small_sample():
+    """bench.py's CPU baseline for the backward leg (the oracle timed on a bounded sample)."""
+    import numpy as np
+    import torch
+
+    import bench
+    from chunked_linear_attention_chunk_b200 import synth
+
+    x = synth.make_inputs(1, 96, 2, 16, 16, "bf16", seed=5, s0_std=0.1)
+    dO = torch.from_numpy(np.random.default_rng(5).normal(size=(1, 96, 2, 16)).astype(np.float32)).to(torch.bfloat16)
+    r = bench.cpu_baseline_bwd(x, dO, 64)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    assert "first 64 of 96 tokens" in r["sample"]

@@ -100,3 +100,37 @@ def test_one_rank_backward_is_the_plain_backward():
                           dST=dST.numpy())
     for n in ref:
         assert np.allclose(g[n].numpy(), ref[n], rtol=1e-9, atol=1e-12), n
+
+
+CUT3 = [0, 50, 50, 90]  # three ranks, the middle one with an empty segment
+
+
+def _rank_bwd3(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from chunked_linear_attention_chunk_b200.sp import sp_chunk_bwd
+        x = _inputs()
+        dO, dST = _grads()
+        seg = [x[n][:, CUT3[rank]:CUT3[rank + 1]] for n in NAMES]
+        g = sp_chunk_bwd(*seg, dO[:, CUT3[rank]:CUT3[rank + 1]], S0=x["S0"].double(), dS_T=dST,
+                         ops=OracleSegmentOps())
+        for n, t in g.items():
+            if t is not None:
+                np.save(os.path.join(out_dir, f"{n}{rank}.npy"), t.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_ranks_backward_with_an_empty_segment(tmp_path):
+    mp.spawn(_rank_bwd3, args=(3, _free_port(), str(tmp_path)), nprocs=3, join=True)
+    x = _inputs()
+    dO, dST = _grads()
+    ref = oracle.backward(*(x[n].numpy() for n in NAMES), dO.numpy(), -5.0, S0=x["S0"].numpy().astype(np.float64),
+                          dST=dST.numpy())
+    for r in range(3):
+        for n in ("dq", "dk", "dv", "da", "dbeta"):
+            got = np.load(tmp_path / f"{n}{r}.npy")
+            assert got.shape[1] == CUT3[r + 1] - CUT3[r]
+            assert np.allclose(got, ref[n][:, CUT3[r]:CUT3[r + 1]], rtol=1e-8, atol=1e-11), (r, n)
+        assert np.allclose(np.load(tmp_path / f"dS0{r}.npy"), ref["dS0"], rtol=1e-8, atol=1e-11), r

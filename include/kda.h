@@ -1,7 +1,8 @@
 /*
  * kda.h -- C ABI of libkda: the chunked forward of KDA incremental linear attention
- * (a gated delta rule with per-channel decay) with the lower-bounded decay gate, and
- * its single-token decode step, for NVIDIA B200 (sm_100a).
+ * (a gated delta rule with per-channel decay) with the lower-bounded decay gate, its
+ * backward (the gradients of every input), and its single-token decode step, for NVIDIA
+ * B200 (sm_100a).
  *
  * The operation.  The pages ("Trillion-Scale MoE Multimodal Models: Practical
  * Techniques for Ultra-Long Context ...", section 3; "Breaking Through
@@ -34,10 +35,11 @@
  *     invocations and may be made from several host threads.
  *   - Errors detected inside a kernel (a bounded wait that ran out) are recorded in a
  *     per-device status word and reported by kda_device_status().
- *   - libkda_debug.so is the same library built with KDA_DEBUG_CHECKS: its prep and scan
- *     CTAs check the record and token ranges they derive from their grid coordinates
- *     against the buffers they were given and, on a mismatch, record KDA_ERR_DEVICE_BOUNDS
- *     and return without touching memory.
+ *   - libkda_debug.so is the same library built with KDA_DEBUG_CHECKS: its prep, scan,
+ *     state-gradient scan and gradient-kernel CTAs check the record and token ranges they
+ *     derive from their grid coordinates against the buffers they were given and, on a
+ *     mismatch, record KDA_ERR_DEVICE_BOUNDS and return without touching memory.
+ *   - Gradients (kda_chunk_bwd*) are float32 in the layouts of their inputs.
  */
 #ifndef KDA_H
 #define KDA_H

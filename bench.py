@@ -343,6 +343,66 @@ def run_reference(args):
     return 0
 
 
+def stage_metrics(tokens, token_heads, states, ms, world, hbm_peak, bf16_peak, peak_kind):
+    """tokens/s, TFLOP/s and the path roofline of one chunked-forward step of ``ms``."""
+    alg = token_heads * BYTES_PER_TOKEN_HEAD + 2 * states * 128 * 128 * 4
+    gbs = alg / (ms * 1e-3) / 1e9
+    tflops = token_heads * FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "value": world * tokens / (ms * 1e-3), "unit": UNIT, "tflops": tflops,
+            "pct_bf16_peak": tflops / bf16_peak,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "peak_kind": peak_kind, "kernels": "prep + scan of every kda_chunk_fwd call of the step",
+                         "algorithmic_bytes": alg}}
+
+
+def time_stage(kda, sw, rank, world, device, hbm_peak, bf16_peak, peak_kind, args):
+    """One step of a context stage on its own seeded inputs: the 8K stage is one kda_chunk_fwd
+    over B4 H16 T8192; the 1M stage is 16 kda_chunk_fwd calls over consecutive 64K segments of
+    one sequence (each segment drawn from its own seed), the state carried in place."""
+    names = ("q", "k", "v", "a", "beta")
+    B, H, D = sw.B, sw.H, sw.dk
+    if sw.segment:
+        nseg = sw.T // sw.segment
+        segs = []
+        for i in range(nseg):
+            if rank == 0:
+                xi = synth.workload_inputs(sw, segment_index=i)
+            else:  # every rank its own sequence
+                xi = synth.make_inputs(B, sw.segment, H, D, D, sw.dtype, rank_seed(sw.seed * 1000 + i, rank),
+                                       sw.s0_std)
+            segs.append({n: xi[n].to(device) for n in names})
+            if i == 0:
+                S0 = xi["S0"].to(device)
+            del xi
+        Tc = sw.segment
+    else:
+        xi = synth.make_inputs(B, sw.T, H, D, D, sw.dtype, rank_seed(sw.seed, rank), sw.s0_std, sw.adversarial)
+        segs = [{n: xi[n].to(device) for n in names}]
+        S0 = xi["S0"].to(device)
+        del xi
+        Tc = sw.T
+    S = torch.empty_like(S0)
+    o = torch.empty((B, Tc, H, D), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace(B, Tc, H, D, D), dtype=torch.uint8, device=device)
+
+    def step():
+        S.copy_(S0)
+        for sd in segs:
+            kda.kda_chunk_fwd(*(sd[n] for n in names), G_MIN, S0=S, o=o, S_T=S, workspace=ws)
+
+    steps = max(2, min(args.steps, 10 if not sw.segment else 3))
+    with ClockSampler(device.index) as clk:
+        ms = time_steps(step, steps, 3, world, device)
+    assert kda.kda_device_status(device) == 0
+    out = {"workload": sw.name, "B": B, "T": sw.T, "H": H, "dk": D, "dv": D, "steps": steps,
+           "calls_per_step": len(segs), "gpu_launches_per_step": 2 * len(segs),
+           "l2": "inputs exceed the 126 MB L2; no flush"}
+    out.update(stage_metrics(B * sw.T, B * sw.T * H, B * H, ms, world, hbm_peak, bf16_peak, peak_kind))
+    out["clocks"] = clk.summary()
+    del segs, ws, o
+    return out
+
+
 def run_libkda(args):
     import chunked_linear_attention_chunk_b200 as kda
 
@@ -407,6 +467,16 @@ def run_libkda(args):
     tflops = token_heads * FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
     prep_traffic = measured_traffic_per_token_head("prep")
     scan_traffic = measured_traffic_per_token_head("scan")
+
+    # ---- the other context stages: 8K (B4 H16 T8192) and 1M (B1 H16 T1048576 as 16 calls of
+    # 64K tokens with the state carried in place), each through kda_chunk_fwd on its own inputs
+    stages = None
+    if args.only != "decode" and not args.no_stages:
+        stages = {}
+        for key, sw in (("8k", synth.STAGE_8K), ("1m", synth.STAGE_1M)):
+            if key == "8k" and w is synth.STAGE_8K:
+                continue
+            stages[key] = time_stage(kda, sw, rank, world, device, hbm_peak, bf16_peak, peak_kind, args)
 
     # ---- the ablation: unbounded log-sigmoid gate, element-wise diagonal tiles (same inputs)
     abl = None
@@ -588,27 +658,29 @@ def run_libkda(args):
 
     # ---- decode step: N=256, H=32, d=128, fp32 state, chained steps
     dw = synth.DECODE
-    dec_steps = 200 if args.only != "decode" else max(args.steps, 1)
+    # (the configured 1000 chained steps, every step with its own seeded token set, all of them
+    # resident on the device: 8.4 GB of tokens; the warm-up steps have sets of their own)
+    dec_steps = dw.steps if args.only != "decode" else max(args.steps, 1)
+    dec_warm = max(args.warmup, 3)
     dec_ms = float("nan")
     dclk = None
     if args.only != "chunk":
         S = synth.decode_state(dw).to(device)
-        n_sets = 50
         toks = []
-        for s in range(n_sets):
-            t = synth.decode_tokens(dw, rank_seed(s, rank))
+        for t in synth.decode_token_sets(dw, range(dec_warm + dec_steps), seed_of=lambda i: rank_seed(i, rank)):
             toks.append({n: t[n].to(device) for n in names})
         od = torch.empty((dw.N, dw.H, dw.dv), dtype=torch.bfloat16, device=device)
         counter = [0]
 
         def dec_step():
-            t = toks[counter[0] % n_sets]
+            t = toks[counter[0]]
             counter[0] += 1
             kda.kda_decode_step(*(t[n] for n in names), S, G_MIN, o=od)
 
         with ClockSampler(local) as dclk:
-            dec_ms = time_steps(dec_step, dec_steps, max(args.warmup, 3), world, device)
+            dec_ms = time_steps(dec_step, dec_steps, dec_warm, world, device)
         assert kda.kda_device_status(device) == 0
+        del toks
     units = dw.N * dw.H
     dec_bytes = units * (2 * dw.dk * dw.dv * 4 + 3 * dw.dk * 2 + dw.dv * 2 + 2 + dw.dv * 2)
     dec_gbs = world * dec_bytes / (dec_ms * 1e-3) / 1e9
@@ -646,6 +718,8 @@ def run_libkda(args):
     }
     if abl is not None:
         line["ablation"] = abl
+    if stages:
+        line["stages"] = stages
     if vl is not None:
         line["varlen"] = vl
     if spl is not None:
@@ -682,6 +756,7 @@ def main(argv=None):
     ap.add_argument("--no-varlen", action="store_true", help="skip timing the packed variable-length batch")
     ap.add_argument("--no-sp", action="store_true", help="skip timing the sequence-parallel leg")
     ap.add_argument("--no-bwd", action="store_true", help="skip timing the backward leg")
+    ap.add_argument("--no-stages", action="store_true", help="skip timing the 8K and 1M context stages")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

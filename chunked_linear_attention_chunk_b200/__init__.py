@@ -449,6 +449,11 @@ def kda_chunk_fwd_noalloc(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None
     _check_cuda(q, k, v, a, beta, S0, o, S_T)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    for t in (k, v, a, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, a, beta must share one dtype")
+    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if S_T is None and return_state:

@@ -32,6 +32,8 @@
 // warp streams the records through a 3-stage mbarrier pipeline with bulk copies, and per
 // chunk one tcgen05 round computes [N S, Q' S] while four consumer warps, one TMEM lane
 // (= one state row or chunk row) per thread, keep the fp32 state block in registers.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 
 #include "kda_common.cuh"
@@ -191,8 +193,8 @@ struct PrepLayout {
     static constexpr uint32_t REm = RBeta + kC * 4;        // e^{G_{m_I}}
     static constexpr uint32_t REl = REm + kTiles * D * 4;  // e^{G_last - G_{m_I}}
     static constexpr uint32_t RDd = REl + kTiles * D * 4;  // bf16 [6][D]  e^{G_{m_I} - G_{m_J}}
-    static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarriers: round 1, then units U1..U4
-    static constexpr uint32_t RTmem = RBar + 5 * 8;
+    static constexpr uint32_t RBar = RDd + 6 * D * 2;      // mbarriers: round 1, U1..U4, a, q|k|v
+    static constexpr uint32_t RTmem = RBar + 7 * 8;
     static constexpr uint32_t Bytes = RTmem + 8;
     static_assert(RG % 1024 == 0 && RP % 1024 == 0, "operand alignment");
     // two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
@@ -307,12 +309,24 @@ __device__ __forceinline__ void diag_pair(int p, int &r, int &j)
     j = p - r * (r + 1) / 2;
 }
 
+// The token tensors as TMA tensor maps over this GPU's memory: dims (innermost first)
+// {D, H, T, B} for a regular batch, {D, H, T} for a packed one; boxes of 64 channels x one
+// head x 64 tokens land with the 128-byte swizzle, which is the token-major operand layout
+// (one 128-byte row per token, a 64-channel block per 8 KB).
+struct TokenMaps {
+    CUtensorMap q, k, v, a;
+};
+
+// Warps of the fused gate / cumulative-sum / decay-factor pass: one per (16-token tile,
+// 64-channel half), a lane per channel pair.
+template <int D>
+constexpr int kFusedWarps = kTiles * (D / 64);
+
 template <int D, bool kLogSig>
 __global__ void __launch_bounds__(kPrepThreads, 2)
-    prep_kernel(SeqMap map, int H, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
-                const __nv_bfloat16 *__restrict__ beta, float g_min, const float *__restrict__ A_log,
-                unsigned char *__restrict__ ws, unsigned int *status)
+    prep_kernel(const __grid_constant__ TokenMaps tm, SeqMap map, int H, const __nv_bfloat16 *__restrict__ beta,
+                const float *__restrict__ gtab, bool per_head_tab, unsigned char *__restrict__ ws,
+                unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char prep_smem[];
     using L = PrepLayout<D>;
@@ -327,15 +341,21 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     unsigned char *sm = prep_smem;
     constexpr int LDA = kC + 1;
     constexpr int CPR = D / 8;  // 16-byte chunks per token row
-    float *sG = reinterpret_cast<float *>(sm + L::RG);   // [64][D]
+    constexpr int NFW = kFusedWarps<D>;
+    float *sG = reinterpret_cast<float *>(sm + L::RG);   // [64][D] (ablation only)
     float *sA = reinterpret_cast<float *>(sm + L::RA);   // [64][65]
     float *sT = reinterpret_cast<float *>(sm + L::RT);   // [64][65]
     float *sBeta = reinterpret_cast<float *>(sm + L::RBeta);
     __nv_bfloat16 *sEm = reinterpret_cast<__nv_bfloat16 *>(sm + L::REm);  // hi [4][D] | lo [4][D]
     __nv_bfloat16 *sEl = reinterpret_cast<__nv_bfloat16 *>(sm + L::REl);
     __nv_bfloat16 *sDd = reinterpret_cast<__nv_bfloat16 *>(sm + L::RDd);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::RBar);
+    // per-(tile, channel) totals and local mid-tile values of the cumulative sum, in P's slot
+    // (P is written from step 4 on)
+    float *sTot = reinterpret_cast<float *>(sm + L::RP);
+    float *sMid = sTot + kTiles * D;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::RBar);  // round 1, U1..U4, a, q|k|v
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::RTmem);
+    static_assert(2 * kTiles * D * 4 <= kC * kC * 2, "cumulative-sum tables fit P's slot");
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = lane >> 2, tq = lane & 3;
@@ -352,215 +372,218 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     const int n = loc.n, h = loc.h;
     unsigned char *rec = ws + loc.rec * R::Bytes;
-    const int64_t rowstride = (int64_t)H * D;  // elements between consecutive tokens
-    const int64_t base = (loc.tok0 * H + h) * D;
+    const float *tab = gtab + (per_head_tab ? (size_t)h * kGateTableEntries : 0);
 
-    // -- 0. async loads into the swizzled token-major operands (zero past the sequence):
-    //       a first (the gate needs it), then q, k, v, which land during steps 1-2
-    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
-        const int r = i / CPR, c8 = (i % CPR) * 8;
-        const bool ok = r < n;
-        const int64_t off = base + (ok ? (int64_t)r * rowstride : 0) + c8;
-        cp_async_16_zfill(sm + L::RX + tok_off(r, c8), a + off, ok);
-    }
-    cp_async_commit();
-    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
-        const int r = i / CPR, c8 = (i % CPR) * 8;
-        const bool ok = r < n;
-        const int64_t off = base + (ok ? (int64_t)r * rowstride : 0) + c8;
-        const uint32_t d = tok_off(r, c8);
-        cp_async_16_zfill(sm + L::RQ + d, q + off, ok);
-        cp_async_16_zfill(sm + L::RK + d, k + off, ok);
-        cp_async_16_zfill(sm + L::RV + d, v + off, ok);
-    }
-    cp_async_commit();
-    if (tid < kC)
-        sBeta[tid] = tid < n ? __bfloat162float(beta[(loc.tok0 + tid) * H + h]) : 0.0f;
+    // -- 0. one thread issues the tensor copies of the chunk's a, then q, k, v (64 tokens x 64
+    //       channels per box; a regular batch reads zeros past its sequence, a packed one
+    //       reads the next sequence's tokens there, which step 1 masks); the other warps load
+    //       beta and allocate tensor memory meanwhile
+    uint64_t *bar_a = bar + 5, *bar_qkv = bar + 6;
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i)
+        for (int i = 0; i < 7; ++i)
             mbar_init(bar + i, 1);
         fence_mbar_init_cluster();
+        constexpr uint32_t kBox = (uint32_t)kC * 64 * 2;
+        const int b = map.cu ? 0 : (int)(blockIdx.y / H), t0 = map.cu ? 0 : (int)blockIdx.x * kC;
+        auto load = [&](const CUtensorMap *m, uint32_t dst, uint64_t *bb) {
+            for (int cb = 0; cb < D / 64; ++cb) {
+                if (map.cu)
+                    tma_load_3d(sm + dst + cb * kBox, m, cb * 64, h, (int)loc.tok0, bb);
+                else
+                    tma_load_4d(sm + dst + cb * kBox, m, cb * 64, h, t0, b, bb);
+            }
+        };
+        mbar_arrive_expect_tx(bar_a, (D / 64) * kBox);
+        load(&tm.a, L::RX, bar_a);
+        mbar_arrive_expect_tx(bar_qkv, 3 * (D / 64) * kBox);
+        load(&tm.q, L::RQ, bar_qkv);
+        load(&tm.k, L::RK, bar_qkv);
+        load(&tm.v, L::RV, bar_qkv);
     }
     if (warp == 0)
         tc::tmem_alloc(tslot, 2 * D);
-    cp_async_wait<1>();  // a is in; q, k, v may still be in flight
+    if (tid >= kPrepThreads - kC) {
+        const int r = tid - (kPrepThreads - kC);
+        sBeta[r] = r < n ? __bfloat162float(beta[(loc.tok0 + r) * H + h]) : 0.0f;
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tslot;
 
-    // -- 1. gate g = g_min sigmoid(a) (0 past the sequence) fused with its inclusive
-    //       cumulative sum over tokens: kPrepThreads / D threads per channel, each summing
-    //       its run of tokens; later runs then add the totals of the earlier ones
+    // -- 1. fused pass, warp (tile I, channel half), lane = channel pair c0, c0 + 1:
+    //       g from the table (0 past the sequence), its inclusive cumulative sum G over the
+    //       tile in registers, the tiles' totals exchanged through shared memory; then the
+    //       per-(tile, channel) scalars and Gamma_C = e^{G_last}.
+    //       Bounded gate: one reference per tile, its middle token m_I (row and column role
+    //       alike).  Unbounded gate: the row role of tile I takes G just before the tile (b_I;
+    //       0 for I = 0), the column role of tile J the tile's last token (e_J), so every
+    //       off-diagonal factor is at most 1 whatever g is.
+    float dA[kDiagSlots] = {}, dP[kDiagSlots] = {};
     {
-        constexpr int TPC = kCoreThreads / D;
-        constexpr int LEN = kC / TPC;
-        const bool core = tid < kCoreThreads;
-        const int c = tid % D, part = tid / D;
-        const float scale = A_log ? __expf(A_log[h]) : 1.0f;  // e^A on the gate's argument
-        float gv[LEN];
-        float run = 0.0f;
-        if (core) {
+        const bool fw = warp < NFW;
+        const int I = warp % kTiles, c0 = (warp / kTiles) * 64 + 2 * lane;
+        float G0[kTile], G1[kTile];  // G of tokens 16 I + s, channels c0 and c0 + 1
+        float rr0 = 0.f, rr1 = 0.f, cr0 = 0.f, cr1 = 0.f, gl0 = 0.f, gl1 = 0.f;
+        if (fw) {
+            mbar_wait_bounded(bar_a, 0, status);
+            uint32_t ab[kTile];
 #pragma unroll
-            for (int r = 0; r < LEN; ++r) {
-                const int t = part * LEN + r;
-                const float av = scale * __bfloat162float(
-                                             *reinterpret_cast<const __nv_bfloat16 *>(sm + L::RX + tc::mnmaj_sw128(t, c, kC)));
-                float g;
+            for (int s2 = 0; s2 < kTile; ++s2)
+                ab[s2] = *reinterpret_cast<const uint32_t *>(sm + L::RX + tok_off(I * kTile + s2, c0));
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < kTile; ++s2) {
+                const bool ok = I * kTile + s2 < n;
+                const float g0 = __ldg(tab + (ab[s2] & 0xffffu)), g1 = __ldg(tab + (ab[s2] >> 16));
+                x0 += ok ? g0 : 0.f;
+                x1 += ok ? g1 : 0.f;
+                G0[s2] = x0;
+                G1[s2] = x1;
+            }
+            *reinterpret_cast<float2 *>(&sTot[I * D + c0]) = make_float2(x0, x1);
+            *reinterpret_cast<float2 *>(&sMid[I * D + c0]) = make_float2(G0[kRef], G1[kRef]);
+            asm volatile("bar.sync 1, %0;" ::"n"(NFW * 32) : "memory");
+            // offsets of every tile (sums in tile order), this tile's references
+            float off0[kTiles], off1[kTiles];
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int J = 0; J < kTiles; ++J) {
+                off0[J] = a0;
+                off1[J] = a1;
+                const float2 t = *reinterpret_cast<const float2 *>(&sTot[J * D + c0]);
+                a0 += t.x;
+                a1 += t.y;
+            }
+            gl0 = a0, gl1 = a1;
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int J = 0; J < kTiles; ++J)
+                if (J == I)
+                    o0 = off0[J], o1 = off1[J];
+#pragma unroll
+            for (int s2 = 0; s2 < kTile; ++s2) {
+                G0[s2] += o0;
+                G1[s2] += o1;
+            }
+            // column reference of tile J (a G value; J is a compile-time index wherever used)
+            auto col_ref = [&](int J, int ch) -> float {
+                const float o = ch ? off1[J] : off0[J];
                 if constexpr (kLogSig)
-                    g = gate_logsigmoid_fast(av);
+                    return o + sTot[J * D + c0 + ch];
                 else
-                    g = gate_bounded_fast(av, g_min);
-                run += t < n ? g : 0.0f;
-                gv[r] = run;
+                    return o + sMid[J * D + c0 + ch];
+            };
+            // this tile's row and column references
+            if constexpr (kLogSig) {
+                rr0 = o0, rr1 = o1;
+                cr0 = o0 + sTot[I * D + c0], cr1 = o1 + sTot[I * D + c0 + 1];
+            } else {
+                rr0 = cr0 = G0[kRef];
+                rr1 = cr1 = G1[kRef];
+            }
+            {  // e^{row ref} and e^{G_last - col ref} as bf16 hi / lo pairs
+                const float em0 = __expf(rr0), em1 = __expf(rr1);
+                const float el0 = __expf(gl0 - cr0), el1 = __expf(gl1 - cr1);
+                const uint32_t emh = pack_bf16x2(em0, em1), elh = pack_bf16x2(el0, el1);
+                const float2 emf = unpack_bf16x2(emh), elf = unpack_bf16x2(elh);
+                *reinterpret_cast<uint32_t *>(&sEm[I * D + c0]) = emh;
+                *reinterpret_cast<uint32_t *>(&sEm[(kTiles + I) * D + c0]) = pack_bf16x2(em0 - emf.x, em1 - emf.y);
+                *reinterpret_cast<uint32_t *>(&sEl[I * D + c0]) = elh;
+                *reinterpret_cast<uint32_t *>(&sEl[(kTiles + I) * D + c0]) = pack_bf16x2(el0 - elf.x, el1 - elf.y);
+            }
+#pragma unroll
+            for (int J = 0; J < kTiles - 1; ++J)  // e^{row ref I - col ref J}, J < I
+                if (J < I)
+                    *reinterpret_cast<uint32_t *>(&sDd[(I * (I - 1) / 2 + J) * D + c0]) =
+                        pack_bf16x2(__expf(rr0 - col_ref(J, 0)), __expf(rr1 - col_ref(J, 1)));
+            if (I == kTiles - 1)
+                *reinterpret_cast<float2 *>(rec + R::Gam + c0 * 4) = make_float2(__expf(gl0), __expf(gl1));
+            if constexpr (kLogSig) {  // the element-wise diagonal tiles read G
+#pragma unroll
+                for (int s2 = 0; s2 < kTile; ++s2)
+                    *reinterpret_cast<float2 *>(&sG[(I * kTile + s2) * D + c0]) = make_float2(G0[s2], G1[s2]);
             }
         }
-        if (core)
+
+        if constexpr (kLogSig) {
+            // -- 1a. unbounded gate only: the diagonal tiles element by element from the raw
+            //        q, k and G (their decay cannot be factored), held in registers until step 4
+            __syncthreads();
+            mbar_wait_bounded(bar_qkv, 0, status);
+            const int It = tid >> 6;
 #pragma unroll
-            for (int r = 0; r < LEN; ++r)
-                sG[(part * LEN + r) * D + c] = gv[r];
-        __syncthreads();
-        float off = 0.0f;
-        for (int p = 0; p < part && core; ++p)
-            off += sG[(p * LEN + LEN - 1) * D + c];
-        __syncthreads();
-        if (core && part > 0)
+            for (int s = 0; s < kDiagSlots; ++s) {
+                const int p = (tid & 63) + 64 * s;
+                if (tid < kCoreThreads && p < kDiagPairs) {
+                    int r, j;
+                    diag_pair(p, r, j);
+                    const int tr = It * kTile + r, tj = It * kTile + j;
+                    float sa = 0.0f, sp = 0.0f;
+                    if (tr < n) {
+                        for (int c8 = 0; c8 < D; c8 += 8) {
+                            const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tr, c8));
+                            const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(tr, c8));
+                            const uint4 ju = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tj, c8));
+                            const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w},
+                                           jw[4] = {ju.x, ju.y, ju.z, ju.w};
 #pragma unroll
-            for (int r = 0; r < LEN; ++r)
-                sG[(part * LEN + r) * D + c] = gv[r] + off;
+                            for (int w = 0; w < 4; ++w) {
+                                const float2 kr = unpack_bf16x2(kw[w]), qr = unpack_bf16x2(qw[w]),
+                                             kj = unpack_bf16x2(jw[w]);
+                                const float2 gr = *reinterpret_cast<const float2 *>(&sG[tr * D + c8 + 2 * w]);
+                                const float2 gj = *reinterpret_cast<const float2 *>(&sG[tj * D + c8 + 2 * w]);
+                                const float e0 = __expf(gr.x - gj.x), e1 = __expf(gr.y - gj.y);
+                                sa = fmaf(kr.x * kj.x, e0, sa);
+                                sa = fmaf(kr.y * kj.y, e1, sa);
+                                sp = fmaf(qr.x * kj.x, e0, sp);
+                                sp = fmaf(qr.y * kj.y, e1, sp);
+                            }
+                        }
+                    }
+                    dA[s] = j < r ? sBeta[tr] * sa : 0.0f;
+                    dP[s] = sp;
+                }
+            }
+            __syncthreads();  // raw q, k are overwritten next
+        }
+
+        // -- 2. decay factors, in place: Kr = k e^{G - row ref}, Qr = q e^{G - row ref}
+        //       (over k, q) and Ec = k e^{col ref - G} (over a); rows past the sequence are
+        //       zero in all three and in v (a packed batch loaded the next sequence there)
+        if (fw) {
+            mbar_wait_bounded(bar_qkv, 0, status);
+#pragma unroll
+            for (int s2 = 0; s2 < kTile; ++s2) {
+                const int r = I * kTile + s2;
+                const uint32_t d = tok_off(r, c0);
+                const float x0 = G0[s2] - rr0, x1 = G1[s2] - rr1;
+                const float y0 = cr0 - G0[s2], y1 = cr1 - G1[s2];
+                uint32_t kr = 0u, qr = 0u, ec = 0u;
+                if (r < n) {
+                    const float2 kk = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + L::RK + d));
+                    const float2 qq = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + L::RQ + d));
+                    const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(y0), i1 = __expf(y1);
+                    kr = pack_bf16x2(kk.x * e0, kk.y * e1);
+                    qr = pack_bf16x2(qq.x * e0, qq.y * e1);
+                    ec = pack_bf16x2(kk.x * i0, kk.y * i1);
+                } else {
+                    *reinterpret_cast<uint32_t *>(sm + L::RV + d) = 0u;
+                }
+                *reinterpret_cast<uint32_t *>(sm + L::RK + d) = kr;
+                *reinterpret_cast<uint32_t *>(sm + L::RQ + d) = qr;
+                *reinterpret_cast<uint32_t *>(sm + L::RX + d) = ec;
+            }
+        }
     }
-    cp_async_wait<0>();  // q, k, v are in (read from step 3a on)
     __syncthreads();
 
-    // -- 2. per-(tile, channel) decay scalars (bf16) and Gamma_C (record)
-    //       Bounded gate: one reference per tile, its middle token m_I (row and column
-    //       role alike).  Unbounded gate: the row role of tile I takes G just before the
-    //       tile (b_I; 0 for I = 0), the column role of tile J the tile's last token
-    //       (e_J), so every off-diagonal factor is at most 1 whatever g is.
-    auto row_ref = [&](int I, int c) -> float {
-        if constexpr (kLogSig)
-            return I > 0 ? sG[(I * kTile - 1) * D + c] : 0.0f;
-        else
-            return sG[(I * kTile + kRef) * D + c];
-    };
-    auto col_ref = [&](int J, int c) -> float {
-        if constexpr (kLogSig)
-            return sG[(J * kTile + kTile - 1) * D + c];
-        else
-            return sG[(J * kTile + kRef) * D + c];
-    };
-    for (int i = tid; i < kTiles * D; i += kPrepThreads) {
-        const int I = i / D, c = i % D;
-        const float em = __expf(row_ref(I, c)), el = __expf(sG[(kC - 1) * D + c] - col_ref(I, c));
-        const __nv_bfloat16 emh = __float2bfloat16(em), elh = __float2bfloat16(el);
-        sEm[i] = emh;
-        sEm[kTiles * D + i] = __float2bfloat16(em - __bfloat162float(emh));
-        sEl[i] = elh;
-        sEl[kTiles * D + i] = __float2bfloat16(el - __bfloat162float(elh));
-    }
-    for (int i = tid; i < 6 * D; i += kPrepThreads) {
-        const int p = i / D, c = i % D;
-        const int I = p < 1 ? 1 : (p < 3 ? 2 : 3);
-        const int J = p - I * (I - 1) / 2;
-        sDd[i] = __float2bfloat16(__expf(row_ref(I, c) - col_ref(J, c)));
-    }
-    {
-        float *gGam = reinterpret_cast<float *>(rec + R::Gam);
-        for (int c = tid; c < D; c += kPrepThreads)
-            gGam[c] = __expf(sG[(kC - 1) * D + c]);
-    }
-
-    // -- 3a. unbounded gate only: the diagonal tiles element by element from the raw q, k
-    //        and G (their decay cannot be factored), held in registers until step 4
-    float dA[kDiagSlots] = {}, dP[kDiagSlots] = {};
-    if constexpr (kLogSig) {
-        const int I = tid >> 6;
-#pragma unroll
-        for (int s = 0; s < kDiagSlots; ++s) {
-            const int p = (tid & 63) + 64 * s;
-            if (tid < kCoreThreads && p < kDiagPairs) {
-                int r, j;
-                diag_pair(p, r, j);
-                const int tr = I * kTile + r, tj = I * kTile + j;
-                float sa = 0.0f, sp = 0.0f;
-                for (int c8 = 0; c8 < D; c8 += 8) {
-                    const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tr, c8));
-                    const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(tr, c8));
-                    const uint4 ju = *reinterpret_cast<const uint4 *>(sm + L::RK + tok_off(tj, c8));
-                    const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w},
-                                   jw[4] = {ju.x, ju.y, ju.z, ju.w};
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float2 kr = unpack_bf16x2(kw[w]), qr = unpack_bf16x2(qw[w]), kj = unpack_bf16x2(jw[w]);
-                        const float2 gr = *reinterpret_cast<const float2 *>(&sG[tr * D + c8 + 2 * w]);
-                        const float2 gj = *reinterpret_cast<const float2 *>(&sG[tj * D + c8 + 2 * w]);
-                        const float e0 = __expf(gr.x - gj.x), e1 = __expf(gr.y - gj.y);
-                        sa = fmaf(kr.x * kj.x, e0, sa);
-                        sa = fmaf(kr.y * kj.y, e1, sa);
-                        sp = fmaf(qr.x * kj.x, e0, sp);
-                        sp = fmaf(qr.y * kj.y, e1, sp);
-                    }
-                }
-                dA[s] = j < r ? sBeta[tr] * sa : 0.0f;
-                dP[s] = sp;
-            }
-        }
-        __syncthreads();  // raw q, k are overwritten next
-    }
-
-    // -- 3. decay factors E = e^{G - G_ref} (row role) and e^{G_ref' - G} (column role):
-    //       Kr = k E and Qr = q E in place of k and q, Ec in place of a
-    for (int i = tid; i < kC * CPR; i += kPrepThreads) {
-        const int r = i / CPR, c8 = (i % CPR) * 8;
-        const int m = kLogSig ? (r / kTile) * kTile - 1 : (r / kTile) * kTile + kRef;  // row reference token
-        const int mc = kLogSig ? (r / kTile) * kTile + kTile - 1 : m;                   // column reference token
-        const uint32_t d = tok_off(r, c8);
-        const uint4 ku = *reinterpret_cast<const uint4 *>(sm + L::RK + d);
-        const uint4 qu = *reinterpret_cast<const uint4 *>(sm + L::RQ + d);
-        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w};
-        const uint32_t qw[4] = {qu.x, qu.y, qu.z, qu.w};
-        const float4 G0 = *reinterpret_cast<const float4 *>(&sG[r * D + c8]);
-        const float4 G1 = *reinterpret_cast<const float4 *>(&sG[r * D + c8 + 4]);
-        const float4 zero4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        const float4 M0 = m >= 0 ? *reinterpret_cast<const float4 *>(&sG[m * D + c8]) : zero4;
-        const float4 M1 = m >= 0 ? *reinterpret_cast<const float4 *>(&sG[m * D + c8 + 4]) : zero4;
-        const float x[8] = {G0.x - M0.x, G0.y - M0.y, G0.z - M0.z, G0.w - M0.w,
-                            G1.x - M1.x, G1.y - M1.y, G1.z - M1.z, G1.w - M1.w};
-        float y[8];  // column exponent G_{mc} - G
-        if constexpr (kLogSig) {
-            const float4 C0 = *reinterpret_cast<const float4 *>(&sG[mc * D + c8]);
-            const float4 C1 = *reinterpret_cast<const float4 *>(&sG[mc * D + c8 + 4]);
-            const float yy[8] = {C0.x - G0.x, C0.y - G0.y, C0.z - G0.z, C0.w - G0.w,
-                                 C1.x - G1.x, C1.y - G1.y, C1.z - G1.z, C1.w - G1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                y[e] = yy[e];
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                y[e] = -x[e];
-        }
-        uint32_t kr[4], qr[4], ec[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float2 kk = unpack_bf16x2(kw[p]), qq = unpack_bf16x2(qw[p]);
-            const float e0 = __expf(x[2 * p]), e1 = __expf(x[2 * p + 1]);
-            const float i0 = __expf(y[2 * p]), i1 = __expf(y[2 * p + 1]);
-            kr[p] = pack_bf16x2(kk.x * e0, kk.y * e1);
-            qr[p] = pack_bf16x2(qq.x * e0, qq.y * e1);
-            ec[p] = pack_bf16x2(kk.x * i0, kk.y * i1);
-        }
-        *reinterpret_cast<uint4 *>(sm + L::RK + d) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
-        *reinterpret_cast<uint4 *>(sm + L::RQ + d) = make_uint4(qr[0], qr[1], qr[2], qr[3]);
-        *reinterpret_cast<uint4 *>(sm + L::RX + d) = make_uint4(ec[0], ec[1], ec[2], ec[3]);
-    }
-    // upper blocks of P are zero
+    // upper blocks of P are zero (its slot held the cumulative-sum tables until here)
     for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
         const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
         if (j / kTile > r / kTile)
             *reinterpret_cast<uint32_t *>(sm + L::RP + tc::kmaj_sw128(r, j, kC)) = 0u;
     }
-    __syncthreads();
 
     // -- 4. dense 16-token tile products A and P, one warp per (row tile I, column tile
     //       J <= I): row operands Kr, Qr of tile I (scaled by e^{G_{m_I} - G_{m_J}} when
@@ -930,10 +953,13 @@ struct ScanSmem {
     static constexpr uint32_t kStageBytes = Rec<D>::Shared + Rec<D>::Blk;  // shared part + own value block
     static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
     alignas(1024) unsigned char stage[kStages][kStageStride];
-    alignas(1024) unsigned char sbuf[D * kBV * 2];  // S block, bf16, MN-major 64-byte swizzle (row = key channel)
-    uint64_t full[kStages];                         // stage filled (arrive + bytes)
-    uint64_t empty[kStages];                        // stage released by the consumers
-    uint64_t mma_bar;                               // tcgen05 MMA batch completed
+    // the entering state of chunk c as the bf16 MMA operand, in sbuf[c % 2] (MN-major 64-byte
+    // swizzle, row = key channel): Q' S of chunk c may still read it while S of c + 1 is written
+    alignas(1024) unsigned char sbuf[2][D * kBV * 2];
+    uint64_t full[kStages];   // stage filled (arrive + bytes)
+    uint64_t empty[kStages];  // stage free: two arrivals, the consumers' and the MMAs' that read it
+    uint64_t mma_n;           // N S of the chunk completed (and all before it)
+    uint64_t mma_q[2];        // Q' S of chunk c completed, in mma_q[c % 2]
     uint32_t tmem_slot;
 };
 
@@ -969,7 +995,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     using SM = ScanSmem<D>;
     using R = Rec<D>;
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
-    constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N S; [kBV, 2 kBV): Q' S
+    // TMEM columns: [0, kBV) N S; [kBV (1 + c % 2), + kBV) Q' S of chunk c
+    constexpr uint32_t kTmemCols = 4 * kBV;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // Column blocks past D / kBV (affine mode only) carry the transfer map instead of the
     // state: they start from the identity, add no Bm and write M_out.
@@ -994,9 +1021,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.empty[s], 2);
         }
-        mbar_init(&sm.mma_bar, 1);
+        mbar_init(&sm.mma_n, 1);
+        mbar_init(&sm.mma_q[0], 1);
+        mbar_init(&sm.mma_q[1], 1);
         fence_mbar_init_cluster();
     }
     if (warp == 0)
@@ -1004,7 +1033,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = sm.tmem_slot;  // columns [0, kBV): N S; [kBV, 2 kBV): Q' S
+    const uint32_t tmem = sm.tmem_slot;
 
     if (warp == kScanWarps) {
         // ---------------- producer: one lane issues the bulk copies
@@ -1043,7 +1072,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 S[j + 2] = v.z;
                 S[j + 3] = v.w;
             }
-            store_state(sm.sbuf, row, S);
+            store_state(sm.sbuf[0], row, S);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -1051,8 +1080,36 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc::fence_after_sync();
 
         const uint32_t id_k = tc::idesc_bf16(128, kBV, false, true);  // A K-major, B MN-major
-        const uint32_t sbuf_a = smem_u32(sm.sbuf);
-        uint32_t mma_phase = 0;
+        const bool orow = o && warp < 2;  // chunk rows 0..63 = TMEM lanes 0..63: warps 0 and 1
+        uint4 opre[kBV / 8];              // this row's O' of the chunk whose output is pending
+        // O = Q' S + O' of chunk c, run one chunk late while the tensor core works on the next
+        // chunk's N S (Q' S of c in TMEM, O' copied to registers before the stage was freed)
+        auto out_epilogue = [&](int c) {
+            if (!orow)
+                return;
+            mbar_wait_bounded(&sm.mma_q[c & 1], (c >> 1) & 1, status);
+            tc::fence_after_sync();
+            uint32_t y[kBV];
+            tc::ld_32x32b_x32(lane_addr + kBV * (1 + (c & 1)), y);
+            tc::wait_ld();
+            const int t = c * kC + row;
+            if (t < seq.len) {
+                uint4 *op = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8) {
+                    const uint32_t ow[4] = {opre[j / 8].x, opre[j / 8].y, opre[j / 8].z, opre[j / 8].w};
+                    uint32_t r4[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 of = unpack_bf16x2(ow[p]);
+                        r4[p] = pack_bf16x2(of.x + __uint_as_float(y[j + 2 * p]), of.y + __uint_as_float(y[j + 2 * p + 1]));
+                    }
+                    op[j / 8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+                }
+            }
+        };
+
+        uint32_t n_phase = 0;
         for (int c = 0; c < NT; ++c) {
             const int s = c % kStages;
             if constexpr (kSave) {
@@ -1067,20 +1124,30 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             const unsigned char *st = sm.stage[s];
             const uint32_t st_a = smem_u32(st);
 
-            // [N S | Q' S] in one round (rows past N (D = 64) and past Q' are don't-cares)
+            // N S first (the state chain waits for it), then Q' S (only the output needs it),
+            // each completing on its own barrier; the MMAs' reads of the stage end with Q' S,
+            // whose completion is also one of the two arrivals that free the stage (rows past
+            // N (D = 64) and past Q' are don't-cares)
             if (tid == 0) {
                 tc::fence_after_sync();
+                const uint32_t sb = smem_u32(sm.sbuf[c & 1]);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
+                    const uint64_t bd = tc::smem_desc(sb + ks * 1024, 0, 512, tc::kSw64);
                     const uint64_t an =
                         tc::smem_desc(st_a + R::Nm + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
+                    tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(&sm.mma_n);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t bd = tc::smem_desc(sb + ks * 1024, 0, 512, tc::kSw64);
                     const uint64_t aq =
                         tc::smem_desc(st_a + R::Qp + (ks >> 2) * (kC * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
-                    tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + kBV * (1 + (c & 1)), aq, bd, id_k, ks > 0 ? 1u : 0u);
                 }
-                tc::commit(&sm.mma_bar);
+                tc::commit(&sm.mma_q[c & 1]);
+                tc::commit(&sm.empty[s]);
             }
             // Diag(Gamma) S + Bm while the tensor core runs (stage data is in since `full`)
             if (srow) {
@@ -1098,12 +1165,20 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     }
                 }
             }
-            mbar_wait_bounded(&sm.mma_bar, mma_phase, status);
-            mma_phase ^= 1;
+            // the previous chunk's output while N S runs
+            if (c > 0)
+                out_epilogue(c - 1);
+            // this chunk's O' rows, so the stage can be freed at the end of the iteration
+            if (orow) {
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8)
+                    opre[j / 8] = *reinterpret_cast<const uint4 *>(st + R::Shared + R::BmBlk + tc::mnmaj_sw64(row, j));
+            }
+            mbar_wait_bounded(&sm.mma_n, n_phase, status);
+            n_phase ^= 1;
             tc::fence_after_sync();
-
-            const unsigned char *blkp = st + R::Shared;
-            // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk
+            // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk.  sbuf[(c + 1) % 2]
+            // was last read by Q' S of chunk c - 1, which completed before N S of chunk c.
             if (srow) {
                 uint32_t d[kBV];
                 tc::ld_32x32b_x32(lane_addr, d);
@@ -1111,37 +1186,21 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kBV; ++j)
                     S[j] -= __uint_as_float(d[j]);
-                store_state(sm.sbuf, row, S);
+                store_state(sm.sbuf[(c + 1) & 1], row, S);
                 tc::fence_smem_to_async();
-            }
-            // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
-            if (o && warp < 2) {
-                uint32_t y[kBV];
-                tc::ld_32x32b_x32(lane_addr + kBV, y);
-                tc::wait_ld();
-                const int t = c * kC + row;
-                if (t < seq.len) {
-                    uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
-#pragma unroll
-                    for (int j = 0; j < kBV; j += 8) {
-                        const uint4 ou = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
-                        const uint32_t ow[4] = {ou.x, ou.y, ou.z, ou.w};
-                        uint32_t r4[4];
-#pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            const float2 of = unpack_bf16x2(ow[p]);
-                            r4[p] = pack_bf16x2(of.x + __uint_as_float(y[j + 2 * p]),
-                                                of.y + __uint_as_float(y[j + 2 * p + 1]));
-                        }
-                        orow[j / 8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
-                    }
-                }
             }
             tc::fence_before_sync();
             consumer_sync();
             tc::fence_after_sync();
             if (tid == 0)
-                mbar_arrive_local(&sm.empty[s]);
+                mbar_arrive_local(&sm.empty[s]);  // the consumers' arrival: Bm and O' are read
+        }
+        if (NT > 0) {
+            out_epilogue(NT - 1);
+            // every MMA has completed before the tensor memory is released (commits track all
+            // earlier MMAs of the issuing thread)
+            if (tid == 0)
+                mbar_wait_bounded(&sm.mma_q[(NT - 1) & 1], ((NT - 1) >> 1) & 1, status);
         }
 
         float *Sout = xfer ? M_out : S_T;
@@ -1557,7 +1616,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_chunk_kernel(SeqMap map, int H, int nunits, const __nv_bfloat16 *__restrict__ qg,
                      const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ vg,
                      const __nv_bfloat16 *__restrict__ ag, const __nv_bfloat16 *__restrict__ betag, float g_min,
-                     const float *__restrict__ A_log, const __nv_bfloat16 *__restrict__ dOg,
+                     const float *__restrict__ A_log, const float *__restrict__ gtab,
+                     const __nv_bfloat16 *__restrict__ dOg,
                      const float *__restrict__ Hs, const float *__restrict__ dHs, float *scratch,
                      float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ da,
                      float *__restrict__ dbeta, float *__restrict__ dA_part, unsigned int *status)
@@ -1598,8 +1658,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float *S = Hs + loc.rec * (size_t)D * D;
         const float *dSn = dHs + loc.rec * (size_t)D * D;
         auto tix = [&](int r) { return (tok0 + r) * H + h; };  // token-head row index
-        // the gate's argument is scale * a (scale = e^{A_log[h]}, or 1)
+        // the gate's argument is scale * a (scale = e^{A_log[h]}, or 1); g itself comes from the
+        // gate table the forward prep used (per head with the scale)
         const float scale = A_log ? __expf(A_log[h]) : 1.0f;
+        const float *tab = gtab + (A_log ? (size_t)h * kGateTableEntries : 0);
 
         // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da
 #pragma unroll 4
@@ -1607,11 +1669,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int r = e / D, c = e % D;
             const bool ok = r < n;
             const size_t gi = (size_t)tix(ok ? r : 0) * D + c;
-            const float av = scale * __bfloat162float(ag[gi]);
+            const __nv_bfloat16 ab = ag[gi];
+            const float av = scale * __bfloat162float(ab);
             const float sg = __fdividef(1.f, 1.f + __expf(-av));
             sq[r * LDD + c] = ok ? __bfloat162float(qg[gi]) : 0.f;
             sk[r * LDD + c] = ok ? __bfloat162float(kg[gi]) : 0.f;
-            sG[r * LDD + c] = ok ? gate_bounded_fast(av, g_min) : 0.f;
+            sG[r * LDD + c] = ok ? __ldg(tab + __bfloat16_as_ushort(ab)) : 0.f;
             Gp[e] = g_min * sg * (1.f - sg) * scale;
             Bv[e] = ok ? __bfloat162float(vg[gi]) : 0.f;
             dOs[e] = ok ? __bfloat162float(dOg[gi]) : 0.f;
@@ -1971,21 +2034,66 @@ __global__ void __launch_bounds__(kRedThreads)
         dA_log[h] = buf[0];
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime (the library does not link the driver).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// One token tensor [B, T, H, D] (B = 0: a packed [T, H, D]) of bf16 as a tensor map with boxes
+// of 64 channels x 1 head x 64 tokens, 128-byte swizzle, zeros outside the tensor.
+cudaError_t make_token_map(CUtensorMap *m, const void *base, int D, int H, int64_t T, int B)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)(B > 0 ? B : 1)};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B > 0 ? 4 : 3, const_cast<void *>(base), dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The gate table (launch_gate_table) lives in the workspace at `gtab`; the prep looks g up in it.
 template <int D, bool kLogSig>
 cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, const void *k, const void *v,
-                          const void *a, const void *beta, float g_min, const float *A_log, void *ws, cudaStream_t s)
+                          const void *a, const void *beta, float g_min, const float *A_log, void *ws, float *gtab,
+                          cudaStream_t s)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
-    const size_t smem = PrepLayout<D>::Bytes;
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel<D, kLogSig>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    TokenMaps tm;
+    const int B = m.cu ? 0 : m.nseq;
+    cudaError_t e = make_token_map(&tm.q, q, D, H, m.T, B);
+    if (e == cudaSuccess)
+        e = make_token_map(&tm.k, k, D, H, m.T, B);
+    if (e == cudaSuccess)
+        e = make_token_map(&tm.v, v, D, H, m.T, B);
+    if (e == cudaSuccess)
+        e = make_token_map(&tm.a, a, D, H, m.T, B);
+    if (e == cudaSuccess)
+        e = launch_gate_table(kLogSig, (double)g_min, A_log, H, gtab, s);
     if (e != cudaSuccess)
         return e;
-    prep_kernel<D, kLogSig><<<grid, kPrepThreads, smem, s>>>(
-        m, H, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-        static_cast<const __nv_bfloat16 *>(beta), g_min, A_log, static_cast<unsigned char *>(ws), status);
+    const size_t smem = PrepLayout<D>::Bytes;
+    e = cudaFuncSetAttribute(prep_kernel<D, kLogSig>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    prep_kernel<D, kLogSig><<<grid, kPrepThreads, smem, s>>>(tm, m, H, static_cast<const __nv_bfloat16 *>(beta), gtab,
+                                                             A_log != nullptr && !kLogSig,
+                                                             static_cast<unsigned char *>(ws), status);
     return cudaGetLastError();
 }
 
@@ -2009,14 +2117,17 @@ cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S
 
 cudaError_t launch_prep(const SeqMap &m, int H, int D, dim3 grid, const void *q, const void *k, const void *v,
                         const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log, void *ws,
-                        cudaStream_t s)
+                        float *gtab, cudaStream_t s)
 {
     if (logsigmoid)
-        return D == 64 ? launch_prep_d<64, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s)
-                       : launch_prep_d<128, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s);
-    return D == 64 ? launch_prep_d<64, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s)
-                   : launch_prep_d<128, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, s);
+        return D == 64 ? launch_prep_d<64, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s)
+                       : launch_prep_d<128, true>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s);
+    return D == 64 ? launch_prep_d<64, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s)
+                   : launch_prep_d<128, false>(m, H, grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s);
 }
+
+// Bytes of the gate tables a workspace reserves: one per head (the per-head scale needs them).
+size_t gate_table_bytes(int H) { return (size_t)H * kGateTableEntries * 4; }
 
 cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const float *S0, void *o, float *S_T,
                         cudaStream_t s, float *M_out = nullptr)
@@ -2030,19 +2141,20 @@ cudaError_t launch_scan(const SeqMap &m, int H, int D, const void *ws, const flo
 // record, in record order), the per-chunk partials of dL/dA_log, and the per-CTA scratch slots
 // of bwd_chunk_kernel.
 struct BwdLayout {
-    size_t table, states, dstates, parts, scratch, total;
+    size_t table, gtab, states, dstates, parts, scratch, total;
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D, int nseq_packed = 0)
+BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D, int H, int nseq_packed = 0)
 {
     const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
     const size_t blk = (size_t)D * D * 4;
     const size_t slot = (size_t)(D == 64 ? BwdSlot<64>::floats : BwdSlot<128>::floats) * 4;
     BwdLayout l;
     l.table = (size_t)nrec * rec;
-    l.states = round256(l.table + (nseq_packed ? (size_t)(nseq_packed + 1) * 4 : 0));
+    l.gtab = round256(l.table + (nseq_packed ? (size_t)(nseq_packed + 1) * 4 : 0));
+    l.states = round256(l.gtab + gate_table_bytes(H));
     l.dstates = l.states + (size_t)nrec * blk;
     l.parts = l.dstates + (size_t)nrec * blk;
     l.scratch = round256(l.parts + (size_t)nrec * 4);
@@ -2063,7 +2175,8 @@ cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits,
     float *Hs = reinterpret_cast<float *>(base + l.states), *dHs = reinterpret_cast<float *>(base + l.dstates);
     float *parts = dA_log ? reinterpret_cast<float *>(base + l.parts) : nullptr;
     float *scratch = reinterpret_cast<float *>(base + l.scratch);
-    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, A_log, ws, s);
+    float *gtab = reinterpret_cast<float *>(base + l.gtab);
+    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s);
     if (e == cudaSuccess)
         e = launch_scan_d<D>(m, H, ws, S0, nullptr, nullptr, nullptr, s, Hs);
     if (e != cudaSuccess)
@@ -2084,8 +2197,8 @@ cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits,
     bwd_chunk_kernel<D><<<grid, kBwdThreads, BwdSmem<D>::bytes, s>>>(
         m, H, (int)nunits, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(a),
-        static_cast<const __nv_bfloat16 *>(beta), g_min, A_log, static_cast<const __nv_bfloat16 *>(dO), Hs, dHs,
-        scratch, dq, dk, dv, da, dbeta, parts, status);
+        static_cast<const __nv_bfloat16 *>(beta), g_min, A_log, gtab, static_cast<const __nv_bfloat16 *>(dO), Hs,
+        dHs, scratch, dq, dk, dv, da, dbeta, parts, status);
     e = cudaGetLastError();
     if (e != cudaSuccess || !dA_log)
         return e;
@@ -2153,19 +2266,22 @@ size_t varlen_records(int N, int T) { return ((size_t)T + kC - 1) / kC + (size_t
 
 }  // namespace
 
-size_t chunk_bf16_workspace(int B, int T, int H, int D)
+size_t chunk_bf16_records(int B, int T, int H, int D)
 {
     const size_t NT = ((size_t)T + kC - 1) / kC;
     const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
     return (size_t)B * H * NT * rec;
 }
 
+size_t chunk_bf16_workspace(int B, int T, int H, int D) { return chunk_bf16_records(B, T, H, D) + gate_table_bytes(H); }
+
 cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
                              const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log,
                              void *workspace, cudaStream_t s)
 {
     const SeqMap m = regular_map(B, T, H);
-    return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, s);
+    float *gtab = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + chunk_bf16_records(B, T, H, D));
+    return launch_prep(m, H, D, dim3(m.NT, B * H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, gtab, s);
 }
 
 cudaError_t launch_scan_bf16(int B, int T, int H, int D, const void *workspace, const float *S0, void *o,
@@ -2183,13 +2299,13 @@ cudaError_t launch_scan_affine_bf16(int B, int T, int H, int D, const void *work
 size_t chunk_bf16_bwd_workspace(int B, int T, int H, int D)
 {
     const SeqMap m = regular_map(B, T, H);
-    return bwd_layout(m.nrec, m.nrec, D).total;
+    return bwd_layout(m.nrec, m.nrec, D, H).total;
 }
 
 void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *dstates)
 {
     const SeqMap m = regular_map(B, T, H);
-    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D);
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, H);
     *states = l.states;
     *dstates = l.dstates;
 }
@@ -2201,7 +2317,7 @@ cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, con
 {
     const SeqMap m = regular_map(B, T, H);
     const dim3 grid(m.NT, B * H);
-    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D);
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, H);
     return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk, dv,
                                       da, dbeta, dS0, dA_log, workspace, s)
                    : launch_bwd_d<128>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk,
@@ -2211,7 +2327,7 @@ cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, con
 size_t chunk_bf16_bwd_varlen_workspace(int N, int T, int H, int D)
 {
     const int64_t nrec = (int64_t)H * (int64_t)varlen_records(N, T);
-    return bwd_layout(nrec, nrec, D, N).total;
+    return bwd_layout(nrec, nrec, D, H, N).total;
 }
 
 cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
@@ -2230,7 +2346,7 @@ cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H,
     m.NT = (int)varlen_records(N, T);
     m.nrec = (int64_t)H * m.NT;
     m.ntok = T;
-    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, N);
+    const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, H, N);
     int32_t *choff = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + l.table);
     m.choff = choff;
     seq_table_kernel<<<1, kTableThreads, 0, s>>>(cu, N, T, choff, status);
@@ -2312,7 +2428,7 @@ size_t chunk_bf16_varlen_workspace(int N, int T, int H, int D)
 {
     const size_t rec = D == 64 ? Rec<64>::Bytes : Rec<128>::Bytes;
     const size_t table = ((size_t)(N + 1) * 4 + 255) / 256 * 256;
-    return (size_t)H * varlen_records(N, T) * rec + table;
+    return (size_t)H * varlen_records(N, T) * rec + table + gate_table_bytes(H);
 }
 
 cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,
@@ -2337,7 +2453,9 @@ cudaError_t launch_chunk_bf16_varlen(int N, const int32_t *cu, int T, int H, int
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    e = launch_prep(m, H, D, dim3(m.NT, H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, s);
+    float *gtab = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(choff) +
+                                            ((size_t)(N + 1) * 4 + 255) / 256 * 256);
+    e = launch_prep(m, H, D, dim3(m.NT, H), q, k, v, a, beta, g_min, logsigmoid, A_log, workspace, gtab, s);
     if (e != cudaSuccess)
         return e;
     return launch_scan(m, H, D, workspace, S0, o, S_T, s);

@@ -90,12 +90,44 @@ __global__ void __launch_bounds__(256) gate_heads_kernel(const Tin *__restrict__
         float y[V];
 #pragma unroll
         for (int j = 0; j < V; ++j)
-            y[j] = __double2float_rn(g_min / (1.0 + exp(-((double)x[j] * scale))));
+            y[j] = gate_heads_exact(x[j], scale, g_min);
         float4 *out = reinterpret_cast<float4 *>(g + i * V);
 #pragma unroll
         for (int j = 0; j < V / 4; ++j)
             __stcs(out + j, make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]));
     }
+}
+
+// The gate of every bfloat16 bit pattern of the pre-activation: tab[bits], or with a per-head
+// scale tab[h * 65536 + bits].  The entries come from the same fp64 functions as the
+// stand-alone gate kernels, so a lookup gives exactly what kda_gate_fwd (kda_gate_fwd_heads)
+// returns for that input.  The chunk kernels read g this way, one table per call.
+__global__ void __launch_bounds__(256) gate_table_kernel(int logsigmoid, double g_min, const float *__restrict__ A_log,
+                                                         int nh, float *__restrict__ tab)
+{
+    const int64_t n = (int64_t)nh << 16;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float a = bf16_bits_to_float((uint16_t)(i & 0xffff));
+        float g;
+        if (logsigmoid)
+            g = gate_logsigmoid_exact(a);
+        else if (A_log)
+            g = gate_heads_exact(a, exp((double)A_log[i >> 16]), g_min);
+        else
+            g = gate_bounded_exact(a, g_min);
+        tab[i] = g;
+    }
+}
+
+cudaError_t launch_gate_table(bool logsigmoid, double g_min, const float *A_log, int H, float *tab, cudaStream_t s)
+{
+    const int nh = (A_log && !logsigmoid) ? H : 1;
+    int64_t blocks = (((int64_t)nh << 16) + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    blocks = blocks > cap ? cap : blocks;
+    gate_table_kernel<<<(unsigned)blocks, 256, 0, s>>>(logsigmoid ? 1 : 0, g_min, logsigmoid ? nullptr : A_log, nh,
+                                                        tab);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gate_heads(const void *a, kda_dtype dt, double g_min, const float *A_log, int64_t n_tok, int H,

@@ -27,19 +27,13 @@ int num_sms()
     return n;
 }
 
+// Looked up on every launch (it allocates nothing): a cached address could outlive the
+// context it belongs to (cudaDeviceReset, another context made current on the device).
 unsigned int *device_status_ptr()
 {
-    static unsigned int *cache[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
-        return nullptr;
-    if (dev < 64 && cache[dev])
-        return cache[dev];
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess)
         return nullptr;
-    if (dev < 64)
-        cache[dev] = static_cast<unsigned int *>(p);
     return static_cast<unsigned int *>(p);
 }
 
@@ -286,20 +280,31 @@ kda_status copy_state(const ChunkShape &sh, const float *S0, float *S_T, cudaStr
     return from_cuda(cudaMemsetAsync(S_T, 0, (size_t)sh.ns * 4, s));
 }
 
-// Validation and dispatch shared by kda_chunk_fwd and kda_chunk_fwd_logsigmoid.
-kda_status chunk_fwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
-                          const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
-                          const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
-                          kda_stream_t stream)
+}  // namespace
+
+namespace kda {
+
+// Every check of one chunk-forward problem (shape, gate, alignment, aliasing and, when
+// `check_ws` is set, the workspace size), done once on the whole problem before anything is
+// launched.  Shared by kda_chunk_fwd, kda_chunk_fwd_logsigmoid and kda_chunk_fwd_noalloc.
+kda_status validate_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                              const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                              const float *S0, const void *o, const float *S_T, const void *workspace,
+                              size_t ws_bytes, bool check_ws)
 {
     ChunkShape sh;
     kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
     if (st == KDA_OK)
         st = check_gate(gate, g_min, dtype);
+    if (st != KDA_OK)
+        return st;
+    if (!check_ws) {  // the caller supplies its own scratch; only the overlap checks use the range
+        sh.ws = workspace ? ws_bytes : 0;
+        ws_bytes = sh.ws;
+    }
+    st = check_prep_args(sh, q, k, v, a, beta, workspace, ws_bytes);
     if (st == KDA_OK)
-        st = check_prep_args(sh, q, k, v, a, beta, workspace, ws_bytes);
-    if (st == KDA_OK)
-        st = check_scan_args(sh, workspace, ws_bytes, S0, o, S_T);
+        st = check_scan_args(sh, workspace, ws_bytes, S0, const_cast<void *>(o), const_cast<float *>(S_T));
     if (st != KDA_OK)
         return st;
     // the outputs must not overlap the inputs either
@@ -309,20 +314,47 @@ kda_status chunk_fwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, 
                             Range(beta, sh.ntok * es)})
         if (overlaps(ro, in) || overlaps(rST, in))
             return KDA_ERR_ALIAS;
+    return KDA_OK;
+}
 
-    cudaStream_t s = (cudaStream_t)stream;
-    if (T == 0)
+// The launches of one validated chunk-forward problem.
+kda_status dispatch_chunk_fwd(int B, int T, int H, int dk, kda_dtype dtype, const void *q, const void *k,
+                              const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                              const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s)
+{
+    if (T == 0) {
+        ChunkShape sh;
+        sh.ns = (int64_t)B * H * dk * dk;
         return copy_state(sh, S0, S_T, s);
+    }
     if (dtype == KDA_F32)
         return from_cuda(launch_chunk_f32(B, T, H, dk, static_cast<const float *>(q), static_cast<const float *>(k),
                                           static_cast<const float *>(v), static_cast<const float *>(a),
                                           static_cast<const float *>(beta), g_min, S0, static_cast<float *>(o), S_T,
                                           s));
-    st = from_cuda(
+    kda_status st = from_cuda(
         launch_prep_bf16(B, T, H, dk, q, k, v, a, beta, g_min, gate == KDA_GATE_LOGSIGMOID, nullptr, workspace, s));
     if (st != KDA_OK)
         return st;
     return from_cuda(launch_scan_bf16(B, T, H, dk, workspace, S0, o, S_T, s));
+}
+
+}  // namespace kda
+
+namespace {
+
+// Validation and dispatch shared by kda_chunk_fwd and kda_chunk_fwd_logsigmoid.
+kda_status chunk_fwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                          const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                          const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                          kda_stream_t stream)
+{
+    const kda_status st = validate_chunk_fwd(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, gate, S0, o, S_T,
+                                             workspace, ws_bytes, true);
+    if (st != KDA_OK)
+        return st;
+    return dispatch_chunk_fwd(B, T, H, dk, dtype, q, k, v, a, beta, g_min, gate, S0, o, S_T, workspace,
+                              (cudaStream_t)stream);
 }
 
 }  // namespace

@@ -1,6 +1,7 @@
 // kda_common.cuh -- device helpers shared by the libkda kernels (sm_100a).
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (the type only; the encoder is reached through the runtime)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -30,6 +31,21 @@ constexpr bool kDebugChecks = false;
 __device__ __forceinline__ float gate_bounded_exact(float a, double g_min)
 {
     return __double2float_rn(g_min / (1.0 + exp(-(double)a)));
+}
+
+// The gate with a per-head scale on its argument, g = g_min * sigmoid(scale * a), the
+// product formed in float64 too: one rounding from the fp64 value.
+__device__ __forceinline__ float gate_heads_exact(float a, double scale, double g_min)
+{
+    return __double2float_rn(g_min / (1.0 + exp(-((double)a * scale))));
+}
+
+// Unbounded gate g = log sigmoid(a) = min(a, 0) - log(1 + e^{-|a|}), evaluated in float64
+// and rounded once.
+__device__ __forceinline__ float gate_logsigmoid_exact(float a)
+{
+    const double x = (double)a;
+    return __double2float_rn(fmin(x, 0.0) - log1p(exp(-fabs(x))));
 }
 
 // Same gate in float32 with the hardware exponential and divide (the chunk kernels'
@@ -218,6 +234,28 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Tiled tensor copies (TMA) of one box of a tensor map in this GPU's memory into this CTA's
+// shared memory, completing on `bar` (no multicast).  Coordinates are in elements, innermost
+// first; the innermost one times the element size is a multiple of 16 bytes at every call.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *tm, int x, int y, int z, int w,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -19,6 +19,11 @@ cudaError_t launch_gate(const void *a, kda_dtype dt, double g_min, float *g, int
 cudaError_t launch_gate_heads(const void *a, kda_dtype dt, double g_min, const float *A_log, int64_t n_tok, int H,
                               int dk, float *g, cudaStream_t s);
 
+// The gate of all 65536 bfloat16 inputs (per head with A_log, H x 65536 entries), from the
+// same fp64 functions as the kernels above: the chunk kernels look g up in it.
+constexpr size_t kGateTableEntries = 65536;
+cudaError_t launch_gate_table(bool logsigmoid, double g_min, const float *A_log, int H, float *tab, cudaStream_t s);
+
 // K5: float32 CUDA-core chunked forward (16-token chunks).
 cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const float *k, const float *v,
                              const float *a, const float *beta, float g_min, const float *S0, float *o,
@@ -28,6 +33,9 @@ cudaError_t launch_chunk_f32(int B, int T, int H, int D, const float *q, const f
 // chunk) into the workspace; the scan walks them.  `logsigmoid` selects the unbounded gate
 // g = log sigmoid(a) with element-wise diagonal tiles (g_min is then not used).  A_log
 // (nullable, [H]) scales the gate's argument by e^{A_log[h]}.
+// The workspace holds the records, then one gate table per head (the per-head scale needs
+// them; without it only the first is written): chunk_bf16_records + H x 65536 floats.
+size_t chunk_bf16_records(int B, int T, int H, int D);
 size_t chunk_bf16_workspace(int B, int T, int H, int D);
 cudaError_t launch_prep_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
                              const void *a, const void *beta, float g_min, bool logsigmoid, const float *A_log,
@@ -69,6 +77,16 @@ cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H,
                                          const float *A_log, const float *S0, const void *dO, const float *dS_T,
                                          float *dq, float *dk, float *dv, float *da, float *dbeta, float *dS0,
                                          float *dA_log, void *workspace, cudaStream_t s);
+// All checks of one kda_chunk_fwd problem, on the whole (B, T) problem at once; with
+// check_ws false the workspace range is only used for the overlap checks (its size is the
+// caller's business).  dispatch_chunk_fwd launches a problem that passed them.
+kda_status validate_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                              const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                              const float *S0, const void *o, const float *S_T, const void *workspace,
+                              size_t ws_bytes, bool check_ws);
+kda_status dispatch_chunk_fwd(int B, int T, int H, int dk, kda_dtype dtype, const void *q, const void *k,
+                              const void *v, const void *a, const void *beta, float g_min, kda_gate gate,
+                              const float *S0, void *o, float *S_T, void *workspace, cudaStream_t s);
 // K4: single-token decode step.
 cudaError_t launch_decode(int N, int H, int D, kda_dtype dt, const void *q, const void *k, const void *v,
                           const void *a, const void *beta, float g_min, float *S, void *o, cudaStream_t s);

@@ -10,11 +10,9 @@
 // keeps until the process exits.  Nothing here allocates.
 //
 // The scratch holds the per-chunk records of kda_chunk_fwd for one stretch of whole
-// 64-token chunks of one batch element at a time, plus a carry slot for the state when
-// the caller passes no S_T.  Longer inputs are processed stretch by stretch with the
+// 64-token chunks of one batch element at a time and the gate table after them, plus a
+// carry slot for the state when the caller passes no S_T.  Longer inputs are processed stretch by stretch with the
 // float32 state carried between calls, which gives exactly the same result as one call.
-#include <mutex>
-
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -25,27 +23,18 @@ constexpr size_t kScratchBytes = (size_t)64 << 20;  // 64 MiB per device
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::mutex g_setup_mutex;
-void *g_scratch_ptr[64] = {nullptr};
-
-// Device address of the scratch array on the current device, looked up once per device.
+// Device address of the scratch array in the current device's context.  Host code only
+// holds a stand-in for the array's name, so the address is looked up on every call (this
+// allocates nothing); a cached address could outlive its context (cudaDeviceReset, another
+// context made current on the same device).  The first lookup on a device may load the
+// module, which is why the first call should come before any stream capture.
 cudaError_t scratch_ptr(void **out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= 64)
-        return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess)
-            return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -61,27 +50,33 @@ extern "C" kda_status kda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv,
                                             float g_min, const float *S0, void *o, float *S_T,
                                             kda_stream_t stream)
 {
-    if ((dtype != KDA_BF16 && dtype != KDA_F32) || B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1)
-        return KDA_ERR_INVALID_ARG;
-    // The float32 path needs no scratch: the regular entry point allocates nothing either.
+    // Every check runs once on the whole (B, T) problem -- shapes, gate bound, alignment, and
+    // overlaps between any two tensors, across batch elements too -- before anything is
+    // launched.  The scratch is library memory no caller pointer can reach, so it takes no
+    // part in the overlap checks.
+    kda_status st = validate_chunk_fwd(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, KDA_GATE_BOUNDED, S0, o,
+                                       S_T, nullptr, 0, false);
+    if (st != KDA_OK)
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // The float32 path and T = 0 need no scratch.
     if (dtype == KDA_F32 || T == 0)
-        return kda_chunk_fwd(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, S0, o, S_T, nullptr, 0, stream);
+        return dispatch_chunk_fwd(B, T, H, dk, dtype, q, k, v, a, beta, g_min, KDA_GATE_BOUNDED, S0, o, S_T,
+                                  nullptr, s);
 
-    const size_t rec = kda_chunk_fwd_workspace(1, KDA_CHUNK, H, dk, dv, dtype);  // one chunk, all heads
-    if (rec == 0)  // unsupported head dims: let the regular checks name the reason
-        return kda_chunk_fwd(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, S0, o, S_T, nullptr, 0, stream);
+    const size_t rec = chunk_bf16_records(1, KDA_CHUNK, H, dk);  // one chunk of every head
     const size_t state_bytes = ((size_t)H * dk * dv * 4 + 255) / 256 * 256;  // carry slot, one batch element
-    if (state_bytes + rec > kScratchBytes)
+    const size_t table = kGateTableEntries * 4;  // the gate table after the records (no per-head scale here)
+    if (state_bytes + table + rec > kScratchBytes)
         return KDA_ERR_WORKSPACE;  // not even one chunk of all heads fits the fixed scratch
-    const int64_t chunks = (int64_t)((kScratchBytes - state_bytes) / rec);
-    const int64_t stretch = chunks * KDA_CHUNK;  // tokens per call
+    const int64_t chunks = (int64_t)((kScratchBytes - state_bytes - table) / rec);
+    const int64_t stretch = chunks * KDA_CHUNK;  // tokens per launch pair
 
     void *scratch = nullptr;
     if (scratch_ptr(&scratch) != cudaSuccess)
         return KDA_ERR_CUDA;
     float *carry_slot = static_cast<float *>(scratch);
     void *ws = static_cast<unsigned char *>(scratch) + state_bytes;
-    const size_t ws_bytes = kScratchBytes - state_bytes;
 
     const size_t es = 2;  // bf16
     const unsigned char *qb = static_cast<const unsigned char *>(q);
@@ -90,19 +85,18 @@ extern "C" kda_status kda_chunk_fwd_noalloc(int B, int T, int H, int dk, int dv,
     const unsigned char *ab = static_cast<const unsigned char *>(a);
     const unsigned char *bb = static_cast<const unsigned char *>(beta);
     unsigned char *ob = static_cast<unsigned char *>(o);
-    if (!qb || !kb || !vb || !ab || !bb || !ob)
-        return KDA_ERR_INVALID_ARG;
     const size_t state_elems = (size_t)H * dk * dv;
     for (int b = 0; b < B; ++b) {
         const float *s_in = S0 ? S0 + (size_t)b * state_elems : nullptr;
+        // without S_T the state between stretches lives in the carry slot, reused by every
+        // batch element (each one's first stretch starts from its own S0, never the slot)
         float *carry = S_T ? S_T + (size_t)b * state_elems : carry_slot;
         for (int64_t t0 = 0; t0 < T; t0 += stretch) {
             const int len = (int)(T - t0 < stretch ? T - t0 : stretch);
             const size_t tok = (size_t)b * T + (size_t)t0;  // first token row of this stretch
-            const kda_status st = kda_chunk_fwd(
-                1, len, H, dk, dv, dtype, qb + tok * H * dk * es, kb + tok * H * dk * es, vb + tok * H * dv * es,
-                ab + tok * H * dk * es, bb + tok * H * es, g_min, t0 == 0 ? s_in : carry, ob + tok * H * dv * es,
-                carry, ws, ws_bytes, stream);
+            st = dispatch_chunk_fwd(1, len, H, dk, dtype, qb + tok * H * dk * es, kb + tok * H * dk * es,
+                                    vb + tok * H * dv * es, ab + tok * H * dk * es, bb + tok * H * es, g_min,
+                                    KDA_GATE_BOUNDED, t0 == 0 ? s_in : carry, ob + tok * H * dv * es, carry, ws, s);
             if (st != KDA_OK)
                 return st;
         }

@@ -33,6 +33,28 @@ import torch.distributed as dist
 import chunked_linear_attention_chunk_b200 as kda
 
 
+class DistComm:
+    """The exchange steps over torch.distributed (the default): all-gather and all-reduce in
+    ``group``; a single process without a process group is world 1."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+
+    def all_gather(self, x):
+        if self.world == 1:
+            return [x]
+        xs = [torch.empty_like(x) for _ in range(self.world)]
+        dist.all_gather(xs, x.contiguous(), group=self.group)
+        return xs
+
+    def all_reduce_(self, x):
+        if self.world > 1:
+            dist.all_reduce(x, group=self.group)
+        return x
+
+
 class LibkdaSegmentOps:
     """The per-segment steps on this rank's GPU, through libkda (bf16 tokens)."""
 
@@ -63,58 +85,44 @@ class LibkdaSegmentOps:
                                  dS_T=None if dS_T is None else dS_T.contiguous(), A_log=self.A_log)
 
 
-def sp_chunk_fwd(q, k, v, a, beta, S0=None, group=None, ops=None):
+def sp_chunk_fwd(q, k, v, a, beta, S0=None, group=None, ops=None, comm=None):
     """This rank's segment of a sequence-parallel chunked forward.
 
     q, k, a [B, T_r, H, dk]; v [B, T_r, H, dv]; beta [B, T_r, H]: the segment of every
     batch sequence this rank holds; rank r holds the r-th segment in sequence order
     (segments may differ in length).  S0 [B, H, dk, dv] is the sequence's initial state,
     the same on every rank (or None for zeros).  Returns (o for this segment, the whole
-    sequence's final state), the latter identical on every rank."""
+    sequence's final state), the latter identical on every rank.  ``comm`` replaces the
+    torch.distributed exchange (``DistComm(group)``) with another one of the same methods."""
     ops = ops if ops is not None else LibkdaSegmentOps()
-    world = dist.get_world_size(group) if dist.is_initialized() else 1
-    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    comm = comm if comm is not None else DistComm(group)
     handle, S_zero, M = ops.maps(q, k, v, a, beta)
-    if world > 1:
-        Zs = [torch.empty_like(S_zero) for _ in range(world)]
-        Ms = [torch.empty_like(M) for _ in range(world)]
-        dist.all_gather(Zs, S_zero.contiguous(), group=group)
-        dist.all_gather(Ms, M.contiguous(), group=group)
-    else:
-        Zs, Ms = [S_zero], [M]
+    Zs, Ms = comm.all_gather(S_zero), comm.all_gather(M)
     S_in = ops.combine(torch.stack(Ms), torch.stack(Zs), S0)
-    o, _ = ops.forward(handle, S_in[rank])
-    return o, S_in[world]
+    o, _ = ops.forward(handle, S_in[comm.rank])
+    return o, S_in[comm.world]
 
 
-def _gather(x, world, group):
-    if world == 1:
-        return [x]
-    xs = [torch.empty_like(x) for _ in range(world)]
-    dist.all_gather(xs, x.contiguous(), group=group)
-    return xs
-
-
-def sp_chunk_bwd(q, k, v, a, beta, dO, S0=None, dS_T=None, group=None, ops=None):
+def sp_chunk_bwd(q, k, v, a, beta, dO, S0=None, dS_T=None, group=None, ops=None, comm=None):
     """This rank's segment of a sequence-parallel backward (the segments as in
     ``sp_chunk_fwd``; dO is this segment's dL/do, dS_T the gradient of the whole sequence's
     final state, the same on every rank, or None).  Returns the ``kda_chunk_bwd`` dict of
     this segment's token gradients, with dS0 the gradient of the sequence's initial state
     (identical on every rank) and, given A_log, dA_log summed over all segments."""
     ops = ops if ops is not None else LibkdaSegmentOps()
-    world = dist.get_world_size(group) if dist.is_initialized() else 1
-    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    comm = comm if comm is not None else DistComm(group)
+    world, rank = comm.world, comm.rank
     tokens = (q, k, v, a, beta)
     _, S_zero, M = ops.maps(*tokens)
-    Ms = _gather(M, world, group)
-    S_in = ops.combine(torch.stack(Ms), torch.stack(_gather(S_zero, world, group)), S0)
+    Ms = comm.all_gather(M)
+    S_in = ops.combine(torch.stack(Ms), torch.stack(comm.all_gather(S_zero)), S0)
     dZ = ops.backward(tokens, S_in[rank], dO, None)["dS0"]
-    dZs = _gather(dZ, world, group)
+    dZs = comm.all_gather(dZ)
     # suffix over the segments in reverse order: X[j + 1] = M[R-1-j]^T X[j] + dZ[R-1-j], X[0] = dS_T
     Mt = torch.stack([Ms[world - 1 - j].transpose(-1, -2) for j in range(world)])
     X = ops.combine(Mt, torch.stack([dZs[world - 1 - j] for j in range(world)]), dS_T)
     g = ops.backward(tokens, S_in[rank], dO, X[world - 1 - rank])
     g["dS0"] = X[world]
-    if g.get("dA_log") is not None and world > 1:
-        dist.all_reduce(g["dA_log"], group=group)
+    if g.get("dA_log") is not None:
+        comm.all_reduce_(g["dA_log"])
     return g

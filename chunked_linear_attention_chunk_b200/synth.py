@@ -124,7 +124,7 @@ def adversarial_range(T: int):
 def make_inputs(B, T, H, dk, dv, dtype="bf16", seed=0, s0_std=0.1, adversarial=False):
     """Draw one batch.  Returns a dict of CPU tensors:
     q, k, a [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H] (all ``dtype``); S0 [B,H,dk,dv] float32
-    (zeros when ``s0_std`` is 0)."""
+    (zeros when ``s0_std`` is 0; left out when it is None)."""
     q = _unit_rows(_normal(seed, _Q, (B, T, H, dk)))
     k = _unit_rows(_normal(seed, _K, (B, T, H, dk)))
     v = _normal(seed, _V, (B, T, H, dv))
@@ -133,11 +133,13 @@ def make_inputs(B, T, H, dk, dv, dtype="bf16", seed=0, s0_std=0.1, adversarial=F
         s, e = adversarial_range(T)
         a[:, s:e] = np.float32(ADV_VALUE)
     beta = _sigmoid32(_normal(seed, _BETA, (B, T, H)))
+    out = {n: _cast(x, dtype) for n, x in (("q", q), ("k", k), ("v", v), ("a", a), ("beta", beta))}
+    if s0_std is None:  # token tensors only
+        return out
     if s0_std > 0:
         S0 = _normal(seed, _S0, (B, H, dk, dv), std=s0_std)
     else:
         S0 = np.zeros((B, H, dk, dv), np.float32)
-    out = {n: _cast(x, dtype) for n, x in (("q", q), ("k", k), ("v", v), ("a", a), ("beta", beta))}
     out["S0"] = torch.from_numpy(S0)
     return out
 
@@ -160,8 +162,24 @@ def decode_state(w: DecodeWorkload):
 def decode_tokens(w: DecodeWorkload, step: int, dtype="bf16"):
     """Token set of one decode step: q, k, a [N,H,dk]; v [N,H,dv]; beta [N,H]."""
     seed = w.seed * 1000 + step
-    x = make_inputs(w.N, 1, w.H, w.dk, w.dv, dtype, seed, 0.0, False)
+    x = make_inputs(w.N, 1, w.H, w.dk, w.dv, dtype, seed, None, False)
     return {n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "a", "beta")}
+
+
+def decode_token_sets(w: DecodeWorkload, steps, seed_of=None, workers=None):
+    """Token sets of consecutive decode steps, in order (``decode_tokens(w, seed_of(i))`` for
+    each i in ``steps``), drawn a bounded number of steps ahead on a thread pool."""
+    steps = list(steps)
+    seed_of = seed_of or (lambda i: i)
+    workers = workers or min(16, os.cpu_count() or 1)
+    ahead = 2 * workers
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = [ex.submit(decode_tokens, w, seed_of(i)) for i in steps[:ahead]]
+        for j in range(len(steps)):
+            if j + ahead < len(steps):
+                futs.append(ex.submit(decode_tokens, w, seed_of(steps[j + ahead])))
+            yield futs[j].result()
+            futs[j] = None
 
 
 def to_numpy32(t: torch.Tensor) -> np.ndarray:

@@ -147,7 +147,10 @@ size_t kda_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, kda_dtype dt
  *              is rejected.
  *   workspace  device scratch of at least kda_chunk_fwd_workspace(...) bytes, 16-byte
  *              aligned, overlapping no tensor argument (may be NULL when that size is
- *              0).  Its contents on entry are ignored and on exit unspecified.
+ *              0).  Its contents on entry are ignored and on exit unspecified: the
+ *              bf16 path writes its per-chunk records there, then a table of the gate at
+ *              every bfloat16 input (the values kda_gate_fwd returns, one float each),
+ *              from which the kernels read g.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.
  */
 kda_status kda_chunk_fwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q,
@@ -352,8 +355,12 @@ kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const 
  * until the process exits.  It allocates nothing and computes exactly what kda_chunk_fwd
  * computes: inputs longer than the scratch holds are processed in stretches of whole
  * 64-token chunks with the float32 state carried between them.
- *   - The first call on a device looks up the scratch array's device address (once per
- *     device, with that device current); make that first call before any stream capture.
+ *   - Every call looks up the scratch array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing); the first such lookup on a device
+ *     may load the library's module there, so make the first call before any stream
+ *     capture.
+ *   - All checks (shapes, alignment, overlaps between any two tensors, across batch
+ *     elements too) run on the whole problem before the first launch, as in kda_chunk_fwd.
  *   - All calls share the one array, and it keeps whatever the last call left there;
  *     nothing in it needs to start at zero.  Calls whose GPU work overlaps (other
  *     streams, other host threads) race on the array: serialise them.

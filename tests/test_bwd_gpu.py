@@ -137,6 +137,48 @@ def test_bwd_repeatable():
         assert np.array_equal(a[n], b[n]), n
 
 
+def test_bwd_repeatable_full_size_and_packed():
+    """Five calls at the full 64K-token stage (B1 T65536 H32 d128, 1024 chunks per head over
+    the 148 persistent gradient CTAs, each CTA reusing its scratch slot for about 220
+    chunks) and three over a packed batch with the per-head gate scale: every gradient is
+    bitwise the same from call to call.  Each element of every gradient is produced by one
+    thread from values written before a CTA barrier, with no atomics, so nothing may vary."""
+    w = synth.STAGE_64K
+    x = synth.workload_inputs(w)
+    rng = np.random.default_rng(741)
+    dO = torch.from_numpy(rng.normal(size=(w.B, w.T, w.H, w.dv)).astype(np.float32)).to(torch.bfloat16).cuda()
+    d = {n: x[n].cuda() for n in NAMES}
+    S0 = x["S0"].cuda()
+    ws = torch.empty(kda.kda_chunk_bwd_workspace(w.B, w.T, w.H, w.dk, w.dv), dtype=torch.uint8, device="cuda")
+    first = None
+    for _ in range(5):
+        g = kda.kda_chunk_bwd(*(d[n] for n in NAMES), dO, G_MIN, S0=S0, workspace=ws)
+        torch.cuda.synchronize()
+        assert kda.kda_device_status() == 0
+        if first is None:
+            first = {n: t.clone() for n, t in g.items() if t is not None}
+        else:
+            for n, t in first.items():
+                assert torch.equal(g[n], t), n
+    del first, g, ws, d, dO
+    lengths = [700, 1, 64, 3000, 129]
+    xp, dOp, dSTp, S0p, cu = _packed(lengths, 4, 128, seed=742)
+    A_log = torch.from_numpy((np.random.default_rng(743).normal(size=4) * 0.5).astype(np.float32)).cuda()
+    dp = {n: xp[n][0].cuda() for n in NAMES}
+    cu_d = torch.from_numpy(cu).cuda()
+    ref = None
+    for _ in range(3):
+        g = kda.kda_chunk_bwd_varlen(*(dp[n] for n in NAMES), dOp[0].cuda(), cu_d, G_MIN, S0=S0p.cuda(),
+                                     dS_T=dSTp.cuda(), A_log=A_log)
+        torch.cuda.synchronize()
+        assert kda.kda_device_status() == 0
+        if ref is None:
+            ref = {n: t.clone() for n, t in g.items() if t is not None}
+        else:
+            for n, t in ref.items():
+                assert torch.equal(g[n], t), n
+
+
 def test_bwd_full_size_sampled_heads():
     """The 64K-token stage (B1 T65536 H32 d128, bench inputs) against the oracle on two
     sampled heads (the oracle runs them alone: heads are independent)."""

@@ -35,6 +35,43 @@ def test_decode_config_chained_steps():
         assert err_s(S.cpu().numpy(), S_ref) <= 1e-5
 
 
+def test_decode_config_1000_chained_steps():
+    """The decode workload as configured: N=256 sequences x H=32 heads, d=128, fp32 state
+    ~N(0, 0.1), 1000 chained steps, each with its own seeded token set, the state updated in
+    place on the GPU.  The (n, h) units are independent, so the fp64 oracle follows a sample
+    of 64 of the 8192 units through all 1000 steps: o is compared at 11 sampled steps and
+    the state after the last step.
+
+    Tolerance for the state after 1000 steps: every step rounds a handful of float32
+    operations (decay, two dot products, the rank-1 update: relative 2^-24 each, a few ulp
+    for the fast exponential), and the step map is non-expansive (decay factors <= 1, the
+    erase I - beta k k^T with |k| = 1 and 0 < beta < 1), so rounding errors add up at most
+    linearly: 1000 steps x ~2^-20 ~ 1e-3 of the state's scale.  o is bf16 (2e-2)."""
+    w = synth.DECODE
+    steps = 1000
+    rng = np.random.default_rng(1234)
+    units = np.unique(np.concatenate([[0, w.N * w.H - 1], rng.choice(w.N * w.H, 62, replace=False)]))
+    un, uh = units // w.H, units % w.H
+    S_cpu = synth.decode_state(w)
+    S = S_cpu.cuda()
+    S_ref = S_cpu.numpy()[un, uh].astype(np.float64)[:, None]  # [units, 1, dk, dv]
+    check_at = set(range(0, steps, 100)) | {steps - 1}
+    worst_o = 0.0
+    for step, tok in enumerate(synth.decode_token_sets(w, range(steps))):
+        d = {n: t.cuda(non_blocking=False) for n, t in tok.items()}
+        o = kda.kda_decode_step(*(d[n] for n in NAMES), S, G_MIN)
+        sub = {n: synth.to_numpy32(tok[n])[un, uh][:, None] for n in NAMES}
+        o_ref, S_ref = oracle.decode(*(sub[n] for n in NAMES), S_ref, G_MIN)
+        if step in check_at:
+            got = o.float().cpu().numpy()[un, uh][:, None]
+            worst_o = max(worst_o, _err_tok(got, o_ref))
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    assert worst_o <= TOL_BF16_O, worst_o
+    es = err_s(S.cpu().numpy()[un, uh][:, None], S_ref)
+    assert es <= 1e-3, es
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_decode_f32(D):
     x = synth.make_inputs(5, 1, 3, D, D, "f32", seed=600 + D, s0_std=0.1)

@@ -75,3 +75,48 @@ def test_gate_heads_bit_exact(dtype):
     torch.cuda.synchronize()
     ref = oracle.gate_heads(a.float().numpy(), A_log.numpy(), -5.0)
     assert np.array_equal(g.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def _records_bytes(B, T, H, D):
+    rec = D * D * 2 + 64 * D * 2 + D * 4 + D * D * 2 + 64 * D * 2
+    return B * H * ((T + 63) // 64) * rec
+
+
+@pytest.mark.parametrize("g_min", [-5.0, -0.25])
+def test_chunk_path_gate_table_is_bit_exact(g_min):
+    """The chunk path reads g from a table of the gate at all 65536 bfloat16 inputs, which the
+    prep writes into the workspace (after the records) with the fp64 function of kda_gate_fwd.
+    The table equals the oracle's gate bit for bit, so every g the hot path uses does too."""
+    g_min = float(np.float32(g_min))
+    B, T, H, D = 1, 200, 2, 128
+    x = synth.make_inputs(B, T, H, D, D, "bf16", seed=41, s0_std=0.1)
+    d = {n: x[n].cuda() for n in ("q", "k", "v", "a", "beta")}
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace(B, T, H, D, D), dtype=torch.uint8, device="cuda")
+    kda.kda_chunk_fwd_prep(d["q"], d["k"], d["v"], d["a"], d["beta"], ws, g_min)
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    off = _records_bytes(B, T, H, D)
+    assert ws.numel() >= off + 65536 * 4
+    tab = ws[off:off + 65536 * 4].cpu().numpy().view(np.float32)
+    a = _all_bf16()
+    _same_bits(tab, oracle.gate(a.float().numpy(), g_min))
+    # the table is indexed by the input's bits: entry i is the gate of bf16 pattern i
+    assert tab[0] == np.float32(oracle.gate(np.zeros(1, np.float32), g_min)[0])
+
+
+def test_chunk_path_gate_table_per_head_is_bit_exact():
+    """With the per-head scale the prep writes one table per head, each equal to
+    kda_gate_fwd_heads (and the oracle) at every bfloat16 input of that head."""
+    B, T, H, D = 1, 70, 3, 64
+    x = synth.make_inputs(B, T, H, D, D, "bf16", seed=42, s0_std=0.1)
+    d = {n: x[n].cuda() for n in ("q", "k", "v", "a", "beta")}
+    A_log = torch.tensor([0.4, -0.7, 1.1])
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace(B, T, H, D, D), dtype=torch.uint8, device="cuda")
+    kda.kda_chunk_fwd_prep(d["q"], d["k"], d["v"], d["a"], d["beta"], ws, -5.0, A_log=A_log.cuda())
+    torch.cuda.synchronize()
+    off = _records_bytes(B, T, H, D)
+    tab = ws[off:off + H * 65536 * 4].cpu().numpy().view(np.float32).reshape(H, 65536)
+    a = _all_bf16().float().numpy()
+    for h in range(H):
+        ref = oracle.gate_heads(a.reshape(1, 1, 65536), A_log[h:h + 1].numpy(), -5.0).reshape(-1)
+        _same_bits(tab[h], ref)

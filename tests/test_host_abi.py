@@ -55,13 +55,15 @@ def test_status_strings(L):
 
 def test_workspace_size(L):
     f = L.kda_chunk_fwd_workspace
-    # per chunk record: N (D x D) + Q' (64 x D) bf16, Gamma (D f32), Bm (D x D) + O' (64 x D) bf16
+    # per chunk record: N (D x D) + Q' (64 x D) bf16, Gamma (D f32), Bm (D x D) + O' (64 x D) bf16;
+    # after the records, one gate table of 65536 floats per head
     rec128 = 128 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 128 * 128 * 2 + 64 * 128 * 2
-    assert f(1, 64, 1, 128, 128, kda.KDA_BF16) == rec128
-    assert f(2, 65, 3, 128, 128, kda.KDA_BF16) == 2 * 3 * 2 * rec128
-    assert f(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec128
+    tab = 65536 * 4
+    assert f(1, 64, 1, 128, 128, kda.KDA_BF16) == rec128 + tab
+    assert f(2, 65, 3, 128, 128, kda.KDA_BF16) == 2 * 3 * 2 * rec128 + 3 * tab
+    assert f(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec128 + 32 * tab
     rec64 = 64 * 64 * 2 + 64 * 64 * 2 + 64 * 4 + 64 * 64 * 2 + 64 * 64 * 2
-    assert f(1, 100, 1, 64, 64, kda.KDA_BF16) == 2 * rec64
+    assert f(1, 100, 1, 64, 64, kda.KDA_BF16) == 2 * rec64 + tab
     assert f(1, 100, 1, 64, 64, kda.KDA_F32) == 0
     assert f(1, 0, 1, 128, 128, kda.KDA_BF16) == 0
     assert f(0, 64, 1, 128, 128, kda.KDA_BF16) == 0
@@ -243,7 +245,7 @@ def test_varlen_entry_validates(L):
     n = T * H * D * 2
     ws_need = L.kda_chunk_fwd_varlen_workspace(N, T, H, D, D, kda.KDA_BF16)
     rec = 128 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 128 * 128 * 2 + 64 * 128 * 2
-    assert ws_need == H * ((T + 63) // 64 + N) * rec + 256
+    assert ws_need == H * ((T + 63) // 64 + N) * rec + 256 + H * 65536 * 4  # records, chunk table, gate tables
     assert L.kda_chunk_fwd_varlen_workspace(N, T, H, D, D, kda.KDA_F32) == 0
     ins = [BASE + i * (n + 4096) for i in range(5)]
     cu = BASE * 2
@@ -399,3 +401,39 @@ def test_chunk_bwd_varlen_entry_validates(L):
     assert bwd(dq=ins[1]) == ALIAS
     assert bwd(w=cu) == ALIAS                             # workspace over cu_seqlens
     assert bwd(dA=BASE * 3) == INVALID
+
+
+def _noalloc(L, B=2, T=64, H=1, dk=128, dv=128, dt=kda.KDA_BF16, q=None, S0=None, o=None, ST=None, g_min=-5.0):
+    es = 2 if dt == kda.KDA_BF16 else 4
+    n = B * T * H * dk * es
+    q = BASE if q is None else q
+    o = BASE + 5 * (n + 4096) if o is None else o
+    P = ctypes.c_void_p
+    return L.kda_chunk_fwd_noalloc(B, T, H, dk, dv, dt, P(q), P(BASE + (n + 4096)), P(BASE + 2 * (n + 4096)),
+                                   P(BASE + 3 * (n + 4096)), P(BASE + 4 * (n + 4096)), ctypes.c_float(g_min),
+                                   P(S0), P(o), P(ST), None)
+
+
+def test_noalloc_validates_the_whole_problem_before_launching(L):
+    """The no-workspace entry runs its batch elements one by one, but every check covers
+    the whole (B, T) problem first: an overlap that only exists between different batch
+    elements is refused with ALIAS, before anything is launched (no GPU is needed to see it)."""
+    B, T, H, d = 2, 64, 1, 128
+    per_o = T * H * d * 2           # bytes of o per batch element
+    per_s = H * d * d * 4           # bytes of S per batch element
+    O = BASE * 2
+    # S0 of batch element 1 starts where o (element 0) starts: o[0] overlaps S0[1] only
+    assert O - per_s + per_s == O and per_o > 0
+    assert _noalloc(L, B=B, S0=O - per_s, o=O, ST=BASE * 4) == ALIAS
+    S = BASE * 3
+    # S_T of element 0 lies on q of element 1
+    q_elem1 = BASE + T * H * d * 2
+    assert _noalloc(L, B=B, ST=q_elem1, S0=None) == ALIAS
+    # the same problems through kda_chunk_fwd are refused the same way
+    assert _chunk(L, B=B, ST=q_elem1) == ALIAS
+    # and the ordinary argument checks hold
+    assert _noalloc(L, g_min=-6.0) == UNSUPPORTED
+    assert _noalloc(L, dk=96, dv=96) == UNSUPPORTED
+    assert _noalloc(L, q=BASE + 8) == ALIGN
+    assert _noalloc(L, o=BASE) == ALIAS
+    assert _noalloc(L, S0=S, ST=S + 4096) == ALIAS

@@ -953,13 +953,10 @@ struct ScanSmem {
     static constexpr uint32_t kStageBytes = Rec<D>::Shared + Rec<D>::Blk;  // shared part + own value block
     static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
     alignas(1024) unsigned char stage[kStages][kStageStride];
-    // the entering state of chunk c as the bf16 MMA operand, in sbuf[c % 2] (MN-major 64-byte
-    // swizzle, row = key channel): Q' S of chunk c may still read it while S of c + 1 is written
-    alignas(1024) unsigned char sbuf[2][D * kBV * 2];
-    uint64_t full[kStages];   // stage filled (arrive + bytes)
-    uint64_t empty[kStages];  // stage free: two arrivals, the consumers' and the MMAs' that read it
-    uint64_t mma_n;           // N S of the chunk completed (and all before it)
-    uint64_t mma_q[2];        // Q' S of chunk c completed, in mma_q[c % 2]
+    alignas(1024) unsigned char sbuf[D * kBV * 2];  // S block, bf16, MN-major 64-byte swizzle (row = key channel)
+    uint64_t full[kStages];                         // stage filled (arrive + bytes)
+    uint64_t empty[kStages];                        // stage released by the consumers
+    uint64_t mma_bar;                               // tcgen05 MMA batch completed
     uint32_t tmem_slot;
 };
 
@@ -995,8 +992,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     using SM = ScanSmem<D>;
     using R = Rec<D>;
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
-    // TMEM columns: [0, kBV) N S; [kBV (1 + c % 2), + kBV) Q' S of chunk c
-    constexpr uint32_t kTmemCols = 4 * kBV;
+    constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N S; [kBV, 2 kBV): Q' S
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // Column blocks past D / kBV (affine mode only) carry the transfer map instead of the
     // state: they start from the identity, add no Bm and write M_out.
@@ -1021,11 +1017,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 2);
+            mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.mma_n, 1);
-        mbar_init(&sm.mma_q[0], 1);
-        mbar_init(&sm.mma_q[1], 1);
+        mbar_init(&sm.mma_bar, 1);
         fence_mbar_init_cluster();
     }
     if (warp == 0)
@@ -1033,7 +1027,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = sm.tmem_slot;
+    const uint32_t tmem = sm.tmem_slot;  // columns [0, kBV): N S; [kBV, 2 kBV): Q' S
 
     if (warp == kScanWarps) {
         // ---------------- producer: one lane issues the bulk copies
@@ -1072,7 +1066,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 S[j + 2] = v.z;
                 S[j + 3] = v.w;
             }
-            store_state(sm.sbuf[0], row, S);
+            store_state(sm.sbuf, row, S);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -1080,36 +1074,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc::fence_after_sync();
 
         const uint32_t id_k = tc::idesc_bf16(128, kBV, false, true);  // A K-major, B MN-major
-        const bool orow = o && warp < 2;  // chunk rows 0..63 = TMEM lanes 0..63: warps 0 and 1
-        uint4 opre[kBV / 8];              // this row's O' of the chunk whose output is pending
-        // O = Q' S + O' of chunk c, run one chunk late while the tensor core works on the next
-        // chunk's N S (Q' S of c in TMEM, O' copied to registers before the stage was freed)
-        auto out_epilogue = [&](int c) {
-            if (!orow)
-                return;
-            mbar_wait_bounded(&sm.mma_q[c & 1], (c >> 1) & 1, status);
-            tc::fence_after_sync();
-            uint32_t y[kBV];
-            tc::ld_32x32b_x32(lane_addr + kBV * (1 + (c & 1)), y);
-            tc::wait_ld();
-            const int t = c * kC + row;
-            if (t < seq.len) {
-                uint4 *op = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
-#pragma unroll
-                for (int j = 0; j < kBV; j += 8) {
-                    const uint32_t ow[4] = {opre[j / 8].x, opre[j / 8].y, opre[j / 8].z, opre[j / 8].w};
-                    uint32_t r4[4];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float2 of = unpack_bf16x2(ow[p]);
-                        r4[p] = pack_bf16x2(of.x + __uint_as_float(y[j + 2 * p]), of.y + __uint_as_float(y[j + 2 * p + 1]));
-                    }
-                    op[j / 8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
-                }
-            }
-        };
-
-        uint32_t n_phase = 0;
+        const uint32_t sbuf_a = smem_u32(sm.sbuf);
+        uint32_t mma_phase = 0;
         for (int c = 0; c < NT; ++c) {
             const int s = c % kStages;
             if constexpr (kSave) {
@@ -1124,30 +1090,20 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             const unsigned char *st = sm.stage[s];
             const uint32_t st_a = smem_u32(st);
 
-            // N S first (the state chain waits for it), then Q' S (only the output needs it),
-            // each completing on its own barrier; the MMAs' reads of the stage end with Q' S,
-            // whose completion is also one of the two arrivals that free the stage (rows past
-            // N (D = 64) and past Q' are don't-cares)
+            // [N S | Q' S] in one round (rows past N (D = 64) and past Q' are don't-cares)
             if (tid == 0) {
                 tc::fence_after_sync();
-                const uint32_t sb = smem_u32(sm.sbuf[c & 1]);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t bd = tc::smem_desc(sb + ks * 1024, 0, 512, tc::kSw64);
+                    const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
                     const uint64_t an =
                         tc::smem_desc(st_a + R::Nm + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
-                    tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
-                }
-                tc::commit(&sm.mma_n);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t bd = tc::smem_desc(sb + ks * 1024, 0, 512, tc::kSw64);
                     const uint64_t aq =
                         tc::smem_desc(st_a + R::Qp + (ks >> 2) * (kC * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
-                    tc::mma_bf16(tmem + kBV * (1 + (c & 1)), aq, bd, id_k, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
                 }
-                tc::commit(&sm.mma_q[c & 1]);
-                tc::commit(&sm.empty[s]);
+                tc::commit(&sm.mma_bar);
             }
             // Diag(Gamma) S + Bm while the tensor core runs (stage data is in since `full`)
             if (srow) {
@@ -1165,20 +1121,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     }
                 }
             }
-            // the previous chunk's output while N S runs
-            if (c > 0)
-                out_epilogue(c - 1);
-            // this chunk's O' rows, so the stage can be freed at the end of the iteration
-            if (orow) {
-#pragma unroll
-                for (int j = 0; j < kBV; j += 8)
-                    opre[j / 8] = *reinterpret_cast<const uint4 *>(st + R::Shared + R::BmBlk + tc::mnmaj_sw64(row, j));
-            }
-            mbar_wait_bounded(&sm.mma_n, n_phase, status);
-            n_phase ^= 1;
+            mbar_wait_bounded(&sm.mma_bar, mma_phase, status);
+            mma_phase ^= 1;
             tc::fence_after_sync();
-            // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk.  sbuf[(c + 1) % 2]
-            // was last read by Q' S of chunk c - 1, which completed before N S of chunk c.
+
+            const unsigned char *blkp = st + R::Shared;
+            // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk
             if (srow) {
                 uint32_t d[kBV];
                 tc::ld_32x32b_x32(lane_addr, d);
@@ -1186,21 +1134,37 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kBV; ++j)
                     S[j] -= __uint_as_float(d[j]);
-                store_state(sm.sbuf[(c + 1) & 1], row, S);
+                store_state(sm.sbuf, row, S);
                 tc::fence_smem_to_async();
+            }
+            // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
+            if (o && warp < 2) {
+                uint32_t y[kBV];
+                tc::ld_32x32b_x32(lane_addr + kBV, y);
+                tc::wait_ld();
+                const int t = c * kC + row;
+                if (t < seq.len) {
+                    uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
+#pragma unroll
+                    for (int j = 0; j < kBV; j += 8) {
+                        const uint4 ou = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
+                        const uint32_t ow[4] = {ou.x, ou.y, ou.z, ou.w};
+                        uint32_t r4[4];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const float2 of = unpack_bf16x2(ow[p]);
+                            r4[p] = pack_bf16x2(of.x + __uint_as_float(y[j + 2 * p]),
+                                                of.y + __uint_as_float(y[j + 2 * p + 1]));
+                        }
+                        orow[j / 8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+                    }
+                }
             }
             tc::fence_before_sync();
             consumer_sync();
             tc::fence_after_sync();
             if (tid == 0)
-                mbar_arrive_local(&sm.empty[s]);  // the consumers' arrival: Bm and O' are read
-        }
-        if (NT > 0) {
-            out_epilogue(NT - 1);
-            // every MMA has completed before the tensor memory is released (commits track all
-            // earlier MMAs of the issuing thread)
-            if (tid == 0)
-                mbar_wait_bounded(&sm.mma_q[(NT - 1) & 1], ((NT - 1) >> 1) & 1, status);
+                mbar_arrive_local(&sm.empty[s]);
         }
 
         float *Sout = xfer ? M_out : S_T;
@@ -1441,8 +1405,8 @@ constexpr int kBwdSlots = 148;  // one CTA per SM of a 148-SM part
 template <int D>
 struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blocks
     static constexpr int CD = kC * D;
-    static constexpr int Kb = 0, Kh = Kb + CD, Qb = Kh + CD;
-    static constexpr int Bk = Qb + CD;   // diag(beta) Kbar, later dBk
+    static constexpr int Kb = 0, Kh = Kb + CD;
+    static constexpr int Bk = Kh + CD;   // diag(beta) Kbar, later dBk
     static constexpr int Bv = Bk + CD;   // diag(beta) V, later dBv
     static constexpr int W = Bv + CD;    // W, then dW, then the pairwise dq
     static constexpr int U = W + CD;     // Utilde, U, then dk
@@ -1635,7 +1599,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *const sseg = bsm + SL::seg, *const sred = bsm + SL::red;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *sl = scratch + (size_t)blockIdx.x * L::floats;
-    float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Qb = sl + L::Qb, *const Bk = sl + L::Bk;
+    float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Bk = sl + L::Bk;
     float *const Bv = sl + L::Bv, *const W = sl + L::W, *const U = sl + L::U, *const dOs = sl + L::dO;
     float *const dU = sl + L::dU, *const dKh = sl + L::dKh, *const dQb = sl + L::dQb, *const Gp = sl + L::Gp;
     float *const Xg = sl + L::X;
@@ -1698,7 +1662,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float kv = sk[r * LDD + c];
             Kb[e] = kv * e1;
             Kh[e] = kv * eh;
-            Qb[e] = sq[r * LDD + c] * e1;
             Bk[e] = sbeta[r] * kv * e1;
             Bv[e] *= sbeta[r];
         }

@@ -6,8 +6,10 @@
 One step = one chunked forward over the 64K-stage batch (B=1, H=32, T=65536,
 dk=dv=128, bf16 inputs, fp32 state, the 5% a=+8 slice): gate, cumulative decay,
 dense 16-token tile products, WY/UT solve and the state scan, i.e. the whole hot path.
-It is issued as kda_chunk_fwd_prep + kda_chunk_fwd_scan (the two launches kda_chunk_fwd
-makes) so that CUDA events between them time each kernel during the timed steps.
+It is issued as kda_chunk_fwd_prep + kda_chunk_fwd_scan (the same launches kda_chunk_fwd
+makes: the gate table and the prep, then the scan) so that CUDA events between them time
+each stage during the timed steps.  The 8K and 1M context stages are timed too, under
+``stages``.
 Inputs (2.69 GB) exceed the 126 MB L2, so no flush is needed between steps.
 The log-sigmoid ablation (element-wise diagonal tiles) is timed on the same inputs and
 reported under ``ablation``.
@@ -395,7 +397,7 @@ def time_stage(kda, sw, rank, world, device, hbm_peak, bf16_peak, peak_kind, arg
         ms = time_steps(step, steps, 3, world, device)
     assert kda.kda_device_status(device) == 0
     out = {"workload": sw.name, "B": B, "T": sw.T, "H": H, "dk": D, "dv": D, "steps": steps,
-           "calls_per_step": len(segs), "gpu_launches_per_step": 2 * len(segs),
+           "calls_per_step": len(segs), "gpu_launches_per_step": 3 * len(segs),
            "l2": "inputs exceed the 126 MB L2; no flush"}
     out.update(stage_metrics(B * sw.T, B * sw.T * H, B * H, ms, world, hbm_peak, bf16_peak, peak_kind))
     out["clocks"] = clk.summary()
@@ -427,7 +429,7 @@ def run_libkda(args):
     need = kda.kda_chunk_fwd_workspace(B, T, H, D, D)
     ws = torch.empty(need, dtype=torch.uint8, device=device)
 
-    # One step is kda_chunk_fwd issued as its two stages (the same two launches the single
+    # One step is kda_chunk_fwd issued as its two stages (the same launches the single
     # call makes), with CUDA events around each on the launching stream during the timed
     # steps, so each kernel's own duration is measured live.
     stream = torch.cuda.current_stream(device)
@@ -507,7 +509,7 @@ def run_libkda(args):
         assert kda.kda_device_status(device) == 0
         vl = {"workload": f"packed 64K axis, H={H} d={D}: {Nd} documents, log-uniform lengths 16..16384 "
                           f"(min {int(lengths.min())}, max {int(lengths.max())})",
-              "ms_per_step": vl_ms, "value": world * tokens / (vl_ms * 1e-3), "unit": UNIT, "gpu_launches_per_step": 3,
+              "ms_per_step": vl_ms, "value": world * tokens / (vl_ms * 1e-3), "unit": UNIT, "gpu_launches_per_step": 4,
               "roofline_path_frac": (token_heads * BYTES_PER_TOKEN_HEAD + 2 * Nd * H * D * D * 4) / (vl_ms * 1e-3)
               / 1e9 / hbm_peak}
 
@@ -529,7 +531,7 @@ def run_libkda(args):
         assert kda.kda_device_status(device) == 0
         spl = {"workload": f"one {T}-token sequence in {world} segment(s) of {seg}, H={H} d={D}",
                "ms_per_step": sp_ms, "value": tokens / (sp_ms * 1e-3), "unit": UNIT, "segments": world,
-               "gpu_launches_per_step": 4, "collectives_per_step": 2 if world > 1 else 0}
+               "gpu_launches_per_step": 5, "collectives_per_step": 2 if world > 1 else 0}
         del sd, xs
 
     # ---- backward: the gradients of every input for the same workload and inputs, one
@@ -557,10 +559,10 @@ def run_libkda(args):
         bwd = {"what": "kda_chunk_bwd: dq, dk, dv, da, dbeta, dS0 (float32) from dL/do",
                "cpu_baseline": bwd_cpu,
                "ms_per_step": bwd_ms, "value": world * tokens / (bwd_ms * 1e-3), "unit": UNIT,
-               "gpu_launches_per_step": 4, "vs_forward_time": bwd_ms / ms, "workspace_bytes": ws_b.numel(),
+               "gpu_launches_per_step": 5, "vs_forward_time": bwd_ms / ms, "workspace_bytes": ws_b.numel(),
                "roofline": {"bound": "hbm", "achieved": bwd_gbs, "peak": hbm_peak, "unit": "GB/s",
                             "frac": bwd_gbs / hbm_peak, "peak_kind": peak_kind,
-                            "kernels": "the whole backward path (four launches)",
+                            "kernels": "the whole backward path (five launches)",
                             "algorithmic_bytes_per_step": bwd_bytes},
                "dominant_kernel": {"kernel": "bwd_chunk_kernel (per-chunk gradients)",
                                    "algorithmic_bytes_per_token_head": BWD_CHUNK_BYTES_PER_TOKEN_HEAD,
@@ -582,7 +584,7 @@ def run_libkda(args):
             assert kda.kda_device_status(device) == 0
             bwd["packed"] = {"workload": f"the varlen leg's {len(lengths)} documents on the 64K axis",
                              "ms_per_step": bvl_ms, "value": world * tokens / (bvl_ms * 1e-3), "unit": UNIT,
-                             "gpu_launches_per_step": 5}
+                             "gpu_launches_per_step": 6}
             del ws_vb, gv
         del dO
 
@@ -697,10 +699,10 @@ def run_libkda(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "how": "kda_chunk_fwd from pinned host buffers; upload, compute and read-back on three "
                        "streams, double-buffered, so step i's read-back overlaps step i+1's upload"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "roofline": {"bound": "hbm", "achieved": prep_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": prep_gbs / hbm_peak, "peak_kind": peak_kind,
-                     "kernel": "prep_kernel (dominant; one launch per step)",
+                     "kernel": "prep_kernel (dominant; one launch per step, timed with the 3-us gate-table launch before it)",
                      "algorithmic_bytes_per_launch": prep_bytes, "ms_per_launch": prep_ms,
                      "traffic": None if prep_traffic is None else prep_traffic * token_heads,
                      "path": {"kernels": "prep + scan (one kda_chunk_fwd)", "achieved": achieved_gbs,

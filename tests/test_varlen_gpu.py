@@ -87,3 +87,53 @@ def test_invalid_cu_seqlens_is_reported_on_device():
     assert torch.equal(ST.cpu(), S0)              # nothing ran: the state passes through
     assert not o.any()                            # and no output was written
     assert kda.kda_device_status() == 0
+
+
+@pytest.mark.parametrize("gate", [kda.KDA_GATE_BOUNDED, kda.KDA_GATE_LOGSIGMOID])
+def test_varlen_tail_chunk_ignores_the_next_sequence(gate):
+    """A sequence whose last chunk is partial gets the next sequence's tokens in the rest of
+    that chunk's tiles (the tensor copies read the packed axis); the prep must mask them.  With
+    the next sequence all NaN, the first sequence's o and S_T must equal a packed batch of the
+    first sequence alone, bit for bit; lengths 70 and 1 leave 58 and 63 foreign rows in the
+    tail chunk."""
+    H, D = 2, 128
+    for L0 in (70, 1):
+        x, S0, _ = _packed([L0, 90], H, D, seed=1240 + L0)
+        cu2 = torch.tensor([0, L0, L0 + 90], dtype=torch.int32, device="cuda")
+        cu1 = torch.tensor([0, L0], dtype=torch.int32, device="cuda")
+        d = to_dev(x)
+        poisoned = {n: d[n][0].clone() for n in NAMES}
+        for n in NAMES:
+            poisoned[n][L0:] = float("nan")
+        o2, S2 = kda.kda_chunk_fwd_varlen(*(poisoned[n] for n in NAMES), cu2, G_MIN, gate, S0=S0.cuda())
+        o1, S1 = kda.kda_chunk_fwd_varlen(*(d[n][0][:L0].contiguous() for n in NAMES), cu1, G_MIN, gate,
+                                          S0=S0[:1].cuda())
+        torch.cuda.synchronize()
+        assert kda.kda_device_status() == 0
+        assert torch.equal(o2[:L0], o1), L0
+        assert torch.equal(S2[0], S1[0]), L0
+        assert torch.isnan(S2[1]).any()          # the second sequence did run on its NaN tokens
+
+
+def test_varlen_backward_tail_chunk_ignores_the_next_sequence():
+    """The same for the packed backward: with the next sequence all NaN (inputs and dL/do),
+    every gradient of the first sequence equals the packed backward of that sequence alone."""
+    H, D, L0 = 2, 128, 70
+    x, S0, _ = _packed([L0, 90], H, D, seed=1250)
+    cu2 = torch.tensor([0, L0, L0 + 90], dtype=torch.int32, device="cuda")
+    cu1 = torch.tensor([0, L0], dtype=torch.int32, device="cuda")
+    d = to_dev(x)
+    gen = torch.Generator().manual_seed(1251)
+    dO = torch.randn((L0 + 90, H, D), generator=gen).to(torch.bfloat16).cuda()
+    poisoned = {n: d[n][0].clone() for n in NAMES}
+    dOp = dO.clone()
+    for t in list(poisoned.values()) + [dOp]:
+        t[L0:] = float("nan")
+    g2 = kda.kda_chunk_bwd_varlen(*(poisoned[n] for n in NAMES), dOp, cu2, G_MIN, S0=S0.cuda())
+    g1 = kda.kda_chunk_bwd_varlen(*(d[n][0][:L0].contiguous() for n in NAMES), dO[:L0].contiguous(), cu1, G_MIN,
+                                  S0=S0[:1].cuda())
+    torch.cuda.synchronize()
+    assert kda.kda_device_status() == 0
+    for n in ("dq", "dk", "dv", "da", "dbeta"):
+        assert torch.equal(g2[n][:L0], g1[n]), n
+    assert torch.equal(g2["dS0"][0], g1["dS0"][0])

@@ -1419,10 +1419,27 @@ struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blo
     static constexpr int floats = X + kC * kC;
 };
 
-constexpr int kGTM = 64, kGTK = 32;  // output tiles of 64 x TN (TN = 64 or 128), K steps of 32
-constexpr int kGLDA = kGTK + 4;       // conflict-free fragment reads (B: TN + 8)
-constexpr int kGStage = kGTM * kGLDA + kGTK * (128 + 8);
-constexpr int kGPA = kGTM * kGTK / kBwdThreads;
+// Operand sources of cta_gemm.  "K" = consecutive along the contraction index, "M" / "N" =
+// consecutive along the output row / column index.  Global ones (the scratch slot, the saved
+// states) are staged into shared memory by 16-byte cp.async copies; shared ones are read in
+// place.
+enum GemmSrc : int {
+    kGlobK,  // A(i, k) = p[i * ld + k]  or  B(k, j) = p[j * ld + k]
+    kGlobMN, // A(i, k) = p[k * ld + i]  or  B(k, j) = p[k * ld + j]
+    kSmemK,  // as kGlobK, in shared memory
+    kSmemM,  // A only: as kGlobMN, in shared memory
+};
+
+constexpr int kGKS = 16;    // contraction step per pipeline stage
+constexpr int kGStages = 3; // cp.async ring depth
+// one stage: A 64 x 16 (K-consecutive rows padded to 20, or 16 x 64 padded to 72), B 16 x TN
+// (N-consecutive rows padded to TN + 8) or TN x 16 (K-consecutive, 16-byte chunks XOR-swizzled)
+constexpr int kGStageA = kC * (kGKS + 4);
+constexpr int kGStageB = kGKS * (128 + 8);
+constexpr int kGStageFloats = kGStageA + kGStageB;
+constexpr int kGStage = kGStages * kGStageFloats;
+static_assert(kGKS * 72 <= kGStageA && 128 * kGKS <= kGStageB, "stage layouts fit");
+static_assert(2 * 16 * 256 <= kGStage, "the partial-sum exchange fits the ring");
 
 template <int D>
 struct BwdSmem {  // float offsets in shared memory
@@ -1432,101 +1449,186 @@ struct BwdSmem {  // float offsets in shared memory
     static constexpr int Ap = G + kC * LDD, P = Ap + kC * LDC, T = P + kC * LDC;
     static constexpr int dT = T + kC * LDC;  // scratch of the block solve, then dT, then dP
     static constexpr int dA = dT + kC * LDC;
-    static constexpr int stage = dA + kC * LDC;
+    static constexpr int stage = dA + kC * LDC;  // cta_gemm's ring (16-byte aligned)
+    static constexpr int seg = stage;  // after the contractions: row-segment sums of dG, then of dKhat * Khat
     static constexpr int beta = stage + kGStage;
     static constexpr int dGam = beta + kC;
-    static constexpr int seg = dGam + D;  // row-segment sums: of dG, then of dKhat * Khat
-    static constexpr int red = seg + 2 * kBwdThreads;  // per-warp partial sums of dA_log
+    static constexpr int red = dGam + D;  // per-warp partial sums of dA_log
     static constexpr int floats = red + kBwdWarps;
     static constexpr size_t bytes = (size_t)floats * 4;
+    static_assert(stage % 4 == 0, "cp.async destinations are 16-byte aligned");
+    static_assert(2 * kBwdThreads <= kGStage, "segment sums fit the ring");
     static_assert(bytes <= 232448, "shared memory per block");
 };
 
-// Strided fp32 matrix view: element (i, j) at p[i * rs + j * cs] (shared or global memory).
-struct MatV {
-    const float *p;
-    int rs, cs;
-    __device__ __forceinline__ float at(int i, int j) const { return p[(int64_t)i * rs + (int64_t)j * cs]; }
-};
-
-// C[M x N] = A[M x K] B[K x N] on the whole CTA (M, N, K multiples of 64, TN, 32); every
-// output element goes to epi(i, j, value) exactly once, from a thread fixed by (M, N).
-// Operands are staged through shared memory as TF32 in 64 x 32 / 32 x TN tiles, the next
-// tile fetched into registers while the tensor cores work on the current one; warp w
-// computes rows 16 (w / 4) .. + 16 and columns TN/4 (w % 4) .. + TN/4 of each 64 x TN tile.
-template <int TN, class Epi>
-__device__ void cta_gemm(int M, int N, int K, MatV A, MatV B, uint32_t *stage, Epi epi)
+template <int TN>
+__device__ __forceinline__ int gemm_bk_off(int j, int k)  // (k, j) of a staged K-consecutive B
 {
-    constexpr int kGTN = TN, kGLDB = TN + 8, kGPB = kGTK * TN / kBwdThreads, NF = TN / 32;
-    uint32_t *sA = stage, *sB = stage + kGTM * kGLDA;
+    return j * kGKS + ((((k >> 2) ^ (j >> 1)) & 3) << 2) + (k & 3);
+}
+
+// ldmatrix of four 8 x 4 fp32 blocks (each row 16 bytes): thread T receives element
+// (T / 4, T % 4) of block q in r[q]; lane l gives the address of row l % 8 of block l / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float *row_ptr)
+{
+    ldmatrix_x4(r, row_ptr);
+}
+
+// C[64 x TN] = A[64 x K] B[K x TN] on the whole CTA (K a multiple of 16); every output pair
+// (j even) goes to epi(i, j, c_ij, c_i,j+1) exactly once.  With acc_in, the pair handed over is
+// acc_in[i, j..j+1] + sign * C (all of a thread's acc_in values are loaded together, before its
+// first store, so a read-modify-write of one array costs one memory round trip, not one per
+// element).  TF32 mma.sync with fp32
+// accumulation; operands enter the tensor cores as their fp32 bit patterns (the hardware
+// uses the TF32 part).  The contraction is split between two groups of eight warps: per
+// 16-wide step, group 0 takes its first 8 indices and group 1 the rest, each warp a 32 x TN/4
+// tile, and the two partial sums meet in shared memory at the end.  The global operands move
+// through a three-stage ring of shared-memory tiles, one CTA barrier per step.  Starts and
+// ends with every thread past a barrier.
+template <int TN, int SA, int SB, class Epi>
+__device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb, float *stage, Epi epi,
+                         const float *acc_in = nullptr, int ld_in = 0, float sign = 1.f)
+{
+    static_assert(TN == 64 || TN == 128, "output tile width");
+    static_assert(SB != kSmemM, "B in place is K-consecutive");
+    constexpr int NF = TN / 32, LDBN = TN + 8;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int wm = (warp >> 2) * 16, wn = (warp & 3) * (TN / 4);
-    float ra[kGPA], rb[kGPB];
-    auto fetch = [&](int m0, int n0, int k0) {
-#pragma unroll
-        for (int p = 0; p < kGPA; ++p) {
-            const int e = tid + p * kBwdThreads;
-            const int i = A.cs == 1 ? e / kGTK : e % kGTM, kk = A.cs == 1 ? e % kGTK : e / kGTM;
-            ra[p] = A.at(m0 + i, k0 + kk);
+    const int grp = warp >> 3, wl = warp & 7;
+    const int wm = (wl >> 2) * 32, wn = (wl & 3) * (TN / 4), kk = grp * 8;
+    const int lr = lane & 7, lq = lane >> 3;  // ldmatrix: row within a block, block
+    const int nk = K / kGKS;
+    auto issue = [&](int s, int slot) {
+        float *sA = stage + slot * kGStageFloats, *sB = sA + kGStageA;
+        const int k0 = s * kGKS;
+        if constexpr (SA == kGlobK) {
+            if (tid < kC * 4) {
+                const int i = tid >> 2, c = tid & 3;
+                cp_async_16(sA + i * (kGKS + 4) + 4 * c, A + (size_t)i * lda + k0 + 4 * c);
+            }
+        } else if constexpr (SA == kGlobMN) {
+            if (tid < kGKS * (kC / 4)) {
+                const int k = tid / (kC / 4), c = tid % (kC / 4);
+                cp_async_16(sA + k * 72 + 4 * c, A + (size_t)(k0 + k) * lda + 4 * c);
+            }
         }
-#pragma unroll
-        for (int p = 0; p < kGPB; ++p) {
-            const int e = tid + p * kBwdThreads;
-            const int kk = B.cs == 1 ? e / kGTN : e % kGTK, j = B.cs == 1 ? e % kGTN : e / kGTK;
-            rb[p] = B.at(k0 + kk, n0 + j);
+        if constexpr (SB == kGlobMN) {
+            if (tid < kGKS * (TN / 4)) {
+                const int k = tid / (TN / 4), c = tid % (TN / 4);
+                cp_async_16(sB + k * LDBN + 4 * c, B + (size_t)(k0 + k) * ldb + 4 * c);
+            }
+        } else if constexpr (SB == kGlobK) {
+            if (tid < TN * 4) {
+                const int j = tid >> 2, c = tid & 3;
+                cp_async_16(sB + gemm_bk_off<TN>(j, 4 * c), B + (size_t)j * ldb + k0 + 4 * c);
+            }
         }
     };
-    fetch(0, 0, 0);
-    for (int m0 = 0; m0 < M; m0 += kGTM)
-        for (int n0 = 0; n0 < N; n0 += kGTN) {
-            float acc[NF][4] = {};
-            for (int k0 = 0; k0 < K; k0 += kGTK) {
-                __syncthreads();  // the previous tile's readers are done
+    // A fragments of the warp's two 16-row blocks at contraction offset kk of step k0
+    auto load_a = [&](const float *sA, int k0, uint32_t (&af)[2][4]) {
 #pragma unroll
-                for (int p = 0; p < kGPA; ++p) {
-                    const int e = tid + p * kBwdThreads;
-                    const int i = A.cs == 1 ? e / kGTK : e % kGTM, kk = A.cs == 1 ? e % kGTK : e / kGTM;
-                    sA[i * kGLDA + kk] = to_tf32(ra[p]);
+        for (int mf = 0; mf < 2; ++mf) {
+            const int r0 = wm + mf * 16;
+            if constexpr (SA == kGlobK || SA == kSmemK) {
+                const int row = r0 + (lq & 1) * 8 + lr, col = kk + (lq >> 1) * 4;
+                ldsm_x4(af[mf], SA == kGlobK ? sA + row * (kGKS + 4) + col : A + row * lda + k0 + col);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = r0 + g + (q & 1) * 8, k = kk + t + (q >> 1) * 4;
+                    af[mf][q] = __float_as_uint(SA == kGlobMN ? sA[k * 72 + i] : A[(k0 + k) * lda + i]);
                 }
-#pragma unroll
-                for (int p = 0; p < kGPB; ++p) {
-                    const int e = tid + p * kBwdThreads;
-                    const int kk = B.cs == 1 ? e / kGTN : e % kGTK, j = B.cs == 1 ? e % kGTN : e / kGTK;
-                    sB[kk * kGLDB + j] = to_tf32(rb[p]);
-                }
-                __syncthreads();
-                // the next tile, in this output tile or the next one
-                if (k0 + kGTK < K)
-                    fetch(m0, n0, k0 + kGTK);
-                else if (n0 + kGTN < N)
-                    fetch(m0, n0 + kGTN, 0);
-                else if (m0 + kGTM < M)
-                    fetch(m0 + kGTM, 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < kGTK; kk += 8) {
-                    uint32_t af[4];
-                    af[0] = sA[(wm + g) * kGLDA + kk + t];
-                    af[1] = sA[(wm + g + 8) * kGLDA + kk + t];
-                    af[2] = sA[(wm + g) * kGLDA + kk + t + 4];
-                    af[3] = sA[(wm + g + 8) * kGLDA + kk + t + 4];
-#pragma unroll
-                    for (int nt = 0; nt < NF; ++nt) {
-                        uint32_t bf[2];
-                        bf[0] = sB[(kk + t) * kGLDB + wn + nt * 8 + g];
-                        bf[1] = sB[(kk + t + 4) * kGLDB + wn + nt * 8 + g];
-                        mma_tf32_1688(acc[nt], af, bf);
-                    }
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NF; ++nt) {
-                const int i = m0 + wm + g, j = n0 + wn + nt * 8 + 2 * t;
-                epi(i, j, acc[nt][0]);
-                epi(i, j + 1, acc[nt][1]);
-                epi(i + 8, j, acc[nt][2]);
-                epi(i + 8, j + 1, acc[nt][3]);
             }
         }
+    };
+    auto load_b = [&](const float *sB, int k0, uint32_t (&bf)[NF][2]) {
+        if constexpr (SB == kGlobMN) {
+#pragma unroll
+            for (int nf = 0; nf < NF; ++nf) {
+                const int j = wn + nf * 8 + g;
+                bf[nf][0] = __float_as_uint(sB[(kk + t) * LDBN + j]);
+                bf[nf][1] = __float_as_uint(sB[(kk + t + 4) * LDBN + j]);
+            }
+        } else {
+            // rows j (K-consecutive): block q of an x4 = (column block, k half)
+            auto addr = [&](int j, int k) -> const float * {
+                return SB == kGlobK ? sB + gemm_bk_off<TN>(j, k) : B + j * ldb + k0 + k;
+            };
+            if constexpr (NF == 4) {
+#pragma unroll
+                for (int hk = 0; hk < 2; ++hk) {
+                    uint32_t r[4];
+                    ldsm_x4(r, addr(wn + lq * 8 + lr, kk + hk * 4));
+#pragma unroll
+                    for (int nf = 0; nf < 4; ++nf)
+                        bf[nf][hk] = r[nf];
+                }
+            } else {
+                uint32_t r[4];
+                ldsm_x4(r, addr(wn + (lq & 1) * 8 + lr, kk + (lq >> 1) * 4));
+                bf[0][0] = r[0], bf[1][0] = r[1], bf[0][1] = r[2], bf[1][1] = r[3];
+            }
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < kGStages - 1; ++s) {
+        if (s < nk)
+            issue(s, s);
+        cp_async_commit();
+    }
+    float acc[2][NF][4] = {};
+    for (int s = 0; s < nk; ++s) {
+        cp_async_wait<kGStages - 2>();
+        __syncthreads();  // stage s is in for every thread; stage s - 1 is no longer read
+        if (s + kGStages - 1 < nk)
+            issue(s + kGStages - 1, (s + kGStages - 1) % kGStages);
+        cp_async_commit();
+        const float *sA = stage + (s % kGStages) * kGStageFloats, *sB = sA + kGStageA;
+        uint32_t af[2][4], bf[NF][2];
+        load_a(sA, s * kGKS, af);
+        load_b(sB, s * kGKS, bf);
+#pragma unroll
+        for (int mf = 0; mf < 2; ++mf)
+#pragma unroll
+            for (int nf = 0; nf < NF; ++nf)
+                mma_tf32_1688(acc[mf][nf], af[mf], bf[nf]);
+    }
+    float2 prev[NF][2];
+    if (acc_in) {
+#pragma unroll
+        for (int nf = 0; nf < NF; ++nf)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                prev[nf][hh] = *reinterpret_cast<const float2 *>(acc_in + (wm + grp * 16 + g + 8 * hh) * ld_in +
+                                                                 wn + nf * 8 + 2 * t);
+    }
+    // partial sums: group g finishes row block mf = g of its tile and hands the other over
+    cp_async_wait<0>();
+    __syncthreads();  // the ring is free
+    float *xch = stage;  // [2][NF * 4][256]: row block, value, thread of the group
+    const int gt = wl * 32 + lane;
+#pragma unroll
+    for (int nf = 0; nf < NF; ++nf)
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            xch[((1 - grp) * NF * 4 + nf * 4 + v) * 256 + gt] = grp ? acc[0][nf][v] : acc[1][nf][v];
+    __syncthreads();
+#pragma unroll
+    for (int nf = 0; nf < NF; ++nf) {
+        float c[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            c[v] = (grp ? acc[1][nf][v] : acc[0][nf][v]) + xch[(grp * NF * 4 + nf * 4 + v) * 256 + gt];
+        const int i = wm + grp * 16 + g, j = wn + nf * 8 + 2 * t;
+        if (acc_in) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                c[2 * hh] = fmaf(sign, c[2 * hh], prev[nf][hh].x);
+                c[2 * hh + 1] = fmaf(sign, c[2 * hh + 1], prev[nf][hh].y);
+            }
+        }
+        epi(i, j, c[0], c[1]);
+        epi(i + 8, j, c[2], c[3]);
+    }
     __syncthreads();
 }
 
@@ -1594,7 +1696,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *const sq = bsm + SL::q, *const sk = bsm + SL::k, *const sG = bsm + SL::G;
     float *const sAp = bsm + SL::Ap, *const sP = bsm + SL::P, *const sT = bsm + SL::T;
     float *const sdT = bsm + SL::dT, *const sdA = bsm + SL::dA;
-    uint32_t *const stage = reinterpret_cast<uint32_t *>(bsm + SL::stage);
+    float *const stage = bsm + SL::stage;
     float *const sbeta = bsm + SL::beta, *const sdGam = bsm + SL::dGam;
     float *const sseg = bsm + SL::seg, *const sred = bsm + SL::red;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1627,21 +1729,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float scale = A_log ? __expf(A_log[h]) : 1.0f;
         const float *tab = gtab + (A_log ? (size_t)h * kGateTableEntries : 0);
 
-        // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da
-#pragma unroll 4
-        for (int e = tid; e < CD; e += kBwdThreads) {
-            const int r = e / D, c = e % D;
+        // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da; eight channels
+        //    per item (16-byte loads)
+        for (int it = tid; it < CD / 8; it += kBwdThreads) {
+            const int r = it / (D / 8), c = (it % (D / 8)) * 8, e = r * D + c;
             const bool ok = r < n;
             const size_t gi = (size_t)tix(ok ? r : 0) * D + c;
-            const __nv_bfloat16 ab = ag[gi];
-            const float av = scale * __bfloat162float(ab);
-            const float sg = __fdividef(1.f, 1.f + __expf(-av));
-            sq[r * LDD + c] = ok ? __bfloat162float(qg[gi]) : 0.f;
-            sk[r * LDD + c] = ok ? __bfloat162float(kg[gi]) : 0.f;
-            sG[r * LDD + c] = ok ? __ldg(tab + __bfloat16_as_ushort(ab)) : 0.f;
-            Gp[e] = g_min * sg * (1.f - sg) * scale;
-            Bv[e] = ok ? __bfloat162float(vg[gi]) : 0.f;
-            dOs[e] = ok ? __bfloat162float(dOg[gi]) : 0.f;
+            const uint4 au = __ldg(reinterpret_cast<const uint4 *>(ag + gi));
+            uint4 qu = __ldg(reinterpret_cast<const uint4 *>(qg + gi)), ku = __ldg(reinterpret_cast<const uint4 *>(kg + gi));
+            uint4 vu = __ldg(reinterpret_cast<const uint4 *>(vg + gi)), du = __ldg(reinterpret_cast<const uint4 *>(dOg + gi));
+            if (!ok)
+                qu = ku = vu = du = make_uint4(0u, 0u, 0u, 0u);
+            const float bt = ok ? __bfloat162float(betag[tix(r)]) : 0.f;  // Bv = beta v
+            const uint32_t aw[4] = {au.x, au.y, au.z, au.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w},
+                           kw[4] = {ku.x, ku.y, ku.z, ku.w}, vw[4] = {vu.x, vu.y, vu.z, vu.w},
+                           dw[4] = {du.x, du.y, du.z, du.w};
+            float fq[8], fk[8], fg[8], fp[8], fv[8], fd[8];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 q2 = unpack_bf16x2(qw[w]), k2 = unpack_bf16x2(kw[w]), v2 = unpack_bf16x2(vw[w]),
+                             d2 = unpack_bf16x2(dw[w]), a2 = unpack_bf16x2(aw[w]);
+                fq[2 * w] = q2.x, fq[2 * w + 1] = q2.y;
+                fk[2 * w] = k2.x, fk[2 * w + 1] = k2.y;
+                fv[2 * w] = bt * v2.x, fv[2 * w + 1] = bt * v2.y;
+                fd[2 * w] = d2.x, fd[2 * w + 1] = d2.y;
+                fg[2 * w] = ok ? __ldg(tab + (aw[w] & 0xffffu)) : 0.f;
+                fg[2 * w + 1] = ok ? __ldg(tab + (aw[w] >> 16)) : 0.f;
+                const float s0 = __fdividef(1.f, 1.f + __expf(-scale * a2.x)), s1 = __fdividef(1.f, 1.f + __expf(-scale * a2.y));
+                fp[2 * w] = g_min * s0 * (1.f - s0) * scale;
+                fp[2 * w + 1] = g_min * s1 * (1.f - s1) * scale;
+            }
+#pragma unroll
+            for (int h4 = 0; h4 < 8; h4 += 4) {
+                *reinterpret_cast<float4 *>(sq + r * LDD + c + h4) = make_float4(fq[h4], fq[h4 + 1], fq[h4 + 2], fq[h4 + 3]);
+                *reinterpret_cast<float4 *>(sk + r * LDD + c + h4) = make_float4(fk[h4], fk[h4 + 1], fk[h4 + 2], fk[h4 + 3]);
+                *reinterpret_cast<float4 *>(sG + r * LDD + c + h4) = make_float4(fg[h4], fg[h4 + 1], fg[h4 + 2], fg[h4 + 3]);
+                *reinterpret_cast<float4 *>(Gp + e + h4) = make_float4(fp[h4], fp[h4 + 1], fp[h4 + 2], fp[h4 + 3]);
+                *reinterpret_cast<float4 *>(Bv + e + h4) = make_float4(fv[h4], fv[h4 + 1], fv[h4 + 2], fv[h4 + 3]);
+                *reinterpret_cast<float4 *>(dOs + e + h4) = make_float4(fd[h4], fd[h4 + 1], fd[h4 + 2], fd[h4 + 3]);
+            }
         }
         for (int r = tid; r < kC; r += kBwdThreads)
             sbeta[r] = r < n ? __bfloat162float(betag[tix(r)]) : 0.f;
@@ -1663,7 +1789,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             Kb[e] = kv * e1;
             Kh[e] = kv * eh;
             Bk[e] = sbeta[r] * kv * e1;
-            Bv[e] *= sbeta[r];
         }
         if (warp < kTiles * (kTiles + 1) / 2) {
             int I = 0, J = warp;  // warp -> (I, J), J <= I, row by row
@@ -1732,16 +1857,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             __syncthreads();
         }
         // 6. dense contractions
-        const MatV Tn{sT, LDC, 1}, Tt{sT, 1, LDC};
-        cta_gemm<D>(kC, D, kC, Tn, MatV{Bk, D, 1}, stage, [&](int i, int j, float x) { W[i * D + j] = x; });
-        cta_gemm<D>(kC, D, kC, Tn, MatV{Bv, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] = x; });
-        cta_gemm<D>(kC, D, D, MatV{W, D, 1}, MatV{S, D, 1}, stage, [&](int i, int j, float x) { U[i * D + j] -= x; });
-        cta_gemm<D>(kC, D, D, MatV{Kh, D, 1}, MatV{dSn, D, 1}, stage, [&](int i, int j, float x) { dU[i * D + j] = x; });
-        cta_gemm<D>(kC, D, kC, MatV{sP, 1, LDC}, MatV{dOs, D, 1}, stage,
-                 [&](int i, int j, float x) { dU[i * D + j] += x; });
-        cta_gemm<D>(kC, D, D, MatV{U, D, 1}, MatV{dSn, 1, D}, stage, [&](int i, int j, float x) { dKh[i * D + j] = x; });
-        cta_gemm<D>(kC, D, D, MatV{dOs, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { dQb[i * D + j] = x; });
-        cta_gemm<D>(kC, D, D, MatV{dU, D, 1}, MatV{S, 1, D}, stage, [&](int i, int j, float x) { W[i * D + j] = -x; });
+        // A operand T: kSmemK over sT; T^T: kSmemM over sT.  Row-major 64 x D blocks of the slot
+        // are kGlobK as A, kGlobMN as B; S and dS' (row-major D x D) are kGlobMN as B, and their
+        // transposes kGlobK.
+        auto st2 = [](float *p, float x0, float x1) { *reinterpret_cast<float2 *>(p) = make_float2(x0, x1); };
+        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, x0, x1); });
+        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, Bv, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); });
+        cta_gemm<D, kGlobK, kGlobMN>(D, W, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); }, U, D, -1.f);
+        cta_gemm<D, kGlobK, kGlobMN>(D, Kh, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); });
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sP, LDC, dOs, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); }, dU, D);
+        cta_gemm<D, kGlobK, kGlobK>(D, U, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dKh + i * D + j, x0, x1); });
+        cta_gemm<D, kGlobK, kGlobK>(D, dOs, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(dQb + i * D + j, x0, x1); });
+        cta_gemm<D, kGlobK, kGlobK>(D, dU, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, -x0, -x1); });
         float *const dW = W;
         // dGamma_i = sum_j dS'_ij S_ij, warp per row
 #pragma unroll
@@ -1757,23 +1884,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0)
                 sdGam[i] = acc;
         }
-        cta_gemm<64>(kC, kC, D, MatV{dW, D, 1}, MatV{Bk, 1, D}, stage,
-                 [&](int i, int j, float x) { sdT[i * LDC + j] = x; });
-        cta_gemm<64>(kC, kC, D, MatV{dU, D, 1}, MatV{Bv, 1, D}, stage,
-                 [&](int i, int j, float x) { sdT[i * LDC + j] += x; });
-        cta_gemm<D>(kC, D, kC, Tt, MatV{dW, D, 1}, stage, [&](int i, int j, float x) { Bk[i * D + j] = x; });
-        cta_gemm<D>(kC, D, kC, Tt, MatV{dU, D, 1}, stage, [&](int i, int j, float x) { Bv[i * D + j] = x; });
-        cta_gemm<64>(kC, kC, kC, MatV{sdT, LDC, 1}, Tt, stage, [&](int i, int j, float x) { Xg[i * kC + j] = x; });
-        cta_gemm<64>(kC, kC, kC, Tt, MatV{Xg, kC, 1}, stage,
-                 [&](int i, int j, float x) { sdA[i * LDC + j] = j < i ? -x : 0.f; });
-        cta_gemm<64>(kC, kC, D, MatV{dOs, D, 1}, MatV{U, 1, D}, stage,
-                 [&](int i, int j, float x) { sdT[i * LDC + j] = j <= i ? x : 0.f; });
+        cta_gemm<64, kGlobK, kGlobK>(D, dW, D, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); });
+        cta_gemm<64, kGlobK, kGlobK>(D, dU, D, Bv, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); }, sdT, LDC);
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dW, D, stage, [&](int i, int j, float x0, float x1) { st2(Bk + i * D + j, x0, x1); });
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dU, D, stage, [&](int i, int j, float x0, float x1) { st2(Bv + i * D + j, x0, x1); });
+        cta_gemm<64, kSmemK, kSmemK>(kC, sdT, LDC, sT, LDC, stage, [&](int i, int j, float x0, float x1) { st2(Xg + i * kC + j, x0, x1); });
+        cta_gemm<64, kSmemM, kGlobMN>(kC, sT, LDC, Xg, kC, stage, [&](int i, int j, float x0, float x1) {
+            st2(sdA + i * LDC + j, j < i ? -x0 : 0.f, j + 1 < i ? -x1 : 0.f);
+        });
+        cta_gemm<64, kGlobK, kGlobK>(D, dOs, D, U, D, stage, [&](int i, int j, float x0, float x1) {
+            st2(sdT + i * LDC + j, j <= i ? x0 : 0.f, j + 1 <= i ? x1 : 0.f);
+        });
         float *const dBk = Bk, *const dBv = Bv, *const sdP = sdT;  // dA' = diag(beta) dA
-        // 7. pairwise products backward, rows: for r in tile I, channels of one 32-wide quarter,
-        //    dq_r = sum_{s<=r} dP_rs k_s E_rs,  dk_r = sum_{s<r} dA'_rs k_s E_rs,  dG_r = q_r dq_r + k_r dk_r
-        //    (E_rs = e^{G_r - G_s} per channel), one warp per (I, 32-channel quarter).  dq -> W, dk -> U, dG -> dO.
+        // 7. pairwise products backward, one warp per (tile I, 32-channel quarter); E_rs = e^{G_r - G_s}
+        //    per channel.  Rows of tile I:
+        //      dq_r = sum_{s<=r} dP_rs k_s E_rs,  dk_r = sum_{s<r} dA'_rs k_s E_rs,  dG_r = q_r dq_r + k_r dk_r;
+        //    columns of tile J = I (each row tile I' >= J with its own reference):
+        //      dk_s += sum_{r>=s} (dP_rs q_r + dA'_rs k_r) E_rs,  dG_s -= k_s (that sum).
+        //    The row tile I has I + 1 tile pairs and the column tile 4 - I, five per warp.  Both
+        //    passes give a thread the same (token, channel) elements, so it sums them in registers
+        //    and stores dq -> W, dk -> U and dG -> dO once.
         if (warp < kTiles * NQ) {
             const int I = warp / NQ, c0 = (warp % NQ) * 32, g = lane >> 2, t = lane & 3;
+            float vq[4][4] = {}, vk[4][4] = {};
             for (int pass = 0; pass < 2; ++pass) {  // 0: tiles J < I (reference 16 I), 1: J = I (middle)
                 const int m = pass == 0 ? I * kTile : I * kTile + kRef;
                 float aq[4][4] = {}, ak[4][4] = {};
@@ -1807,35 +1940,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int x = 0; x < 4; ++x) {
                         const int r = I * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
                         const float f = __expf(sG[r * LDD + c] - sG[m * LDD + c]);
-                        const float vq = aq[nf][x] * f, vk = ak[nf][x] * f;
-                        const float dg = sq[r * LDD + c] * vq + sk[r * LDD + c] * vk;
-                        if (pass == 0) {
-                            W[r * D + c] = vq;
-                            U[r * D + c] = vk;
-                            dOs[r * D + c] = dg;
-                        } else {
-                            W[r * D + c] += vq;
-                            U[r * D + c] += vk;
-                            dOs[r * D + c] += dg;
-                        }
+                        vq[nf][x] = fmaf(aq[nf][x], f, vq[nf][x]);
+                        vk[nf][x] = fmaf(ak[nf][x], f, vk[nf][x]);
                     }
             }
-        }
-        __syncthreads();
-        //    columns: dk_s += sum_{r>=s} (dP_rs q_r + dA'_rs k_r) E_rs and dG_s -= k_s (that sum), one
-        //    warp per (column tile J, quarter); each row tile I >= J has its own reference.
-        if (warp < kTiles * NQ) {
-            const int J = warp / NQ, c0 = (warp % NQ) * 32, g = lane >> 2, t = lane & 3;
+            const int J = I;
             float tot[4][4] = {};
-            for (int I = J; I < kTiles; ++I) {
-                const int m = I > J ? I * kTile : I * kTile + kRef;
+            for (int Ir = J; Ir < kTiles; ++Ir) {
+                const int m = Ir > J ? Ir * kTile : Ir * kTile + kRef;
                 float acc[4][4] = {};
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                     uint32_t fp[4], fa[4];
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {  // A(s, r) = dP_rs: s = row of the product
-                        const int s = J * kTile + g + (x & 1) * 8, r = I * kTile + ks * 8 + t + (x >> 1) * 4;
+                        const int s = J * kTile + g + (x & 1) * 8, r = Ir * kTile + ks * 8 + t + (x >> 1) * 4;
                         fp[x] = to_tf32(sdP[r * LDC + s]);
                         fa[x] = to_tf32(sbeta[r] * sdA[r * LDC + s]);
                     }
@@ -1844,7 +1963,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         uint32_t bq[2], bk[2];
 #pragma unroll
                         for (int x = 0; x < 2; ++x) {
-                            const int r = I * kTile + ks * 8 + t + x * 4, c = c0 + nf * 8 + g;
+                            const int r = Ir * kTile + ks * 8 + t + x * 4, c = c0 + nf * 8 + g;
                             const float f = __expf(sG[r * LDD + c] - sG[m * LDD + c]);
                             bq[x] = to_tf32(sq[r * LDD + c] * f);
                             bk[x] = to_tf32(sk[r * LDD + c] * f);
@@ -1864,28 +1983,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int nf = 0; nf < 4; ++nf)
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int s = J * kTile + g + (x >> 1) * 8, c = c0 + nf * 8 + 2 * t + (x & 1);
-                    U[s * D + c] += tot[nf][x];
-                    dOs[s * D + c] -= sk[s * LDD + c] * tot[nf][x];
+                for (int hh = 0; hh < 2; ++hh) {  // element pairs (x = 2 hh, 2 hh + 1): channels c, c + 1
+                    const int r = I * kTile + g + hh * 8, c = c0 + nf * 8 + 2 * t;
+                    const float2 q2 = *reinterpret_cast<const float2 *>(sq + r * LDD + c);
+                    const float2 k2 = *reinterpret_cast<const float2 *>(sk + r * LDD + c);
+                    const float q0 = vq[nf][2 * hh], q1 = vq[nf][2 * hh + 1];
+                    const float k0 = vk[nf][2 * hh], k1 = vk[nf][2 * hh + 1];
+                    const float t0 = tot[nf][2 * hh], t1 = tot[nf][2 * hh + 1];
+                    *reinterpret_cast<float2 *>(W + r * D + c) = make_float2(q0, q1);
+                    *reinterpret_cast<float2 *>(U + r * D + c) = make_float2(k0 + t0, k1 + t1);
+                    *reinterpret_cast<float2 *>(dOs + r * D + c) =
+                        make_float2(q2.x * q0 + k2.x * (k0 - t0), q2.y * q1 + k2.y * (k1 - t1));
                 }
         }
         __syncthreads();
-        // 8. the decay-scaled operands' gradients; outputs dq, dk, dv; dG -> sq
-#pragma unroll 4
-        for (int e = tid; e < CD; e += kBwdThreads) {
-            const int r = e / D, c = e % D;
-            const float Gv = sG[r * LDD + c], e1 = __expf(Gv), eh = __expf(sG[(kC - 1) * LDD + c] - Gv);
-            const float kv = sk[r * LDD + c];
-            const float dkb = sbeta[r] * dBk[e];
-            const float dqv = W[e] + dQb[e] * e1;
-            const float dkv = U[e] + dkb * e1 + dKh[e] * eh;
-            sq[r * LDD + c] = dOs[e] + (dQb[e] * sq[r * LDD + c] + dkb * kv) * e1 - dKh[e] * kv * eh;
+        // 8. the decay-scaled operands' gradients; outputs dq, dk, dv; dG -> sq.  Four channels per
+        //    item (16-byte accesses).
+        for (int it = tid; it < CD / 4; it += kBwdThreads) {
+            const int r = it / (D / 4), c = (it % (D / 4)) * 4, e = r * D + c;
+            const float4 G4 = *reinterpret_cast<const float4 *>(sG + r * LDD + c);
+            const float4 Gl = *reinterpret_cast<const float4 *>(sG + (kC - 1) * LDD + c);
+            const float4 k4 = *reinterpret_cast<const float4 *>(sk + r * LDD + c);
+            const float4 q4 = *reinterpret_cast<const float4 *>(sq + r * LDD + c);
+            const float4 w4 = *reinterpret_cast<const float4 *>(W + e), dq4 = *reinterpret_cast<const float4 *>(dQb + e);
+            const float4 u4 = *reinterpret_cast<const float4 *>(U + e), bk4 = *reinterpret_cast<const float4 *>(dBk + e);
+            const float4 kh4 = *reinterpret_cast<const float4 *>(dKh + e), o4 = *reinterpret_cast<const float4 *>(dOs + e);
+            const float4 bv4 = *reinterpret_cast<const float4 *>(dBv + e);
+            const float br = sbeta[r];
+            const float Gv[4] = {G4.x, G4.y, G4.z, G4.w}, Gt[4] = {Gl.x, Gl.y, Gl.z, Gl.w};
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w}, dqb[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+            const float uv[4] = {u4.x, u4.y, u4.z, u4.w}, bkv[4] = {bk4.x, bk4.y, bk4.z, bk4.w};
+            const float khv[4] = {kh4.x, kh4.y, kh4.z, kh4.w}, ov[4] = {o4.x, o4.y, o4.z, o4.w};
+            const float bvv[4] = {bv4.x, bv4.y, bv4.z, bv4.w};
+            float oq[4], ok4[4], ov4[4], og[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float e1 = __expf(Gv[u]), eh = __expf(Gt[u] - Gv[u]);
+                const float dkb = br * bkv[u];
+                oq[u] = wv[u] + dqb[u] * e1;
+                ok4[u] = uv[u] + dkb * e1 + khv[u] * eh;
+                og[u] = ov[u] + (dqb[u] * qv[u] + dkb * kv[u]) * e1 - khv[u] * kv[u] * eh;
+                ov4[u] = br * bvv[u];
+            }
+            *reinterpret_cast<float4 *>(sq + r * LDD + c) = make_float4(og[0], og[1], og[2], og[3]);
             if (r < n) {
                 const size_t gi = (size_t)tix(r) * D + c;
-                dq[gi] = dqv;
-                dk[gi] = dkv;
-                dv[gi] = sbeta[r] * dBv[e];
+                *reinterpret_cast<float4 *>(dq + gi) = make_float4(oq[0], oq[1], oq[2], oq[3]);
+                *reinterpret_cast<float4 *>(dk + gi) = make_float4(ok4[0], ok4[1], ok4[2], ok4[3]);
+                *reinterpret_cast<float4 *>(dv + gi) = make_float4(ov4[0], ov4[1], ov4[2], ov4[3]);
             }
         }
         __syncthreads();

@@ -1408,8 +1408,8 @@ struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blo
     static constexpr int Kb = 0, Kh = Kb + CD;
     static constexpr int Bk = Kh + CD;   // diag(beta) Kbar, later dBk
     static constexpr int Bv = Bk + CD;   // diag(beta) V, later dBv
-    static constexpr int W = Bv + CD;    // W, then dW, then the pairwise dq
-    static constexpr int U = W + CD;     // Utilde, U, then dk
+    static constexpr int W = Bv + CD;    // Bv - Bk S, then dW, then the pairwise dq
+    static constexpr int U = W + CD;     // U, then dk
     static constexpr int dO = U + CD;    // dO, then the pairwise dG
     static constexpr int dU = dO + CD;
     static constexpr int dKh = dU + CD;
@@ -1474,7 +1474,8 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float *row_ptr)
     ldmatrix_x4(r, row_ptr);
 }
 
-// C[64 x TN] = A[64 x K] B[K x TN] on the whole CTA (K a multiple of 16); every output pair
+// C[64 x TN] = A[64 x K] B[K x TN] (+ A2[64 x K2] B2[K2 x TN], operands of the same kinds) on the
+// whole CTA (K, K2 multiples of 16); every output pair
 // (j even) goes to epi(i, j, c_ij, c_i,j+1) exactly once.  With acc_in, the pair handed over is
 // acc_in[i, j..j+1] + sign * C (all of a thread's acc_in values are loaded together, before its
 // first store, so a read-modify-write of one array costs one memory round trip, not one per
@@ -1487,7 +1488,8 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float *row_ptr)
 // ends with every thread past a barrier.
 template <int TN, int SA, int SB, class Epi>
 __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb, float *stage, Epi epi,
-                         const float *acc_in = nullptr, int ld_in = 0, float sign = 1.f)
+                         const float *acc_in = nullptr, int ld_in = 0, float sign = 1.f, int K2 = 0,
+                         const float *A2 = nullptr, int lda2 = 0, const float *B2 = nullptr, int ldb2 = 0)
 {
     static_assert(TN == 64 || TN == 128, "output tile width");
     static_assert(SB != kSmemM, "B in place is K-consecutive");
@@ -1496,10 +1498,18 @@ __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb
     const int grp = warp >> 3, wl = warp & 7;
     const int wm = (wl >> 2) * 32, wn = (wl & 3) * (TN / 4), kk = grp * 8;
     const int lr = lane & 7, lq = lane >> 3;  // ldmatrix: row within a block, block
-    const int nk = K / kGKS;
+    const int nk1 = K / kGKS, nk = nk1 + K2 / kGKS;
+    // step s of the contraction: its operands and its offset inside them
+    auto seg = [&](int s, const float *&Ap, int &la, const float *&Bp, int &lb) -> int {
+        const bool second = s >= nk1;
+        Ap = second ? A2 : A, la = second ? lda2 : lda, Bp = second ? B2 : B, lb = second ? ldb2 : ldb;
+        return (second ? s - nk1 : s) * kGKS;
+    };
     auto issue = [&](int s, int slot) {
         float *sA = stage + slot * kGStageFloats, *sB = sA + kGStageA;
-        const int k0 = s * kGKS;
+        const float *A, *B;
+        int lda, ldb;
+        const int k0 = seg(s, A, lda, B, ldb);
         if constexpr (SA == kGlobK) {
             if (tid < kC * 4) {
                 const int i = tid >> 2, c = tid & 3;
@@ -1524,7 +1534,7 @@ __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb
         }
     };
     // A fragments of the warp's two 16-row blocks at contraction offset kk of step k0
-    auto load_a = [&](const float *sA, int k0, uint32_t (&af)[2][4]) {
+    auto load_a = [&](const float *sA, const float *A, int lda, int k0, uint32_t (&af)[2][4]) {
 #pragma unroll
         for (int mf = 0; mf < 2; ++mf) {
             const int r0 = wm + mf * 16;
@@ -1540,7 +1550,7 @@ __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb
             }
         }
     };
-    auto load_b = [&](const float *sB, int k0, uint32_t (&bf)[NF][2]) {
+    auto load_b = [&](const float *sB, const float *B, int ldb, int k0, uint32_t (&bf)[NF][2]) {
         if constexpr (SB == kGlobMN) {
 #pragma unroll
             for (int nf = 0; nf < NF; ++nf) {
@@ -1584,8 +1594,11 @@ __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb
         cp_async_commit();
         const float *sA = stage + (s % kGStages) * kGStageFloats, *sB = sA + kGStageA;
         uint32_t af[2][4], bf[NF][2];
-        load_a(sA, s * kGKS, af);
-        load_b(sB, s * kGKS, bf);
+        const float *Ap, *Bp;
+        int la, lb;
+        const int k0 = seg(s, Ap, la, Bp, lb);
+        load_a(sA, Ap, la, k0, af);
+        load_b(sB, Bp, lb, k0, bf);
 #pragma unroll
         for (int mf = 0; mf < 2; ++mf)
 #pragma unroll
@@ -1728,10 +1741,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // gate table the forward prep used (per head with the scale)
         const float scale = A_log ? __expf(A_log[h]) : 1.0f;
         const float *tab = gtab + (A_log ? (size_t)h * kGateTableEntries : 0);
-
         // 1. inputs (rows past the chunk's tokens are zero, with g = 0), and dg/da; eight channels
         //    per item (16-byte loads)
-        for (int it = tid; it < CD / 8; it += kBwdThreads) {
+        static_assert(CD % (8 * kBwdThreads) == 0, "whole passes over the chunk");
+#pragma unroll
+        for (int pass8 = 0; pass8 < CD / 8 / kBwdThreads; ++pass8) {
+            const int it = tid + pass8 * kBwdThreads;
             const int r = it / (D / 8), c = (it % (D / 8)) * 8, e = r * D + c;
             const bool ok = r < n;
             const size_t gi = (size_t)tix(ok ? r : 0) * D + c;
@@ -1861,9 +1876,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // are kGlobK as A, kGlobMN as B; S and dS' (row-major D x D) are kGlobMN as B, and their
         // transposes kGlobK.
         auto st2 = [](float *p, float x0, float x1) { *reinterpret_cast<float2 *>(p) = make_float2(x0, x1); };
-        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, x0, x1); });
-        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, Bv, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); });
-        cta_gemm<D, kGlobK, kGlobMN>(D, W, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); }, U, D, -1.f);
+        // U = T (Bv - Bk S) = Utilde - W S: X = Bv - Bk S over W's slot, then U = T X
+        cta_gemm<D, kGlobK, kGlobMN>(D, Bk, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, x0, x1); }, Bv, D, -1.f);
+        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, W, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); });
         cta_gemm<D, kGlobK, kGlobMN>(D, Kh, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); });
         cta_gemm<D, kSmemM, kGlobMN>(kC, sP, LDC, dOs, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); }, dU, D);
         cta_gemm<D, kGlobK, kGlobK>(D, U, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dKh + i * D + j, x0, x1); });
@@ -1884,8 +1899,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0)
                 sdGam[i] = acc;
         }
-        cta_gemm<64, kGlobK, kGlobK>(D, dW, D, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); });
-        cta_gemm<64, kGlobK, kGlobK>(D, dU, D, Bv, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); }, sdT, LDC);
+        // dT = dW Bk^T + dU Bv^T, one contraction over both
+        cta_gemm<64, kGlobK, kGlobK>(D, dW, D, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); },
+                                     nullptr, 0, 1.f, D, dU, D, Bv, D);
         cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dW, D, stage, [&](int i, int j, float x0, float x1) { st2(Bk + i * D + j, x0, x1); });
         cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dU, D, stage, [&](int i, int j, float x0, float x1) { st2(Bv + i * D + j, x0, x1); });
         cta_gemm<64, kSmemK, kSmemK>(kC, sdT, LDC, sT, LDC, stage, [&](int i, int j, float x0, float x1) { st2(Xg + i * kC + j, x0, x1); });

@@ -205,12 +205,13 @@ struct PrepLayout {
 __device__ __forceinline__ uint32_t tok_off(int r, int c8) { return tc::mnmaj_sw128(r, c8, kC); }
 
 // One 16x16 output block of the block substitution, by one warp with tf32 tensor-core
-// MMAs:  X = sum_{K=J}^{I-1} A_IK T_KJ,  T_IJ = -T_II X.  A and T are fp32 [64][kC + 1];
-// X goes through a 16x16 scratch (row stride kC + 1, an unused upper block of A) to turn
-// the accumulator layout into an operand layout.
-__device__ __forceinline__ void solve_block_tf32(const float *A, float *Tm, float *X, int I, int J, int lane)
+// MMAs:  X = diag(rs_I) sum_{K=J}^{I-1} A_IK T_KJ,  T_IJ = -T_II X  (rs = the row scale, or 1
+// without it).  A and T are fp32 [64][LD]; X goes through a 16x16 scratch (row stride LD) to
+// turn the accumulator layout into an operand layout.
+template <int LD>
+__device__ __forceinline__ void solve_block_tf32(const float *A, float *Tm, float *X, int I, int J, int lane,
+                                                 const float *rs = nullptr)
 {
-    constexpr int LD = kC + 1;
     const int g = lane >> 2, t = lane & 3;
     float acc[2][4] = {};
     auto product = [&](const float *Am, int arow, int acol, const float *Bm, int brow, int bcol, int bld) {
@@ -232,12 +233,13 @@ __device__ __forceinline__ void solve_block_tf32(const float *A, float *Tm, floa
     };
     for (int K = J; K < I; ++K)
         product(A, I * kTile, K * kTile, Tm, K * kTile, J * kTile, LD);
+    const float s0 = rs ? rs[I * kTile + g] : 1.0f, s1 = rs ? rs[I * kTile + g + 8] : 1.0f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        X[g * LD + nt * 8 + 2 * t] = acc[nt][0];
-        X[g * LD + nt * 8 + 2 * t + 1] = acc[nt][1];
-        X[(g + 8) * LD + nt * 8 + 2 * t] = acc[nt][2];
-        X[(g + 8) * LD + nt * 8 + 2 * t + 1] = acc[nt][3];
+        X[g * LD + nt * 8 + 2 * t] = s0 * acc[nt][0];
+        X[g * LD + nt * 8 + 2 * t + 1] = s0 * acc[nt][1];
+        X[(g + 8) * LD + nt * 8 + 2 * t] = s1 * acc[nt][2];
+        X[(g + 8) * LD + nt * 8 + 2 * t + 1] = s1 * acc[nt][3];
         acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
     }
     __syncwarp();
@@ -711,7 +713,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     __syncthreads();
     for (int lvl = 1; lvl < kTiles; ++lvl) {  // level lvl: blocks (J + lvl, J), one warp each
         if (warp < kTiles - lvl)
-            solve_block_tf32(sA, sT, sA + (warp + 1) * kTile /* upper block (0, warp+1) of A */, warp + lvl,
+            solve_block_tf32<kC + 1>(sA, sT, sA + (warp + 1) * kTile /* upper block (0, warp+1) of A */, warp + lvl,
                              warp, lane);
         __syncthreads();
     }
@@ -1821,54 +1823,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncthreads();
         // 5. T = (I + A)^{-1}, A = diag(beta) A', unit lower triangular, by 16 x 16 blocks: the
-        //    diagonal blocks by forward substitution (one warp each), then block rows by level,
-        //    T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
-        if (warp < kTiles) {
-            const int b0 = warp * kTile, j = lane & 15;
-            for (int rr = 1; rr < kTile; ++rr) {
-                const int r = b0 + rr;
-                float acc = 0.f;
+        //    diagonal blocks by forward substitution (one lane per column, the column in registers),
+        //    then block rows by level, T_IJ = -T_II diag(beta_I) sum_{K=J}^{I-1} A'_IK T_KJ, one warp
+        //    per block with tf32 tensor-core products.
+        if (warp < kTiles && lane < kTile) {
+            const int I = warp, c = lane;
+            float x[kTile];
 #pragma unroll
-                for (int s = 0; s < kTile - 1; ++s)
-                    if (s >= j && s < rr)
-                        acc = fmaf(sAp[r * LDC + b0 + s], sT[(b0 + s) * LDC + b0 + j], acc);
-                __syncwarp();
-                if (lane < kTile && j < rr)
-                    sT[r * LDC + b0 + j] = -sbeta[r] * acc;
-                __syncwarp();
+            for (int r = 0; r < kTile; ++r)
+                x[r] = r == c ? 1.0f : 0.0f;
+#pragma unroll
+            for (int r = 1; r < kTile; ++r) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int y = 0; y < r; ++y)
+                    acc = fmaf(sAp[(I * kTile + r) * LDC + I * kTile + y], x[y], acc);
+                if (r > c)
+                    x[r] = -sbeta[I * kTile + r] * acc;
             }
+#pragma unroll
+            for (int r = 0; r < kTile; ++r)
+                sT[(I * kTile + r) * LDC + I * kTile + c] = x[r];
         }
         __syncthreads();
         for (int lvl = 1; lvl < kTiles; ++lvl) {
-            if (warp < kTiles - lvl) {
-                const int J = warp, I = warp + lvl;
-                const int rr = lane >> 1, j0 = (lane & 1) * 8, r = I * kTile + rr;
-                float x[8] = {};
-                for (int K = J; K < I; ++K)
-#pragma unroll
-                    for (int s = 0; s < kTile; ++s) {
-                        const float av = sAp[r * LDC + K * kTile + s];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            x[u] = fmaf(av, sT[(K * kTile + s) * LDC + J * kTile + j0 + u], x[u]);
-                    }
-                float *Xs = sdT + warp * kTile * LDC;  // 16 x 16 per warp (sdT is free until step 6)
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    Xs[rr * LDC + j0 + u] = sbeta[r] * x[u];
-                __syncwarp();
-                float y[8] = {};
-#pragma unroll
-                for (int uu = 0; uu < kTile; ++uu) {
-                    const float tv = sT[r * LDC + I * kTile + uu];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        y[u] = fmaf(tv, Xs[uu * LDC + j0 + u], y[u]);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    sT[r * LDC + J * kTile + j0 + u] = -y[u];
-            }
+            if (warp < kTiles - lvl)  // scratch: a 16 x 16 block of sdT per warp (free until step 6)
+                solve_block_tf32<LDC>(sAp, sT, sdT + warp * kTile * LDC, warp + lvl, warp, lane, sbeta);
             __syncthreads();
         }
         // 6. dense contractions

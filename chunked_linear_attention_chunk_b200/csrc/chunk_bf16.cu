@@ -1477,22 +1477,46 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float *row_ptr)
 }
 
 // C[64 x TN] = A[64 x K] B[K x TN] (+ A2[64 x K2] B2[K2 x TN], operands of the same kinds) on the
-// whole CTA (K, K2 multiples of 16); every output pair
-// (j even) goes to epi(i, j, c_ij, c_i,j+1) exactly once.  With acc_in, the pair handed over is
-// acc_in[i, j..j+1] + sign * C (all of a thread's acc_in values are loaded together, before its
-// first store, so a read-modify-write of one array costs one memory round trip, not one per
-// element).  TF32 mma.sync with fp32
+// whole CTA (K, K2 multiples of 16), written as the GemmOut says, each output pair (j even) once
+// (a thread loads all its acc_in values before its first store, so a read-modify-write of one
+// array costs one memory round trip, not one per element).  TF32 mma.sync with fp32
 // accumulation; operands enter the tensor cores as their fp32 bit patterns (the hardware
 // uses the TF32 part).  The contraction is split between two groups of eight warps: per
 // 16-wide step, group 0 takes its first 8 indices and group 1 the rest, each warp a 32 x TN/4
 // tile, and the two partial sums meet in shared memory at the end.  The global operands move
 // through a three-stage ring of shared-memory tiles, one CTA barrier per step.  Starts and
 // ends with every thread past a barrier.
-template <int TN, int SA, int SB, class Epi>
-__device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb, float *stage, Epi epi,
-                         const float *acc_in = nullptr, int ld_in = 0, float sign = 1.f, int K2 = 0,
-                         const float *A2 = nullptr, int lda2 = 0, const float *B2 = nullptr, int ldb2 = 0)
+// Where cta_gemm puts its result: dst[i, j] = sign * C[i, j] (+ acc_in[i, j]), rows of ld floats
+// (global or shared memory); with mask 1 only j < i is kept (0 elsewhere), with mask 2 j <= i.
+struct GemmOut {
+    float *dst;
+    int ld;
+    float sign;
+    const float *acc_in;
+    int ld_in;
+    int mask;
+};
+
+// One copy of the code per operand-kind combination (not per call site), so the gradient
+// kernel's instruction footprint stays small.
+template <int TN, int SA, int SB>
+__device__ __noinline__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb, float *stage, GemmOut out,
+                                      int K2 = 0, const float *A2 = nullptr, int lda2 = 0, const float *B2 = nullptr,
+                                      int ldb2 = 0)
 {
+    const float *const acc_in = out.acc_in;
+    const int ld_in = out.ld_in;
+    const float sign = out.sign;
+    auto epi = [&](int i, int j, float x0, float x1) {
+        if (out.mask == 1) {
+            x0 = j < i ? x0 : 0.f;
+            x1 = j + 1 < i ? x1 : 0.f;
+        } else if (out.mask == 2) {
+            x0 = j <= i ? x0 : 0.f;
+            x1 = j + 1 <= i ? x1 : 0.f;
+        }
+        *reinterpret_cast<float2 *>(out.dst + i * out.ld + j) = make_float2(x0, x1);
+    };
     static_assert(TN == 64 || TN == 128, "output tile width");
     static_assert(SB != kSmemM, "B in place is K-consecutive");
     constexpr int NF = TN / 32, LDBN = TN + 8;
@@ -1634,12 +1658,10 @@ __device__ void cta_gemm(int K, const float *A, int lda, const float *B, int ldb
         for (int v = 0; v < 4; ++v)
             c[v] = (grp ? acc[1][nf][v] : acc[0][nf][v]) + xch[(grp * NF * 4 + nf * 4 + v) * 256 + gt];
         const int i = wm + grp * 16 + g, j = wn + nf * 8 + 2 * t;
-        if (acc_in) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                c[2 * hh] = fmaf(sign, c[2 * hh], prev[nf][hh].x);
-                c[2 * hh + 1] = fmaf(sign, c[2 * hh + 1], prev[nf][hh].y);
-            }
+        for (int hh = 0; hh < 2; ++hh) {
+            c[2 * hh] = acc_in ? fmaf(sign, c[2 * hh], prev[nf][hh].x) : sign * c[2 * hh];
+            c[2 * hh + 1] = acc_in ? fmaf(sign, c[2 * hh + 1], prev[nf][hh].y) : sign * c[2 * hh + 1];
         }
         epi(i, j, c[0], c[1]);
         epi(i + 8, j, c[2], c[3]);
@@ -1855,15 +1877,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // A operand T: kSmemK over sT; T^T: kSmemM over sT.  Row-major 64 x D blocks of the slot
         // are kGlobK as A, kGlobMN as B; S and dS' (row-major D x D) are kGlobMN as B, and their
         // transposes kGlobK.
-        auto st2 = [](float *p, float x0, float x1) { *reinterpret_cast<float2 *>(p) = make_float2(x0, x1); };
         // U = T (Bv - Bk S) = Utilde - W S: X = Bv - Bk S over W's slot, then U = T X
-        cta_gemm<D, kGlobK, kGlobMN>(D, Bk, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, x0, x1); }, Bv, D, -1.f);
-        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, W, D, stage, [&](int i, int j, float x0, float x1) { st2(U + i * D + j, x0, x1); });
-        cta_gemm<D, kGlobK, kGlobMN>(D, Kh, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); });
-        cta_gemm<D, kSmemM, kGlobMN>(kC, sP, LDC, dOs, D, stage, [&](int i, int j, float x0, float x1) { st2(dU + i * D + j, x0, x1); }, dU, D);
-        cta_gemm<D, kGlobK, kGlobK>(D, U, D, dSn, D, stage, [&](int i, int j, float x0, float x1) { st2(dKh + i * D + j, x0, x1); });
-        cta_gemm<D, kGlobK, kGlobK>(D, dOs, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(dQb + i * D + j, x0, x1); });
-        cta_gemm<D, kGlobK, kGlobK>(D, dU, D, S, D, stage, [&](int i, int j, float x0, float x1) { st2(W + i * D + j, -x0, -x1); });
+        cta_gemm<D, kGlobK, kGlobMN>(D, Bk, D, S, D, stage, GemmOut{W, D, -1.f, Bv, D, 0});
+        cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, W, D, stage, GemmOut{U, D, 1.f, nullptr, 0, 0});
+        cta_gemm<D, kGlobK, kGlobMN>(D, Kh, D, dSn, D, stage, GemmOut{dU, D, 1.f, nullptr, 0, 0});
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sP, LDC, dOs, D, stage, GemmOut{dU, D, 1.f, dU, D, 0});
+        cta_gemm<D, kGlobK, kGlobK>(D, U, D, dSn, D, stage, GemmOut{dKh, D, 1.f, nullptr, 0, 0});
+        cta_gemm<D, kGlobK, kGlobK>(D, dOs, D, S, D, stage, GemmOut{dQb, D, 1.f, nullptr, 0, 0});
+        cta_gemm<D, kGlobK, kGlobK>(D, dU, D, S, D, stage, GemmOut{W, D, -1.f, nullptr, 0, 0});
         float *const dW = W;
         // dGamma_i = sum_j dS'_ij S_ij, warp per row
 #pragma unroll
@@ -1880,17 +1901,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 sdGam[i] = acc;
         }
         // dT = dW Bk^T + dU Bv^T, one contraction over both
-        cta_gemm<64, kGlobK, kGlobK>(D, dW, D, Bk, D, stage, [&](int i, int j, float x0, float x1) { st2(sdT + i * LDC + j, x0, x1); },
-                                     nullptr, 0, 1.f, D, dU, D, Bv, D);
-        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dW, D, stage, [&](int i, int j, float x0, float x1) { st2(Bk + i * D + j, x0, x1); });
-        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dU, D, stage, [&](int i, int j, float x0, float x1) { st2(Bv + i * D + j, x0, x1); });
-        cta_gemm<64, kSmemK, kSmemK>(kC, sdT, LDC, sT, LDC, stage, [&](int i, int j, float x0, float x1) { st2(Xg + i * kC + j, x0, x1); });
-        cta_gemm<64, kSmemM, kGlobMN>(kC, sT, LDC, Xg, kC, stage, [&](int i, int j, float x0, float x1) {
-            st2(sdA + i * LDC + j, j < i ? -x0 : 0.f, j + 1 < i ? -x1 : 0.f);
-        });
-        cta_gemm<64, kGlobK, kGlobK>(D, dOs, D, U, D, stage, [&](int i, int j, float x0, float x1) {
-            st2(sdT + i * LDC + j, j <= i ? x0 : 0.f, j + 1 <= i ? x1 : 0.f);
-        });
+        cta_gemm<64, kGlobK, kGlobK>(D, dW, D, Bk, D, stage, GemmOut{sdT, LDC, 1.f, nullptr, 0, 0}, D, dU, D, Bv, D);
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dW, D, stage, GemmOut{Bk, D, 1.f, nullptr, 0, 0});
+        cta_gemm<D, kSmemM, kGlobMN>(kC, sT, LDC, dU, D, stage, GemmOut{Bv, D, 1.f, nullptr, 0, 0});
+        cta_gemm<64, kSmemK, kSmemK>(kC, sdT, LDC, sT, LDC, stage, GemmOut{Xg, kC, 1.f, nullptr, 0, 0});
+        cta_gemm<64, kSmemM, kGlobMN>(kC, sT, LDC, Xg, kC, stage, GemmOut{sdA, LDC, -1.f, nullptr, 0, 1});
+        cta_gemm<64, kGlobK, kGlobK>(D, dOs, D, U, D, stage, GemmOut{sdT, LDC, 1.f, nullptr, 0, 2});
         float *const dBk = Bk, *const dBv = Bv, *const sdP = sdT;  // dA' = diag(beta) dA
         // 7. pairwise products backward, one warp per (tile I, 32-channel quarter); E_rs = e^{G_r - G_s}
         //    per channel.  Rows of tile I:

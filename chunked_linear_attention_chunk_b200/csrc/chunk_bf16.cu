@@ -1418,7 +1418,8 @@ struct BwdSlot {  // float offsets inside one scratch slot, 64 x D row-major blo
     static constexpr int dQb = dKh + CD;
     static constexpr int Gp = dQb + CD;  // dg/da = g_min sigma(a) (1 - sigma(a))
     static constexpr int X = Gp + CD;    // dT T^T, 64 x 64
-    static constexpr int floats = X + kC * kC;
+    static constexpr int P = X + kC * kC;  // the pairwise products P, 64 x 64
+    static constexpr int floats = P + kC * kC;
 };
 
 // Operand sources of cta_gemm.  "K" = consecutive along the contraction index, "M" / "N" =
@@ -1432,10 +1433,10 @@ enum GemmSrc : int {
     kSmemM,  // A only: as kGlobMN, in shared memory
 };
 
-constexpr int kGKS = 16;    // contraction step per pipeline stage
-constexpr int kGStages = 3; // cp.async ring depth
-// one stage: A 64 x 16 (K-consecutive rows padded to 20, or 16 x 64 padded to 72), B 16 x TN
-// (N-consecutive rows padded to TN + 8) or TN x 16 (K-consecutive, 16-byte chunks XOR-swizzled)
+constexpr int kGKS = 32;    // contraction step per pipeline stage
+constexpr int kGStages = 2; // cp.async stages (double buffer)
+// one stage: A 64 x 32 (K-consecutive rows padded to 36, or 32 x 64 padded to 72), B 32 x TN
+// (N-consecutive rows padded to TN + 8) or TN x 32 (K-consecutive, 16-byte chunks XOR-swizzled)
 constexpr int kGStageA = kC * (kGKS + 4);
 constexpr int kGStageB = kGKS * (128 + 8);
 constexpr int kGStageFloats = kGStageA + kGStageB;
@@ -1448,7 +1449,7 @@ struct BwdSmem {  // float offsets in shared memory
     static constexpr int LDD = D + 4;    // conflict-free mma fragment reads
     static constexpr int LDC = kC + 4;
     static constexpr int q = 0, k = q + kC * LDD, G = k + kC * LDD;  // q later holds dG
-    static constexpr int Ap = G + kC * LDD, P = Ap + kC * LDC, T = P + kC * LDC;
+    static constexpr int Ap = G + kC * LDD, T = Ap + kC * LDC;
     static constexpr int dT = T + kC * LDC;  // scratch of the block solve, then dT, then dP
     static constexpr int dA = dT + kC * LDC;
     static constexpr int stage = dA + kC * LDC;  // cta_gemm's ring (16-byte aligned)
@@ -1466,7 +1467,7 @@ struct BwdSmem {  // float offsets in shared memory
 template <int TN>
 __device__ __forceinline__ int gemm_bk_off(int j, int k)  // (k, j) of a staged K-consecutive B
 {
-    return j * kGKS + ((((k >> 2) ^ (j >> 1)) & 3) << 2) + (k & 3);
+    return j * kGKS + ((((k >> 2) ^ j) & 7) << 2) + (k & 3);
 }
 
 // ldmatrix of four 8 x 4 fp32 blocks (each row 16 bytes): thread T receives element
@@ -1476,16 +1477,6 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float *row_ptr)
     ldmatrix_x4(r, row_ptr);
 }
 
-// C[64 x TN] = A[64 x K] B[K x TN] (+ A2[64 x K2] B2[K2 x TN], operands of the same kinds) on the
-// whole CTA (K, K2 multiples of 16), written as the GemmOut says, each output pair (j even) once
-// (a thread loads all its acc_in values before its first store, so a read-modify-write of one
-// array costs one memory round trip, not one per element).  TF32 mma.sync with fp32
-// accumulation; operands enter the tensor cores as their fp32 bit patterns (the hardware
-// uses the TF32 part).  The contraction is split between two groups of eight warps: per
-// 16-wide step, group 0 takes its first 8 indices and group 1 the rest, each warp a 32 x TN/4
-// tile, and the two partial sums meet in shared memory at the end.  The global operands move
-// through a three-stage ring of shared-memory tiles, one CTA barrier per step.  Starts and
-// ends with every thread past a barrier.
 // Where cta_gemm puts its result: dst[i, j] = sign * C[i, j] (+ acc_in[i, j]), rows of ld floats
 // (global or shared memory); with mask 1 only j < i is kept (0 elsewhere), with mask 2 j <= i.
 struct GemmOut {
@@ -1497,6 +1488,16 @@ struct GemmOut {
     int mask;
 };
 
+// C[64 x TN] = A[64 x K] B[K x TN] (+ A2[64 x K2] B2[K2 x TN], operands of the same kinds) on the
+// whole CTA (K, K2 multiples of 32), written as the GemmOut says, each output pair (j even) once
+// (a thread loads all its acc_in values before its first store, so a read-modify-write of one
+// array costs one memory round trip, not one per element).  TF32 mma.sync with fp32
+// accumulation; operands enter the tensor cores as their fp32 bit patterns (the hardware
+// uses the TF32 part).  The contraction is split between two groups of eight warps: per
+// 32-wide step, group 0 takes its first 16 indices and group 1 the rest, each warp a 32 x TN/4
+// tile, and the two partial sums meet in shared memory at the end.  The global operands move
+// through two shared-memory stages (double buffer), one CTA barrier per step.  Starts and
+// ends with every thread past a barrier.
 // One copy of the code per operand-kind combination (not per call site), so the gradient
 // kernel's instruction footprint stays small.
 template <int TN, int SA, int SB>
@@ -1522,7 +1523,7 @@ __device__ __noinline__ void cta_gemm(int K, const float *A, int lda, const floa
     constexpr int NF = TN / 32, LDBN = TN + 8;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const int grp = warp >> 3, wl = warp & 7;
-    const int wm = (wl >> 2) * 32, wn = (wl & 3) * (TN / 4), kk = grp * 8;
+    const int wm = (wl >> 2) * 32, wn = (wl & 3) * (TN / 4);
     const int lr = lane & 7, lq = lane >> 3;  // ldmatrix: row within a block, block
     const int nk1 = K / kGKS, nk = nk1 + K2 / kGKS;
     // step s of the contraction: its operands and its offset inside them
@@ -1536,31 +1537,28 @@ __device__ __noinline__ void cta_gemm(int K, const float *A, int lda, const floa
         const float *A, *B;
         int lda, ldb;
         const int k0 = seg(s, A, lda, B, ldb);
+        constexpr int CPR = kGKS / 4;  // 16-byte chunks per K-consecutive row
+        static_assert(kC * CPR == kBwdThreads && kGKS * (kC / 4) == kBwdThreads, "one A chunk per thread");
         if constexpr (SA == kGlobK) {
-            if (tid < kC * 4) {
-                const int i = tid >> 2, c = tid & 3;
-                cp_async_16(sA + i * (kGKS + 4) + 4 * c, A + (size_t)i * lda + k0 + 4 * c);
-            }
+            const int i = tid / CPR, c = tid % CPR;
+            cp_async_16(sA + i * (kGKS + 4) + 4 * c, A + (size_t)i * lda + k0 + 4 * c);
         } else if constexpr (SA == kGlobMN) {
-            if (tid < kGKS * (kC / 4)) {
-                const int k = tid / (kC / 4), c = tid % (kC / 4);
-                cp_async_16(sA + k * 72 + 4 * c, A + (size_t)(k0 + k) * lda + 4 * c);
-            }
+            const int k = tid / (kC / 4), c = tid % (kC / 4);
+            cp_async_16(sA + k * 72 + 4 * c, A + (size_t)(k0 + k) * lda + 4 * c);
         }
-        if constexpr (SB == kGlobMN) {
-            if (tid < kGKS * (TN / 4)) {
-                const int k = tid / (TN / 4), c = tid % (TN / 4);
+#pragma unroll
+        for (int e = tid; e < kGKS * TN / 4; e += kBwdThreads) {
+            if constexpr (SB == kGlobMN) {
+                const int k = e / (TN / 4), c = e % (TN / 4);
                 cp_async_16(sB + k * LDBN + 4 * c, B + (size_t)(k0 + k) * ldb + 4 * c);
-            }
-        } else if constexpr (SB == kGlobK) {
-            if (tid < TN * 4) {
-                const int j = tid >> 2, c = tid & 3;
+            } else if constexpr (SB == kGlobK) {
+                const int j = e / CPR, c = e % CPR;
                 cp_async_16(sB + gemm_bk_off<TN>(j, 4 * c), B + (size_t)j * ldb + k0 + 4 * c);
             }
         }
     };
     // A fragments of the warp's two 16-row blocks at contraction offset kk of step k0
-    auto load_a = [&](const float *sA, const float *A, int lda, int k0, uint32_t (&af)[2][4]) {
+    auto load_a = [&](const float *sA, const float *A, int lda, int k0, int kk, uint32_t (&af)[2][4]) {
 #pragma unroll
         for (int mf = 0; mf < 2; ++mf) {
             const int r0 = wm + mf * 16;
@@ -1576,7 +1574,7 @@ __device__ __noinline__ void cta_gemm(int K, const float *A, int lda, const floa
             }
         }
     };
-    auto load_b = [&](const float *sB, const float *B, int ldb, int k0, uint32_t (&bf)[NF][2]) {
+    auto load_b = [&](const float *sB, const float *B, int ldb, int k0, int kk, uint32_t (&bf)[NF][2]) {
         if constexpr (SB == kGlobMN) {
 #pragma unroll
             for (int nf = 0; nf < NF; ++nf) {
@@ -1619,17 +1617,21 @@ __device__ __noinline__ void cta_gemm(int K, const float *A, int lda, const floa
             issue(s + kGStages - 1, (s + kGStages - 1) % kGStages);
         cp_async_commit();
         const float *sA = stage + (s % kGStages) * kGStageFloats, *sB = sA + kGStageA;
-        uint32_t af[2][4], bf[NF][2];
         const float *Ap, *Bp;
         int la, lb;
         const int k0 = seg(s, Ap, la, Bp, lb);
-        load_a(sA, Ap, la, k0, af);
-        load_b(sB, Bp, lb, k0, bf);
 #pragma unroll
-        for (int mf = 0; mf < 2; ++mf)
+        for (int h = 0; h < 2; ++h) {  // this group's two 8-wide slices of the step
+            const int kk = grp * 16 + h * 8;
+            uint32_t af[2][4], bf[NF][2];
+            load_a(sA, Ap, la, k0, kk, af);
+            load_b(sB, Bp, lb, k0, kk, bf);
 #pragma unroll
-            for (int nf = 0; nf < NF; ++nf)
-                mma_tf32_1688(acc[mf][nf], af[mf], bf[nf]);
+            for (int mf = 0; mf < 2; ++mf)
+#pragma unroll
+                for (int nf = 0; nf < NF; ++nf)
+                    mma_tf32_1688(acc[mf][nf], af[mf], bf[nf]);
+        }
     }
     float2 prev[NF][2];
     if (acc_in) {
@@ -1710,7 +1712,7 @@ __device__ void pair_fwd_tile(const float *sq, const float *sk, const float *sG,
         for (int x = 0; x < 4; ++x) {
             const int r = r0 + g + (x >> 1) * 8, s = s0 + nt * 8 + 2 * t + (x & 1);
             Ap[r * LDC + s] = s < r ? aA[nt][x] : 0.f;
-            P[r * LDC + s] = s <= r ? aP[nt][x] : 0.f;
+            P[r * kC + s] = s <= r ? aP[nt][x] : 0.f;  // P: row stride kC (the scratch slot)
         }
 }
 
@@ -1731,7 +1733,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr int NQ = D / 32;  // 32-channel quarters (per warp) of the pairwise backward
     extern __shared__ __align__(16) float bsm[];
     float *const sq = bsm + SL::q, *const sk = bsm + SL::k, *const sG = bsm + SL::G;
-    float *const sAp = bsm + SL::Ap, *const sP = bsm + SL::P, *const sT = bsm + SL::T;
+    float *const sAp = bsm + SL::Ap, *const sT = bsm + SL::T;
     float *const sdT = bsm + SL::dT, *const sdA = bsm + SL::dA;
     float *const stage = bsm + SL::stage;
     float *const sbeta = bsm + SL::beta, *const sdGam = bsm + SL::dGam;
@@ -1741,7 +1743,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *const Kb = sl + L::Kb, *const Kh = sl + L::Kh, *const Bk = sl + L::Bk;
     float *const Bv = sl + L::Bv, *const W = sl + L::W, *const U = sl + L::U, *const dOs = sl + L::dO;
     float *const dU = sl + L::dU, *const dKh = sl + L::dKh, *const dQb = sl + L::dQb, *const Gp = sl + L::Gp;
-    float *const Xg = sl + L::X;
+    float *const Xg = sl + L::X, *const Pg = sl + L::P;  // P: 64 x 64, row stride kC
 
     for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
         // regular batch: unit = (b*H + h) * NT + chunk; packed batch: unit = h * NT + chunk slot
@@ -1835,13 +1837,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 J -= I + 1;
                 ++I;
             }
-            pair_fwd_tile<D>(sq, sk, sG, sAp, sP, I, J, lane);
+            pair_fwd_tile<D>(sq, sk, sG, sAp, Pg, I, J, lane);
         }
         for (int e = tid; e < kC * kC; e += kBwdThreads) {
             const int r = e / kC, s = e % kC;
             sT[r * LDC + s] = r == s ? 1.f : 0.f;
             if (s / kTile > r / kTile)  // tiles above the diagonal (the pairwise tiles write the rest)
-                sAp[r * LDC + s] = sP[r * LDC + s] = 0.f;
+                sAp[r * LDC + s] = Pg[r * kC + s] = 0.f;
         }
         __syncthreads();
         // 5. T = (I + A)^{-1}, A = diag(beta) A', unit lower triangular, by 16 x 16 blocks: the
@@ -1881,7 +1883,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         cta_gemm<D, kGlobK, kGlobMN>(D, Bk, D, S, D, stage, GemmOut{W, D, -1.f, Bv, D, 0});
         cta_gemm<D, kSmemK, kGlobMN>(kC, sT, LDC, W, D, stage, GemmOut{U, D, 1.f, nullptr, 0, 0});
         cta_gemm<D, kGlobK, kGlobMN>(D, Kh, D, dSn, D, stage, GemmOut{dU, D, 1.f, nullptr, 0, 0});
-        cta_gemm<D, kSmemM, kGlobMN>(kC, sP, LDC, dOs, D, stage, GemmOut{dU, D, 1.f, dU, D, 0});
+        cta_gemm<D, kGlobMN, kGlobMN>(kC, Pg, kC, dOs, D, stage, GemmOut{dU, D, 1.f, dU, D, 0});
         cta_gemm<D, kGlobK, kGlobK>(D, U, D, dSn, D, stage, GemmOut{dKh, D, 1.f, nullptr, 0, 0});
         cta_gemm<D, kGlobK, kGlobK>(D, dOs, D, S, D, stage, GemmOut{dQb, D, 1.f, nullptr, 0, 0});
         cta_gemm<D, kGlobK, kGlobK>(D, dU, D, S, D, stage, GemmOut{W, D, -1.f, nullptr, 0, 0});

@@ -2019,10 +2019,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float4 Gl = *reinterpret_cast<const float4 *>(sG + (kC - 1) * LDD + c);
             const float4 k4 = *reinterpret_cast<const float4 *>(sk + r * LDD + c);
             const float4 q4 = *reinterpret_cast<const float4 *>(sq + r * LDD + c);
-            const float4 w4 = *reinterpret_cast<const float4 *>(W + e), dq4 = *reinterpret_cast<const float4 *>(dQb + e);
-            const float4 u4 = *reinterpret_cast<const float4 *>(U + e), bk4 = *reinterpret_cast<const float4 *>(dBk + e);
-            const float4 kh4 = *reinterpret_cast<const float4 *>(dKh + e), o4 = *reinterpret_cast<const float4 *>(dOs + e);
-            const float4 bv4 = *reinterpret_cast<const float4 *>(dBv + e);
+            // explicit global loads: they may run ahead of this thread's shared-memory stores
+            const float4 w4 = __ldcg(reinterpret_cast<const float4 *>(W + e)), dq4 = __ldcg(reinterpret_cast<const float4 *>(dQb + e));
+            const float4 u4 = __ldcg(reinterpret_cast<const float4 *>(U + e)), bk4 = __ldcg(reinterpret_cast<const float4 *>(dBk + e));
+            const float4 kh4 = __ldcg(reinterpret_cast<const float4 *>(dKh + e)), o4 = __ldcg(reinterpret_cast<const float4 *>(dOs + e));
+            const float4 bv4 = __ldcg(reinterpret_cast<const float4 *>(dBv + e));
             const float br = sbeta[r];
             const float Gv[4] = {G4.x, G4.y, G4.z, G4.w}, Gt[4] = {Gl.x, Gl.y, Gl.z, Gl.w};
             const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
@@ -2060,7 +2061,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int u = 0; u < SR; ++u) {
                 const int r = r0 + u;
                 loc += sq[r * LDD + c];
-                lkh = fmaf(dKh[r * D + c] * sk[r * LDD + c], __expf(Gl - sG[r * LDD + c]), lkh);
+                lkh = fmaf(__ldcg(dKh + r * D + c) * sk[r * LDD + c], __expf(Gl - sG[r * LDD + c]), lkh);
             }
             sseg[sgi * D + c] = loc;
             sseg[kBwdThreads + sgi * D + c] = lkh;
@@ -2071,7 +2072,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float gp[SR];
 #pragma unroll
             for (int u = 0; u < SR; ++u)
-                gp[u] = Gp[(r0 + u) * D + c];
+                gp[u] = __ldcg(Gp + (r0 + u) * D + c);
             float acc = sdGam[c] * __expf(sG[(kC - 1) * LDD + c]);
             for (int s2 = 0; s2 < NSEG; ++s2)
                 acc += sseg[kBwdThreads + s2 * D + c];
@@ -2098,27 +2099,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     sred[warp] = dal;
             }
         }
-        // 10. dbeta_r = sum_c dBk_rc Kbar_rc + sum_c dBv_rc v_rc + sum_s dA_rs A'_rs; warp per row
+        // 10. dbeta_r = sum_c dBk_rc Kbar_rc + sum_c dBv_rc v_rc + sum_s dA_rs A'_rs; warp per row,
+        //     the warp's rows summed together (rows past the chunk read row 0 and store nothing)
+        {
+            constexpr int RPW = kC / kBwdWarps;
+            float acc[RPW];
 #pragma unroll
-        for (int rr = 0; rr < kC / kBwdWarps; ++rr) {
-            const int r = warp + rr * kBwdWarps;
-            if (r >= n)
-                break;
-            float acc = 0.f;
+            for (int rr = 0; rr < RPW; ++rr) {
+                const int r = warp + rr * kBwdWarps, rv = r < n ? r : 0;
+                float a = 0.f;
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                const int c = lane + 32 * cc;
-                acc += dBk[r * D + c] * Kb[r * D + c] +
-                       dBv[r * D + c] * __bfloat162float(vg[(size_t)tix(r) * D + c]);
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    const int c = lane + 32 * cc;
+                    a += __ldcg(dBk + r * D + c) * __ldcg(Kb + r * D + c) +
+                         __ldcg(dBv + r * D + c) * __bfloat162float(vg[(size_t)tix(rv) * D + c]);
+                }
+#pragma unroll
+                for (int ss = 0; ss < kC / 32; ++ss)
+                    a += sdA[r * LDC + lane + 32 * ss] * sAp[r * LDC + lane + 32 * ss];
+                acc[rr] = a;
             }
 #pragma unroll
-            for (int ss = 0; ss < kC / 32; ++ss)
-                acc += sdA[r * LDC + lane + 32 * ss] * sAp[r * LDC + lane + 32 * ss];
+            for (int rr = 0; rr < RPW; ++rr) {
+                float a = acc[rr];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0)
-                dbeta[tix(r)] = acc;
+                for (int o = 16; o > 0; o >>= 1)
+                    a += __shfl_xor_sync(0xffffffffu, a, o);
+                const int r = warp + rr * kBwdWarps;
+                if (lane == 0 && r < n)
+                    dbeta[tix(r)] = a;
+            }
         }
         __syncthreads();  // shared memory and the slot are reused by the next chunk
         if (dA_part && tid == 0) {

@@ -1393,9 +1393,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 
 // ------------------------------------------------------------------ per-chunk gradients
 // Persistent: kBwdSlots CTAs of 512 threads walk the chunks.  q, k, G and the chunk's 64 x 64
-// matrices stay in shared memory; the 64 x D intermediates live in a float32 scratch slot of
-// the workspace per CTA (written and read back by the same CTA; L2 holds part of it).  Dense
-// contractions go through cta_gemm (TF32 mma.sync, fp32 accumulation).  The pairwise decay
+// matrices A', T, dT and dA stay in shared memory; P and the 64 x D intermediates live in a
+// float32 scratch slot of the workspace per CTA (written and read back by the same CTA; L2
+// holds part of it).  Dense contractions go through cta_gemm (TF32 mma.sync, fp32
+// accumulation).  The pairwise decay
 // products are 16 x 16 tile pairs on the same mma, with the decay factored through a
 // reference token of the ROW tile (the forward's prep uses the column tile's middle token;
 // either factoring is exact): the row tile's first token for tiles below the diagonal (both

@@ -950,17 +950,34 @@ constexpr int kScanWarps = 4;                        // consumer warps (one TMEM
 constexpr int kScanThreads = (kScanWarps + 1) * 32;  // + one producer warp
 constexpr int kStages = 3;
 
-template <int D>
+template <int D, bool kSave>
 struct ScanSmem {
     static constexpr uint32_t kStageBytes = Rec<D>::Shared + Rec<D>::Blk;  // shared part + own value block
     static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
     alignas(1024) unsigned char stage[kStages][kStageStride];
     alignas(1024) unsigned char sbuf[D * kBV * 2];  // S block, bf16, MN-major 64-byte swizzle (row = key channel)
+    // kSave: the float32 block entering a chunk, double-buffered, for the tensor store
+    alignas(1024) unsigned char hbuf[2][kSave ? D * kBV * 4 : 16];
     uint64_t full[kStages];                         // stage filled (arrive + bytes)
     uint64_t empty[kStages];                        // stage released by the consumers
     uint64_t mma_bar;                               // tcgen05 MMA batch completed
     uint32_t tmem_slot;
 };
+
+// Byte offset of (row, column j < kBV) in a saved float32 state block as the tensor store
+// reads it: rows of kBV floats (128 B), 16-byte chunks XOR (row & 7) (the 128-byte swizzle).
+__device__ __forceinline__ uint32_t hblk_off(int row, int j)
+{
+    return (uint32_t)row * 128u + ((uint32_t)((j >> 2) ^ (row & 7)) << 4) + (uint32_t)(j & 3) * 4u;
+}
+
+// One thread row's kBV floats into a saved-block buffer.
+__device__ __forceinline__ void stage_state_f32(unsigned char *buf, int row, const float (&S)[kBV])
+{
+#pragma unroll
+    for (int j = 0; j < kBV; j += 4)
+        *reinterpret_cast<float4 *>(buf + hblk_off(row, j)) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+}
 
 __device__ __forceinline__ void consumer_sync()
 {
@@ -988,10 +1005,10 @@ template <int D, bool kAffine, bool kSave>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, float *__restrict__ M_out,
-                float *__restrict__ Hs, unsigned int *status)
+                const __grid_constant__ CUtensorMap hs_map, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char scan_smem[];
-    using SM = ScanSmem<D>;
+    using SM = ScanSmem<D, kSave>;
     using R = Rec<D>;
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
     constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N S; [kBV, 2 kBV): Q' S
@@ -1069,6 +1086,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 S[j + 3] = v.w;
             }
             store_state(sm.sbuf, row, S);
+            if constexpr (kSave)
+                stage_state_f32(sm.hbuf[0], row, S);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -1080,14 +1099,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         uint32_t mma_phase = 0;
         for (int c = 0; c < NT; ++c) {
             const int s = c % kStages;
-            if constexpr (kSave) {
-                if (srow) {
-                    float4 *hp = reinterpret_cast<float4 *>(Hs + ((seq.rec0 + c) * D + row) * D + col0);
-#pragma unroll
-                    for (int j = 0; j < kBV; j += 4)
-                        hp[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-                }
-            }
             mbar_wait_bounded(&sm.full[s], (c / kStages) & 1, status);
             const unsigned char *st = sm.stage[s];
             const uint32_t st_a = smem_u32(st);
@@ -1095,6 +1106,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             // [N S | Q' S] in one round (rows past N (D = 64) and past Q' are don't-cares)
             if (tid == 0) {
                 tc::fence_after_sync();
+                if constexpr (kSave) {
+                    // the block entering chunk c, staged by every row thread before the last
+                    // consumer barrier; wait until the store of chunk c - 1 has read its buffer,
+                    // which the rows refill (for chunk c + 1) only after this round's MMAs
+                    tma_store_2d(&hs_map, col0, (int)((seq.rec0 + c) * D), sm.hbuf[c & 1]);
+                    bulk_commit();
+                    bulk_wait_read_1();
+                }
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
@@ -1137,6 +1156,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 for (int j = 0; j < kBV; ++j)
                     S[j] -= __uint_as_float(d[j]);
                 store_state(sm.sbuf, row, S);
+                if constexpr (kSave) {
+                    if (c + 1 < NT)
+                        stage_state_f32(sm.hbuf[(c + 1) & 1], row, S);
+                }
                 tc::fence_smem_to_async();
             }
             // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
@@ -1169,6 +1192,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 mbar_arrive_local(&sm.empty[s]);
         }
 
+        if constexpr (kSave) {
+            if (tid == 0)
+                bulk_wait_all();  // the last blocks are written before the CTA leaves
+        }
         float *Sout = xfer ? M_out : S_T;
         if (Sout && srow)
 #pragma unroll
@@ -1216,6 +1243,7 @@ struct DScanSmem {
     alignas(1024) unsigned char stage[kStages][kStageStride];
     alignas(1024) unsigned char sbuf[D * kBV * 2];   // dS' block, bf16, MN-major 64-byte swizzle
     alignas(1024) unsigned char obuf[kC * kBV * 2];  // dO block of the chunk, same layout (row = token)
+    alignas(1024) unsigned char hbuf[2][D * kBV * 4];  // float32 block for the tensor store, double-buffered
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t mma_bar;
@@ -1225,8 +1253,8 @@ struct DScanSmem {
 template <int D>
 __global__ void __launch_bounds__(kScanThreads, 1)
     dscan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const __nv_bfloat16 *__restrict__ dO,
-                 const float *__restrict__ dS_T, float *__restrict__ dHs, float *__restrict__ dS0,
-                 unsigned int *status)
+                 const float *__restrict__ dS_T, const __grid_constant__ CUtensorMap dhs_map,
+                 float *__restrict__ dS0, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char dscan_smem[];
     using SM = DScanSmem<D>;
@@ -1316,12 +1344,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         uint32_t mma_phase = 0;
         for (int i = 0; i < NT; ++i) {
             const int c = NT - 1 - i, s = i % kStages;
-            // dS' of chunk c (the gradient of the state after it) is what the rows hold now
+            // dS' of chunk c (the gradient of the state after it) is what the rows hold now; its
+            // float32 block goes out by a tensor store (buffer i & 1: the store of iteration i - 2
+            // has read it, thread 0 waited for that before the last barrier of iteration i - 1)
             if (srow) {
-                float4 *hp = reinterpret_cast<float4 *>(dHs + ((seq.rec0 + c) * D + row) * D + col0);
-#pragma unroll
-                for (int j = 0; j < kBV; j += 4)
-                    hp[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                stage_state_f32(sm.hbuf[i & 1], row, S);
                 store_state(sm.sbuf, row, S);
             }
             if (trow) {
@@ -1340,6 +1367,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             const uint32_t st_a = smem_u32(st);
             if (tid == 0) {
                 tc::fence_after_sync();
+                tma_store_2d(&dhs_map, col0, (int)((seq.rec0 + c) * D), sm.hbuf[i & 1]);
+                bulk_commit();
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint64_t an = tc::smem_desc(st_a + R::Nm + ks * 2048, D * 128, 1024, tc::kSw128);
@@ -1372,12 +1401,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 for (int j = 0; j < kBV; ++j)
                     S[j] += __uint_as_float(y[j]) - __uint_as_float(d[j]);
             }
+            if (tid == 0)
+                bulk_wait_read_1();  // the store of iteration i - 1 has read buffer (i + 1) & 1
             tc::fence_before_sync();
             consumer_sync();
             tc::fence_after_sync();
             if (tid == 0)
                 mbar_arrive_local(&sm.empty[s]);
         }
+        if (tid == 0)
+            bulk_wait_all();  // the last blocks are written before the CTA leaves
         if (dS0 && srow)
 #pragma unroll
             for (int j = 0; j < kBV; j += 4)
@@ -2199,6 +2232,25 @@ cudaError_t make_token_map(CUtensorMap *m, const void *base, int D, int H, int64
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// A float32 array of D x D state blocks (one per record) as a tensor map of nrec * D rows of D
+// floats, boxes of 32 columns x D rows with the 128-byte swizzle (the scans' saved blocks).
+cudaError_t make_state_map(CUtensorMap *m, float *base, int64_t nrec, int D)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    if (nrec * D >= ((int64_t)1 << 31))  // row coordinates are 32-bit
+        return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(nrec * D)};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)kBV, (cuuint32_t)D};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // The gate table (launch_gate_table) lives in the workspace at `gtab`; the prep looks g up in it.
 template <int D, bool kLogSig>
 cudaError_t launch_prep_d(const SeqMap &m, int H, dim3 grid, const void *q, const void *k, const void *v,
@@ -2238,14 +2290,18 @@ cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
-    const size_t smem = sizeof(ScanSmem<D>) + 1024;  // + alignment slack
+    // + alignment slack; the state-saving variant holds two more float32 blocks
+    const size_t smem = (Hs ? sizeof(ScanSmem<D, true>) : sizeof(ScanSmem<D, false>)) + 1024;
     // with M_out: the state blocks and, after them, as many transfer-map blocks
     auto kernel = Hs ? scan_kernel<D, false, true> : M_out ? scan_kernel<D, true, false> : scan_kernel<D, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
+    CUtensorMap hs_map{};
+    if (Hs && (e = make_state_map(&hs_map, Hs, m.nrec, D)) != cudaSuccess)
+        return e;
     kernel<<<dim3((M_out ? 2 : 1) * (D / kBV), m.nseq * H), kScanThreads, smem, s>>>(
-        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, M_out, Hs, status);
+        m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, M_out, hs_map, status);
     return cudaGetLastError();
 }
 
@@ -2319,8 +2375,12 @@ cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits,
     e = cudaFuncSetAttribute(dscan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
+    CUtensorMap dhs_map{};
+    if ((e = make_state_map(&dhs_map, dHs, m.nrec, D)) != cudaSuccess)
+        return e;
     dscan_kernel<D><<<dim3(D / kBV, m.nseq * H), kScanThreads, smem, s>>>(
-        m, H, static_cast<const unsigned char *>(ws), static_cast<const __nv_bfloat16 *>(dO), dS_T, dHs, dS0, status);
+        m, H, static_cast<const unsigned char *>(ws), static_cast<const __nv_bfloat16 *>(dO), dS_T, dhs_map, dS0,
+        status);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;

@@ -259,6 +259,16 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *tm, in
         : "memory");
 }
 
+// Tiled tensor store (TMA) of one box from this CTA's shared memory to a tensor map in this
+// GPU's memory, tracked by bulk groups; coordinates as for the loads (never negative).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, int x, int y, const void *src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+
 // Bulk (non-tensor) async copy shared -> global, tracked by bulk groups.
 __device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes)
 {

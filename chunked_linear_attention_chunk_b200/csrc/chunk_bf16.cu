@@ -999,8 +999,9 @@ __device__ __forceinline__ void store_state(unsigned char *sbuf, int row, const 
                        pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
 }
 
-// kSave: also write the fp32 state entering every chunk to Hs (one D x D block per record,
-// indexed like the records), for the backward.
+// kSave: also write the fp32 state entering every chunk to the state array of hs_map (one
+// D x D block per record, indexed like the records), for the backward: the rows stage their
+// block in shared memory and one thread stores it with a 2-D tensor store per chunk.
 template <int D, bool kAffine, bool kSave>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
@@ -1232,7 +1233,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 // One CTA per (32-column block of dv, sequence*head), chunks in reverse order.  Per chunk one
 // tcgen05 round computes [N^T dS' | Q'^T dO]: N and Q' are the record's K-major operands,
 // read here as MN-major (transposed) A operands; dS' (bf16 copy) and the chunk's dO block
-// are MN-major B operands.  The fp32 gradient block stays in registers, one row per thread.
+// are MN-major B operands.  The fp32 gradient block stays in registers, one row per thread;
+// every chunk's block (the gradient of the state after it) leaves by a 2-D tensor store.
 template <int D>
 struct DScanSmem {
     // An M = 128 MN-major read of Q' (and of N when D = 64) covers two 64-row MN blocks; past

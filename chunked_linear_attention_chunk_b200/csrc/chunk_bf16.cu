@@ -446,14 +446,18 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             *reinterpret_cast<float2 *>(&sTot[I * D + c0]) = make_float2(x0, x1);
             *reinterpret_cast<float2 *>(&sMid[I * D + c0]) = make_float2(G0[kRef], G1[kRef]);
             asm volatile("bar.sync 1, %0;" ::"n"(NFW * 32) : "memory");
-            // offsets of every tile (sums in tile order), this tile's references
-            float off0[kTiles], off1[kTiles];
+            // offsets of every tile (sums in tile order), this tile's references; every tile's total
+            // and local reference value read here, before this warp's stores below
+            float off0[kTiles], off1[kTiles], ref0[kTiles], ref1[kTiles];
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int J = 0; J < kTiles; ++J) {
                 off0[J] = a0;
                 off1[J] = a1;
                 const float2 t = *reinterpret_cast<const float2 *>(&sTot[J * D + c0]);
+                const float2 m = kLogSig ? t : *reinterpret_cast<const float2 *>(&sMid[J * D + c0]);
+                ref0[J] = m.x;
+                ref1[J] = m.y;
                 a0 += t.x;
                 a1 += t.y;
             }
@@ -469,13 +473,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                 G1[s2] += o1;
             }
             // column reference of tile J (a G value; J is a compile-time index wherever used)
-            auto col_ref = [&](int J, int ch) -> float {
-                const float o = ch ? off1[J] : off0[J];
-                if constexpr (kLogSig)
-                    return o + sTot[J * D + c0 + ch];
-                else
-                    return o + sMid[J * D + c0 + ch];
-            };
+            auto col_ref = [&](int J, int ch) -> float { return ch ? off1[J] + ref1[J] : off0[J] + ref0[J]; };
             // this tile's row and column references
             if constexpr (kLogSig) {
                 rr0 = o0, rr1 = o1;
@@ -555,6 +553,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         //       zero in all three and in v (a packed batch loaded the next sequence there)
         if (fw) {
             mbar_wait_bounded(bar_qkv, 0, status);
+            // the tile's k and q first: the stores below go to the same arrays, so loads placed
+            // after them could not be moved ahead
+            uint32_t kw[kTile], qw[kTile];
+#pragma unroll
+            for (int s2 = 0; s2 < kTile; ++s2) {
+                const uint32_t d = tok_off(I * kTile + s2, c0);
+                kw[s2] = *reinterpret_cast<const uint32_t *>(sm + L::RK + d);
+                qw[s2] = *reinterpret_cast<const uint32_t *>(sm + L::RQ + d);
+            }
 #pragma unroll
             for (int s2 = 0; s2 < kTile; ++s2) {
                 const int r = I * kTile + s2;
@@ -563,8 +570,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                 const float y0 = cr0 - G0[s2], y1 = cr1 - G1[s2];
                 uint32_t kr = 0u, qr = 0u, ec = 0u;
                 if (r < n) {
-                    const float2 kk = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + L::RK + d));
-                    const float2 qq = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + L::RQ + d));
+                    const float2 kk = unpack_bf16x2(kw[s2]);
+                    const float2 qq = unpack_bf16x2(qw[s2]);
                     const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(y0), i1 = __expf(y1);
                     kr = pack_bf16x2(kk.x * e0, kk.y * e1);
                     qr = pack_bf16x2(qq.x * e0, qq.y * e1);
@@ -676,6 +683,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     //         start T = (I + A)^{-1} with the 16x16 diagonal blocks (forward substitution,
     //         one lane per column).  Then block substitution level by level.
     if (warp >= kTiles) {
+        // each item's loads before its stores (they write the arrays they read)
         for (int i = tid - kTiles * 32; i < kC * CPR; i += kPrepThreads - kTiles * 32) {
             const int r = i / CPR, c8 = (i % CPR) * 8;
             const int tile = r / kTile;
@@ -684,12 +692,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             const uint4 eml = *reinterpret_cast<const uint4 *>(&sEm[(kTiles + tile) * D + c8]);
             const uint4 elh = *reinterpret_cast<const uint4 *>(&sEl[tile * D + c8]);
             const uint4 ell = *reinterpret_cast<const uint4 *>(&sEl[(kTiles + tile) * D + c8]);
-            uint4 *pk = reinterpret_cast<uint4 *>(sm + L::RK + d);
-            uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + d);
-            uint4 *px = reinterpret_cast<uint4 *>(sm + L::RX + d);
-            *pk = mul8_hilo(*pk, emh, eml);
-            *pq = mul8_hilo(*pq, emh, eml);
-            *px = mul8_hilo(*px, elh, ell);
+            const uint4 vk = *reinterpret_cast<const uint4 *>(sm + L::RK + d);
+            const uint4 vq = *reinterpret_cast<const uint4 *>(sm + L::RQ + d);
+            const uint4 vx = *reinterpret_cast<const uint4 *>(sm + L::RX + d);
+            *reinterpret_cast<uint4 *>(sm + L::RK + d) = mul8_hilo(vk, emh, eml);
+            *reinterpret_cast<uint4 *>(sm + L::RQ + d) = mul8_hilo(vq, emh, eml);
+            *reinterpret_cast<uint4 *>(sm + L::RX + d) = mul8_hilo(vx, elh, ell);
         }
     } else if (lane < kTile) {
         const int I = warp, c = lane;
@@ -720,13 +728,27 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     // T diag(beta) as the K-major A operand (over A's place), written twice: as rows 0..63
     // and again as rows 64..127 of the M = 128 MMA, so TMEM lanes 64..127 hold a second copy
     // of the result and all four lane quarters can drain it
-    for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
-        const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
-        const bool upper = j / kTile > r / kTile;  // those blocks of T are zero and never written
-        const uint32_t tb =
-            upper ? 0u : pack_bf16x2(sT[r * LDA + j] * sBeta[j], sT[r * LDA + j + 1] * sBeta[j + 1]);
-        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) = tb;
-        *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(kC + r, j, kC)) = tb;
+    {  // every load first (T's region is not the one written, but the compiler cannot tell)
+        constexpr int NIT = (kC * (kC / 2) + kPrepThreads - 1) / kPrepThreads;
+        float t0[NIT], t1[NIT], b0[NIT], b1[NIT];
+#pragma unroll
+        for (int it = 0; it < NIT; ++it) {
+            const int i = tid + it * kPrepThreads, r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+            const bool live = i < kC * (kC / 2) && j / kTile <= r / kTile;  // blocks above: zero
+            t0[it] = live ? sT[r * LDA + j] : 0.f;
+            t1[it] = live ? sT[r * LDA + j + 1] : 0.f;
+            b0[it] = live ? sBeta[j] : 0.f;
+            b1[it] = live ? sBeta[j + 1] : 0.f;
+        }
+#pragma unroll
+        for (int it = 0; it < NIT; ++it) {
+            const int i = tid + it * kPrepThreads, r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+            if (i < kC * (kC / 2)) {
+                const uint32_t tb = pack_bf16x2(t0[it] * b0[it], t1[it] * b1[it]);
+                *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(r, j, kC)) = tb;
+                *reinterpret_cast<uint32_t *>(sm + L::RG + tc::kmaj_sw128(kC + r, j, kC)) = tb;
+            }
+        }
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -866,11 +888,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         for (int c0 = 0; c0 < D / 2; c0 += 32) {
             uint32_t x[32];
             tc::ld_32x32b_x32(tc::taddr(tmem, (warp & 3) * 32, D + chalf + c0), x);
+            uint4 qbs[4];  // Qbar's four 8-column chunks, loaded before any of them is written back
+#pragma unroll
+            for (int j = 0; j < 32; j += 8)
+                qbs[j / 8] = *reinterpret_cast<const uint4 *>(sm + L::RQ + tok_off(lrow, chalf + c0 + j));
             tc::wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {
                 uint4 *pq = reinterpret_cast<uint4 *>(sm + L::RQ + tok_off(lrow, chalf + c0 + j));
-                const uint4 qb = *pq;
+                const uint4 qb = qbs[j / 8];
                 const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
                 uint32_t o4[4];
 #pragma unroll

@@ -1122,6 +1122,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc::fence_after_sync();
 
         const uint32_t id_k = tc::idesc_bf16(128, kBV, false, true);  // A K-major, B MN-major
+        // The MMA round is issued from warp 2 so that warps 0 and 1 (TMEM lanes 0..63, the chunk's
+        // rows) can finish a chunk's output after the closing barrier while the next round runs.
+        constexpr int kIssuer = 64;
         const uint32_t sbuf_a = smem_u32(sm.sbuf);
         uint32_t mma_phase = 0;
         for (int c = 0; c < NT; ++c) {
@@ -1131,7 +1134,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             const uint32_t st_a = smem_u32(st);
 
             // [N S | Q' S] in one round (rows past N (D = 64) and past Q' are don't-cares)
-            if (tid == 0) {
+            if (tid == kIssuer) {
                 tc::fence_after_sync();
                 if constexpr (kSave) {
                     // the block entering chunk c, staged by every row thread before the last
@@ -1174,10 +1177,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             tc::fence_after_sync();
 
             const unsigned char *blkp = st + R::Shared;
+            const bool orow_w = o && warp < 2;  // O = Q' S + O' for chunk rows 0..63 (warps 0 and 1)
+            uint32_t y[kBV];
+            uint4 ou[kBV / 8];
             // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk
             if (srow) {
                 uint32_t d[kBV];
                 tc::ld_32x32b_x32(lane_addr, d);
+                if (orow_w)
+                    tc::ld_32x32b_x32(lane_addr + kBV, y);
                 tc::wait_ld();
 #pragma unroll
                 for (int j = 0; j < kBV; ++j)
@@ -1189,18 +1197,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 }
                 tc::fence_smem_to_async();
             }
-            // O = Q' S + O' for chunk rows 0..63 (TMEM lanes 0..63: warps 0 and 1)
-            if (o && warp < 2) {
-                uint32_t y[kBV];
-                tc::ld_32x32b_x32(lane_addr + kBV, y);
-                tc::wait_ld();
+            // the O' rows too before the barrier (the stage is released after it)
+            if (orow_w) {
+#pragma unroll
+                for (int j = 0; j < kBV; j += 8)
+                    ou[j / 8] = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
+            }
+            tc::fence_before_sync();
+            consumer_sync();
+            tc::fence_after_sync();
+            if (tid == kIssuer)
+                mbar_arrive_local(&sm.empty[s]);
+            if (orow_w) {  // the output while the next chunk's round runs
                 const int t = c * kC + row;
                 if (t < seq.len) {
                     uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
 #pragma unroll
                     for (int j = 0; j < kBV; j += 8) {
-                        const uint4 ou = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
-                        const uint32_t ow[4] = {ou.x, ou.y, ou.z, ou.w};
+                        const uint32_t ow[4] = {ou[j / 8].x, ou[j / 8].y, ou[j / 8].z, ou[j / 8].w};
                         uint32_t r4[4];
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
@@ -1212,15 +1226,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     }
                 }
             }
-            tc::fence_before_sync();
-            consumer_sync();
-            tc::fence_after_sync();
-            if (tid == 0)
-                mbar_arrive_local(&sm.empty[s]);
         }
 
         if constexpr (kSave) {
-            if (tid == 0)
+            if (tid == kIssuer)
                 bulk_wait_all();  // the last blocks are written before the CTA leaves
         }
         float *Sout = xfer ? M_out : S_T;

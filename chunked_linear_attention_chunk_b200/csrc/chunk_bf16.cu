@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     // -- 4b/5. warps 4 and up: chunk-referenced operands in place (Kbar = Kr e^{G_m},
     //         Qbar = Qr e^{G_m}, Khat = Ec e^{G_last - G_m}); at the same time warps 0..3
     //         start T = (I + A)^{-1} with the 16x16 diagonal blocks (forward substitution,
-    //         one lane per column).  Then block substitution level by level.
+    //         one lane per column).  Then block substitution, one warp per block column.
     if (warp >= kTiles) {
         // each item's loads before its stores (they write the arrays they read)
         for (int i = tid - kTiles * 32; i < kC * CPR; i += kPrepThreads - kTiles * 32) {
@@ -719,12 +719,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             sT[(I * kTile + r) * LDA + I * kTile + c] = x[r];
     }
     __syncthreads();
-    for (int lvl = 1; lvl < kTiles; ++lvl) {  // level lvl: blocks (J + lvl, J), one warp each
-        if (warp < kTiles - lvl)
-            solve_block_tf32<kC + 1>(sA, sT, sA + (warp + 1) * kTile /* upper block (0, warp+1) of A */, warp + lvl,
-                             warp, lane);
-        __syncthreads();
+    // block column J on warp J, top to bottom: block (I, J) needs only T_KJ (J <= K < I, this
+    // warp's own earlier blocks) and the diagonal T_II, so the warps need no CTA barrier between
+    if (warp < kTiles - 1) {
+        for (int I = warp + 1; I < kTiles; ++I) {
+            solve_block_tf32<kC + 1>(sA, sT, sA + (warp + 1) * kTile /* upper block (0, warp+1) of A */, I, warp,
+                                     lane);
+            __syncwarp();
+        }
     }
+    __syncthreads();
     // T diag(beta) as the K-major A operand (over A's place), written twice: as rows 0..63
     // and again as rows 64..127 of the M = 128 MMA, so TMEM lanes 64..127 hold a second copy
     // of the result and all four lane quarters can drain it
@@ -1919,8 +1923,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncthreads();
         // 5. T = (I + A)^{-1}, A = diag(beta) A', unit lower triangular, by 16 x 16 blocks: the
         //    diagonal blocks by forward substitution (one lane per column, the column in registers),
-        //    then block rows by level, T_IJ = -T_II diag(beta_I) sum_{K=J}^{I-1} A'_IK T_KJ, one warp
-        //    per block with tf32 tensor-core products.
+        //    then the blocks below, T_IJ = -T_II diag(beta_I) sum_{K=J}^{I-1} A'_IK T_KJ, one warp per
+        //    block column with tf32 tensor-core products.
         if (warp < kTiles && lane < kTile) {
             const int I = warp, c = lane;
             float x[kTile];
@@ -1941,11 +1945,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 sT[(I * kTile + r) * LDC + I * kTile + c] = x[r];
         }
         __syncthreads();
-        for (int lvl = 1; lvl < kTiles; ++lvl) {
-            if (warp < kTiles - lvl)  // scratch: a 16 x 16 block of sdT per warp (free until step 6)
-                solve_block_tf32<LDC>(sAp, sT, sdT + warp * kTile * LDC, warp + lvl, warp, lane, sbeta);
-            __syncthreads();
+        if (warp < kTiles - 1) {  // block column J on warp J, top to bottom (no CTA barrier between)
+            for (int I = warp + 1; I < kTiles; ++I) {
+                // scratch: a 16 x 16 block of sdT per warp (free until step 6)
+                solve_block_tf32<LDC>(sAp, sT, sdT + warp * kTile * LDC, I, warp, lane, sbeta);
+                __syncwarp();
+            }
         }
+        __syncthreads();
         // 6. dense contractions
         // A operand T: kSmemK over sT; T^T: kSmemM over sT.  Row-major 64 x D blocks of the slot
         // are kGlobK as A, kGlobMN as B; S and dS' (row-major D x D) are kGlobMN as B, and their

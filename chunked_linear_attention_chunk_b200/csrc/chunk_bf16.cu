@@ -462,11 +462,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                 a1 += t.y;
             }
             gl0 = a0, gl1 = a1;
-            float o0 = 0.f, o1 = 0.f;
+            float o0 = 0.f, o1 = 0.f, ti0 = 0.f, ti1 = 0.f;
 #pragma unroll
             for (int J = 0; J < kTiles; ++J)
                 if (J == I)
-                    o0 = off0[J], o1 = off1[J];
+                    o0 = off0[J], o1 = off1[J], ti0 = ref0[J], ti1 = ref1[J];
+            // the tables in P's slot are read: the warps the front end leaves idle may zero P
+            asm volatile("bar.arrive 2, %0;" ::"n"(kPrepThreads) : "memory");
 #pragma unroll
             for (int s2 = 0; s2 < kTile; ++s2) {
                 G0[s2] += o0;
@@ -477,7 +479,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             // this tile's row and column references
             if constexpr (kLogSig) {
                 rr0 = o0, rr1 = o1;
-                cr0 = o0 + sTot[I * D + c0], cr1 = o1 + sTot[I * D + c0 + 1];
+                cr0 = o0 + ti0, cr1 = o1 + ti1;  // the tile's total (ref is the total here)
             } else {
                 rr0 = cr0 = G0[kRef];
                 rr1 = cr1 = G1[kRef];
@@ -503,6 +505,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
                 for (int s2 = 0; s2 < kTile; ++s2)
                     *reinterpret_cast<float2 *>(&sG[(I * kTile + s2) * D + c0]) = make_float2(G0[s2], G1[s2]);
+            }
+        } else {
+            // upper blocks of P are zero (its slot holds the cumulative-sum tables until every
+            // front-end warp has read them)
+            asm volatile("bar.sync 2, %0;" ::"n"(kPrepThreads) : "memory");
+            for (int i = tid - NFW * 32; i < kC * (kC / 2); i += kPrepThreads - NFW * 32) {
+                const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
+                if (j / kTile > r / kTile)
+                    *reinterpret_cast<uint32_t *>(sm + L::RP + tc::kmaj_sw128(r, j, kC)) = 0u;
             }
         }
 
@@ -587,12 +598,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     __syncthreads();
 
-    // upper blocks of P are zero (its slot held the cumulative-sum tables until here)
-    for (int i = tid; i < kC * (kC / 2); i += kPrepThreads) {
-        const int r = i / (kC / 2), j = (i % (kC / 2)) * 2;
-        if (j / kTile > r / kTile)
-            *reinterpret_cast<uint32_t *>(sm + L::RP + tc::kmaj_sw128(r, j, kC)) = 0u;
-    }
 
     // -- 4. dense 16-token tile products A and P, one warp per (row tile I, column tile
     //       J <= I): row operands Kr, Qr of tile I (scaled by e^{G_{m_I} - G_{m_J}} when

@@ -566,7 +566,8 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
     kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
     if (st != KDA_OK)
         return st;
-    if (dtype != KDA_BF16 || (int64_t)B * H * (((int64_t)T + 63) / 64) > 0x7fffffff)
+    // the saved state arrays are addressed as (records x dk) rows with 32-bit coordinates
+    if (dtype != KDA_BF16 || (int64_t)B * H * (((int64_t)T + 63) / 64) * dk > 0x7fffffff)
         return KDA_ERR_UNSUPPORTED;
     st = check_gmin(g_min);
     if (st != KDA_OK)
@@ -636,7 +637,7 @@ kda_status kda_chunk_bwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, 
     if (st != KDA_OK)
         return st;
     if (dk != dv || (dk != 64 && dk != 128) || dtype != KDA_BF16 || T > kMaxPackedTokens || (int64_t)N * H > 65535 ||
-        (int64_t)H * (((int64_t)T + 63) / 64 + N) > 0x7fffffff)
+        (int64_t)H * (((int64_t)T + 63) / 64 + N) * dk > 0x7fffffff)
         return KDA_ERR_UNSUPPORTED;
     if (!cu_seqlens || (dA_log && !A_log))
         return KDA_ERR_INVALID_ARG;

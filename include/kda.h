@@ -302,8 +302,9 @@ kda_status kda_state_combine(int R, int B, int H, int dk, int dv, const float *M
  *                that order, from the byte offsets kda_chunk_bwd_offsets gives), then the
  *                gradient kernel's scratch.
  * The outputs must not overlap each other, an input or the workspace.
- * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, ALIAS, WORKSPACE, CUDA.  T == 0 writes dS0 =
- * dS_T (or zeros), dA_log = 0, and nothing else.
+ * Errors: INVALID_ARG, UNSUPPORTED (also when B * H * ceil(T / 64) * dk >= 2^31: the saved
+ * state arrays are written as that many rows of dv floats, by row index), ALIGNMENT, ALIAS,
+ * WORKSPACE, CUDA.  T == 0 writes dS0 = dS_T (or zeros), dA_log = 0, and nothing else.
  *
  * kda_chunk_bwd_varlen -- the same over a packed batch of N sequences on one token axis, as
  * kda_chunk_fwd_varlen lays it out (cu_seqlens on the device and checked there; each

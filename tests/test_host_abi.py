@@ -344,6 +344,11 @@ def test_chunk_bwd_entry_validates(L):
 
     assert bwd(dtype=kda.KDA_F32) == UNSUPPORTED
     assert bwd(dk=96) == UNSUPPORTED
+    # the saved state arrays are (records x dk) rows addressed with 32-bit row indices
+    big = lambda T_, H_, dk_: L.kda_chunk_bwd(1, T_, H_, dk_, dk_, kda.KDA_BF16, *([P(BASE)] * 5), ctypes.c_float(-5.0),
+                                              None, None, P(BASE), None, *([P(BASE)] * 5), None, None, P(BASE), 1, None)
+    assert big(64 * (1 << 16), 256, 128) == UNSUPPORTED   # 2^24 records x 128 rows each
+    assert big(64 * (1 << 16), 256, 64) != UNSUPPORTED    # 2^24 records x 64 rows: within range
     assert bwd(g_min=0.0) == INVALID
     assert bwd(q=0) == INVALID
     assert bwd(dO=0) == INVALID

@@ -1161,7 +1161,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     const uint64_t aq =
                         tc::smem_desc(st_a + R::Qp + (ks >> 2) * (kC * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
                     tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
+                    if constexpr (!kSave)  // the state-saving scan forms no output
+                        tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
                 }
                 tc::commit(&sm.mma_bar);
             }
@@ -1186,7 +1187,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             tc::fence_after_sync();
 
             const unsigned char *blkp = st + R::Shared;
-            const bool orow_w = o && warp < 2;  // O = Q' S + O' for chunk rows 0..63 (warps 0 and 1)
+            const bool orow_w = !kSave && o && warp < 2;  // O = Q' S + O' for chunk rows 0..63 (warps 0, 1)
             uint32_t y[kBV];
             uint4 ou[kBV / 8];
             // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk

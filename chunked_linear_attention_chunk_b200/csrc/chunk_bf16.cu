@@ -985,16 +985,28 @@ constexpr int kScanWarps = 4;                        // consumer warps (one TMEM
 constexpr int kScanThreads = (kScanWarps + 1) * 32;  // + one producer warp
 constexpr int kStages = 3;
 
-template <int D, bool kSave>
+// Threads of a forward scan CTA over kW value blocks: four consumer warps per block (warp w
+// reads TMEM lane quarter w % 4 and block w / 4), one producer warp.
+template <int kW>
+constexpr int scan_threads() { return (kScanWarps * kW + 1) * 32; }
+
+// kW value blocks per CTA: 1, or 2 where one block per CTA would take more than one wave of
+// the GPU's SMs (the two blocks then share the stage's N and Q'; at D = 128 two stages fit
+// the shared memory, not three).
+template <int D, bool kSave, int kW = 1>
 struct ScanSmem {
-    static constexpr uint32_t kStageBytes = Rec<D>::Shared + Rec<D>::Blk;  // shared part + own value block
+    static constexpr uint32_t kStageBytes = Rec<D>::Shared + kW * Rec<D>::Blk;  // shared part + own value blocks
     static constexpr uint32_t kStageStride = (kStageBytes + 1023) / 1024 * 1024;
-    alignas(1024) unsigned char stage[kStages][kStageStride];
-    alignas(1024) unsigned char sbuf[D * kBV * 2];  // S block, bf16, MN-major 64-byte swizzle (row = key channel)
+    static constexpr int kSt =
+        kW == 1 || kStages * kStageStride + (uint32_t)D * kBV * kW * 2 + 2048 <= 232448 - 1024 ? kStages : 2;
+    alignas(1024) unsigned char stage[kSt][kStageStride];
+    // S block, bf16, MN-major (row = key channel): the 64-byte swizzle over 32 columns (kW = 1),
+    // the 128-byte swizzle over 64 (kW = 2)
+    alignas(1024) unsigned char sbuf[D * kBV * kW * 2];
     // kSave: the float32 block entering a chunk, double-buffered, for the tensor store
     alignas(1024) unsigned char hbuf[2][kSave ? D * kBV * 4 : 16];
-    uint64_t full[kStages];                         // stage filled (arrive + bytes)
-    uint64_t empty[kStages];                        // stage released by the consumers
+    uint64_t full[kSt];                             // stage filled (arrive + bytes)
+    uint64_t empty[kSt];                            // stage released by the consumers
     uint64_t mma_bar;                               // tcgen05 MMA batch completed
     uint32_t tmem_slot;
 };
@@ -1014,9 +1026,10 @@ __device__ __forceinline__ void stage_state_f32(unsigned char *buf, int row, con
         *reinterpret_cast<float4 *>(buf + hblk_off(row, j)) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
 }
 
+template <int kW = 1>
 __device__ __forceinline__ void consumer_sync()
 {
-    asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kScanWarps * kW * 32) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar)
@@ -1034,26 +1047,38 @@ __device__ __forceinline__ void store_state(unsigned char *sbuf, int row, const 
                        pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
 }
 
+// Columns [c0, c0 + kBV) of row `row` of a 64-column state block as the bf16 MMA operand
+// (MN-major, 128-byte swizzle).
+__device__ __forceinline__ void store_state_w(unsigned char *sbuf, int row, int c0, const float (&S)[kBV])
+{
+#pragma unroll
+    for (int j = 0; j < kBV; j += 8)
+        *reinterpret_cast<uint4 *>(sbuf + tc::mnmaj_sw128(row, c0 + j, 128)) =
+            make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
+                       pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+}
+
 // kSave: also write the fp32 state entering every chunk to the state array of hs_map (one
 // D x D block per record, indexed like the records), for the backward: the rows stage their
 // block in shared memory and one thread stores it with a 2-D tensor store per chunk.
-template <int D, bool kAffine, bool kSave>
-__global__ void __launch_bounds__(kScanThreads, 1)
+template <int D, bool kAffine, bool kSave, int kW = 1>
+__global__ void __launch_bounds__(scan_threads<kW>(), 1)
     scan_kernel(SeqMap map, int H, const unsigned char *__restrict__ ws, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, float *__restrict__ M_out,
                 const __grid_constant__ CUtensorMap hs_map, unsigned int *status)
 {
     extern __shared__ __align__(1024) unsigned char scan_smem[];
-    using SM = ScanSmem<D, kSave>;
+    using SM = ScanSmem<D, kSave, kW>;
     using R = Rec<D>;
+    static_assert(kW == 1 || (kW == 2 && !kAffine && !kSave && D / kBV % 2 == 0), "wide scan: plain forward only");
     SM &sm = *reinterpret_cast<SM *>(scan_smem + ((1024u - (smem_u32(scan_smem) & 1023u)) & 1023u));
-    constexpr uint32_t kTmemCols = 2 * kBV;  // [0, kBV): N S; [kBV, 2 kBV): Q' S
+    constexpr uint32_t kTmemCols = 2 * kBV * kW;  // [0, kW kBV): N S; [kW kBV, 2 kW kBV): Q' S
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // Column blocks past D / kBV (affine mode only) carry the transfer map instead of the
     // state: they start from the identity, add no Bm and write M_out.
     constexpr int NB = D / kBV;
     const bool xfer = kAffine && blockIdx.x >= NB;
-    const int blk = xfer ? blockIdx.x - NB : blockIdx.x, col0 = blk * kBV;
+    const int blk = xfer ? blockIdx.x - NB : blockIdx.x, col0 = blk * kBV * kW;
     const SeqLoc seq = locate_seq(map, H);
     if constexpr (kDebugChecks) {
         // the records this CTA reads and the token rows it can write (an invalid packed-batch
@@ -1070,7 +1095,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const unsigned char *recs = ws + seq.rec0 * R::Bytes;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < SM::kSt; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -1082,27 +1107,29 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = sm.tmem_slot;  // columns [0, kBV): N S; [kBV, 2 kBV): Q' S
+    const uint32_t tmem = sm.tmem_slot;
 
-    if (warp == kScanWarps) {
+    if (warp == kScanWarps * kW) {
         // ---------------- producer: one lane issues the bulk copies
         if (lane == 0) {
             for (int c = 0; c < NT; ++c) {
-                const int s = c % kStages;
-                if (c >= kStages)
-                    mbar_wait_bounded(&sm.empty[s], ((c / kStages) - 1) & 1, status);
+                const int s = c % SM::kSt;
+                if (c >= SM::kSt)
+                    mbar_wait_bounded(&sm.empty[s], ((c / SM::kSt) - 1) & 1, status);
                 mbar_arrive_expect_tx(&sm.full[s], SM::kStageBytes);
                 const unsigned char *rec = recs + (size_t)c * R::Bytes;
                 bulk_g2s(sm.stage[s], rec, R::Shared, &sm.full[s]);
-                bulk_g2s(sm.stage[s] + R::Shared, rec + R::Shared + blk * R::Blk, R::Blk, &sm.full[s]);
+                bulk_g2s(sm.stage[s] + R::Shared, rec + R::Shared + blk * kW * R::Blk, kW * R::Blk, &sm.full[s]);
             }
         }
         __syncwarp();
     } else {
-        // ---------------- consumers: thread `row` owns TMEM lane `row`
-        const int row = warp * 32 + lane;
+        // ---------------- consumers: thread `row` owns TMEM lane `row`; warp w takes lane
+        // quarter w % 4 of value block w / 4 (the columns from ccol on)
+        const int q4 = kW == 1 ? warp : (warp & 3), wc = kW == 1 ? 0 : (warp >> 2);
+        const int row = q4 * 32 + lane, ccol = col0 + wc * kBV;
         const bool srow = row < D;  // owns state row `row` (key channel)
-        const uint32_t lane_addr = tc::taddr(tmem, (uint32_t)warp * 32, 0);
+        const uint32_t lane_addr = tc::taddr(tmem, (uint32_t)q4 * 32, (uint32_t)(wc * kBV));
         float S[kBV];
         if (srow) {
 #pragma unroll
@@ -1114,31 +1141,34 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     v.z = row == col0 + j + 2 ? 1.f : 0.f;
                     v.w = row == col0 + j + 3 ? 1.f : 0.f;
                 } else if (S0) {
-                    v = *reinterpret_cast<const float4 *>(&S0[((size_t)bh * D + row) * D + col0 + j]);
+                    v = *reinterpret_cast<const float4 *>(&S0[((size_t)bh * D + row) * D + ccol + j]);
                 }
                 S[j] = v.x;
                 S[j + 1] = v.y;
                 S[j + 2] = v.z;
                 S[j + 3] = v.w;
             }
-            store_state(sm.sbuf, row, S);
+            if constexpr (kW == 1)
+                store_state(sm.sbuf, row, S);
+            else
+                store_state_w(sm.sbuf, row, wc * kBV, S);
             if constexpr (kSave)
                 stage_state_f32(sm.hbuf[0], row, S);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
-        consumer_sync();
+        consumer_sync<kW>();
         tc::fence_after_sync();
 
-        const uint32_t id_k = tc::idesc_bf16(128, kBV, false, true);  // A K-major, B MN-major
+        const uint32_t id_k = tc::idesc_bf16(128, kBV * kW, false, true);  // A K-major, B MN-major
         // The MMA round is issued from warp 2 so that warps 0 and 1 (TMEM lanes 0..63, the chunk's
         // rows) can finish a chunk's output after the closing barrier while the next round runs.
         constexpr int kIssuer = 64;
         const uint32_t sbuf_a = smem_u32(sm.sbuf);
         uint32_t mma_phase = 0;
         for (int c = 0; c < NT; ++c) {
-            const int s = c % kStages;
-            mbar_wait_bounded(&sm.full[s], (c / kStages) & 1, status);
+            const int s = c % SM::kSt;
+            mbar_wait_bounded(&sm.full[s], (c / SM::kSt) & 1, status);
             const unsigned char *st = sm.stage[s];
             const uint32_t st_a = smem_u32(st);
 
@@ -1155,21 +1185,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 }
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t bd = tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64);
+                    const uint64_t bd = kW == 1 ? tc::smem_desc(sbuf_a + ks * 1024, 0, 512, tc::kSw64)
+                                                : tc::smem_desc(sbuf_a + ks * 2048, D * 128, 1024, tc::kSw128);
                     const uint64_t an =
                         tc::smem_desc(st_a + R::Nm + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
                     const uint64_t aq =
                         tc::smem_desc(st_a + R::Qp + (ks >> 2) * (kC * 128) + (ks & 3) * 32, 16, 1024, tc::kSw128);
                     tc::mma_bf16(tmem, an, bd, id_k, ks > 0 ? 1u : 0u);
                     if constexpr (!kSave)  // the state-saving scan forms no output
-                        tc::mma_bf16(tmem + kBV, aq, bd, id_k, ks > 0 ? 1u : 0u);
+                        tc::mma_bf16(tmem + kBV * kW, aq, bd, id_k, ks > 0 ? 1u : 0u);
                 }
                 tc::commit(&sm.mma_bar);
             }
             // Diag(Gamma) S + Bm while the tensor core runs (stage data is in since `full`)
             if (srow) {
                 const float g = reinterpret_cast<const float *>(st + R::Gam)[row];
-                const unsigned char *bmp = st + R::Shared;
+                const unsigned char *bmp = st + R::Shared + wc * R::Blk;
 #pragma unroll
                 for (int j = 0; j < kBV; j += 8) {
                     const uint4 bu = *reinterpret_cast<const uint4 *>(bmp + tc::mnmaj_sw64(row, j));
@@ -1186,8 +1217,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             mma_phase ^= 1;
             tc::fence_after_sync();
 
-            const unsigned char *blkp = st + R::Shared;
-            const bool orow_w = !kSave && o && warp < 2;  // O = Q' S + O' for chunk rows 0..63 (warps 0, 1)
+            const unsigned char *blkp = st + R::Shared + wc * R::Blk;
+            const bool orow_w = !kSave && o && q4 < 2;  // O = Q' S + O' for chunk rows 0..63 (quarters 0, 1)
             uint32_t y[kBV];
             uint4 ou[kBV / 8];
             // S <- (Diag(Gamma) S + Bm) - N S; bf16 copy for the next chunk
@@ -1195,12 +1226,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 uint32_t d[kBV];
                 tc::ld_32x32b_x32(lane_addr, d);
                 if (orow_w)
-                    tc::ld_32x32b_x32(lane_addr + kBV, y);
+                    tc::ld_32x32b_x32(lane_addr + kBV * kW, y);
                 tc::wait_ld();
 #pragma unroll
                 for (int j = 0; j < kBV; ++j)
                     S[j] -= __uint_as_float(d[j]);
-                store_state(sm.sbuf, row, S);
+                if constexpr (kW == 1)
+                    store_state(sm.sbuf, row, S);
+                else
+                    store_state_w(sm.sbuf, row, wc * kBV, S);
                 if constexpr (kSave) {
                     if (c + 1 < NT)
                         stage_state_f32(sm.hbuf[(c + 1) & 1], row, S);
@@ -1214,14 +1248,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     ou[j / 8] = *reinterpret_cast<const uint4 *>(blkp + R::BmBlk + tc::mnmaj_sw64(row, j));
             }
             tc::fence_before_sync();
-            consumer_sync();
+            consumer_sync<kW>();
             tc::fence_after_sync();
             if (tid == kIssuer)
                 mbar_arrive_local(&sm.empty[s]);
             if (orow_w) {  // the output while the next chunk's round runs
                 const int t = c * kC + row;
                 if (t < seq.len) {
-                    uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + col0);
+                    uint4 *orow = reinterpret_cast<uint4 *>(o + ((seq.tok0 + t) * H + h) * D + ccol);
 #pragma unroll
                     for (int j = 0; j < kBV; j += 8) {
                         const uint32_t ow[4] = {ou[j / 8].x, ou[j / 8].y, ou[j / 8].z, ou[j / 8].w};
@@ -1246,7 +1280,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if (Sout && srow)
 #pragma unroll
             for (int j = 0; j < kBV; j += 4)
-                *reinterpret_cast<float4 *>(&Sout[((size_t)bh * D + row) * D + col0 + j]) =
+                *reinterpret_cast<float4 *>(&Sout[((size_t)bh * D + row) * D + ccol + j]) =
                     make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     tc::fence_before_sync();
@@ -2340,11 +2374,31 @@ cudaError_t launch_scan_d(const SeqMap &m, int H, const void *ws, const float *S
     unsigned int *status = device_status_ptr();
     if (!status)
         return cudaErrorInvalidDevice;
+    cudaError_t e;
+    if (!Hs && !M_out) {
+        // the plain forward: two value blocks per CTA where one per CTA would need more CTAs
+        // than the GPU has SMs (one scan CTA fits an SM), so the chains run in one wave
+        int dev = 0, nsm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        if ((int64_t)m.nseq * H * (D / kBV) > nsm) {
+            const size_t smem2 = sizeof(ScanSmem<D, false, 2>) + 1024;
+            e = cudaFuncSetAttribute(scan_kernel<D, false, false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem2);
+            if (e != cudaSuccess)
+                return e;
+            scan_kernel<D, false, false, 2><<<dim3(D / kBV / 2, m.nseq * H), scan_threads<2>(), smem2, s>>>(
+                m, H, static_cast<const unsigned char *>(ws), S0, static_cast<__nv_bfloat16 *>(o), S_T, nullptr,
+                CUtensorMap{}, status);
+            return cudaGetLastError();
+        }
+    }
     // + alignment slack; the state-saving variant holds two more float32 blocks
     const size_t smem = (Hs ? sizeof(ScanSmem<D, true>) : sizeof(ScanSmem<D, false>)) + 1024;
     // with M_out: the state blocks and, after them, as many transfer-map blocks
     auto kernel = Hs ? scan_kernel<D, false, true> : M_out ? scan_kernel<D, true, false> : scan_kernel<D, false, false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     CUtensorMap hs_map{};

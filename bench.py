@@ -63,7 +63,7 @@ BWD_CHUNK_BYTES_PER_TOKEN_HEAD = BWD_BYTES_PER_TOKEN_HEAD + 2 * 128 * 128 * 4 //
 # C^2/3; Gamma scaling dk dv / C), C = 16.
 FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 128 * (3 * 16 - 1) + 2 * 16 * 128 + 16 * 16 / 3 + 128 * 128 / 16
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "chunk_fwd_traffic.json")
-WORKLOADS = {"64k": synth.STAGE_64K, "8k": synth.STAGE_8K}
+WORKLOADS = {"64k": synth.STAGE_64K, "8k": synth.STAGE_8K, "16k": synth.PROFILE_16K}
 
 
 def peaks():
@@ -752,7 +752,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="64k",
-                    help="64k (the benchmark workload) or 8k (a smaller case for profiler captures)")
+                    help="64k (the benchmark workload); 8k or 16k (smaller cases for profiler captures; 16k has the 64K stage's 32 heads, so its scan takes the same one-block form)")
     ap.add_argument("--only", choices=("all", "chunk", "decode"), default="all")
     ap.add_argument("--no-ablation", action="store_true", help="skip timing the log-sigmoid ablation path")
     ap.add_argument("--no-varlen", action="store_true", help="skip timing the packed variable-length batch")

@@ -53,6 +53,8 @@ class Workload:
 TINY = Workload("tiny_B1_H2_T256_d64_f32", 1, 256, 2, 64, 64, "f32", 1000, 0.0)
 STAGE_8K = Workload("8k_B4_H16_T8192_d128_bf16", 4, 8192, 16, 128, 128, "bf16", 1001, 0.1)
 STAGE_64K = Workload("64k_B1_H32_T65536_d128_bf16_adv5pct", 1, 65536, 32, 128, 128, "bf16", 1002, 0.1, adversarial=True)
+# a quarter of the 64K stage (its 32 heads, 16384 tokens): a small case of the same kernel forms
+PROFILE_16K = Workload("16k_B1_H32_T16384_d128_bf16", 1, 16384, 32, 128, 128, "bf16", 1005, 0.1)
 STAGE_1M = Workload("1m_B1_H16_T1048576_d128_bf16_seg64k", 1, 1048576, 16, 128, 128, "bf16", 1004, 0.1, segment=65536)
 
 

@@ -31,7 +31,9 @@
 // K3 (scan) runs one CTA per (32-column block of the value dim, batch*head); a producer
 // warp streams the records through a 3-stage mbarrier pipeline with bulk copies, and per
 // chunk one tcgen05 round computes [N S, Q' S] while four consumer warps, one TMEM lane
-// (= one state row or chunk row) per thread, keep the fp32 state block in registers.
+// (= one state row or chunk row) per thread, keep the fp32 state block in registers.  With
+// more such chains than SMs, one CTA takes two blocks (eight consumer warps, an N = 64
+// round, two stages) so that all chains run in one wave.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

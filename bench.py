@@ -359,49 +359,77 @@ def stage_metrics(tokens, token_heads, states, ms, world, hbm_peak, bf16_peak, p
 
 def time_stage(kda, sw, rank, world, device, hbm_peak, bf16_peak, peak_kind, args):
     """One step of a context stage on its own seeded inputs: the 8K stage is one kda_chunk_fwd
-    over B4 H16 T8192; the 1M stage is 16 kda_chunk_fwd calls over consecutive 64K segments of
-    one sequence (each segment drawn from its own seed), the state carried in place."""
+    over B4 H16 T8192; the 1M stage is one sequence of 16 consecutive 64K segments (each drawn
+    from its own seed), the state carried from segment to segment.  The 1M step is one
+    kda_chunk_fwd_segmented call (64K stretches, each stretch's prep overlapping the scan of the
+    one before); the same work as 16 kda_chunk_fwd calls is timed beside it
+    (`sequential_calls`) and both are checked to give the same final state bit for bit."""
     names = ("q", "k", "v", "a", "beta")
     B, H, D = sw.B, sw.H, sw.dk
+    seq = None
     if sw.segment:
-        nseg = sw.T // sw.segment
-        segs = []
+        nseg, seg = sw.T // sw.segment, sw.segment
+        full = {n: torch.empty((B, sw.T, H) + (() if n == "beta" else (D,)), dtype=torch.bfloat16, device=device)
+                for n in names}
         for i in range(nseg):
             if rank == 0:
                 xi = synth.workload_inputs(sw, segment_index=i)
             else:  # every rank its own sequence
-                xi = synth.make_inputs(B, sw.segment, H, D, D, sw.dtype, rank_seed(sw.seed * 1000 + i, rank),
-                                       sw.s0_std)
-            segs.append({n: xi[n].to(device) for n in names})
+                xi = synth.make_inputs(B, seg, H, D, D, sw.dtype, rank_seed(sw.seed * 1000 + i, rank), sw.s0_std)
+            for n in names:
+                full[n][:, i * seg:(i + 1) * seg].copy_(xi[n])
             if i == 0:
                 S0 = xi["S0"].to(device)
             del xi
-        Tc = sw.segment
+        o = torch.empty((B, sw.T, H, D), dtype=torch.bfloat16, device=device)
+        S = torch.empty_like(S0)
+        ws = torch.empty(kda.kda_chunk_fwd_workspace(B, seg, H, D, D), dtype=torch.uint8, device=device)
+        ws2 = torch.empty(kda.kda_chunk_fwd_segmented_workspace(B, sw.T, H, D, D, seg), dtype=torch.uint8,
+                          device=device)
+
+        def step_calls():
+            S.copy_(S0)
+            for i in range(nseg):
+                sl = slice(i * seg, (i + 1) * seg)
+                kda.kda_chunk_fwd(*(full[n][:, sl] for n in names), G_MIN, S0=S, o=o[:, sl], S_T=S, workspace=ws)
+
+        def step():
+            S.copy_(S0)
+            kda.kda_chunk_fwd_segmented(*(full[n] for n in names), seg, G_MIN, S0=S, o=o, S_T=S, workspace=ws2)
+
+        steps = max(2, min(args.steps, 3))
+        ms_calls = time_steps(step_calls, steps, 3, world, device)
+        S_calls = S.clone()
+        seq = {"ms_per_step": ms_calls, "value": B * sw.T * world / (ms_calls * 1e-3), "unit": "tokens/s",
+               "calls_per_step": nseg}
+        calls = 1
     else:
         xi = synth.make_inputs(B, sw.T, H, D, D, sw.dtype, rank_seed(sw.seed, rank), sw.s0_std, sw.adversarial)
-        segs = [{n: xi[n].to(device) for n in names}]
+        x = {n: xi[n].to(device) for n in names}
         S0 = xi["S0"].to(device)
         del xi
-        Tc = sw.T
-    S = torch.empty_like(S0)
-    o = torch.empty((B, Tc, H, D), dtype=torch.bfloat16, device=device)
-    ws = torch.empty(kda.kda_chunk_fwd_workspace(B, Tc, H, D, D), dtype=torch.uint8, device=device)
+        S = torch.empty_like(S0)
+        o = torch.empty((B, sw.T, H, D), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(kda.kda_chunk_fwd_workspace(B, sw.T, H, D, D), dtype=torch.uint8, device=device)
+        nseg, calls = 1, 1
 
-    def step():
-        S.copy_(S0)
-        for sd in segs:
-            kda.kda_chunk_fwd(*(sd[n] for n in names), G_MIN, S0=S, o=o, S_T=S, workspace=ws)
+        def step():
+            S.copy_(S0)
+            kda.kda_chunk_fwd(*(x[n] for n in names), G_MIN, S0=S, o=o, S_T=S, workspace=ws)
 
-    steps = max(2, min(args.steps, 10 if not sw.segment else 3))
+        steps = max(2, min(args.steps, 10))
     with ClockSampler(device.index) as clk:
         ms = time_steps(step, steps, 3, world, device)
     assert kda.kda_device_status(device) == 0
     out = {"workload": sw.name, "B": B, "T": sw.T, "H": H, "dk": D, "dv": D, "steps": steps,
-           "calls_per_step": len(segs), "gpu_launches_per_step": 3 * len(segs),
+           "calls_per_step": calls, "gpu_launches_per_step": 3 * nseg,
            "l2": "inputs exceed the 126 MB L2; no flush"}
+    if seq is not None:
+        out["entry"] = f"kda_chunk_fwd_segmented, {sw.segment}-token stretches"
+        seq["same_final_state"] = bool(torch.equal(S, S_calls))
+        out["sequential_calls"] = seq
     out.update(stage_metrics(B * sw.T, B * sw.T * H, B * H, ms, world, hbm_peak, bf16_peak, peak_kind))
     out["clocks"] = clk.summary()
-    del segs, ws, o
     return out
 
 

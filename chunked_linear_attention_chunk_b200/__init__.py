@@ -64,6 +64,8 @@ EXPORTS = (
     "kda_chunk_bwd",
     "kda_chunk_bwd_varlen_workspace",
     "kda_chunk_bwd_varlen",
+    "kda_chunk_fwd_segmented_workspace",
+    "kda_chunk_fwd_segmented",
 )
 
 
@@ -133,6 +135,10 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_bwd_varlen_workspace.restype = S
     L.kda_chunk_bwd_varlen.argtypes = [I, P, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     L.kda_chunk_bwd_varlen.restype = I
+    L.kda_chunk_fwd_segmented_workspace.argtypes = [I, I, I, I, I, I]
+    L.kda_chunk_fwd_segmented_workspace.restype = S
+    L.kda_chunk_fwd_segmented.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, S, P]
+    L.kda_chunk_fwd_segmented.restype = I
     _lib = L
     return L
 
@@ -221,6 +227,39 @@ def kda_chunk_fwd(q, k, v, a, beta, g_min: float = -5.0, S0=None, o=None, S_T=No
                              float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
                              _stream(q.device))
     _raise(st, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_chunk_fwd_segmented_workspace(B: int, T: int, H: int, dk: int, dv: int, seg_T: int) -> int:
+    return int(lib().kda_chunk_fwd_segmented_workspace(B, T, H, dk, dv, seg_T))
+
+
+def kda_chunk_fwd_segmented(q, k, v, a, beta, seg_T: int, g_min: float = -5.0, S0=None, o=None, S_T=None,
+                            workspace=None):
+    """``kda_chunk_fwd`` (bf16) taken ``seg_T`` tokens at a time (a multiple of 64), the prep of
+    each stretch overlapping the scan of the one before; bit for bit the same result.  Returns
+    (o, S_T); S_T may be S0 (in place)."""
+    _check_cuda(q, k, v, a, beta, S0, o, S_T, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    for t in (k, v, a, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, a, beta must share one dtype")
+    if k.shape != q.shape or a.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch: q,k,a [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(lib().kda_chunk_fwd_segmented_workspace(B, T, H, dk, dv, int(seg_T)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd_segmented(B, T, H, dk, dv, code, int(seg_T), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                       _ptr(beta), float(g_min), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                       ws_bytes, _stream(q.device))
+    _raise(st, "kda_chunk_fwd_segmented")
     return o, S_T
 
 

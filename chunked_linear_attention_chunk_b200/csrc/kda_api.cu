@@ -498,6 +498,106 @@ kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *w
     return from_cuda(launch_scan_bf16(B, T, H, dk, workspace, S0, o, S_T, (cudaStream_t)stream));
 }
 
+// Two stretches' records, each slot rounded up to 256 bytes.
+size_t kda_chunk_fwd_segmented_workspace(int B, int T, int H, int dk, int dv, int seg_T)
+{
+    if (seg_T < KDA_CHUNK || seg_T % KDA_CHUNK != 0 || T < 0)
+        return 0;
+    const size_t slot = kda_chunk_fwd_workspace(1, T < seg_T ? T : seg_T, H, dk, dv, KDA_BF16);
+    if (B < 1 || slot == 0)
+        return 0;
+    return 2 * ((slot + 255) / 256 * 256);
+}
+
+kda_status kda_chunk_fwd_segmented(int B, int T, int H, int dk, int dv, kda_dtype dtype, int seg_T, const void *q,
+                                   const void *k, const void *v, const void *a, const void *beta, float g_min,
+                                   const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                                   kda_stream_t stream)
+{
+    ChunkShape sh;
+    kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
+    if (st != KDA_OK)
+        return st;
+    if (dtype != KDA_BF16)
+        return KDA_ERR_UNSUPPORTED;
+    if (seg_T < KDA_CHUNK || seg_T % KDA_CHUNK != 0 || !S_T)
+        return KDA_ERR_INVALID_ARG;
+    // every check of kda_chunk_fwd on the whole problem, the workspace range included
+    st = validate_chunk_fwd(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, KDA_GATE_BOUNDED, S0, o, S_T,
+                            workspace, ws_bytes, false);
+    if (st != KDA_OK)
+        return st;
+    const cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0)
+        return copy_state(sh, S0, S_T, s);
+    const size_t need = kda_chunk_fwd_segmented_workspace(B, T, H, dk, dv, seg_T);
+    if (!workspace || ws_bytes < need)
+        return KDA_ERR_WORKSPACE;
+    const int nseg = (T + seg_T - 1) / seg_T, units = B * nseg;
+    const size_t slot = need / 2;
+    unsigned char *ws[2] = {static_cast<unsigned char *>(workspace), static_cast<unsigned char *>(workspace) + slot};
+    const int64_t tok = (int64_t)H * dk * 2, st_elems = (int64_t)H * dk * dv;  // bytes per token row; state floats
+    auto at = [](const void *p, int64_t off) { return static_cast<const unsigned char *>(p) + off; };
+
+    // two streams of this call (released once their work is done): the preps at the lowest
+    // priority, the scans at the highest, so that a scan's CTAs are placed ahead of the next
+    // prep's; both start after the work already on `stream`, which waits for the last scan
+    int lo = 0, hi = 0;
+    cudaStream_t sp = nullptr, sc = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_prep = nullptr, ev_scan[2] = {nullptr, nullptr};
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e == cudaSuccess)
+        e = cudaStreamCreateWithPriority(&sp, cudaStreamNonBlocking, lo);
+    if (e == cudaSuccess)
+        e = cudaStreamCreateWithPriority(&sc, cudaStreamNonBlocking, hi);
+    for (cudaEvent_t *ev : {&ev_start, &ev_prep, &ev_scan[0], &ev_scan[1]})
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e == cudaSuccess)
+        e = cudaEventRecord(ev_start, s);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(sp, ev_start, 0);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(sc, ev_start, 0);
+    // unit u = (batch element b, stretch i): the prep on `sp` (after the scan that last read its
+    // slot), the scan on `sc` after that prep, the state carried in S_T
+    int last = -1;  // the last unit whose scan is recorded
+    for (int u = 0; u < units && e == cudaSuccess; ++u) {
+        const int b = u / nseg, i = u % nseg, t0 = i * seg_T, len = T - t0 < seg_T ? T - t0 : seg_T;
+        const int64_t row = (int64_t)b * T + t0;  // first token row of the stretch
+        if (u >= 2)
+            e = cudaStreamWaitEvent(sp, ev_scan[u & 1], 0);
+        if (e == cudaSuccess)
+            e = launch_prep_bf16(1, len, H, dk, at(q, row * tok), at(k, row * tok), at(v, row * tok),
+                                 at(a, row * tok), at(beta, row * H * 2), g_min, false, nullptr, ws[u & 1], sp);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(ev_prep, sp);
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(sc, ev_prep, 0);
+        if (e == cudaSuccess) {
+            float *Sb = S_T + (int64_t)b * st_elems;
+            const float *Sin = i > 0 ? Sb : (S0 ? S0 + (int64_t)b * st_elems : nullptr);
+            e = launch_scan_bf16(1, len, H, dk, ws[u & 1], Sin, static_cast<unsigned char *>(o) + row * (int64_t)H * dv * 2,
+                                 Sb, sc);
+        }
+        if (e == cudaSuccess && (e = cudaEventRecord(ev_scan[u & 1], sc)) == cudaSuccess)
+            last = u;
+    }
+    if (last >= 0) {  // later work on `stream` follows the last scan, which follows every prep
+        const cudaError_t ej = cudaStreamWaitEvent(s, ev_scan[last & 1], 0);
+        if (e == cudaSuccess)
+            e = ej;
+    }
+    // (destroying an event or a stream whose work is pending releases it once that work is done)
+    for (cudaEvent_t ev : {ev_start, ev_prep, ev_scan[0], ev_scan[1]})
+        if (ev)
+            cudaEventDestroy(ev);
+    for (cudaStream_t st2 : {sp, sc})
+        if (st2)
+            cudaStreamDestroy(st2);
+    return from_cuda(e);
+}
+
 kda_status kda_decode_step(int N, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k, const void *v,
                            const void *a, const void *beta, float g_min, float *S, void *o, kda_stream_t stream)
 {

@@ -245,6 +245,41 @@ kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *w
                               const float *S0, void *o, float *S_T, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_segmented -- the bf16 chunked forward of long sequences, taken seg_T tokens
+ * at a time with the state carried, the prep of each stretch overlapping the scan of the one
+ * before it.  The result equals kda_chunk_fwd on the whole problem bit for bit (stretches are
+ * whole 64-token chunks and the state is carried in float32 either way).
+ * Passages: the context stages of long-context training, up to 1M tokens ("Trillion-Scale
+ * ..." section 2.3; "Trillion-Parameter MoE ... Engineering" section 5.1), over the chunk
+ * recursion with a constant-size state ("... Engineering" section 3.2).
+ * Why: a stretch's scan is serial over its chunks and occupies one SM per (head, 32 value
+ * columns), so with few heads (the 1M stage's 16: 64 of 148 SMs) most SMs idle while it
+ * runs; the next stretch's prep, which does not depend on the state, fills them.
+ *   B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, S0, o:  as in kda_chunk_fwd; dtype must
+ *              be KDA_BF16 (the bounded gate, as kda_chunk_fwd).
+ *   seg_T      tokens per stretch: a positive multiple of 64.  Each batch element's
+ *              sequence is cut into ceil(T / seg_T) stretches (the last may be shorter), and
+ *              the stretches of all elements run in order, element by element.
+ *   S_T        [B, H, dk, dv] float32, required (it carries the state from stretch to
+ *              stretch); may be the same pointer as S0.
+ *   workspace  at least kda_chunk_fwd_segmented_workspace(...) bytes (two stretches'
+ *              records), 16-byte aligned, overlapping no tensor argument.
+ *   stream     the preps run on it; the scans run on a second stream of the library (one
+ *              per device, created on first use at the highest priority, so that a scan's
+ *              CTAs are placed ahead of the next prep's), ordered by events.  When the call
+ *              returns, every launch is ordered before later work on `stream`.  The call
+ *              creates and destroys three CUDA events; it is not meant for stream capture.
+ * Errors: INVALID_ARG (seg_T not a positive multiple of 64, S_T NULL), UNSUPPORTED (dtype
+ * not KDA_BF16, shapes kda_chunk_fwd rejects), ALIGNMENT, ALIAS, WORKSPACE, CUDA.  Every
+ * check is done before the first launch.  T == 0 copies S0 (or zeros) to S_T.
+ */
+size_t kda_chunk_fwd_segmented_workspace(int B, int T, int H, int dk, int dv, int seg_T);
+kda_status kda_chunk_fwd_segmented(int B, int T, int H, int dk, int dv, kda_dtype dtype, int seg_T, const void *q,
+                                   const void *k, const void *v, const void *a, const void *beta, float g_min,
+                                   const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                                   kda_stream_t stream);
+
+/*
  * Sequence parallelism: one long sequence split into R consecutive segments, one per GPU
  * ("Breaking Through ..." section 3: sequence parallelism for the million-token stage).
  * Over a segment the state map is affine, S_out = M S_in + S_zero, with M the product of

@@ -442,3 +442,41 @@ def test_noalloc_validates_the_whole_problem_before_launching(L):
     assert _noalloc(L, q=BASE + 8) == ALIGN
     assert _noalloc(L, o=BASE) == ALIAS
     assert _noalloc(L, S0=S, ST=S + 4096) == ALIAS
+
+
+def _segmented(L, B=1, T=1000, H=2, dk=128, dv=128, dt=kda.KDA_BF16, seg=256, q=None, o=None, S0=None,
+               ST=BASE * 3, ws=None, ws_bytes=None, g_min=-5.0):
+    es = 2 if dt == kda.KDA_BF16 else 4
+    n = B * T * H * max(dk, 1) * es
+    q = BASE if q is None else q
+    k, v, a, beta = (BASE + i * (n + 4096) for i in (1, 2, 3, 4))
+    o = BASE + 5 * (n + 4096) if o is None else o
+    ws = BASE + 6 * (n + 4096) if ws is None else ws
+    need = L.kda_chunk_fwd_segmented_workspace(B, T, H, dk, dv, seg)
+    ws_bytes = need if ws_bytes is None else ws_bytes
+    P = ctypes.c_void_p
+    return L.kda_chunk_fwd_segmented(B, T, H, dk, dv, dt, seg, P(q), P(k), P(v), P(a), P(beta), ctypes.c_float(g_min),
+                                     P(S0), P(o), P(ST), P(ws), ws_bytes, None)
+
+
+def test_segmented_entry_sizes_and_validates(L):
+    """kda_chunk_fwd_segmented: two stretches' records of workspace, and every argument check
+    (its own and kda_chunk_fwd's) before any launch."""
+    f = L.kda_chunk_fwd_segmented_workspace
+    one = L.kda_chunk_fwd_workspace(1, 256, 2, 128, 128, kda.KDA_BF16)
+    assert f(1, 1000, 2, 128, 128, 256) == 2 * ((one + 255) // 256 * 256)
+    assert f(3, 1000, 2, 128, 128, 256) == f(1, 1000, 2, 128, 128, 256)  # per stretch, not per batch
+    short = L.kda_chunk_fwd_workspace(1, 100, 2, 128, 128, kda.KDA_BF16)
+    assert f(1, 100, 2, 128, 128, 256) == 2 * ((short + 255) // 256 * 256)  # T < seg_T
+    for bad in (0, 32, 100, -64):
+        assert f(1, 1000, 2, 128, 128, bad) == 0
+        assert _segmented(L, seg=bad) == INVALID
+    assert _segmented(L, ST=None) == INVALID                 # S_T carries the state
+    assert _segmented(L, dt=kda.KDA_F32) == UNSUPPORTED
+    assert _segmented(L, dk=96, dv=96) == UNSUPPORTED
+    assert _segmented(L, g_min=-6.0) == UNSUPPORTED
+    assert _segmented(L, q=BASE + 8) == ALIGN
+    assert _segmented(L, ws_bytes=f(1, 1000, 2, 128, 128, 256) - 1) == WS
+    assert _segmented(L, ws=0) == WS
+    assert _segmented(L, o=BASE) == ALIAS                    # o over q
+    assert _segmented(L, S0=BASE * 3, ST=BASE * 3 + 4096) == ALIAS

@@ -533,7 +533,7 @@ kda_status kda_chunk_fwd_segmented(int B, int T, int H, int dk, int dv, kda_dtyp
     const size_t need = kda_chunk_fwd_segmented_workspace(B, T, H, dk, dv, seg_T);
     if (!workspace || ws_bytes < need)
         return KDA_ERR_WORKSPACE;
-    const int nseg = (T + seg_T - 1) / seg_T, units = B * nseg;
+    const int64_t nseg = ((int64_t)T + seg_T - 1) / seg_T, units = (int64_t)B * nseg;
     const size_t slot = need / 2;
     unsigned char *ws[2] = {static_cast<unsigned char *>(workspace), static_cast<unsigned char *>(workspace) + slot};
     const int64_t tok = (int64_t)H * dk * 2, st_elems = (int64_t)H * dk * dv;  // bytes per token row; state floats
@@ -561,10 +561,11 @@ kda_status kda_chunk_fwd_segmented(int B, int T, int H, int dk, int dv, kda_dtyp
         e = cudaStreamWaitEvent(sc, ev_start, 0);
     // unit u = (batch element b, stretch i): the prep on `sp` (after the scan that last read its
     // slot), the scan on `sc` after that prep, the state carried in S_T
-    int last = -1;  // the last unit whose scan is recorded
-    for (int u = 0; u < units && e == cudaSuccess; ++u) {
-        const int b = u / nseg, i = u % nseg, t0 = i * seg_T, len = T - t0 < seg_T ? T - t0 : seg_T;
-        const int64_t row = (int64_t)b * T + t0;  // first token row of the stretch
+    int64_t last = -1;  // the last unit whose scan is recorded
+    for (int64_t u = 0; u < units && e == cudaSuccess; ++u) {
+        const int64_t b = u / nseg, i = u % nseg, t0 = i * seg_T;
+        const int len = (int)(T - t0 < seg_T ? T - t0 : seg_T);
+        const int64_t row = b * T + t0;  // first token row of the stretch
         if (u >= 2)
             e = cudaStreamWaitEvent(sp, ev_scan[u & 1], 0);
         if (e == cudaSuccess)
@@ -575,8 +576,8 @@ kda_status kda_chunk_fwd_segmented(int B, int T, int H, int dk, int dv, kda_dtyp
         if (e == cudaSuccess)
             e = cudaStreamWaitEvent(sc, ev_prep, 0);
         if (e == cudaSuccess) {
-            float *Sb = S_T + (int64_t)b * st_elems;
-            const float *Sin = i > 0 ? Sb : (S0 ? S0 + (int64_t)b * st_elems : nullptr);
+            float *Sb = S_T + b * st_elems;
+            const float *Sin = i > 0 ? Sb : (S0 ? S0 + b * st_elems : nullptr);
             e = launch_scan_bf16(1, len, H, dk, ws[u & 1], Sin, static_cast<unsigned char *>(o) + row * (int64_t)H * dv * 2,
                                  Sb, sc);
         }

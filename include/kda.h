@@ -264,11 +264,12 @@ kda_status kda_chunk_fwd_scan(int B, int T, int H, int dk, int dv, const void *w
  *              stretch); may be the same pointer as S0.
  *   workspace  at least kda_chunk_fwd_segmented_workspace(...) bytes (two stretches'
  *              records), 16-byte aligned, overlapping no tensor argument.
- *   stream     the preps run on it; the scans run on a second stream of the library (one
- *              per device, created on first use at the highest priority, so that a scan's
- *              CTAs are placed ahead of the next prep's), ordered by events.  When the call
- *              returns, every launch is ordered before later work on `stream`.  The call
- *              creates and destroys three CUDA events; it is not meant for stream capture.
+ *   stream     the call's work starts after the work already on it and the work queued on
+ *              it later follows the call's.  Inside, the preps run on a stream of the call
+ *              at the lowest priority and the scans on one at the highest (so that a scan's
+ *              CTAs are placed ahead of the next prep's), ordered by events.  The call
+ *              creates two streams and four events and releases them (CUDA frees them once
+ *              their work is done); it is not meant for stream capture.
  * Errors: INVALID_ARG (seg_T not a positive multiple of 64, S_T NULL), UNSUPPORTED (dtype
  * not KDA_BF16, shapes kda_chunk_fwd rejects), ALIGNMENT, ALIAS, WORKSPACE, CUDA.  Every
  * check is done before the first launch.  T == 0 copies S0 (or zeros) to S_T.

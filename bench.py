@@ -595,7 +595,27 @@ def run_libkda(args):
                "dominant_kernel": {"kernel": "bwd_chunk_kernel (per-chunk gradients)",
                                    "algorithmic_bytes_per_token_head": BWD_CHUNK_BYTES_PER_TOKEN_HEAD,
                                    "traffic": None if bwd_traffic is None else bwd_traffic * token_heads}}
-        del ws_b, gout
+        # a training step's two calls on these inputs: the forward, then the backward; the forward
+        # writes its records into the backward's workspace, which kda_chunk_bwd_recorded reuses
+        # instead of running the prep again (kda_chunk_bwd recomputes them)
+        o_t = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=device)
+
+        def train_step(recorded):
+            kda.kda_chunk_fwd(*(d[n] for n in names), G_MIN, S0=S0, o=o_t, workspace=ws_b, return_state=False)
+            if recorded:
+                gout.update(kda.kda_chunk_bwd_recorded(*(d[n] for n in names), dO, ws_b, G_MIN, S0=S0, out=gout))
+            else:
+                gout.update(kda.kda_chunk_bwd(*(d[n] for n in names), dO, G_MIN, S0=S0, workspace=ws_b, out=gout))
+
+        n_tr = max(3, min(args.steps, 5))
+        tr_plain = time_steps(lambda: train_step(False), n_tr, 3, world, device)
+        tr_rec = time_steps(lambda: train_step(True), n_tr, 3, world, device)
+        assert kda.kda_device_status(device) == 0
+        bwd["training_step"] = {"what": "kda_chunk_fwd then kda_chunk_bwd_recorded (the backward reusing the "
+                                        "forward's records from its workspace)",
+                                "ms_per_step": tr_rec, "value": world * tokens / (tr_rec * 1e-3), "unit": UNIT,
+                                "ms_with_kda_chunk_bwd": tr_plain, "gpu_launches_per_step": 6}
+        del ws_b, gout, o_t
         # the same over the packed batch of the varlen leg (documents of mixed length)
         if (B, T, H) == (1, synth.VARLEN_64K_T, synth.VARLEN_64K_H):
             lengths = synth.document_lengths(T)

@@ -66,6 +66,7 @@ EXPORTS = (
     "kda_chunk_bwd_varlen",
     "kda_chunk_fwd_segmented_workspace",
     "kda_chunk_fwd_segmented",
+    "kda_chunk_bwd_recorded",
 )
 
 
@@ -139,6 +140,8 @@ def lib() -> ctypes.CDLL:
     L.kda_chunk_fwd_segmented_workspace.restype = S
     L.kda_chunk_fwd_segmented.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, S, P]
     L.kda_chunk_fwd_segmented.restype = I
+    L.kda_chunk_bwd_recorded.argtypes = L.kda_chunk_bwd.argtypes
+    L.kda_chunk_bwd_recorded.restype = I
     _lib = L
     return L
 
@@ -304,7 +307,7 @@ def _bwd_checks(q, k, v, a, beta, dO, A_log, token_dims):
 
 
 def kda_chunk_bwd(q, k, v, a, beta, dO, g_min: float = -5.0, S0=None, dS_T=None, workspace=None,
-                  return_dS0: bool = True, out=None, A_log=None):
+                  return_dS0: bool = True, out=None, A_log=None, _recorded: bool = False):
     """Gradients of the bf16 chunked forward.  q, k, a [B,T,H,dk], v and dO [B,T,H,dv],
     beta [B,T,H] (bfloat16); S0 and dS_T [B,H,dk,dv] float32 or None (zeros); A_log float32
     [H] or None (the gate's per-head scale e^{A_log[h]}).  Returns a dict of float32 tensors
@@ -319,12 +322,24 @@ def kda_chunk_bwd(q, k, v, a, beta, dO, g_min: float = -5.0, S0=None, dS_T=None,
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().kda_chunk_bwd(B, T, H, dk, dv, KDA_BF16, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
-                             float(g_min), _ptr(A_log), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]),
-                             _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), _ptr(g["dA_log"]),
-                             _ptr(workspace), ws_bytes, _stream(q.device))
-    _raise(st, "kda_chunk_bwd")
+    fn = lib().kda_chunk_bwd_recorded if _recorded else lib().kda_chunk_bwd
+    st = fn(B, T, H, dk, dv, KDA_BF16, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta),
+            float(g_min), _ptr(A_log), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["dq"]), _ptr(g["dk"]),
+            _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), _ptr(g["dA_log"]),
+            _ptr(workspace), ws_bytes, _stream(q.device))
+    _raise(st, "kda_chunk_bwd_recorded" if _recorded else "kda_chunk_bwd")
     return g
+
+
+def kda_chunk_bwd_recorded(q, k, v, a, beta, dO, workspace, g_min: float = -5.0, S0=None, dS_T=None,
+                           return_dS0: bool = True, out=None, A_log=None):
+    """``kda_chunk_bwd`` when ``workspace`` (at least ``kda_chunk_bwd_workspace`` bytes) already
+    holds the records a bf16 ``kda_chunk_fwd`` (or ``kda_chunk_fwd_prep``) wrote into it for the
+    same inputs, g_min and A_log: the backward's own prep is skipped."""
+    if workspace is None:
+        raise ValueError("kda_chunk_bwd_recorded needs the workspace the forward wrote its records to")
+    return kda_chunk_bwd(q, k, v, a, beta, dO, g_min, S0=S0, dS_T=dS_T, workspace=workspace, return_dS0=return_dS0,
+                         out=out, A_log=A_log, _recorded=True)
 
 
 def kda_chunk_bwd_varlen_workspace(N: int, T: int, H: int, dk: int, dv: int) -> int:

@@ -2441,6 +2441,9 @@ struct BwdLayout {
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+// A regular batch's backward workspace starts like the forward's: the records, then the gate
+// table right after them (no padding), so the forward's prep output can be used in place.
+static_assert(Rec<64>::Bytes % 256 == 0 && Rec<128>::Bytes % 256 == 0, "gate table at the forward's offset");
 
 BwdLayout bwd_layout(int64_t nrec, int64_t nunits, int D, int H, int nseq_packed = 0)
 {
@@ -2462,7 +2465,8 @@ template <int D>
 cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits, const BwdLayout &l,
                          const void *q, const void *k, const void *v, const void *a, const void *beta, float g_min,
                          const float *A_log, const float *S0, const void *dO, const float *dS_T, float *dq, float *dk,
-                         float *dv, float *da, float *dbeta, float *dS0, float *dA_log, void *ws, cudaStream_t s)
+                         float *dv, float *da, float *dbeta, float *dS0, float *dA_log, void *ws, cudaStream_t s,
+                         bool have_records = false)
 {
     unsigned int *status = device_status_ptr();
     if (!status)
@@ -2472,7 +2476,10 @@ cudaError_t launch_bwd_d(const SeqMap &m, int H, dim3 prep_grid, int64_t nunits,
     float *parts = dA_log ? reinterpret_cast<float *>(base + l.parts) : nullptr;
     float *scratch = reinterpret_cast<float *>(base + l.scratch);
     float *gtab = reinterpret_cast<float *>(base + l.gtab);
-    cudaError_t e = launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s);
+    // the records and the gate table (same offsets as the forward's workspace) unless the
+    // forward's prep already wrote them there
+    cudaError_t e = have_records ? cudaSuccess
+                                 : launch_prep_d<D, false>(m, H, prep_grid, q, k, v, a, beta, g_min, A_log, ws, gtab, s);
     if (e == cudaSuccess)
         e = launch_scan_d<D>(m, H, ws, S0, nullptr, nullptr, nullptr, s, Hs);
     if (e != cudaSuccess)
@@ -2613,15 +2620,16 @@ void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *
 cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
                                   const void *a, const void *beta, float g_min, const float *A_log, const float *S0,
                                   const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da,
-                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s)
+                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s,
+                                  bool have_records)
 {
     const SeqMap m = regular_map(B, T, H);
     const dim3 grid(m.NT, B * H);
     const BwdLayout l = bwd_layout(m.nrec, m.nrec, D, H);
     return D == 64 ? launch_bwd_d<64>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk, dv,
-                                      da, dbeta, dS0, dA_log, workspace, s)
+                                      da, dbeta, dS0, dA_log, workspace, s, have_records)
                    : launch_bwd_d<128>(m, H, grid, m.nrec, l, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk,
-                                       dv, da, dbeta, dS0, dA_log, workspace, s);
+                                       dv, da, dbeta, dS0, dA_log, workspace, s, have_records);
 }
 
 size_t chunk_bf16_bwd_varlen_workspace(int N, int T, int H, int D)

@@ -657,11 +657,17 @@ kda_status kda_chunk_bwd_offsets(int B, int T, int H, int dk, int dv, size_t *st
     return KDA_OK;
 }
 
-kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
-                         const void *v, const void *a, const void *beta, float g_min, const float *A_log,
-                         const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
-                         float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
-                         kda_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// Validation and dispatch of kda_chunk_bwd and kda_chunk_bwd_recorded (have_records: the
+// workspace holds the forward's records; the prep is not launched).
+kda_status chunk_bwd_impl(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                          const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                          const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
+                          float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
+                          kda_stream_t stream, bool have_records)
 {
     ChunkShape sh;
     kda_status st = check_shape(B, T, H, dk, dv, dtype, sh);
@@ -716,7 +722,31 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
                 return KDA_ERR_ALIAS;
     }
     return from_cuda(launch_chunk_bwd_bf16(B, T, H, dk, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk_, dv_,
-                                           da, dbeta, dS0, dA_log, workspace, s));
+                                           da, dbeta, dS0, dA_log, workspace, s, have_records));
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                         const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                         const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
+                         float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
+                         kda_stream_t stream)
+{
+    return chunk_bwd_impl(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk_, dv_, da,
+                          dbeta, dS0, dA_log, workspace, ws_bytes, stream, false);
+}
+
+kda_status kda_chunk_bwd_recorded(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                                  const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                                  const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_,
+                                  float *dv_, float *da, float *dbeta, float *dS0, float *dA_log, void *workspace,
+                                  size_t ws_bytes, kda_stream_t stream)
+{
+    return chunk_bwd_impl(B, T, H, dk, dv, dtype, q, k, v, a, beta, g_min, A_log, S0, dO, dS_T, dq, dk_, dv_, da,
+                          dbeta, dS0, dA_log, workspace, ws_bytes, stream, true);
 }
 
 size_t kda_chunk_bwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype)

@@ -69,7 +69,10 @@ void chunk_bf16_bwd_offsets(int B, int T, int H, int D, size_t *states, size_t *
 cudaError_t launch_chunk_bwd_bf16(int B, int T, int H, int D, const void *q, const void *k, const void *v,
                                   const void *a, const void *beta, float g_min, const float *A_log, const float *S0,
                                   const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *da,
-                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s);
+                                  float *dbeta, float *dS0, float *dA_log, void *workspace, cudaStream_t s,
+                                  bool have_records = false);
+// (have_records: the workspace already holds the records and gate table the forward's prep
+// wrote for the same inputs, at the same offsets; the prep is not launched again.)
 // The same over a packed batch (cu on the device, checked on the device as in the forward).
 size_t chunk_bf16_bwd_varlen_workspace(int N, int T, int H, int D);
 cudaError_t launch_chunk_bwd_bf16_varlen(int N, const int32_t *cu, int T, int H, int D, const void *q, const void *k,

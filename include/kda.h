@@ -357,6 +357,21 @@ kda_status kda_chunk_bwd(int B, int T, int H, int dk, int dv, kda_dtype dtype, c
                          const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_, float *dv_,
                          float *da, float *dbeta, float *dS0, float *dA_log, void *workspace, size_t ws_bytes,
                          kda_stream_t stream);
+/*
+ * kda_chunk_bwd_recorded -- kda_chunk_bwd for a training step that keeps the forward's
+ * records: the backward's workspace starts with the same layout as kda_chunk_fwd's (the
+ * records, then the gate table), so a bf16 kda_chunk_fwd (or kda_chunk_fwd_prep with the
+ * same gate and A_log) given this workspace writes exactly what kda_chunk_bwd's first launch
+ * would; this call skips that launch and runs the other three.  Same arguments, checks and
+ * errors as kda_chunk_bwd; the gradients equal kda_chunk_bwd's bit for bit when the records
+ * come from the same q, k, v, a, beta, g_min and A_log, ordered before this call.  Other
+ * contents give unspecified gradients but no access outside the buffers.
+ */
+kda_status kda_chunk_bwd_recorded(int B, int T, int H, int dk, int dv, kda_dtype dtype, const void *q, const void *k,
+                                  const void *v, const void *a, const void *beta, float g_min, const float *A_log,
+                                  const float *S0, const void *dO, const float *dS_T, float *dq, float *dk_,
+                                  float *dv_, float *da, float *dbeta, float *dS0, float *dA_log, void *workspace,
+                                  size_t ws_bytes, kda_stream_t stream);
 size_t kda_chunk_bwd_varlen_workspace(int N, int T, int H, int dk, int dv, kda_dtype dtype);
 kda_status kda_chunk_bwd_varlen(int N, const int32_t *cu_seqlens, int T, int H, int dk, int dv, kda_dtype dtype,
                                 float g_min, const float *A_log, const void *q, const void *k, const void *v,

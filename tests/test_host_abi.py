@@ -321,9 +321,10 @@ def test_debug_build_exports_the_same_entry_points():
     assert set(declared_functions()) <= exported
 
 
-def test_chunk_bwd_entry_validates(L):
-    """kda_chunk_bwd rejects every bad argument before a launch (fake pointers: none of
-    these calls may pass validation)."""
+@pytest.mark.parametrize("entry", ["kda_chunk_bwd", "kda_chunk_bwd_recorded"])
+def test_chunk_bwd_entry_validates(L, entry):
+    """kda_chunk_bwd (and kda_chunk_bwd_recorded, which shares its checks) rejects every bad
+    argument before a launch (fake pointers: none of these calls may pass validation)."""
     P = ctypes.c_void_p
     B, T, H, D = 1, 64, 1, 128
     nb = B * T * H * D * 2
@@ -338,14 +339,14 @@ def test_chunk_bwd_entry_validates(L):
 
     def bwd(dtype=kda.KDA_BF16, g_min=-5.0, q=ins[0], dO=ins[5], dq=outs[0], dbeta=outs[4], w=ws, wb=need,
             S0=None, dST=None, dS0=None, dk=D, A=None, dA=None):
-        return L.kda_chunk_bwd(B, T, H, dk, dk, dtype, P(q), P(ins[1]), P(ins[2]), P(ins[3]), P(ins[4]),
-                               ctypes.c_float(g_min), P(A), P(S0), P(dO), P(dST), P(dq), P(outs[1]), P(outs[2]),
-                               P(outs[3]), P(dbeta), P(dS0), P(dA), P(w), wb, None)
+        return getattr(L, entry)(B, T, H, dk, dk, dtype, P(q), P(ins[1]), P(ins[2]), P(ins[3]), P(ins[4]),
+                                 ctypes.c_float(g_min), P(A), P(S0), P(dO), P(dST), P(dq), P(outs[1]), P(outs[2]),
+                                 P(outs[3]), P(dbeta), P(dS0), P(dA), P(w), wb, None)
 
     assert bwd(dtype=kda.KDA_F32) == UNSUPPORTED
     assert bwd(dk=96) == UNSUPPORTED
     # the saved state arrays are (records x dk) rows addressed with 32-bit row indices
-    big = lambda T_, H_, dk_: L.kda_chunk_bwd(1, T_, H_, dk_, dk_, kda.KDA_BF16, *([P(BASE)] * 5), ctypes.c_float(-5.0),
+    big = lambda T_, H_, dk_: getattr(L, entry)(1, T_, H_, dk_, dk_, kda.KDA_BF16, *([P(BASE)] * 5), ctypes.c_float(-5.0),
                                               None, None, P(BASE), None, *([P(BASE)] * 5), None, None, P(BASE), 1, None)
     assert big(64 * (1 << 16), 256, 128) == UNSUPPORTED   # 2^24 records x 128 rows each
     assert big(64 * (1 << 16), 256, 64) != UNSUPPORTED    # 2^24 records x 64 rows: within range
